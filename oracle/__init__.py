@@ -1,0 +1,192 @@
+"""The CPU oracle for the KV-cache compression path -- TEST INFRASTRUCTURE.
+
+A plain, slow, obviously correct restatement of what the path computes (the C source
+``kvq_oracle.c`` holds the arithmetic; this module only marshals numpy arrays through
+ctypes).  Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import it.  It shares no code with the CUDA library.
+
+Pinned by ``tests/test_oracle_pins.py`` against worked examples, invariants, closed forms
+and brute force (see that file); no function here is "parity unpinned".
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+F32, F16 = 0, 1
+KEYS_INT8, KEYS_QJL = 0, 1
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        I32 = ctypes.c_int
+        lib.ora_half_to_double.argtypes = [ctypes.c_uint16]
+        lib.ora_half_to_double.restype = ctypes.c_double
+        lib.ora_double_to_half.argtypes = [ctypes.c_double]
+        lib.ora_double_to_half.restype = ctypes.c_uint16
+        lib.ora_quantize_int8.argtypes = [P, I32, I64, I64, P, P]
+        lib.ora_dequantize_int8.argtypes = [P, P, I64, I64, P, I32]
+        lib.ora_int8_scores.argtypes = [P, I32, P, P, I64, I64, P]
+        lib.ora_qjl_encode.argtypes = [P, I64, I32, P, I32, P, P, P]
+        lib.ora_qjl_query_sketch.argtypes = [P, I32, I64, I32, P, I32, P, P]
+        lib.ora_qjl_estimate.argtypes = [P, P, ctypes.c_double, I32]
+        lib.ora_qjl_estimate.restype = ctypes.c_double
+        lib.ora_qjl_scores.argtypes = [P, I64, P, P, I64, I32, P]
+        lib.ora_decode_attention.argtypes = [I64, I64, I64, I64, I32, P, I32, P, P, P, P, P,
+                                             I32, P, P, ctypes.c_float, P, P, P]
+        for f in ("ora_quantize_int8", "ora_dequantize_int8", "ora_int8_scores",
+                  "ora_qjl_encode", "ora_qjl_query_sketch", "ora_qjl_scores",
+                  "ora_decode_attention"):
+            getattr(lib, f).restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dtype_code(a):
+    if a.dtype == np.float16:
+        return F16
+    if a.dtype == np.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {a.dtype}")
+
+
+def _check(rc, name):
+    if rc != 0:
+        raise ValueError(f"{name} returned {rc}")
+
+
+def half_to_double(bits: int) -> float:
+    return _load().ora_half_to_double(int(bits))
+
+
+def double_to_half(x: float) -> int:
+    return _load().ora_double_to_half(float(x))
+
+
+def quantize_int8(x: np.ndarray):
+    """Per-row absmax INT8: returns (codes int8 [n, d], scales fp32 [n])."""
+    x = np.ascontiguousarray(x)
+    n, d = x.shape
+    codes = np.empty((n, d), np.int8)
+    scales = np.empty((n,), np.float32)
+    _check(_load().ora_quantize_int8(_ptr(x), _dtype_code(x), n, d, _ptr(codes), _ptr(scales)),
+           "ora_quantize_int8")
+    return codes, scales
+
+
+def dequantize_int8(codes: np.ndarray, scales: np.ndarray, out_dtype=np.float32):
+    codes = np.ascontiguousarray(codes, np.int8)
+    scales = np.ascontiguousarray(scales, np.float32)
+    n, d = codes.shape
+    out = np.empty((n, d), out_dtype)
+    _check(_load().ora_dequantize_int8(_ptr(codes), _ptr(scales), n, d, _ptr(out),
+                                       _dtype_code(out)), "ora_dequantize_int8")
+    return out
+
+
+def int8_scores(q: np.ndarray, codes: np.ndarray, scales: np.ndarray):
+    q = np.ascontiguousarray(q)
+    codes = np.ascontiguousarray(codes, np.int8)
+    scales = np.ascontiguousarray(scales, np.float32)
+    n, d = codes.shape
+    assert q.shape == (d,)
+    out = np.empty((n,), np.float32)
+    _check(_load().ora_int8_scores(_ptr(q), _dtype_code(q), _ptr(codes), _ptr(scales), n, d,
+                                   _ptr(out)), "ora_int8_scores")
+    return out
+
+
+def qjl_encode(keys_f16: np.ndarray, S: np.ndarray, want_u: bool = False):
+    """Sign sketch of fp16 keys [n, d] with sketch matrix S [m, d] (any float dtype, used
+    in fp64).  Returns (words uint32 [n, m/32], norms fp16 [n][, u fp64 [n, m]])."""
+    keys = np.ascontiguousarray(keys_f16, np.float16)
+    S64 = np.ascontiguousarray(S, np.float64)
+    n, d = keys.shape
+    m = S64.shape[0]
+    assert S64.shape[1] == d
+    words = np.empty((n, m // 32), np.uint32)
+    norms = np.empty((n,), np.float16)
+    u = np.empty((n, m), np.float64) if want_u else None
+    _check(_load().ora_qjl_encode(_ptr(keys), n, d, _ptr(S64), m, _ptr(words), _ptr(norms),
+                                  _ptr(u)), "ora_qjl_encode")
+    return (words, norms, u) if want_u else (words, norms)
+
+
+def qjl_query_sketch(q: np.ndarray, S: np.ndarray):
+    """v = S q for each row of q [n, d]; returns (v64 [n, m], v32 [n, m])."""
+    q = np.ascontiguousarray(q)
+    S64 = np.ascontiguousarray(S, np.float64)
+    n, d = q.shape
+    m = S64.shape[0]
+    v64 = np.empty((n, m), np.float64)
+    v32 = np.empty((n, m), np.float32)
+    _check(_load().ora_qjl_query_sketch(_ptr(q), _dtype_code(q), n, d, _ptr(S64), m, _ptr(v64),
+                                        _ptr(v32)), "ora_qjl_query_sketch")
+    return v64, v32
+
+
+def qjl_estimate(v: np.ndarray, key_words: np.ndarray, key_norm: float) -> float:
+    v = np.ascontiguousarray(v, np.float64)
+    w = np.ascontiguousarray(key_words, np.uint32)
+    return _load().ora_qjl_estimate(_ptr(v), _ptr(w), float(key_norm), v.shape[0])
+
+
+def qjl_scores(v: np.ndarray, words: np.ndarray, norms_f16: np.ndarray):
+    v = np.ascontiguousarray(np.atleast_2d(v), np.float64)
+    words = np.ascontiguousarray(words, np.uint32)
+    norms = np.ascontiguousarray(norms_f16, np.float16)
+    nq, m = v.shape
+    nk = words.shape[0]
+    out = np.empty((nq, nk), np.float32)
+    _check(_load().ora_qjl_scores(_ptr(v), nq, _ptr(words), _ptr(norms), nk, m, _ptr(out)),
+           "ora_qjl_scores")
+    return out
+
+
+def decode_attention(q_f16, *, k_codes=None, k_scales=None, k_words=None, k_norms=None,
+                     S=None, v_codes=None, v_scales=None, sm_scale=0.0,
+                     want_out=True, want_scores=False, want_probs=False):
+    """One decode step.  q [B, Hq, D] fp16; INT8 keys [B, Hkv, T, D] + [B, Hkv, T] or
+    QJL keys words [B, Hkv, T, m/32] + norms [B, Hkv, T] + S [m, D]; INT8 values.
+    Returns a dict with 'out' [B, Hq, D], 'scores' / 'probs' [B, Hq, T] as requested."""
+    q = np.ascontiguousarray(q_f16, np.float16)
+    B, Hq, D = q.shape
+    qjl = k_words is not None
+    if qjl:
+        k_words = np.ascontiguousarray(k_words, np.uint32)
+        k_norms = np.ascontiguousarray(k_norms, np.float16)
+        Hkv, T = k_words.shape[1], k_words.shape[2]
+        S64 = np.ascontiguousarray(S, np.float64)
+        m = S64.shape[0]
+    else:
+        k_codes = np.ascontiguousarray(k_codes, np.int8)
+        k_scales = np.ascontiguousarray(k_scales, np.float32)
+        Hkv, T = k_codes.shape[1], k_codes.shape[2]
+        S64, m = None, 0
+    if want_out:
+        v_codes = np.ascontiguousarray(v_codes, np.int8)
+        v_scales = np.ascontiguousarray(v_scales, np.float32)
+    out = np.empty((B, Hq, D), np.float32) if want_out else None
+    scores = np.empty((B, Hq, T), np.float32) if want_scores else None
+    probs = np.empty((B, Hq, T), np.float32) if want_probs else None
+    rc = _load().ora_decode_attention(
+        B, Hq, Hkv, T, D, _ptr(q), KEYS_QJL if qjl else KEYS_INT8,
+        _ptr(k_codes) if not qjl else None, _ptr(k_scales) if not qjl else None,
+        _ptr(k_words) if qjl else None, _ptr(k_norms) if qjl else None, _ptr(S64), m,
+        _ptr(v_codes) if want_out else None, _ptr(v_scales) if want_out else None,
+        float(sm_scale), _ptr(out), _ptr(scores), _ptr(probs))
+    _check(rc, "ora_decode_attention")
+    return {"out": out, "scores": scores, "probs": probs}

@@ -1,0 +1,359 @@
+"""Pins for the CPU oracle: each test checks it against something other than itself --
+hand-worked examples from the pages' equations, invariants, closed forms, library
+routines for special cases, and fp64 brute force on tiny inputs.  CPU only.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+import oracle
+from kv_cache_quantization_absmax_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------------------------
+# fp16 conversions (IEEE binary16) against numpy's own conversions
+# ----------------------------------------------------------------------------------
+
+def test_half_to_double_all_patterns():
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = bits.view(np.float16).astype(np.float64)
+    got = np.array([oracle.half_to_double(int(b)) for b in bits])
+    finite = np.isfinite(ref)
+    assert np.array_equal(got[finite], ref[finite])
+    assert np.array_equal(np.isinf(got), np.isinf(ref))
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+
+
+def test_double_to_half_round_to_nearest_even():
+    rng = np.random.default_rng(123)
+    xs = np.concatenate([
+        rng.standard_normal(20000) * 10.0 ** rng.uniform(-9, 5, 20000),
+        # exact midpoints between neighbouring halves exercise ties-to-even
+        (np.arange(0, 4096, dtype=np.float64) + 0.5) * 2.0 ** -24,
+        (np.arange(1024, 2048, dtype=np.float64) + 0.5) * 2.0 ** -3,
+        [0.0, -0.0, 65504.0, 65519.99, 65520.0, 1e9, -1e9, 2.0 ** -25, 2.0 ** -25 * 1.0001],
+    ])
+    with np.errstate(over="ignore"):
+        ref = xs.astype(np.float16).view(np.uint16)
+    got = np.array([oracle.double_to_half(float(x)) for x in xs], dtype=np.uint16)
+    assert np.array_equal(got, ref)
+
+
+# ----------------------------------------------------------------------------------
+# INT8 absmax quantization (Q-TensorFormer section 6, INT8 equation)
+# ----------------------------------------------------------------------------------
+
+def _fl32_nearest(fr: Fraction) -> Fraction:
+    """Nearest fp32 value (ties to even) of an exact rational, by exact arithmetic;
+    used only to validate the hand-worked fixture values themselves."""
+    if fr == 0:
+        return Fraction(0)
+    sign = -1 if fr < 0 else 1
+    a = abs(fr)
+    e = math.floor(math.log2(a.numerator) - math.log2(a.denominator))
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    e = max(e, -126)
+    quantum = Fraction(2) ** (e - 23)
+    n = round(a / quantum)          # Python rounds Fractions half to even
+    return sign * n * quantum
+
+
+@pytest.mark.parametrize("case", _golden("int8_worked_examples.json")["cases"],
+                         ids=lambda c: c["name"])
+def test_int8_worked_examples(case):
+    dt = np.float32 if case["dtype"] == "f32" else np.float16
+    x = np.array([float.fromhex(v) for v in case["x"]]).astype(dt)
+    assert np.array_equal(x.astype(np.float64), [float.fromhex(v) for v in case["x"]])
+    codes, scales = oracle.quantize_int8(x[None, :])
+    assert float(scales[0]) == float.fromhex(case["scale"])
+    assert codes[0].tolist() == case["codes"]
+    # the fixture's scale is the fp32 value nearest to a / 127 (exact rational check)
+    a = max(abs(Fraction(float(v))) for v in x)
+    assert _fl32_nearest(a / 127) == Fraction(float.fromhex(case["scale"]))
+    # dequantized values are the exact product c * s (formed in fp64, where 8 + 24
+    # significant bits fit) rounded once to fp32
+    xh = oracle.dequantize_int8(codes, scales)
+    exact = np.array(case["codes"], np.float64) * float.fromhex(case["scale"])
+    assert np.array_equal(xh[0], exact.astype(np.float32))
+
+
+def _sweep_like(n, d, dtype, seed):
+    x, _, _ = inputs.sweep_matrix(n * d, d, dtype, seed, n_rows=n)
+    return x
+
+
+@pytest.mark.parametrize("dtype", [np.float32, np.float16])
+@pytest.mark.parametrize("d", [16, 128, 1024])
+def test_int8_invariants(dtype, d):
+    x = _sweep_like(256, d, dtype, seed=d)
+    x[7] = 0                       # a zero row
+    x[9, :] = x[9, 0]              # an all-equal row
+    codes, s = oracle.quantize_int8(x)
+    xf = x.astype(np.float64)
+    a = np.abs(xf).max(axis=1)
+    # zero row: zero scale, zero codes
+    assert s[7] == 0 and not codes[7].any()
+    nz = a > 0
+    # |c| <= 127 and the absmax element maps to exactly +-127 with its sign
+    assert np.abs(codes.astype(np.int32)).max() <= 127
+    j = np.abs(xf).argmax(axis=1)
+    rows = np.nonzero(nz)[0]
+    assert np.array_equal(codes[rows, j[rows]].astype(np.int32),
+                          np.where(xf[rows, j[rows]] > 0, 127, -127))
+    # all-equal row maps every element to the same +-127
+    assert np.all(codes[9] == codes[9, 0]) and abs(int(codes[9, 0])) == 127
+    # round-trip error bound |x - x_hat| <= s/2 (checked in fp64, one fp32 ulp of slack)
+    xh = oracle.dequantize_int8(codes, s).astype(np.float64)
+    err = np.abs(xf - xh)
+    slack = np.spacing(np.abs(xh).astype(np.float32)).astype(np.float64)
+    assert np.all(err <= s.astype(np.float64)[:, None] / 2 + slack)
+    # the scale sits within half an fp32 ulp of a / 127
+    s64 = s.astype(np.float64)
+    assert np.all(np.abs(s64[nz] - a[nz] / 127) <= np.spacing(s[nz]).astype(np.float64) / 2)
+
+
+def test_int8_symmetry_and_power_of_two_scaling():
+    x = _sweep_like(64, 128, np.float32, seed=5)
+    c, s = oracle.quantize_int8(x)
+    cn, sn = oracle.quantize_int8(-x)            # round-half-even is odd-symmetric
+    assert np.array_equal(cn, -c) and np.array_equal(sn, s)
+    c4, s4 = oracle.quantize_int8(x * np.float32(4.0))   # exact rescale by 2^2
+    assert np.array_equal(c4, c) and np.array_equal(s4, s * np.float32(4.0))
+
+
+def test_dequant_fp16_is_rounded_fp32_product():
+    x = _sweep_like(64, 128, np.float16, seed=6)
+    c, s = oracle.quantize_int8(x)
+    f32 = oracle.dequantize_int8(c, s, np.float32)
+    f16 = oracle.dequantize_int8(c, s, np.float16)
+    assert np.array_equal(f16.view(np.uint16), f32.astype(np.float16).view(np.uint16))
+
+
+def test_int8_scores_against_fp64_brute_force():
+    x, q, _ = inputs.sweep_matrix(128 * 1024, 1024, np.float32, 1, n_rows=128)
+    c, s = oracle.quantize_int8(x)
+    got = oracle.int8_scores(q, c, s).astype(np.float64)
+    xh = (c.astype(np.float64) * s.astype(np.float64)[:, None]).astype(np.float32)
+    terms = xh.astype(np.float64) * q.astype(np.float64)[None, :]
+    ref = terms.sum(axis=1)
+    d = x.shape[1]
+    bound = 2 * d * 2.0 ** -24 * np.abs(terms).sum(axis=1)
+    assert np.all(np.abs(got - ref) <= bound)
+    # fp16 query: the same scores as the widened fp32 query
+    q16 = q.astype(np.float16)
+    assert np.array_equal(oracle.int8_scores(q16, c, s), oracle.int8_scores(q16.astype(np.float32), c, s))
+
+
+# ----------------------------------------------------------------------------------
+# QJL sketch and estimator (QJL abstract)
+# ----------------------------------------------------------------------------------
+
+def _tiny_sketch(g):
+    r = np.array(g["rows_0_7"], np.float64)
+    r16 = np.concatenate([r, -r])
+    return np.concatenate([r16, r16])
+
+
+def test_qjl_hand_worked_example():
+    g = _golden("qjl_tiny_example.json")
+    S = _tiny_sketch(g)
+    k = np.array(g["key"], np.float16)[None, :]
+    words, norms, u = oracle.qjl_encode(k, S, want_u=True)
+    assert np.array_equal(u[0, :16], g["projections_0_15"])
+    assert int(words[0, 0]) == int(g["word"], 16)
+    assert int(norms.view(np.uint16)[0]) == int(g["norm_f16_bits"], 16)
+    assert float(norms[0]) == 3.775390625
+    q = np.array(g["query"], np.float16)[None, :]
+    v64, v32 = oracle.qjl_query_sketch(q, S)
+    assert np.array_equal(v64[0, :16], g["query_sketch_0_15"])
+    est = oracle.qjl_estimate(v64[0], words[0], float(norms[0]))
+    expect = math.sqrt(math.pi / 2) / 32 * 3.775390625 * g["signed_sum"]
+    assert est == pytest.approx(expect, rel=1e-15)
+    sc = oracle.qjl_scores(v64, words, norms)
+    assert sc[0, 0] == np.float32(expect)
+
+
+def test_qjl_projection_matches_matmul():
+    S = inputs.sketch_matrix(256, 128)
+    keys = inputs.lognormal_cache(11, 1, 2, 64)[0].reshape(-1, 128)
+    words, norms, u = oracle.qjl_encode(keys, S, want_u=True)
+    ref = keys.astype(np.float64) @ S.astype(np.float64).T
+    assert np.allclose(u, ref, rtol=0, atol=1e-12 * np.abs(ref).max())
+    bits = (u >= 0).astype(np.uint64)
+    packed = np.zeros((keys.shape[0], 8), np.uint64)
+    for i in range(256):
+        packed[:, i // 32] |= bits[:, i] << np.uint64(i % 32)
+    assert np.array_equal(words.astype(np.uint64), packed)
+    nref = np.sqrt((keys.astype(np.float64) ** 2).sum(axis=1)).astype(np.float16)
+    assert np.array_equal(norms.view(np.uint16), nref.view(np.uint16))
+    q = inputs.gaussian_queries(12, 1, 3)[0]
+    v64, v32 = oracle.qjl_query_sketch(q, S)
+    vref = q.astype(np.float64) @ S.astype(np.float64).T
+    assert np.allclose(v64, vref, rtol=0, atol=1e-12 * np.abs(vref).max())
+    assert np.array_equal(v32, v64.astype(np.float32))
+
+
+def test_qjl_estimator_unbiased_over_2000_sketches():
+    """Mean over 2000 independent Gaussian sketches lies within 3 standard errors of the
+    exact inner product (fp64 sketches, seeds 10000..11999)."""
+    k = inputs.lognormal_cache(4, 1, 1, 1)[0].reshape(1, 128)
+    q = inputs.gaussian_queries(40, 1, 1)[0]
+    exact = float(k[0].astype(np.float64) @ q[0].astype(np.float64))
+    est = []
+    for seed in range(10000, 12000):
+        S = inputs.sketch_matrix_f64(256, 128, seed)
+        words, norms = oracle.qjl_encode(k, S)
+        v64, _ = oracle.qjl_query_sketch(q, S)
+        est.append(oracle.qjl_estimate(v64[0], words[0], float(norms[0])))
+    est = np.array(est)
+    se = est.std(ddof=1) / math.sqrt(len(est))
+    assert abs(est.mean() - exact) <= 3 * se, (est.mean(), exact, se)
+    # the 1/m scaling: the spread shrinks like 1/sqrt(m) -- variance is O(|q|^2 |k|^2 / m)
+    assert est.std() < 2.0 * np.linalg.norm(q[0].astype(np.float64)) * np.linalg.norm(
+        k[0].astype(np.float64)) / math.sqrt(256)
+
+
+def test_qjl_parallel_key_and_scaling():
+    S = inputs.sketch_matrix(256, 128)
+    q = inputs.gaussian_queries(13, 1, 1)[0]
+    # k parallel to q (k = q exactly): every bit agrees with the sign of v, so the
+    # estimate is sqrt(pi/2)/m * |k| * sum |v_i| >= 0
+    k = q.copy()
+    words, norms = oracle.qjl_encode(k, S)
+    v64, _ = oracle.qjl_query_sketch(q, S)
+    est = oracle.qjl_estimate(v64[0], words[0], float(norms[0]))
+    assert est == pytest.approx(math.sqrt(math.pi / 2) / 256 * float(norms[0]) * np.abs(v64[0]).sum(),
+                                rel=1e-12)
+    # scaling the key by 4 (exact in fp16) leaves the bits unchanged and scales the estimate
+    k4 = (k.astype(np.float32) * 4).astype(np.float16)
+    w4, n4 = oracle.qjl_encode(k4, S)
+    assert np.array_equal(w4, words)
+    assert float(n4[0]) == 4 * float(norms[0])
+    assert oracle.qjl_estimate(v64[0], w4[0], float(n4[0])) == pytest.approx(4 * est, rel=1e-12)
+    # a zero key: every projection is 0 >= 0, so all bits are set, and the norm is 0
+    wz, nz = oracle.qjl_encode(np.zeros((1, 128), np.float16), S)
+    assert np.all(wz == 0xFFFFFFFF) and float(nz[0]) == 0.0
+
+
+# ----------------------------------------------------------------------------------
+# Decode step: softmax invariants, special cases, fp64 brute force with the page's GQA
+# broadcast (unsqueeze(2).expand(...).reshape(...))
+# ----------------------------------------------------------------------------------
+
+def _tiny_cache(T, D=8, B=1, Hq=4, Hkv=2, seed=0):
+    rng = np.random.default_rng(seed)
+    k = rng.standard_normal((B, Hkv, T, D)).astype(np.float16)
+    v = rng.standard_normal((B, Hkv, T, D)).astype(np.float16)
+    q = rng.standard_normal((B, Hq, D)).astype(np.float16)
+    kc, ks = oracle.quantize_int8(k.reshape(-1, D))
+    vc, vs = oracle.quantize_int8(v.reshape(-1, D))
+    return (k, q, kc.reshape(B, Hkv, T, D), ks.reshape(B, Hkv, T),
+            vc.reshape(B, Hkv, T, D), vs.reshape(B, Hkv, T))
+
+
+def _fl32_product(c, s):
+    """fl32(c * s): the exact fp64 product rounded once to fp32, returned in fp64."""
+    return (c.astype(np.float64) * s.astype(np.float64)[..., None]).astype(np.float32).astype(np.float64)
+
+
+def _brute_force(q, kdeq_or_scores, vdeq, Hq, sigma, scores_given=False):
+    """fp64 attention with the GQA broadcast written as the page's tensor idiom."""
+    import torch
+    qt = torch.tensor(q.astype(np.float64))
+    V = torch.tensor(vdeq)
+    B, Hkv, T, D = V.shape
+    G = Hq // Hkv
+    Ve = V.unsqueeze(2).expand(B, Hkv, G, T, D).reshape(B, Hq, T, D)
+    if scores_given:
+        sc = torch.tensor(kdeq_or_scores)
+    else:
+        K = torch.tensor(kdeq_or_scores)
+        Ke = K.unsqueeze(2).expand(B, Hkv, G, T, D).reshape(B, Hq, T, D)
+        sc = torch.einsum("bhd,bhtd->bht", qt, Ke)
+    p = torch.softmax(sigma * sc, dim=-1)
+    out = torch.einsum("bht,bhtd->bhd", p, Ve)
+    return out.numpy(), sc.numpy(), p.numpy()
+
+
+@pytest.mark.parametrize("T", [1, 5, 33])
+def test_decode_int8_brute_force(T):
+    k, q, kc, ks, vc, vs = _tiny_cache(T)
+    r = oracle.decode_attention(q, k_codes=kc, k_scales=ks, v_codes=vc, v_scales=vs,
+                                want_scores=True, want_probs=True)
+    kdeq = _fl32_product(kc, ks)
+    vdeq = _fl32_product(vc, vs)
+    sigma = float(np.float32(1.0) / np.sqrt(np.float32(8)))
+    out, sc, p = _brute_force(q, kdeq, vdeq, 4, sigma)
+    assert np.allclose(r["scores"], sc, rtol=0, atol=1e-5)
+    assert np.allclose(r["probs"], p, rtol=0, atol=1e-6)
+    assert np.allclose(r["out"], out, rtol=0, atol=1e-5)
+    # softmax rows sum to one
+    assert np.all(np.abs(r["probs"].astype(np.float64).sum(-1) - 1) <= T * 2.0 ** -23)
+    if T == 1:   # a single token: p = 1 exactly and the output is that token's values
+        assert np.array_equal(r["out"], np.repeat(
+            (vc.astype(np.float32) * vs[..., None])[:, :, 0], 2, axis=1))
+
+
+@pytest.mark.parametrize("T", [1, 5, 33])
+def test_decode_qjl_brute_force(T):
+    k, q, _, _, vc, vs = _tiny_cache(T, D=8)
+    S = inputs.sketch_matrix(32, 8, seed=3)
+    B, Hkv, _, D = k.shape
+    words, norms = oracle.qjl_encode(k.reshape(-1, D), S)
+    words = words.reshape(B, Hkv, T, 1)
+    norms = norms.reshape(B, Hkv, T)
+    r = oracle.decode_attention(q, k_words=words, k_norms=norms, S=S, v_codes=vc, v_scales=vs,
+                                want_scores=True, want_probs=True)
+    # brute-force estimator scores from the definition, fp64, per (b, h, t)
+    G = 4 // Hkv
+    v = q.astype(np.float64) @ S.astype(np.float64).T                    # [B, Hq, m]
+    v = v.astype(np.float32).astype(np.float64)                           # stored fp32
+    bits = ((words[..., 0][..., None] >> np.arange(32, dtype=np.uint32)) & 1).astype(np.float64)
+    sgn = 2 * bits - 1                                                   # [B, Hkv, T, 32]
+    sgn_e = np.repeat(sgn, G, axis=1)
+    nrm_e = np.repeat(norms.astype(np.float64), G, axis=1)
+    sc = math.sqrt(math.pi / 2) / 32 * nrm_e * np.einsum("bhm,bhtm->bht", v, sgn_e)
+    vdeq = _fl32_product(vc, vs)
+    sigma = float(np.float32(1.0) / np.sqrt(np.float32(8)))
+    out, _, p = _brute_force(q, sc, vdeq, 4, sigma, scores_given=True)
+    assert np.allclose(r["scores"], sc, rtol=1e-6, atol=1e-6)
+    assert np.allclose(r["probs"], p, rtol=0, atol=1e-6)
+    assert np.allclose(r["out"], out, rtol=0, atol=1e-5)
+
+
+def test_decode_equal_logits_give_mean_of_values():
+    T = 40
+    _, q, kc, ks, vc, vs = _tiny_cache(T)
+    q = np.zeros_like(q)                       # every score is 0
+    r = oracle.decode_attention(q, k_codes=kc, k_scales=ks, v_codes=vc, v_scales=vs,
+                                want_probs=True)
+    assert np.all(r["probs"] == np.float32(1.0) / np.float32(T))
+    vdeq = vc.astype(np.float64) * vs.astype(np.float64)[..., None]
+    mean = np.repeat(vdeq.mean(axis=2), 2, axis=1)
+    assert np.allclose(r["out"], mean, rtol=0, atol=1e-5)
+
+
+def test_decode_gqa_group_mapping():
+    """Query head h reads KV head h // G: give the two KV heads very different values."""
+    T = 6
+    k, q, kc, ks, vc, vs = _tiny_cache(T)
+    vc = vc.copy()
+    vc[:, 0] = 10
+    vc[:, 1] = -10
+    vs = np.ones_like(vs)
+    r = oracle.decode_attention(q, k_codes=kc, k_scales=ks, v_codes=vc, v_scales=vs)
+    assert np.allclose(r["out"][0, :2], 10) and np.allclose(r["out"][0, 2:], -10)
