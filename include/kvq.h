@@ -1,0 +1,197 @@
+/*
+ * kvq.h -- C ABI of libkvq: KV-cache compression and one decode step over the
+ * compressed cache, hand-written CUDA for NVIDIA B200 (sm_100a).
+ *
+ * Conventions shared by every entry point
+ *  - All data pointers are DEVICE pointers owned by the caller.  The library never
+ *    allocates or frees memory and never synchronises the stream; it keeps no state
+ *    between calls other than cached device properties.
+ *  - Calls are asynchronous: KVQ_OK means the work was enqueued on `stream`
+ *    (NULL = the legacy default stream) of the current device.  A fault inside a
+ *    kernel surfaces on the caller's next synchronisation.
+ *  - Arguments are validated on the host before anything is launched; a failed check
+ *    returns its error code and enqueues nothing.  Zero rows/keys return KVQ_OK with
+ *    no launch.
+ *  - KVQ_ERR_CUDA means the CUDA runtime reported an error when the kernel was
+ *    launched (this can also be a sticky error left by earlier asynchronous work).
+ *  - fp16 data is passed as raw IEEE binary16 bit patterns (uint16_t).
+ *  - Rows are contiguous and row-major; 64-bit sizes are used throughout.
+ *  - No C++ exception crosses this boundary.
+ *
+ * Sources (web pages, cited by title and section):
+ *  [INT8]  "Q-TensorFormer" model card, section 6 "Adaptive KV Cache Quantization &
+ *          Attention-Sink Eviction": symmetric INT8, X_hat = clamp(round(X/s8), -128,
+ *          127) * s8 with s8 = max|X| / 127.
+ *  [PAPER] "GPU-Accelerated INT8 Quantization for KV Cache Compression in Large
+ *          Language Models" (arXiv 2601.04719), abstract.
+ *  [QJL]   "QJL: 1-Bit Quantized JL Transform for KV Cache Quantization with Zero
+ *          Overhead" (arXiv 2406.03482), abstract.
+ *  [GQA]   "Q-TensorFormer" model card, section 4 "Grouped-Query Attention (GQA) &
+ *          Multi-Query Attention (MQA)".
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, spelled without CUDA headers. */
+typedef struct CUstream_st* kvq_stream_t;
+
+typedef enum {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, negative size, bad enum ... */
+    KVQ_ERR_UNSUPPORTED = 2,   /* a valid request this build does not implement       */
+    KVQ_ERR_CUDA = 3,          /* the CUDA runtime reported an error at launch         */
+    KVQ_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required           */
+    KVQ_ERR_DEVICE = 5         /* a kernel recorded a device-side error (see below)    */
+} kvq_status;
+
+typedef enum { KVQ_F32 = 0, KVQ_F16 = 1 } kvq_dtype;
+
+typedef enum { KVQ_KEYS_INT8 = 0, KVQ_KEYS_QJL = 1 } kvq_key_format;
+
+#define KVQ_ABI_VERSION 1
+
+int kvq_abi_version(void);
+const char* kvq_status_string(kvq_status s);
+
+/*
+ * kvq_quantize_int8 -- [INT8] with one scale per row ("per token": a row is one head's
+ * head_dim vector); [PAPER] abstract (INT8 KV quantization, 4x smaller than fp32).
+ *   For each row r:  a_r = max_j |x_rj|,   s_r = fl32(a_r / 127),
+ *                    c_rj = clamp(round_half_even(fl32(x_rj / s_r)), -128, 127),
+ *   where the quotient is an IEEE fp32 division by the STORED scale; a row with
+ *   s_r == 0 gets codes 0.  (|x/s| <= 127 whenever s is a normal number, so the clamp
+ *   only binds for rows whose scale is subnormal.)  Results are bit-exact.
+ *   x       [n_rows][d] fp32 or fp16 (x_dtype), 16-byte aligned
+ *   codes   [n_rows][d] int8, 16-byte aligned         (written)
+ *   scales  [n_rows]    fp32, 4-byte aligned          (written)
+ *   d       > 0, multiple of 16, <= 65536
+ *   NaN/Inf inputs give unspecified codes (not checked).
+ */
+kvq_status kvq_quantize_int8(const void* x, kvq_dtype x_dtype, int64_t n_rows, int64_t d,
+                             int8_t* codes, float* scales, kvq_stream_t stream);
+
+/*
+ * kvq_dequantize_int8 -- [INT8] the trailing "* s8": x_hat_rj = fl32(c_rj * s_r); for
+ * fp16 output, that fp32 value rounded to nearest-even fp16.  Bit-exact.
+ *   codes [n_rows][d] int8 (16-byte aligned), scales [n_rows] fp32,
+ *   out   [n_rows][d] fp32 or fp16 (out_dtype), 16-byte aligned (written);
+ *   d > 0, multiple of 16.
+ */
+kvq_status kvq_dequantize_int8(const int8_t* codes, const float* scales, int64_t n_rows,
+                               int64_t d, void* out, kvq_dtype out_dtype, kvq_stream_t stream);
+
+/*
+ * kvq_int8_scores -- [PAPER] "attention score" of one query against INT8 rows:
+ *   scores_r = sum_j q_j * fl32(c_rj * s_r), fp32 accumulation (order unspecified).
+ *   q [d] fp32 or fp16 (q_dtype, 16-byte aligned), codes [n_rows][d] int8 (16-byte
+ *   aligned), scales [n_rows] fp32, scores [n_rows] fp32 (written); d multiple of 16,
+ *   d <= 16384.
+ */
+kvq_status kvq_int8_scores(const void* q, kvq_dtype q_dtype, const int8_t* codes,
+                           const float* scales, int64_t n_rows, int64_t d, float* scores,
+                           kvq_stream_t stream);
+
+/*
+ * kvq_qjl_encode -- [QJL] abstract ("a JL transform followed by sign-bit quantization"):
+ *   u_n = S k_n for each key (fp16 x fp16 products, fp32 accumulation on the tensor
+ *   cores); bit i of key n = [u_n,i >= 0], stored LSB-first, 32 coordinates per word
+ *   (word w holds coordinates 32w .. 32w+31); norm_n = fp16(||k_n||_2).
+ *   keys_f16    [n_keys][d] fp16, 16-byte aligned
+ *   sketch_f16  [m][d] fp16 row-major (the Gaussian JL matrix S), 16-byte aligned
+ *   sign_words  [n_keys][m/32] uint32 (written), 16-byte aligned if m/32 is a multiple
+ *               of 4, else 4-byte aligned
+ *   norms_f16   [n_keys] fp16 (written), 2-byte aligned
+ *   d must be 128 and m a multiple of 32 in [32, 256] (else KVQ_ERR_UNSUPPORTED).
+ *   A bit may differ from the exact (fp64) sign only where |u_i| is within the fp32
+ *   accumulation error of 0.
+ */
+kvq_status kvq_qjl_encode(const uint16_t* keys_f16, int64_t n_keys, int32_t d,
+                          const uint16_t* sketch_f16, int32_t m, uint32_t* sign_words,
+                          uint16_t* norms_f16, kvq_stream_t stream);
+
+/*
+ * kvq_qjl_query_sketch -- [QJL] abstract ("a standard JL transform without
+ * quantization to the other [vector]"): v_n = S q_n in fp32 (tensor cores).
+ *   q_f16 [n_q][d] fp16 (16-byte aligned), sketch_f16 [m][d] fp16 (16-byte aligned),
+ *   v [n_q][m] fp32 (written, 16-byte aligned); d == 128, m multiple of 32 in [32, 256].
+ */
+kvq_status kvq_qjl_query_sketch(const uint16_t* q_f16, int64_t n_q, int32_t d,
+                                const uint16_t* sketch_f16, int32_t m, float* v,
+                                kvq_stream_t stream);
+
+/*
+ * kvq_decode_attention -- one decode step for one query token per head over a
+ * compressed cache ([PAPER] abstract: attention scores over the INT8 cache; [QJL]
+ * abstract: the asymmetric estimator; [GQA] section 4: query head h reads KV head
+ * h / (Hq / Hkv)).
+ *   score_t = INT8 keys: sum_j q_j * fl32(c_tj * s_t);
+ *             QJL keys:  sqrt(pi/2)/m * norm_t * sum_i v_i * (2 b_t,i - 1), v = S q (fp32);
+ *   p_t     = softmax_t(sm_scale * score_t) over all T cached tokens (no mask);
+ *   out     = sum_t p_t * fl32(cv_t * sv_t)   (fp32, [B][Hq][D]).
+ * Layouts (all contiguous):
+ *   q          [B][Hq][D] fp16
+ *   k_codes    [B][Hkv][T][D] int8,  k_scales [B][Hkv][T] fp32      (INT8 keys)
+ *   k_words    [B][Hkv][T][m/32] u32, k_norms [B][Hkv][T] fp16,
+ *   sketch     [m][D] fp16                                          (QJL keys)
+ *   v_codes    [B][Hkv][T][D] int8,  v_scales [B][Hkv][T] fp32      (needed if out)
+ *   out        [B][Hq][D] fp32 or NULL
+ *   scores_out [B][Hq][T] fp32 raw scores (before sm_scale) or NULL
+ * out and scores_out may not both be NULL.  head_dim must be 128 (KVQ_ERR_UNSUPPORTED
+ * otherwise); QJL needs m a multiple of 32 in [32, 256]; Hq % Hkv == 0; T >= 1
+ * (a softmax over no tokens is undefined: KVQ_ERR_INVALID_ARG).  sm_scale == 0 selects
+ * 1/sqrt(head_dim).
+ * workspace: caller-owned device memory of at least kvq_decode_workspace_bytes(a)
+ * bytes, 256-byte aligned (KVQ_ERR_WORKSPACE otherwise).  It holds per-split partial
+ * softmax states and the query sketches; its contents on entry do not matter.
+ * Launches 2 kernels (INT8 keys) or 3 (QJL keys) on `stream`; no host synchronisation.
+ */
+typedef struct kvq_decode_args {
+    int64_t batch;
+    int64_t n_q_heads;
+    int64_t n_kv_heads;
+    int64_t seq_len;
+    int32_t head_dim;
+    int32_t key_format;            /* kvq_key_format */
+    const uint16_t* q_f16;
+    const int8_t* k_codes;
+    const float* k_scales;
+    const uint32_t* k_words;
+    const uint16_t* k_norms_f16;
+    const uint16_t* sketch_f16;
+    int32_t sketch_dim;            /* m */
+    float sm_scale;
+    const int8_t* v_codes;
+    const float* v_scales;
+    float* out;
+    float* scores_out;
+    void* workspace;
+    size_t workspace_bytes;
+} kvq_decode_args;
+
+kvq_status kvq_decode_attention(const kvq_decode_args* a, kvq_stream_t stream);
+
+/* Bytes of workspace kvq_decode_attention needs for these arguments (0 if the
+ * arguments are invalid).  Depends on the current device's SM count. */
+size_t kvq_decode_workspace_bytes(const kvq_decode_args* a);
+
+/*
+ * kvq_device_error -- read and clear the library's device-side error word on the
+ * current device (synchronous: it waits for the device).  Kernels that wait on
+ * barriers give up after a bounded number of polls instead of hanging; when they do,
+ * they record a nonzero code here and skip the rest of their work.  *code = 0 means
+ * no error was recorded.  Returns KVQ_ERR_CUDA if the read itself fails.
+ */
+kvq_status kvq_device_error(uint32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

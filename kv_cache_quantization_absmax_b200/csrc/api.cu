@@ -1,0 +1,182 @@
+// The C ABI (include/kvq.h): host-side argument validation, then dispatch to the
+// kernels.  Nothing here allocates device memory or synchronises a stream.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+#include "kvq_internal.h"
+
+#define KVQ_API extern "C" __attribute__((visibility("default")))
+
+namespace kvq {
+
+int device_sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < 64 && cached[dev] > 0) return cached[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (dev < 64) cached[dev] = n;
+    return n;
+}
+
+}  // namespace kvq
+
+namespace {
+
+inline bool aligned(const void* p, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+inline bool valid_dtype(int t) { return t == KVQ_F32 || t == KVQ_F16; }
+inline kvq_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return KVQ_OK;
+    if (e == cudaErrorNotSupported) return KVQ_ERR_UNSUPPORTED;
+    return KVQ_ERR_CUDA;
+}
+inline cudaStream_t cs(kvq_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+constexpr int64_t kMaxQuantDim = 65536;
+constexpr int64_t kMaxScoreDim = 8192;
+
+bool qjl_dims_ok(int32_t d, int32_t m) {
+    return d == 128 && m >= 32 && m <= 256 && (m % 32) == 0;
+}
+
+// Validation shared by kvq_decode_attention and kvq_decode_workspace_bytes.
+kvq_status check_decode(const kvq_decode_args* a) {
+    if (!a) return KVQ_ERR_INVALID_ARG;
+    if (a->batch < 0 || a->n_q_heads <= 0 || a->n_kv_heads <= 0 || a->seq_len <= 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (a->n_q_heads % a->n_kv_heads != 0) return KVQ_ERR_INVALID_ARG;
+    if (a->key_format != KVQ_KEYS_INT8 && a->key_format != KVQ_KEYS_QJL) return KVQ_ERR_INVALID_ARG;
+    if (a->head_dim <= 0 || a->head_dim % 16 != 0) return KVQ_ERR_INVALID_ARG;
+    if (a->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+    if (!a->out && !a->scores_out) return KVQ_ERR_INVALID_ARG;
+    if (!(a->sm_scale == a->sm_scale) || a->sm_scale < 0.0f) return KVQ_ERR_INVALID_ARG;
+    {
+        // Query heads per KV head served by one CTA: INT8 keys up to 8, QJL keys up to 4
+        // (four 32 KB byte tables fill the shared memory a CTA may use).
+        const int64_t G = a->n_q_heads / a->n_kv_heads;
+        const bool pow2 = G == 1 || G == 2 || G == 4 || G == 8;
+        if (!pow2 || (a->key_format == KVQ_KEYS_QJL && G > 4)) return KVQ_ERR_UNSUPPORTED;
+    }
+    if (a->batch == 0) return KVQ_OK;
+    if (!a->q_f16 || !aligned(a->q_f16, 16)) return KVQ_ERR_INVALID_ARG;
+    if (a->key_format == KVQ_KEYS_INT8) {
+        if (!a->k_codes || !a->k_scales || !aligned(a->k_codes, 16) || !aligned(a->k_scales, 4))
+            return KVQ_ERR_INVALID_ARG;
+    } else {
+        if (a->sketch_dim <= 0 || a->sketch_dim % 32 != 0) return KVQ_ERR_INVALID_ARG;
+        if (!qjl_dims_ok(a->head_dim, a->sketch_dim)) return KVQ_ERR_UNSUPPORTED;
+        if (!a->k_words || !a->k_norms_f16 || !a->sketch_f16) return KVQ_ERR_INVALID_ARG;
+        const uintptr_t wa = ((a->sketch_dim / 32) % 4 == 0) ? 16 : 4;
+        if (!aligned(a->k_words, wa) || !aligned(a->k_norms_f16, 2) || !aligned(a->sketch_f16, 16))
+            return KVQ_ERR_INVALID_ARG;
+    }
+    if (a->out) {
+        if (!a->v_codes || !a->v_scales || !aligned(a->v_codes, 16) || !aligned(a->v_scales, 4) ||
+            !aligned(a->out, 16))
+            return KVQ_ERR_INVALID_ARG;
+    }
+    if (a->scores_out && !aligned(a->scores_out, 4)) return KVQ_ERR_INVALID_ARG;
+    return KVQ_OK;
+}
+
+}  // namespace
+
+KVQ_API int kvq_abi_version(void) { return KVQ_ABI_VERSION; }
+
+KVQ_API const char* kvq_status_string(kvq_status s) {
+    switch (s) {
+        case KVQ_OK: return "ok";
+        case KVQ_ERR_INVALID_ARG: return "invalid argument";
+        case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+        case KVQ_ERR_CUDA: return "CUDA runtime error";
+        case KVQ_ERR_WORKSPACE: return "workspace missing or too small";
+        case KVQ_ERR_DEVICE: return "device-side error recorded";
+    }
+    return "unknown status";
+}
+
+KVQ_API kvq_status kvq_quantize_int8(const void* x, kvq_dtype x_dtype, int64_t n_rows, int64_t d,
+                                     int8_t* codes, float* scales, kvq_stream_t stream) {
+    if (!valid_dtype(x_dtype) || n_rows < 0 || d <= 0 || d % 16 != 0 || d > kMaxQuantDim)
+        return KVQ_ERR_INVALID_ARG;
+    if (n_rows == 0) return KVQ_OK;
+    if (!x || !codes || !scales || !aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 4))
+        return KVQ_ERR_INVALID_ARG;
+    return from_cuda(kvq::launch_quantize_int8(x, x_dtype == KVQ_F16, n_rows, d, codes, scales,
+                                               cs(stream)));
+}
+
+KVQ_API kvq_status kvq_dequantize_int8(const int8_t* codes, const float* scales, int64_t n_rows,
+                                       int64_t d, void* out, kvq_dtype out_dtype,
+                                       kvq_stream_t stream) {
+    if (!valid_dtype(out_dtype) || n_rows < 0 || d <= 0 || d % 16 != 0) return KVQ_ERR_INVALID_ARG;
+    if (n_rows == 0) return KVQ_OK;
+    if (!codes || !scales || !out || !aligned(codes, 16) || !aligned(scales, 4) || !aligned(out, 16))
+        return KVQ_ERR_INVALID_ARG;
+    return from_cuda(kvq::launch_dequantize_int8(codes, scales, n_rows, d, out,
+                                                 out_dtype == KVQ_F16, cs(stream)));
+}
+
+KVQ_API kvq_status kvq_int8_scores(const void* q, kvq_dtype q_dtype, const int8_t* codes,
+                                   const float* scales, int64_t n_rows, int64_t d, float* scores,
+                                   kvq_stream_t stream) {
+    if (!valid_dtype(q_dtype) || n_rows < 0 || d <= 0 || d % 16 != 0 || d > kMaxScoreDim)
+        return KVQ_ERR_INVALID_ARG;
+    if (n_rows == 0) return KVQ_OK;
+    if (!q || !codes || !scales || !scores || !aligned(q, 16) || !aligned(codes, 16) ||
+        !aligned(scales, 4) || !aligned(scores, 4))
+        return KVQ_ERR_INVALID_ARG;
+    return from_cuda(kvq::launch_int8_scores(q, q_dtype == KVQ_F16, codes, scales, n_rows, d,
+                                             scores, cs(stream)));
+}
+
+KVQ_API kvq_status kvq_qjl_encode(const uint16_t* keys_f16, int64_t n_keys, int32_t d,
+                                  const uint16_t* sketch_f16, int32_t m, uint32_t* sign_words,
+                                  uint16_t* norms_f16, kvq_stream_t stream) {
+    if (n_keys < 0 || d <= 0 || d % 16 != 0 || m <= 0 || m % 32 != 0) return KVQ_ERR_INVALID_ARG;
+    if (!qjl_dims_ok(d, m)) return KVQ_ERR_UNSUPPORTED;
+    if (n_keys == 0) return KVQ_OK;
+    const uintptr_t wa = ((m / 32) % 4 == 0) ? 16 : 4;
+    if (!keys_f16 || !sketch_f16 || !sign_words || !norms_f16 || !aligned(keys_f16, 16) ||
+        !aligned(sketch_f16, 16) || !aligned(sign_words, wa) || !aligned(norms_f16, 2))
+        return KVQ_ERR_INVALID_ARG;
+    return from_cuda(kvq::launch_qjl_encode(keys_f16, n_keys, sketch_f16, m, sign_words, norms_f16,
+                                            cs(stream)));
+}
+
+KVQ_API kvq_status kvq_qjl_query_sketch(const uint16_t* q_f16, int64_t n_q, int32_t d,
+                                        const uint16_t* sketch_f16, int32_t m, float* v,
+                                        kvq_stream_t stream) {
+    if (n_q < 0 || d <= 0 || d % 16 != 0 || m <= 0 || m % 32 != 0) return KVQ_ERR_INVALID_ARG;
+    if (!qjl_dims_ok(d, m)) return KVQ_ERR_UNSUPPORTED;
+    if (n_q == 0) return KVQ_OK;
+    if (!q_f16 || !sketch_f16 || !v || !aligned(q_f16, 16) || !aligned(sketch_f16, 16) ||
+        !aligned(v, 16))
+        return KVQ_ERR_INVALID_ARG;
+    return from_cuda(kvq::launch_qjl_query_sketch(q_f16, n_q, sketch_f16, m, v, cs(stream)));
+}
+
+KVQ_API size_t kvq_decode_workspace_bytes(const kvq_decode_args* a) {
+    if (check_decode(a) != KVQ_OK) return 0;
+    return kvq::plan_decode(a, kvq::device_sm_count()).total_bytes;
+}
+
+KVQ_API kvq_status kvq_decode_attention(const kvq_decode_args* a, kvq_stream_t stream) {
+    const kvq_status st = check_decode(a);
+    if (st != KVQ_OK) return st;
+    if (a->batch == 0) return KVQ_OK;
+    const kvq::DecodePlan plan = kvq::plan_decode(a, kvq::device_sm_count());
+    if (!a->workspace || !aligned(a->workspace, 256) || a->workspace_bytes < plan.total_bytes)
+        return KVQ_ERR_WORKSPACE;
+    return from_cuda(kvq::launch_decode(a, plan, cs(stream)));
+}
+
+KVQ_API kvq_status kvq_device_error(uint32_t* code) {
+    if (!code) return KVQ_ERR_INVALID_ARG;
+    return from_cuda(kvq::read_and_clear_device_error(code)) == KVQ_OK ? KVQ_OK : KVQ_ERR_CUDA;
+}

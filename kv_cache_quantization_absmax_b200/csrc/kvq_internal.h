@@ -1,0 +1,42 @@
+// Internal declarations shared by the library's translation units (host side).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq.h"
+
+namespace kvq {
+
+int device_sm_count();  // SM count of the current device (cached per device)
+
+// quantize.cu
+cudaError_t launch_quantize_int8(const void* x, bool f16, int64_t n_rows, int64_t d,
+                                 int8_t* codes, float* scales, cudaStream_t st);
+cudaError_t launch_dequantize_int8(const int8_t* codes, const float* scales, int64_t n_rows,
+                                   int64_t d, void* out, bool f16, cudaStream_t st);
+cudaError_t launch_int8_scores(const void* q, bool q_f16, const int8_t* codes,
+                               const float* scales, int64_t n_rows, int64_t d, float* scores,
+                               cudaStream_t st);
+
+// qjl.cu
+// Returns cudaErrorNotSupported when the driver's tensor-map encoder is unavailable.
+cudaError_t launch_qjl_encode(const uint16_t* keys, int64_t n_keys, const uint16_t* S, int m,
+                              uint32_t* words, uint16_t* norms, cudaStream_t st);
+cudaError_t launch_qjl_query_sketch(const uint16_t* q, int64_t n_q, const uint16_t* S, int m,
+                                    float* v, cudaStream_t st);
+cudaError_t read_and_clear_device_error(uint32_t* code);
+
+// decode.cu
+struct DecodePlan {
+    int64_t units;        // B * Hkv
+    int splits;           // token chunks per unit
+    int64_t chunk;        // tokens per chunk
+    size_t partial_bytes; // per-split softmax states
+    size_t sketch_bytes;  // query sketches (QJL)
+    size_t total_bytes;
+};
+DecodePlan plan_decode(const kvq_decode_args* a, int sm_count);
+cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& plan, cudaStream_t st);
+
+}  // namespace kvq

@@ -1,0 +1,483 @@
+// QJL key sketch and query sketch on the 5th-generation tensor cores (tcgen05).
+//
+// Definition: "QJL: 1-Bit Quantized JL Transform for KV Cache Quantization with Zero
+// Overhead", abstract -- the key is projected by a Gaussian JL matrix S and only the
+// signs of the projection are kept (sign-bit quantization); the query is projected by
+// the same S without quantization; the key's norm is kept for the estimator.
+//
+// u = K S^T for a tile of 128 keys is one dense [128 x 128] x [128 x m] contraction,
+// so it runs as tcgen05.mma (kind::f16, fp16 x fp16 -> fp32 accumulators in tensor
+// memory).  Persistent kernel, one CTA per SM, three warp roles:
+//   warp 0      TMA producer: S once (it stays in shared memory), then 128-key tiles
+//               into a 4-stage ring (two 64-column boxes per tile, 128-byte swizzle);
+//   warp 1      allocates 512 TMEM columns (two m-column accumulators), one thread
+//               issues 8 MMAs (K = 16 each) per tile and commits to an mbarrier;
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator row (one key per thread),
+//               sign bits -> packed words (funnel shift of the sign bits), the key
+//               norm from the tile still in shared memory, 16-byte stores.
+// The epilogue of tile i overlaps the MMA of tile i+1 (double-buffered accumulator)
+// and the TMA loads of tiles i+1..i+4.
+//
+// Norms: the sum of squares is formed in fp64 in index order (each square of an fp16
+// value is exact), square-rooted with IEEE rounding and converted to fp16 with one
+// rounding, so the stored norm is the correctly rounded fp16 of the fp64 norm.
+// Sign bits: bit = 1 iff the fp32 accumulator is >= 0 (-0 is canonicalised to +0); a
+// zero key (sum of squares 0) has all bits set, since every projection is exactly 0.
+//
+// Every mbarrier wait is bounded: after kMaxPolls polls the waiting role records an
+// error code in g_kvq_device_error, raises a CTA-wide abort flag and leaves its loop;
+// the producer then waits (bounded) for its own TMA loads still in flight, the MMA
+// thread for its own MMAs, and TMEM is freed before the CTA exits.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+
+__device__ unsigned int g_kvq_device_error = 0;
+
+namespace {
+
+constexpr int kBM = 128;                 // keys per tile (MMA M)
+constexpr int kDim = 128;                // head_dim (MMA K in total)
+constexpr int kStages = 4;
+constexpr int kHalfBytes = kBM * 64 * 2; // one 64-column box of a key tile: 16 KB
+constexpr int kTileBytes = 2 * kHalfBytes;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccStride = 256;     // TMEM columns between the two accumulators
+constexpr uint32_t kMaxPolls = 1u << 24;
+
+enum : unsigned int {
+    kErrProducer = 0x101,
+    kErrMma = 0x102,
+    kErrEpilogue = 0x103,
+    kErrDrain = 0x104,
+};
+
+// --------------------------------------------------------------------------------
+// PTX wrappers
+// --------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait.  Returns false (after recording `err`) on timeout or when another
+// role has already aborted the CTA.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned int err) {
+    for (uint32_t i = 0; i < kMaxPolls; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 1023u) == 1023u && *abort_flag) return false;
+    }
+    atomicCAS(&g_kvq_device_error, 0u, err);
+    *abort_flag = 1;
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot_smem),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16, one instruction per K = 16 slice.
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// 32 lanes x 32 consecutive 32-bit columns: thread t gets row (lane base + t).
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32"
+        " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
+        " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31},"
+        " [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of 128 bytes,
+// 8-row core groups 1024 bytes apart (stride byte offset), descriptor version 1.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;                 // leading byte offset (unused with swizzle)
+    d |= (uint64_t)(1024u >> 4) << 32;       // stride byte offset
+    d |= (uint64_t)1u << 46;                 // version
+    d |= (uint64_t)2u << 61;                 // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulate, fp16 A and B, both K-major,
+// M = 128, N = n.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+}
+
+struct Smem {
+    uint32_t s_base;      // S: two 64-column halves of m rows x 128 B
+    uint32_t stage_base;  // key stages
+    uint32_t bars;        // mbarriers
+};
+
+template <bool kSketchOut>
+__global__ void __launch_bounds__(kThreads, 1)
+qjl_mma_kernel(const __grid_constant__ CUtensorMap tmap_rows,
+               const __grid_constant__ CUtensorMap tmap_s, int64_t n_rows, int m,
+               uint32_t* __restrict__ words, uint16_t* __restrict__ norms,
+               float* __restrict__ sketch_out) {
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag_storage;
+    volatile int* abort_flag = &abort_flag_storage;
+
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* base_ptr = smem_raw + (base - raw);
+    const uint32_t s_half_bytes = (uint32_t)m * 128u;
+    const uint32_t s_base = base;
+    const uint32_t stage_base = base + 2u * s_half_bytes;
+    const uint32_t bar_base = stage_base + kStages * kTileBytes;
+    auto full_bar = [&](int s) { return bar_base + 8u * s; };
+    auto empty_bar = [&](int s) { return bar_base + 8u * (kStages + s); };
+    auto tfull_bar = [&](int a) { return bar_base + 8u * (2 * kStages + a); };
+    auto tempty_bar = [&](int a) { return bar_base + 8u * (2 * kStages + 2 + a); };
+    const uint32_t s_bar = bar_base + 8u * (2 * kStages + 4);
+    const uint32_t done_bar = bar_base + 8u * (2 * kStages + 5);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t n_tiles = (n_rows + kBM - 1) / kBM;
+
+    if (threadIdx.x == 0) {
+        abort_flag_storage = 0;
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 4);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(tfull_bar(a), 1);
+            mbar_init(tempty_bar(a), 4);
+        }
+        mbar_init(s_bar, 1);
+        mbar_init(done_bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_slot;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_rows)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_s)) : "memory");
+            mbar_arrive_expect_tx(s_bar, 2u * s_half_bytes);
+            tma_load_2d(s_base, &tmap_s, s_bar, 0, 0);
+            tma_load_2d(s_base + s_half_bytes, &tmap_s, s_bar, 64, 0);
+            uint32_t issued_parity[kStages];
+            bool issued[kStages];
+            for (int s = 0; s < kStages; ++s) issued[s] = false, issued_parity[s] = 0;
+            int it = 0;
+            for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+                const int stage = it % kStages;
+                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                if (!mbar_wait(empty_bar(stage), ph ^ 1u, abort_flag, kErrProducer)) break;
+                const uint32_t dst = stage_base + (uint32_t)stage * kTileBytes;
+                mbar_arrive_expect_tx(full_bar(stage), (uint32_t)kTileBytes);
+                tma_load_2d(dst, &tmap_rows, full_bar(stage), 0, (int)(tile * kBM));
+                tma_load_2d(dst + kHalfBytes, &tmap_rows, full_bar(stage), 64, (int)(tile * kBM));
+                issued[stage] = true;
+                issued_parity[stage] = ph;
+            }
+            // Never leave the CTA with a TMA write in flight.
+            mbar_wait(s_bar, 0, abort_flag, kErrDrain);
+            for (int s = 0; s < kStages; ++s)
+                if (issued[s]) {
+                    for (uint32_t i = 0; i < kMaxPolls; ++i)
+                        if (mbar_try_wait(full_bar(s), issued_parity[s])) break;
+                }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            const uint32_t idesc = idesc_f16_f32(m);
+            bool ok = mbar_wait(s_bar, 0, abort_flag, kErrMma);
+            int it = 0;
+            for (int64_t tile = blockIdx.x; ok && tile < n_tiles; tile += gridDim.x, ++it) {
+                const int stage = it % kStages;
+                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                const int acc = it & 1;
+                const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+                if (!mbar_wait(full_bar(stage), ph, abort_flag, kErrMma)) break;
+                if (!mbar_wait(tempty_bar(acc), aph ^ 1u, abort_flag, kErrMma)) break;
+                tc_fence_after();
+                const uint32_t a0 = stage_base + (uint32_t)stage * kTileBytes;
+                const uint32_t d_tmem = tmem_base + (uint32_t)acc * kAccStride;
+#pragma unroll
+                for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint64_t ad = smem_desc_sw128(a0 + kb * kHalfBytes + k * 32);
+                        const uint64_t bd = smem_desc_sw128(s_base + kb * s_half_bytes + k * 32);
+                        tc_mma_f16(d_tmem, ad, bd, idesc, (kb | k) != 0);
+                    }
+                }
+                tc_commit(tfull_bar(acc));
+            }
+            // Wait for every MMA this thread issued before TMEM can be released.
+            tc_commit(done_bar);
+            for (uint32_t i = 0; i < kMaxPolls; ++i)
+                if (mbar_try_wait(done_bar, 0)) break;
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5) ----------------
+        const int quarter = warp & 3;            // TMEM lanes this warp may access
+        const int row = quarter * 32 + lane;     // key row within the tile
+        const int nw = m / 32;
+        int it = 0;
+        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+            const int stage = it % kStages;
+            const int acc = it & 1;
+            const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+            const bool ok = mbar_wait(tfull_bar(acc), aph, abort_flag, kErrEpilogue);
+            if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform: tcgen05.ld is .aligned
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)acc * kAccStride;
+            const int64_t key = tile * kBM + row;
+            if constexpr (!kSketchOut) {
+                uint32_t wbits[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    if (c < nw) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(taddr + (uint32_t)c * 32u, r);
+                        tmem_ld_wait();
+                        uint32_t neg = 0;
+#pragma unroll
+                        for (int j = 31; j >= 0; --j) {
+                            const float v = __fadd_rn(__uint_as_float(r[j]), 0.0f);
+                            neg = __funnelshift_l(__float_as_uint(v), neg, 1);
+                        }
+                        wbits[c] = ~neg;
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(tempty_bar(acc));
+                // Norm from the key tile in shared memory: row `row`, 16-byte chunk c of a
+                // 128-byte swizzled row lives at chunk position c ^ (row & 7).
+                const uint8_t* st = base_ptr + (stage_base - base) + (size_t)stage * kTileBytes;
+                double ss = 0.0;
+#pragma unroll
+                for (int kb = 0; kb < 2; ++kb) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 v = *reinterpret_cast<const uint4*>(
+                            st + kb * kHalfBytes + row * 128 + ((c ^ (row & 7)) << 4));
+                        const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float2 f = __half22float2(h[i]);
+                            ss = __fma_rn((double)f.x, (double)f.x, ss);
+                            ss = __fma_rn((double)f.y, (double)f.y, ss);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty_bar(stage));
+                if (key < n_rows) {
+                    if (ss == 0.0) {
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) wbits[c] = 0xFFFFFFFFu;
+                    }
+                    uint32_t* dst = words + key * nw;
+                    if ((nw & 3) == 0) {
+#pragma unroll
+                        for (int c = 0; c < 8; c += 4)
+                            if (c < nw)
+                                *reinterpret_cast<uint4*>(dst + c) =
+                                    make_uint4(wbits[c], wbits[c + 1], wbits[c + 2], wbits[c + 3]);
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            if (c < nw) dst[c] = wbits[c];
+                    }
+                    const __half hn = __double2half(__dsqrt_rn(ss));
+                    norms[key] = __half_as_ushort(hn);
+                }
+            } else {
+                float* dst = sketch_out + key * m;
+#pragma unroll 1
+                for (int c = 0; c < nw; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(taddr + (uint32_t)c * 32u, r);
+                    tmem_ld_wait();
+                    if (key < n_rows) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<float4*>(dst + c * 32 + j) =
+                                make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                            __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(tempty_bar(acc));
+                    mbar_arrive(empty_bar(stage));
+                }
+            }
+        }
+    }
+
+    __syncwarp();  // reconverge warps 0 and 1, whose lane 0 ran the role loop alone
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, kTmemCols);
+}
+
+// --------------------------------------------------------------------------------
+// Host side
+// --------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D fp16 tensor [rows][128], box = 64 columns x box_rows rows, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* ptr, int64_t rows, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)kDim, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)kDim * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t smem_bytes(int m) {
+    return 1024 /* alignment slack */ + 2u * (size_t)m * 128u + (size_t)kStages * kTileBytes +
+           8u * (2 * kStages + 6);
+}
+
+template <bool kSketchOut>
+cudaError_t launch_mma(const uint16_t* rows, int64_t n_rows, const uint16_t* S, int m,
+                       uint32_t* words, uint16_t* norms, float* sketch, cudaStream_t st) {
+    CUtensorMap map_rows, map_s;
+    if (!make_map(&map_rows, rows, n_rows, kBM)) return cudaErrorNotSupported;
+    if (!make_map(&map_s, S, m, m)) return cudaErrorNotSupported;
+    const size_t smem = smem_bytes(m);
+    cudaError_t e = cudaFuncSetAttribute(qjl_mma_kernel<kSketchOut>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t n_tiles = (n_rows + kBM - 1) / kBM;
+    const int64_t sms = device_sm_count();
+    const int grid = (int)(n_tiles < sms ? n_tiles : sms);
+    qjl_mma_kernel<kSketchOut><<<grid, kThreads, smem, st>>>(map_rows, map_s, n_rows, m, words,
+                                                             norms, sketch);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_qjl_encode(const uint16_t* keys, int64_t n_keys, const uint16_t* S, int m,
+                              uint32_t* words, uint16_t* norms, cudaStream_t st) {
+    return launch_mma<false>(keys, n_keys, S, m, words, norms, nullptr, st);
+}
+
+cudaError_t launch_qjl_query_sketch(const uint16_t* q, int64_t n_q, const uint16_t* S, int m,
+                                    float* v, cudaStream_t st) {
+    return launch_mma<true>(q, n_q, S, m, nullptr, nullptr, v, st);
+}
+
+cudaError_t read_and_clear_device_error(uint32_t* code) {
+    unsigned int v = 0, zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_kvq_device_error, sizeof(v));
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyToSymbol(g_kvq_device_error, &zero, sizeof(zero));
+    *code = v;
+    return e;
+}
+
+}  // namespace kvq

@@ -1,0 +1,230 @@
+"""Thin Python binding over libkvq (include/kvq.h): argument marshalling only.
+
+Every function has the name of the C entry point it calls, takes torch CUDA tensors,
+allocates its outputs with torch (device memory is torch's job; the library allocates
+nothing) and enqueues the work on the current torch stream.  All arithmetic happens in
+the library's CUDA kernels.  There is no fallback: if the library cannot be built or
+loaded, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CUDA, KVQ_ERR_WORKSPACE, KVQ_ERR_DEVICE = range(6)
+KVQ_F32, KVQ_F16 = 0, 1
+KVQ_KEYS_INT8, KVQ_KEYS_QJL = 0, 1
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+
+
+class DecodeArgs(ctypes.Structure):
+    """Mirror of ``kvq_decode_args``."""
+    _fields_ = [
+        ("batch", _I64), ("n_q_heads", _I64), ("n_kv_heads", _I64), ("seq_len", _I64),
+        ("head_dim", _I32), ("key_format", _I32),
+        ("q_f16", _P), ("k_codes", _P), ("k_scales", _P), ("k_words", _P), ("k_norms_f16", _P),
+        ("sketch_f16", _P), ("sketch_dim", _I32), ("sm_scale", ctypes.c_float),
+        ("v_codes", _P), ("v_scales", _P), ("out", _P), ("scores_out", _P),
+        ("workspace", _P), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+class KvqError(RuntimeError):
+    def __init__(self, fn, status):
+        self.status = status
+        super().__init__(f"{fn} failed: {lib.kvq_status_string(status).decode()} (status {status})")
+
+
+def _load():
+    path = _build.build()
+    so = ctypes.CDLL(path)
+    so.kvq_abi_version.restype = ctypes.c_int
+    so.kvq_status_string.argtypes = [ctypes.c_int]
+    so.kvq_status_string.restype = ctypes.c_char_p
+    so.kvq_quantize_int8.argtypes = [_P, ctypes.c_int, _I64, _I64, _P, _P, _P]
+    so.kvq_dequantize_int8.argtypes = [_P, _P, _I64, _I64, _P, ctypes.c_int, _P]
+    so.kvq_int8_scores.argtypes = [_P, ctypes.c_int, _P, _P, _I64, _I64, _P, _P]
+    so.kvq_qjl_encode.argtypes = [_P, _I64, _I32, _P, _I32, _P, _P, _P]
+    so.kvq_qjl_query_sketch.argtypes = [_P, _I64, _I32, _P, _I32, _P, _P]
+    so.kvq_decode_attention.argtypes = [ctypes.POINTER(DecodeArgs), _P]
+    so.kvq_decode_workspace_bytes.argtypes = [ctypes.POINTER(DecodeArgs)]
+    so.kvq_decode_workspace_bytes.restype = ctypes.c_size_t
+    so.kvq_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+    for f in ("kvq_quantize_int8", "kvq_dequantize_int8", "kvq_int8_scores", "kvq_qjl_encode",
+              "kvq_qjl_query_sketch", "kvq_decode_attention", "kvq_device_error"):
+        getattr(so, f).restype = ctypes.c_int
+    if so.kvq_abi_version() != 1:
+        raise RuntimeError(f"libkvq ABI version {so.kvq_abi_version()} != 1")
+    return so
+
+
+lib = _load()
+LIBRARY_PATH = os.path.abspath(_build.LIB)
+
+
+def _check(fn, status):
+    if status != KVQ_OK:
+        raise KvqError(fn, status)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.float16:
+        return KVQ_F16
+    if t.dtype == torch.float32:
+        return KVQ_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("inputs must be contiguous CUDA tensors")
+
+
+def _u16(t):
+    return t.view(torch.int16) if t.dtype == torch.float16 else t
+
+
+# --------------------------------------------------------------------------------------
+
+def kvq_quantize_int8(x, codes=None, scales=None, stream=None):
+    """Per-row absmax INT8 of x [..., D] (fp16/fp32): returns (codes int8 [..., D],
+    scales fp32 [...])."""
+    _need_cuda(x)
+    d = x.shape[-1]
+    n = x.numel() // d if d else 0
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    _check("kvq_quantize_int8", lib.kvq_quantize_int8(_ptr(x), _dtype_code(x), n, d, _ptr(codes),
+                                                      _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def kvq_dequantize_int8(codes, scales, out_dtype=torch.float32, out=None, stream=None):
+    _need_cuda(codes, scales)
+    d = codes.shape[-1]
+    n = codes.numel() // d if d else 0
+    if out is None:
+        out = torch.empty(codes.shape, dtype=out_dtype, device=codes.device)
+    _check("kvq_dequantize_int8", lib.kvq_dequantize_int8(_ptr(codes), _ptr(scales), n, d, _ptr(out),
+                                                          _dtype_code(out), _stream(stream)))
+    return out
+
+
+def kvq_int8_scores(q, codes, scales, out=None, stream=None):
+    """scores_r = sum_j q_j * x_hat_rj for one query q [D] against rows [..., D]."""
+    _need_cuda(q, codes, scales)
+    d = codes.shape[-1]
+    n = codes.numel() // d if d else 0
+    if out is None:
+        out = torch.empty(codes.shape[:-1], dtype=torch.float32, device=codes.device)
+    _check("kvq_int8_scores", lib.kvq_int8_scores(_ptr(q), _dtype_code(q), _ptr(codes), _ptr(scales),
+                                                  n, d, _ptr(out), _stream(stream)))
+    return out
+
+
+def kvq_qjl_encode(keys, sketch, words=None, norms=None, stream=None):
+    """QJL sign sketch of fp16 keys [..., 128] with fp16 S [m, 128]: returns
+    (words uint32-as-int32 [..., m/32], norms fp16 [...])."""
+    _need_cuda(keys, sketch)
+    d = keys.shape[-1]
+    n = keys.numel() // d if d else 0
+    m = sketch.shape[0]
+    if words is None:
+        words = torch.empty(keys.shape[:-1] + (m // 32,), dtype=torch.int32, device=keys.device)
+    if norms is None:
+        norms = torch.empty(keys.shape[:-1], dtype=torch.float16, device=keys.device)
+    _check("kvq_qjl_encode", lib.kvq_qjl_encode(_ptr(keys), n, d, _ptr(sketch), m, _ptr(words),
+                                                _ptr(norms), _stream(stream)))
+    return words, norms
+
+
+def kvq_qjl_query_sketch(q, sketch, out=None, stream=None):
+    _need_cuda(q, sketch)
+    d = q.shape[-1]
+    n = q.numel() // d if d else 0
+    m = sketch.shape[0]
+    if out is None:
+        out = torch.empty(q.shape[:-1] + (m,), dtype=torch.float32, device=q.device)
+    _check("kvq_qjl_query_sketch", lib.kvq_qjl_query_sketch(_ptr(q), n, d, _ptr(sketch), m,
+                                                            _ptr(out), _stream(stream)))
+    return out
+
+
+def make_decode_args(q, *, k_codes=None, k_scales=None, k_words=None, k_norms=None, sketch=None,
+                     v_codes=None, v_scales=None, out=None, scores_out=None, sm_scale=0.0,
+                     workspace=None):
+    """Fill a ``kvq_decode_args`` from tensors (q [B, Hq, D] fp16; cache [B, Hkv, T, ...])."""
+    B, Hq, D = q.shape
+    a = DecodeArgs()
+    a.batch, a.n_q_heads, a.head_dim = B, Hq, D
+    qjl = k_words is not None
+    ref = k_words if qjl else k_codes
+    a.n_kv_heads, a.seq_len = ref.shape[1], ref.shape[2]
+    a.key_format = KVQ_KEYS_QJL if qjl else KVQ_KEYS_INT8
+    a.q_f16 = q.data_ptr()
+    if qjl:
+        a.k_words, a.k_norms_f16, a.sketch_f16 = k_words.data_ptr(), k_norms.data_ptr(), sketch.data_ptr()
+        a.sketch_dim = sketch.shape[0]
+    else:
+        a.k_codes, a.k_scales = k_codes.data_ptr(), k_scales.data_ptr()
+    if v_codes is not None:
+        a.v_codes, a.v_scales = v_codes.data_ptr(), v_scales.data_ptr()
+    a.out = out.data_ptr() if out is not None else None
+    a.scores_out = scores_out.data_ptr() if scores_out is not None else None
+    a.sm_scale = float(sm_scale)
+    if workspace is not None:
+        a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    return a
+
+
+def kvq_decode_workspace_bytes(args: DecodeArgs) -> int:
+    return int(lib.kvq_decode_workspace_bytes(ctypes.byref(args)))
+
+
+def kvq_decode_attention(q, *, k_codes=None, k_scales=None, k_words=None, k_norms=None, sketch=None,
+                         v_codes=None, v_scales=None, want_out=True, want_scores=False,
+                         sm_scale=0.0, workspace=None, out=None, scores_out=None, stream=None):
+    """One decode step; returns (out [B, Hq, D] fp32 or None, scores [B, Hq, T] or None)."""
+    _need_cuda(q, k_codes, k_scales, k_words, k_norms, sketch, v_codes, v_scales)
+    B, Hq, D = q.shape
+    ref = k_words if k_words is not None else k_codes
+    T = ref.shape[2]
+    if want_out and out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    if want_scores and scores_out is None:
+        scores_out = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    a = make_decode_args(q, k_codes=k_codes, k_scales=k_scales, k_words=k_words, k_norms=k_norms,
+                         sketch=sketch, v_codes=v_codes if want_out else None,
+                         v_scales=v_scales if want_out else None, out=out if want_out else None,
+                         scores_out=scores_out if want_scores else None, sm_scale=sm_scale)
+    need = kvq_decode_workspace_bytes(a)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    _check("kvq_decode_attention", lib.kvq_decode_attention(ctypes.byref(a), _stream(stream)))
+    return (out if want_out else None), (scores_out if want_scores else None)
+
+
+def kvq_device_error() -> int:
+    code = ctypes.c_uint32(0)
+    _check("kvq_device_error", lib.kvq_device_error(ctypes.byref(code)))
+    return int(code.value)

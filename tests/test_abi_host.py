@@ -1,0 +1,115 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+entry point include/kvq.h declares, and rejects bad arguments before launching anything.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    from kv_cache_quantization_absmax_b200 import kvq as m
+    return m
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(kvq):
+    names = _declared()
+    assert {"kvq_quantize_int8", "kvq_dequantize_int8", "kvq_qjl_encode",
+            "kvq_decode_attention"} <= set(names)
+    for n in names:
+        assert hasattr(kvq.lib, n), n
+    assert kvq.lib.kvq_abi_version() == 1
+
+
+def test_status_strings(kvq):
+    for s in range(6):
+        assert kvq.lib.kvq_status_string(s)
+
+
+def _p(v):
+    return ctypes.c_void_p(v)
+
+
+A16 = 0x10000          # a 16-byte aligned dummy address (never dereferenced: checks fail first)
+
+
+def test_quantize_rejects_bad_arguments(kvq):
+    L = kvq.lib
+    E = kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_quantize_int8(_p(A16), 1, 10, 100, _p(A16), _p(A16), None) == E   # d % 16
+    assert L.kvq_quantize_int8(_p(A16), 1, -1, 128, _p(A16), _p(A16), None) == E   # n < 0
+    assert L.kvq_quantize_int8(_p(A16), 7, 10, 128, _p(A16), _p(A16), None) == E   # dtype
+    assert L.kvq_quantize_int8(None, 1, 10, 128, _p(A16), _p(A16), None) == E      # null
+    assert L.kvq_quantize_int8(_p(A16 + 8), 1, 10, 128, _p(A16), _p(A16), None) == E  # misaligned
+    assert L.kvq_quantize_int8(_p(A16), 1, 10, 128, _p(A16), _p(A16 + 2), None) == E
+    assert L.kvq_quantize_int8(_p(A16), 1, 10, 1 << 20, _p(A16), _p(A16), None) == E  # too wide
+    assert L.kvq_quantize_int8(None, 1, 0, 128, None, None, None) == kvq.KVQ_OK     # no rows
+    assert L.kvq_dequantize_int8(_p(A16), _p(A16), 10, 24, _p(A16), 0, None) == E
+    assert L.kvq_dequantize_int8(_p(A16), _p(A16), 10, 128, _p(A16 + 4), 0, None) == E
+    assert L.kvq_int8_scores(_p(A16), 0, _p(A16), _p(A16), 10, 16384, _p(A16), None) == E
+
+
+def test_qjl_rejects_bad_arguments(kvq):
+    L = kvq.lib
+    assert L.kvq_qjl_encode(_p(A16), 10, 64, _p(A16), 256, _p(A16), _p(A16), None) == kvq.KVQ_ERR_UNSUPPORTED
+    assert L.kvq_qjl_encode(_p(A16), 10, 128, _p(A16), 512, _p(A16), _p(A16), None) == kvq.KVQ_ERR_UNSUPPORTED
+    assert L.kvq_qjl_encode(_p(A16), 10, 128, _p(A16), 100, _p(A16), _p(A16), None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_qjl_encode(_p(A16), 10, 128, _p(A16), 256, _p(A16 + 4), _p(A16), None) == kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_qjl_encode(_p(A16), 0, 128, _p(A16), 256, None, None, None) == kvq.KVQ_OK
+    assert L.kvq_qjl_query_sketch(_p(A16), 4, 128, _p(A16), 256, _p(A16 + 4), None) == kvq.KVQ_ERR_INVALID_ARG
+
+
+def _args(kvq, **kw):
+    a = kvq.DecodeArgs()
+    a.batch, a.n_q_heads, a.n_kv_heads, a.seq_len, a.head_dim = 1, 8, 2, 100, 128
+    a.key_format = kvq.KVQ_KEYS_INT8
+    a.q_f16 = a.k_codes = a.k_scales = a.v_codes = a.v_scales = a.out = A16
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_decode_rejects_bad_arguments(kvq):
+    L = kvq.lib
+    call = lambda a: L.kvq_decode_attention(ctypes.byref(a), None)
+    E, U = kvq.KVQ_ERR_INVALID_ARG, kvq.KVQ_ERR_UNSUPPORTED
+    assert call(_args(kvq, n_kv_heads=3)) == E                 # Hq % Hkv
+    assert call(_args(kvq, seq_len=0)) == E                    # softmax over nothing
+    assert call(_args(kvq, head_dim=64)) == U
+    assert call(_args(kvq, head_dim=100)) == E
+    assert call(_args(kvq, out=None)) == E                     # nothing requested
+    assert call(_args(kvq, key_format=5)) == E
+    assert call(_args(kvq, n_q_heads=6, n_kv_heads=2)) == U    # G = 3
+    assert call(_args(kvq, k_codes=A16 + 1)) == E
+    assert call(_args(kvq, q_f16=None)) == E
+    assert call(_args(kvq, sm_scale=-1.0)) == E
+    qjl = dict(key_format=kvq.KVQ_KEYS_QJL, k_words=A16, k_norms_f16=A16, sketch_f16=A16)
+    assert call(_args(kvq, sketch_dim=100, **qjl)) == E
+    assert call(_args(kvq, sketch_dim=512, **qjl)) == U
+    assert call(_args(kvq, sketch_dim=256, n_q_heads=16, **qjl)) == U   # QJL with G = 8
+    assert call(_args(kvq, sketch_dim=256, sketch_f16=A16 + 2,
+                      **{k: v for k, v in qjl.items() if k != "sketch_f16"})) == E
+    # valid arguments but no workspace
+    assert call(_args(kvq)) == kvq.KVQ_ERR_WORKSPACE
+    assert L.kvq_decode_workspace_bytes(ctypes.byref(_args(kvq))) > 0
+    assert L.kvq_decode_workspace_bytes(ctypes.byref(_args(kvq, seq_len=0))) == 0
+    # batch 0: nothing to do
+    assert call(_args(kvq, batch=0)) == kvq.KVQ_OK
+
+
+def test_product_path_has_no_cpu_fallback():
+    """The binding loads only libkvq and never the oracle."""
+    src = open(os.path.join(ROOT, "kv_cache_quantization_absmax_b200", "kvq.py")).read()
+    assert "oracle" not in src.replace("never the oracle", "")
+    for f in os.listdir(os.path.join(ROOT, "kv_cache_quantization_absmax_b200", "csrc")):
+        assert "oracle" not in open(os.path.join(ROOT, "kv_cache_quantization_absmax_b200", "csrc", f)).read()

@@ -1,0 +1,163 @@
+"""GPU parity of the fused decode step (scores -> softmax -> sum of INT8 values) against
+the CPU oracle, for INT8 keys and QJL keys, MHA and GQA.
+
+Decode outputs: max-abs error <= 2e-3 against the oracle's fp32-accumulated result.
+INT8 raw scores: the fp32 summation bound.  QJL estimator scores (same sign words and
+norms on both sides): 1e-4 relative to max(|score|, c ||k|| ||S q||_2).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_quantization_absmax_b200 import inputs
+from tests._helpers import score_tolerance, to_np
+
+pytestmark = pytest.mark.gpu
+
+OUT_TOL = 2e-3
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    from kv_cache_quantization_absmax_b200 import kvq as m
+    return m
+
+
+def _int8_cache(seed, B, Hkv, T, Hq):
+    k, v = inputs.lognormal_cache(seed, B, Hkv, T, n_tensors=2)
+    q = inputs.gaussian_queries(seed + 1, B, Hq)
+    kc, ks = oracle.quantize_int8(k.reshape(-1, 128))
+    vc, vs = oracle.quantize_int8(v.reshape(-1, 128))
+    shp = (B, Hkv, T)
+    return q, kc.reshape(shp + (128,)), ks.reshape(shp), vc.reshape(shp + (128,)), vs.reshape(shp)
+
+
+def _cuda(*arrs):
+    return [torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in arrs]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T", [(1, 1, 1, 1), (1, 4, 4, 5), (2, 8, 2, 33), (1, 8, 1, 1000),
+                                        (2, 16, 4, 4097), (1, 8, 8, 300), (1, 16, 2, 2500)])
+def test_decode_int8_parity(kvq, B, Hq, Hkv, T):
+    q, kc, ks, vc, vs = _int8_cache(10 + T, B, Hkv, T, Hq)
+    ref = oracle.decode_attention(q, k_codes=kc, k_scales=ks, v_codes=vc, v_scales=vs,
+                                  want_scores=True)
+    qg, kcg, ksg, vcg, vsg = _cuda(q, kc, ks, vc, vs)
+    out, scores = kvq.kvq_decode_attention(qg, k_codes=kcg, k_scales=ksg, v_codes=vcg,
+                                           v_scales=vsg, want_scores=True)
+    assert np.abs(to_np(out) - ref["out"]).max() <= OUT_TOL
+    # raw scores: fp32 summation bound on the same codes
+    G = Hq // Hkv
+    xh = (kc.astype(np.float64) * ks.astype(np.float64)[..., None])
+    terms = np.abs(np.repeat(xh, G, axis=1) * q.astype(np.float64)[:, :, None, :]).sum(-1)
+    assert np.all(np.abs(to_np(scores).astype(np.float64) - ref["scores"]) <= 2 * 128 * 2.0 ** -24 * terms + 1e-30)
+
+
+def test_decode_scores_only_outlier_layer(kvq):
+    """The one-layer INT8 cache with outlier channels: scores of one fp16 query per head
+    against the dequantized keys (no value pass)."""
+    k, v, q = inputs.outlier_layer(seed=0)
+    kc, ks = oracle.quantize_int8(k.reshape(-1, 128))
+    kc, ks = kc.reshape(k.shape), ks.reshape(k.shape[:-1])
+    ref = oracle.decode_attention(q, k_codes=kc, k_scales=ks, want_out=False, want_scores=True)
+    qg, kcg, ksg = _cuda(q, kc, ks)
+    out, scores = kvq.kvq_decode_attention(qg, k_codes=kcg, k_scales=ksg, want_out=False,
+                                           want_scores=True)
+    assert out is None
+    xh = kc.astype(np.float64) * ks.astype(np.float64)[..., None]
+    terms = np.abs(xh * q.astype(np.float64)[:, :, None, :]).sum(-1)
+    assert np.all(np.abs(to_np(scores).astype(np.float64) - ref["scores"]) <= 2 * 128 * 2.0 ** -24 * terms)
+
+
+def _qjl_cache(seed, B, Hkv, T, Hq, m=256):
+    k, v = inputs.lognormal_cache(seed, B, Hkv, T, n_tensors=2)
+    q = inputs.gaussian_queries(seed + 1, B, Hq)
+    S = inputs.sketch_matrix(m, 128)
+    w, n = oracle.qjl_encode(k.reshape(-1, 128), S)
+    vc, vs = oracle.quantize_int8(v.reshape(-1, 128))
+    shp = (B, Hkv, T)
+    return q, S, w.reshape(shp + (m // 32,)), n.reshape(shp), vc.reshape(shp + (128,)), vs.reshape(shp)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T,m", [(1, 1, 1, 1, 256), (1, 4, 1, 7, 256), (2, 8, 2, 1500, 256),
+                                          (1, 32, 8, 2049, 256), (1, 4, 4, 700, 128), (1, 2, 1, 333, 32)])
+def test_decode_qjl_parity(kvq, B, Hq, Hkv, T, m):
+    q, S, w, n, vc, vs = _qjl_cache(100 + T, B, Hkv, T, Hq, m)
+    ref = oracle.decode_attention(q, k_words=w, k_norms=n, S=S, v_codes=vc, v_scales=vs,
+                                  want_scores=True)
+    qg, Sg, wg, ng, vcg, vsg = _cuda(q, S, w.view(np.int32), n, vc, vs)
+    out, scores = kvq.kvq_decode_attention(qg, k_words=wg, k_norms=ng, sketch=Sg, v_codes=vcg,
+                                           v_scales=vsg, want_scores=True)
+    assert np.abs(to_np(out) - ref["out"]).max() <= OUT_TOL
+    v64, _ = oracle.qjl_query_sketch(q.reshape(-1, 128), S)
+    G = Hq // Hkv
+    tol = score_tolerance(ref["scores"].reshape(B * Hq, T),
+                          np.repeat(n, G, axis=1).reshape(B * Hq, T), v64, m)
+    err = np.abs(to_np(scores).astype(np.float64) - ref["scores"]).reshape(B * Hq, T)
+    assert np.all(err <= tol), float((err / tol).max())
+
+
+def test_decode_int8_llama7b_layer_sampled(kvq):
+    """One layer of the 7B-shaped cache (batch 8, 32 heads, 4096 tokens): GPU quantize
+    then GPU decode; 6 sampled (batch, head) units re-done by the oracle from the fp16
+    cache."""
+    B, H, T = 8, 32, 4096
+    kv = inputs.lognormal_cache_device(3, (2, B, H, T, 128), n_sigma_dims=(0, 2, 4), device="cuda")
+    q = inputs.gaussian_queries_device(33, (B, H, 128), "cuda")
+    kc, ks = kvq.kvq_quantize_int8(kv[0])
+    vc, vs = kvq.kvq_quantize_int8(kv[1])
+    out, _ = kvq.kvq_decode_attention(q, k_codes=kc, k_scales=ks, v_codes=vc, v_scales=vs)
+    out = to_np(out)
+    rng = np.random.default_rng(3)
+    for b, h in zip(rng.integers(0, B, 6), rng.integers(0, H, 6)):
+        k_np = to_np(kv[0, b, h])
+        v_np = to_np(kv[1, b, h])
+        kc_r, ks_r = oracle.quantize_int8(k_np)
+        vc_r, vs_r = oracle.quantize_int8(v_np)
+        ref = oracle.decode_attention(to_np(q[b, h])[None, None], k_codes=kc_r[None, None],
+                                      k_scales=ks_r[None, None], v_codes=vc_r[None, None],
+                                      v_scales=vs_r[None, None])
+        assert np.abs(out[b, h] - ref["out"][0, 0]).max() <= OUT_TOL
+
+
+def test_decode_qjl_gqa_long_context_sampled(kvq):
+    """Long-context GQA cache: batch 4, 32 query / 8 KV heads, 131072 tokens; keys
+    QJL-encoded and values INT8-quantized on the GPU, then one fused decode step.  One
+    sampled KV unit (4 query heads) is re-done end to end by the oracle."""
+    B, Hq, Hkv, T = 4, 32, 8, 131072
+    kv = inputs.lognormal_cache_device(5, (2, B, Hkv, T, 128), n_sigma_dims=(0, 2, 4), device="cuda")
+    q = inputs.gaussian_queries_device(50, (B, Hq, 128), "cuda")
+    S_np = inputs.sketch_matrix(256, 128)
+    S = torch.from_numpy(S_np).cuda()
+    words, norms = kvq.kvq_qjl_encode(kv[0], S)
+    vc, vs = kvq.kvq_quantize_int8(kv[1])
+    out, _ = kvq.kvq_decode_attention(q, k_words=words, k_norms=norms, sketch=S, v_codes=vc,
+                                      v_scales=vs)
+    out = to_np(out)
+    assert kvq.kvq_device_error() == 0
+    b, g = 2, 5
+    k_np = to_np(kv[0, b, g])
+    v_np = to_np(kv[1, b, g])
+    w_r, n_r = oracle.qjl_encode(k_np, S_np)
+    vc_r, vs_r = oracle.quantize_int8(v_np)
+    qs = to_np(q[b, g * 4:(g + 1) * 4])[None]
+    ref = oracle.decode_attention(qs, k_words=w_r[None, None], k_norms=n_r[None, None], S=S_np,
+                                  v_codes=vc_r[None, None], v_scales=vs_r[None, None])
+    assert np.abs(out[b, g * 4:(g + 1) * 4] - ref["out"][0]).max() <= OUT_TOL
+
+
+def test_decode_rejects_bad_workspace(kvq):
+    q, kc, ks, vc, vs = _int8_cache(1, 1, 2, 64, 2)
+    qg, kcg, ksg, vcg, vsg = _cuda(q, kc, ks, vc, vs)
+    out = torch.empty((1, 2, 128), dtype=torch.float32, device="cuda")
+    a = kvq.make_decode_args(qg, k_codes=kcg, k_scales=ksg, v_codes=vcg, v_scales=vsg, out=out)
+    need = kvq.kvq_decode_workspace_bytes(a)
+    assert need > 0
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    a.workspace, a.workspace_bytes = ws.data_ptr(), need - 1
+    import ctypes
+    assert kvq.lib.kvq_decode_attention(ctypes.byref(a), None) == kvq.KVQ_ERR_WORKSPACE
+    a.workspace_bytes = need
+    assert kvq.lib.kvq_decode_attention(ctypes.byref(a), None) == kvq.KVQ_OK
+    torch.cuda.synchronize()
