@@ -1,0 +1,600 @@
+#!/usr/bin/env python
+"""Throughput of the KV-cache compression + compressed-cache decode path on B200.
+
+One step is one pass of the whole path over one batch of synthetic input:
+  7B-shaped cache  (32 layers x {K, V} x [batch 8, 32 heads, 4096 tokens, 128] fp16)
+    1. INT8 per-token absmax quantize of the whole cache            (1 launch)
+    2. one decode step per layer: INT8 scores, softmax, sum of INT8
+       values, one fp16 query per head                              (32 x 2 launches)
+    3. INT8 dequantize of the whole cache back to fp16               (1 launch)
+  long-context GQA cache (batch 4, 32 query / 8 KV heads, 131072 tokens, 128)
+    4. QJL sign sketch of K (m = 256, Gaussian S from seed 7)        (1 launch)
+    5. INT8 quantize of V                                            (1 launch)
+    6. one fused GQA decode step: query sketch, estimator scores,
+       softmax, sum of INT8 values                                   (3 launches)
+The reported value is the algorithmic bytes of the step (each input read once, each
+output written once) divided by the device time of the step, in GB/s; decode keys/s and
+per-row figures are reported beside it.  Inputs (~47 GB resident) are far larger than
+the 126 MB L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Under torchrun each rank runs the same workload on its own GPU (weak scaling, no
+collective on the data path); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "KV quantize/dequant GB/s and compressed-cache decode keys/s; % of HBM peak"
+FALLBACK_HBM_GBS = 6650.0
+
+# ---------------------------------------------------------------------------------
+# Workload geometry and algorithmic bytes (host logic; no GPU needed)
+# ---------------------------------------------------------------------------------
+LLAMA = dict(layers=32, batch=8, heads=32, seq=4096, dim=128)
+GQA = dict(batch=4, q_heads=32, kv_heads=8, seq=131072, dim=128, m=256)
+
+
+def row_bytes(llama=LLAMA, gqa=GQA):
+    """Algorithmic bytes of each row of the step (read once + written once)."""
+    D = llama["dim"]
+    rows_a = llama["layers"] * 2 * llama["batch"] * llama["heads"] * llama["seq"]
+    keys_layer = llama["batch"] * llama["heads"] * llama["seq"]
+    q_layer = llama["batch"] * llama["heads"] * D
+    n_g = gqa["batch"] * gqa["kv_heads"] * gqa["seq"]
+    m = gqa["m"]
+    q_g = gqa["batch"] * gqa["q_heads"] * D
+    return {
+        "quantize_cache": rows_a * (2 * D + D + 4),
+        "decode_int8": llama["layers"] * (keys_layer * 2 * (D + 4) + q_layer * 2 + q_layer * 4),
+        "dequantize_cache": rows_a * (D + 4 + 2 * D),
+        "qjl_encode": n_g * (2 * D + m // 8 + 2) + m * D * 2,
+        "quantize_v": n_g * (2 * D + D + 4),
+        "decode_qjl": n_g * (m // 8 + 2 + D + 4) + m * D * 2 + q_g * 2 + q_g * 4,
+    }
+
+
+def decode_keys(llama=LLAMA, gqa=GQA):
+    return (llama["layers"] * llama["batch"] * llama["heads"] * llama["seq"]
+            + gqa["batch"] * gqa["kv_heads"] * gqa["seq"])
+
+
+LAUNCHES_PER_STEP = 1 + LLAMA["layers"] * 2 + 1 + 1 + 1 + 3
+
+
+def max_over_ranks(value: float, group=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    backend = dist.get_backend(group)
+    dev = torch.device("cuda", torch.cuda.current_device()) if backend == "nccl" else torch.device("cpu")
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())
+
+
+def aggregate(bytes_per_rank: float, n_ranks: int, step_ms_max: float, steps: int) -> float:
+    """Whole-job GB/s: bytes all ranks processed / the slowest rank's time."""
+    return bytes_per_rank * n_ranks * steps / (step_ms_max * steps * 1e-3) / 1e9
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------------
+# Clock sampling during the timed region
+# ---------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="kvq_clocks_", suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "100"]
+            if self.gpu_id:
+                cmd += ["-i", self.gpu_id]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for _, _, flags in rows for n, fl in zip(names, flags) if fl == "Active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_id_for(device_index: int):
+    import torch
+    try:
+        uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------------
+# The device workload
+# ---------------------------------------------------------------------------------
+class Workload:
+    def __init__(self, device, seed_offset=0):
+        import torch
+        from kv_cache_quantization_absmax_b200 import inputs, kvq
+
+        self.kvq = kvq
+        self.torch = torch
+        L, B, H, T, D = (LLAMA[k] for k in ("layers", "batch", "heads", "seq", "dim"))
+        gb, gq, gk, gt, m = (GQA[k] for k in ("batch", "q_heads", "kv_heads", "seq", "m"))
+        dev = device
+        # 7B-shaped cache [L, 2, B, H, T, D] fp16: one sigma per (layer, K/V, head, channel)
+        self.cache = inputs.lognormal_cache_device(3 + seed_offset, (L, 2, B, H, T, D),
+                                                   n_sigma_dims=(0, 1, 3, 5), device=dev)
+        self.q7 = inputs.gaussian_queries_device(30 + seed_offset, (L, B, H, D), dev)
+        self.codes = torch.empty((L, 2, B, H, T, D), dtype=torch.int8, device=dev)
+        self.scales = torch.empty((L, 2, B, H, T), dtype=torch.float32, device=dev)
+        self.deq = torch.empty((L, 2, B, H, T, D), dtype=torch.float16, device=dev)
+        self.out7 = torch.empty((L, B, H, D), dtype=torch.float32, device=dev)
+        # long-context GQA cache [2, B, Hkv, T, D] fp16
+        self.gcache = inputs.lognormal_cache_device(5 + seed_offset, (2, gb, gk, gt, D),
+                                                    n_sigma_dims=(0, 2, 4), device=dev)
+        self.qg = inputs.gaussian_queries_device(50 + seed_offset, (gb, gq, D), dev)
+        self.S = torch.from_numpy(inputs.sketch_matrix(m, D)).to(dev)
+        self.words = torch.empty((gb, gk, gt, m // 32), dtype=torch.int32, device=dev)
+        self.norms = torch.empty((gb, gk, gt), dtype=torch.float16, device=dev)
+        self.vcodes = torch.empty((gb, gk, gt, D), dtype=torch.int8, device=dev)
+        self.vscales = torch.empty((gb, gk, gt), dtype=torch.float32, device=dev)
+        self.outg = torch.empty((gb, gq, D), dtype=torch.float32, device=dev)
+        # decode argument structs and caller-owned workspaces (sized once)
+        self.args7 = []
+        for l in range(L):
+            a = kvq.make_decode_args(self.q7[l], k_codes=self.codes[l, 0], k_scales=self.scales[l, 0],
+                                     v_codes=self.codes[l, 1], v_scales=self.scales[l, 1],
+                                     out=self.out7[l])
+            self.args7.append(a)
+        ws7 = kvq.kvq_decode_workspace_bytes(self.args7[0])
+        self.ws7 = torch.empty(ws7, dtype=torch.uint8, device=dev)
+        for a in self.args7:
+            a.workspace, a.workspace_bytes = self.ws7.data_ptr(), ws7
+        self.argsg = kvq.make_decode_args(self.qg, k_words=self.words, k_norms=self.norms, sketch=self.S,
+                                          v_codes=self.vcodes, v_scales=self.vscales, out=self.outg)
+        wsg = kvq.kvq_decode_workspace_bytes(self.argsg)
+        self.wsg = torch.empty(wsg, dtype=torch.uint8, device=dev)
+        self.argsg.workspace, self.argsg.workspace_bytes = self.wsg.data_ptr(), wsg
+        torch.cuda.synchronize()
+
+    def step(self, stream, ev=None):
+        """Launch the whole path on `stream`; if `ev` (7 events) is given, record row
+        boundaries."""
+        import ctypes
+        kvq = self.kvq
+        lib = kvq.lib
+        s = ctypes.c_void_p(stream.cuda_stream)
+        rec = (lambda i: ev[i].record(stream)) if ev is not None else (lambda i: None)
+        rec(0)
+        kvq.kvq_quantize_int8(self.cache, self.codes, self.scales, stream=stream)
+        rec(1)
+        for a in self.args7:
+            st = lib.kvq_decode_attention(ctypes.byref(a), s)
+            if st != kvq.KVQ_OK:
+                raise kvq.KvqError("kvq_decode_attention", st)
+        rec(2)
+        kvq.kvq_dequantize_int8(self.codes, self.scales, out=self.deq, stream=stream)
+        rec(3)
+        kvq.kvq_qjl_encode(self.gcache[0], self.S, self.words, self.norms, stream=stream)
+        rec(4)
+        kvq.kvq_quantize_int8(self.gcache[1], self.vcodes, self.vscales, stream=stream)
+        rec(5)
+        st = lib.kvq_decode_attention(ctypes.byref(self.argsg), s)
+        if st != kvq.KVQ_OK:
+            raise kvq.KvqError("kvq_decode_attention", st)
+        rec(6)
+
+    def host_buffers(self):
+        """Pinned host copies of the step's inputs, for the end-to-end measurement."""
+        t = self.torch
+        hb = {}
+        for name in ("cache", "q7", "gcache", "qg"):
+            dv = getattr(self, name)
+            h = t.empty(dv.shape, dtype=dv.dtype, pin_memory=True)
+            h.copy_(dv)
+            hb[name] = h
+        hb["out7"] = t.empty(self.out7.shape, dtype=t.float32, pin_memory=True)
+        hb["outg"] = t.empty(self.outg.shape, dtype=t.float32, pin_memory=True)
+        return hb
+
+
+ROW_NAMES = ["quantize_cache", "decode_int8", "dequantize_cache", "qjl_encode", "quantize_v",
+             "decode_qjl"]
+
+
+# ---------------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample of the same workload, single thread)
+# ---------------------------------------------------------------------------------
+class CpuSample:
+    """A bounded sample of each row of the step, drawn once (outside any timing), that
+    the single-threaded C oracle is timed on."""
+
+    def __init__(self, scale: float = 1.0):
+        import numpy as np
+
+        import oracle
+        from kv_cache_quantization_absmax_b200 import inputs
+
+        D, m = 128, GQA["m"]
+        self.D, self.m = D, m
+        self.n_rows = max(1024, int(131072 * scale))      # quantize / dequantize rows
+        self.n_units = max(1, int(8 * scale))             # INT8 decode: units of 4096 tokens
+        self.n_keys = max(512, int(16384 * scale))        # QJL encode keys
+        self.n_gtok = max(1024, int(32768 * scale))       # QJL decode tokens (4 query heads)
+        self.x = inputs.lognormal_cache(3, 1, 1, self.n_rows)[0].reshape(self.n_rows, D)
+        self.c, self.s = oracle.quantize_int8(self.x)
+        T = LLAMA["seq"]
+        kk, vv = inputs.lognormal_cache(31, self.n_units, 1, T, n_tensors=2)
+        kc, ks = oracle.quantize_int8(kk.reshape(-1, D))
+        vc, vs = oracle.quantize_int8(vv.reshape(-1, D))
+        shp = (self.n_units, 1, T)
+        self.dec8 = dict(k_codes=kc.reshape(shp + (D,)), k_scales=ks.reshape(shp),
+                         v_codes=vc.reshape(shp + (D,)), v_scales=vs.reshape(shp))
+        self.q8 = inputs.gaussian_queries(32, self.n_units, 1)
+        self.S = inputs.sketch_matrix(m, D)
+        self.kq = inputs.lognormal_cache(41, 1, 1, self.n_keys)[0].reshape(self.n_keys, D)
+        # the estimator's cost does not depend on the bit values: seeded random sign
+        # words and norms stand in for encoded keys
+        rng = np.random.default_rng(51)
+        w = rng.integers(0, 2 ** 32, (self.n_gtok, m // 32), dtype=np.uint32)
+        n = (np.abs(rng.standard_normal(self.n_gtok)) * 11 + 1).astype(np.float16)
+        vg = inputs.lognormal_cache(52, 1, 1, self.n_gtok)[0]
+        vgc, vgs = oracle.quantize_int8(vg.reshape(-1, D))
+        gs = (1, 1, self.n_gtok)
+        self.decq = dict(k_words=w.reshape(gs + (m // 32,)), k_norms=n.reshape(gs), S=self.S,
+                         v_codes=vgc.reshape(gs + (D,)), v_scales=vgs.reshape(gs))
+        self.qg = inputs.gaussian_queries(53, 1, 4)
+        self.np = np
+        self.description = (
+            f"single-threaded C oracle on a bounded sample of each row: quantize/dequantize "
+            f"{self.n_rows} rows x 128 fp16, INT8 decode {self.n_units} units x {T} tokens, QJL "
+            f"encode {self.n_keys} keys, QJL GQA decode 1 KV unit x {self.n_gtok} tokens x 4 query "
+            f"heads; each row's GB/s is applied to that row's bytes in the full step")
+
+    def rates(self):
+        import oracle
+
+        D, m = self.D, self.m
+        r = {}
+
+        def timed(fn):
+            t0 = time.perf_counter()
+            fn()
+            return time.perf_counter() - t0
+
+        dt = timed(lambda: oracle.quantize_int8(self.x))
+        r["quantize_cache"] = r["quantize_v"] = self.n_rows * (3 * D + 4) / dt / 1e9
+        dt = timed(lambda: oracle.dequantize_int8(self.c, self.s, self.np.float16))
+        r["dequantize_cache"] = self.n_rows * (3 * D + 4) / dt / 1e9
+        dt = timed(lambda: oracle.decode_attention(self.q8, **self.dec8))
+        r["decode_int8"] = self.n_units * LLAMA["seq"] * 2 * (D + 4) / dt / 1e9
+        dt = timed(lambda: oracle.qjl_encode(self.kq, self.S))
+        r["qjl_encode"] = self.n_keys * (2 * D + m // 8 + 2) / dt / 1e9
+        dt = timed(lambda: oracle.decode_attention(self.qg, **self.decq))
+        r["decode_qjl"] = self.n_gtok * (m // 8 + 2 + D + 4) / dt / 1e9
+        return r
+
+
+def cpu_step_gbs(rates):
+    rb = row_bytes()
+    t = sum(rb[k] / 1e9 / rates[k] for k in rb)
+    return sum(rb.values()) / 1e9 / t, t
+
+
+# ---------------------------------------------------------------------------------
+# Arms
+# ---------------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    smp = CpuSample(args.ref_scale)
+    for _ in range(args.warmup):
+        smp.rates()
+    times, per_step = [], []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        rates = smp.rates()
+        times.append(time.perf_counter() - t0)
+        per_step.append(cpu_step_gbs(rates))
+    value = statistics.median(v for v, _ in per_step)
+    step_s = statistics.median(t for _, t in per_step)
+    sample = smp.description
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(step_s * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "sample_wall_s_per_step": round(statistics.median(times), 3),
+        "note": "the CPU oracle as it stands; ms_per_step is the full step extrapolated from "
+                "per-row sample rates",
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config():
+    return {
+        "workload": "llama7b_kv_cache_int8 (32L x {K,V} x [8,32,4096,128] fp16: quantize, 32 decode "
+                    "steps, dequantize) + gqa_long_context_qjl ([4, 32q/8kv, 131072, 128] fp16: QJL "
+                    "encode m=256, INT8 V, fused GQA decode)",
+        "llama_cache": dict(LLAMA), "gqa_cache": dict(GQA),
+        "l2": "inputs larger than L2 (about 47 GB resident per GPU), no flush",
+        "parallelism": "weak-scaled replicas, one per GPU",
+    }
+
+
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    from kv_cache_quantization_absmax_b200 import kvq
+    wl = Workload(dev)
+    stream = torch.cuda.Stream(device=dev)
+    rb = row_bytes()
+    step_bytes = float(sum(rb.values()))
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            wl.step(stream)
+    torch.cuda.synchronize()
+    if kvq.kvq_device_error() != 0:
+        raise RuntimeError("device-side error recorded during warm-up")
+
+    # ---- device-timed region ----
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(gpu_id_for(dev.index))
+    barrier()
+    sampler.start()
+    time.sleep(0.3)
+    t_start.record(stream)
+    with torch.cuda.stream(stream):
+        for k in range(args.steps):
+            wl.step(stream, evs[k])
+    t_end.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    total_ms_max = max_over_ranks(total_ms)
+    ms_step = total_ms_max / args.steps
+    row_ms = {n: statistics.mean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps))
+              for i, n in enumerate(ROW_NAMES)}
+    if kvq.kvq_device_error() != 0:
+        raise RuntimeError("device-side error recorded during the timed region")
+
+    # ---- end to end: pinned host inputs -> device, step, outputs -> host ----
+    e2e = None
+    try:
+        hb = wl.host_buffers()
+        h2d = sum(hb[n].numel() * hb[n].element_size() for n in ("cache", "q7", "gcache", "qg"))
+        d2h = sum(hb[n].numel() * hb[n].element_size() for n in ("out7", "outg"))
+        e_steps = max(1, min(args.steps, args.e2e_steps))
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(e_steps):
+                wl.cache.copy_(hb["cache"], non_blocking=True)
+                wl.q7.copy_(hb["q7"], non_blocking=True)
+                wl.gcache.copy_(hb["gcache"], non_blocking=True)
+                wl.qg.copy_(hb["qg"], non_blocking=True)
+                wl.step(stream)
+                hb["out7"].copy_(wl.out7, non_blocking=True)
+                hb["outg"].copy_(wl.outg, non_blocking=True)
+        e1.record(stream)
+        barrier()
+        e_ms = max_over_ranks(e0.elapsed_time(e1)) / e_steps
+        e2e = {"value": round(aggregate(step_bytes, world, e_ms, 1), 2), "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": round(e_ms, 3), "steps": e_steps}
+        del hb
+    except RuntimeError as exc:  # pinned allocation can fail on a small host
+        e2e = {"value": None, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
+               "unavailable": str(exc)[:200]}
+
+    if rank == 0:
+        peak, peak_kind = load_peaks()
+        dom = max(("quantize_cache", "dequantize_cache"), key=lambda n: row_ms[n])
+        achieved = rb[dom] / (row_ms[dom] * 1e-3) / 1e9
+        traffic = load_traffic(dom)
+        rows = {n: {"ms": round(row_ms[n], 4), "GB/s": round(rb[n] / (row_ms[n] * 1e-3) / 1e9, 1),
+                    "frac_hbm": round(rb[n] / (row_ms[n] * 1e-3) / 1e9 / peak, 4)} for n in ROW_NAMES}
+        dec_ms = row_ms["decode_int8"] + row_ms["decode_qjl"]
+        line = {
+            "metric": METRIC, "value": round(aggregate(step_bytes, world, ms_step, args.steps), 2),
+            "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "storage": "fp16 in; int8 codes + fp32 scales; "
+            "1-bit sign words + fp16 norms", "data": "synthetic", "config": workload_config(),
+            "frac_hbm_step": round(aggregate(step_bytes, 1, ms_step, 1) / peak, 4),
+            "decode_keys_per_s": round(decode_keys() * world / (dec_ms * 1e-3), 1),
+            "rows": rows,
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
+                         "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs"},
+            "e2e": e2e,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            smp = CpuSample(args.cpu_scale)
+            v, _ = cpu_step_gbs(smp.rates())
+            line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                                    "sample": smp.description}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def load_traffic(kernel_row: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if its
+    recorded source hash matches the current kernels (else null)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            tr = json.load(f)
+        from kv_cache_quantization_absmax_b200 import build as kb
+        if tr.get("source_hash") != kb.source_hash():
+            return None
+        v = tr.get("rows", {}).get(kernel_row)
+        return None if v is None else float(v)
+    except Exception:
+        return None
+
+
+def run_profile_case(case: str, reps: int = 3):
+    """Small single-kernel cases for ncu captures (inputs larger than L2, a few GB at most)."""
+    import torch
+    from kv_cache_quantization_absmax_b200 import inputs, kvq
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    B, H, T, D = LLAMA["batch"], LLAMA["heads"], LLAMA["seq"], LLAMA["dim"]
+    if case in ("quantize", "dequantize", "decode_int8"):
+        kv = inputs.lognormal_cache_device(3, (2, B, H, T, D), n_sigma_dims=(0, 2, 4), device=dev)
+        codes, scales = kvq.kvq_quantize_int8(kv)
+        out = torch.empty_like(kv)
+        q = inputs.gaussian_queries_device(30, (B, H, D), dev)
+        for _ in range(reps):
+            if case == "quantize":
+                kvq.kvq_quantize_int8(kv, codes, scales)
+            elif case == "dequantize":
+                kvq.kvq_dequantize_int8(codes, scales, out=out)
+            else:
+                kvq.kvq_decode_attention(q, k_codes=codes[0], k_scales=scales[0], v_codes=codes[1],
+                                         v_scales=scales[1])
+    elif case in ("qjl_encode", "decode_qjl"):
+        gb, gq, gk, gt, m = (GQA[k] for k in ("batch", "q_heads", "kv_heads", "seq", "m"))
+        if case == "qjl_encode":
+            gb = 1
+        kv = inputs.lognormal_cache_device(5, (2, gb, gk, gt, D), n_sigma_dims=(0, 2, 4), device=dev)
+        S = torch.from_numpy(inputs.sketch_matrix(m, D)).to(dev)
+        words, norms = kvq.kvq_qjl_encode(kv[0], S)
+        vc, vs = kvq.kvq_quantize_int8(kv[1])
+        q = inputs.gaussian_queries_device(50, (gb, gq, D), dev)
+        for _ in range(reps):
+            if case == "qjl_encode":
+                kvq.kvq_qjl_encode(kv[0], S, words, norms)
+            else:
+                kvq.kvq_decode_attention(q, k_words=words, k_norms=norms, sketch=S, v_codes=vc,
+                                         v_scales=vs)
+    else:
+        raise SystemExit(f"unknown profile case {case}")
+    torch.cuda.synchronize()
+    if kvq.kvq_device_error() != 0:
+        raise RuntimeError("device-side error recorded")
+    return 0
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["kvq", "reference"], default="kvq")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--ref-scale", type=float, default=2.0,
+                   help="size of the oracle's per-step sample in the reference arm")
+    p.add_argument("--cpu-scale", type=float, default=8.0,
+                   help="size of the oracle sample for the cpu_baseline key")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile-case", default=None,
+                   help="run one small single-kernel case (quantize, dequantize, decode_int8, "
+                        "qjl_encode, decode_qjl) for an ncu capture, then exit")
+    args = p.parse_args(argv)
+    if args.profile_case:
+        return run_profile_case(args.profile_case)
+    if args.warmup < 3 and args.impl == "kvq":
+        print("note: warm-up raised to 3 steps", file=sys.stderr)
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
