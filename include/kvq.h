@@ -182,6 +182,28 @@ kvq_status kvq_decode_attention(const kvq_decode_args* a, kvq_stream_t stream);
 size_t kvq_decode_workspace_bytes(const kvq_decode_args* a);
 
 /*
+ * kvq_decode_attention_noalloc -- kvq_decode_attention for callers that cannot
+ * allocate device memory and cannot lend a workspace (for example code inside a host
+ * engine that has already reserved all device memory through its own allocator, or a
+ * latency-critical path where an allocation, which may synchronise the device, is
+ * not allowed).  No passage on the pages corresponds to it: it is a deployment
+ * variant of the decode step above, with identical arguments and results, except
+ * that a->workspace and a->workspace_bytes are ignored.
+ *   Scratch: a fixed array of kvq_decode_noalloc_max_workspace_bytes() bytes (8 MiB)
+ *   inside the library's device image; every GPU that loads the library keeps it until
+ *   the process exits.  A request needing more than that (see
+ *   kvq_decode_workspace_bytes) returns KVQ_ERR_WORKSPACE and launches nothing.
+ *   The first call on each device looks up the array's device address (a host-side
+ *   runtime call, no allocation); make that first call before any stream capture.
+ *   All calls share the one array and nothing in it needs to start at zero (every
+ *   value read is written earlier in the same call), but calls whose kernels overlap
+ *   on the GPU (different streams, or several host threads) race on it: serialise
+ *   them.  It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+kvq_status kvq_decode_attention_noalloc(const kvq_decode_args* a, kvq_stream_t stream);
+size_t kvq_decode_noalloc_max_workspace_bytes(void);
+
+/*
  * kvq_device_error -- read and clear the library's device-side error word on the
  * current device (synchronous: it waits for the device).  Kernels that wait on
  * barriers give up after a bounded number of polls instead of hanging; when they do,

@@ -57,6 +57,10 @@ def _load():
     so.kvq_decode_workspace_bytes.argtypes = [ctypes.POINTER(DecodeArgs)]
     so.kvq_decode_workspace_bytes.restype = ctypes.c_size_t
     so.kvq_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+    so.kvq_decode_attention_noalloc.argtypes = [ctypes.POINTER(DecodeArgs), _P]
+    so.kvq_decode_attention_noalloc.restype = ctypes.c_int
+    so.kvq_decode_noalloc_max_workspace_bytes.argtypes = []
+    so.kvq_decode_noalloc_max_workspace_bytes.restype = ctypes.c_size_t
     for f in ("kvq_quantize_int8", "kvq_dequantize_int8", "kvq_int8_scores", "kvq_qjl_encode",
               "kvq_qjl_query_sketch", "kvq_decode_attention", "kvq_device_error"):
         getattr(so, f).restype = ctypes.c_int
@@ -221,6 +225,28 @@ def kvq_decode_attention(q, *, k_codes=None, k_scales=None, k_words=None, k_norm
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel()
     _check("kvq_decode_attention", lib.kvq_decode_attention(ctypes.byref(a), _stream(stream)))
+    return (out if want_out else None), (scores_out if want_scores else None)
+
+
+def kvq_decode_attention_noalloc(q, *, k_codes=None, k_scales=None, k_words=None, k_norms=None,
+                                 sketch=None, v_codes=None, v_scales=None, want_out=True,
+                                 want_scores=False, sm_scale=0.0, out=None, scores_out=None,
+                                 stream=None):
+    """The decode step using the library's built-in scratch instead of a workspace
+    (for callers that cannot allocate device memory); see include/kvq.h."""
+    _need_cuda(q, k_codes, k_scales, k_words, k_norms, sketch, v_codes, v_scales)
+    B, Hq, D = q.shape
+    ref = k_words if k_words is not None else k_codes
+    T = ref.shape[2]
+    if want_out and out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    if want_scores and scores_out is None:
+        scores_out = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    a = make_decode_args(q, k_codes=k_codes, k_scales=k_scales, k_words=k_words, k_norms=k_norms,
+                         sketch=sketch, v_codes=v_codes if want_out else None,
+                         v_scales=v_scales if want_out else None, out=out if want_out else None,
+                         scores_out=scores_out if want_scores else None, sm_scale=sm_scale)
+    _check("kvq_decode_attention_noalloc", lib.kvq_decode_attention_noalloc(ctypes.byref(a), _stream(stream)))
     return (out if want_out else None), (scores_out if want_scores else None)
 
 
