@@ -178,5 +178,9 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_decode_args* a, kvq_stream_t s
 
 KVQ_API kvq_status kvq_device_error(uint32_t* code) {
     if (!code) return KVQ_ERR_INVALID_ARG;
-    return from_cuda(kvq::read_and_clear_device_error(code)) == KVQ_OK ? KVQ_OK : KVQ_ERR_CUDA;
+    uint32_t a = 0, b = 0;
+    if (kvq::read_and_clear_device_error(&a) != cudaSuccess) return KVQ_ERR_CUDA;
+    if (kvq::read_and_clear_decode_error(&b) != cudaSuccess) return KVQ_ERR_CUDA;
+    *code = a ? a : b;
+    return KVQ_OK;
 }

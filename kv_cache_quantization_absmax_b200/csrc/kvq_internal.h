@@ -37,6 +37,7 @@ struct DecodePlan {
     size_t total_bytes;
 };
 DecodePlan plan_decode(const kvq_decode_args* a, int sm_count);
+cudaError_t read_and_clear_decode_error(uint32_t* code);
 cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& plan, cudaStream_t st);
 
 }  // namespace kvq

@@ -9,20 +9,30 @@
 // so it runs as tcgen05.mma (kind::f16, fp16 x fp16 -> fp32 accumulators in tensor
 // memory).  Persistent kernel, one CTA per SM, three warp roles:
 //   warp 0      TMA producer: S once (it stays in shared memory), then 128-key tiles
-//               into a 4-stage ring (two 64-column boxes per tile, 128-byte swizzle);
+//               into a 5-stage ring (two 64-column boxes per tile, 128-byte swizzle);
 //   warp 1      allocates 512 TMEM columns (two m-column accumulators), one thread
 //               issues 8 MMAs (K = 16 each) per tile and commits to an mbarrier;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator row (one key per thread),
-//               sign bits -> packed words (funnel shift of the sign bits), the key
-//               norm from the tile still in shared memory, 16-byte stores.
-// The epilogue of tile i overlaps the MMA of tile i+1 (double-buffered accumulator)
-// and the TMA loads of tiles i+1..i+4.
+//   warps 2..9  two epilogue warpgroups; warpgroup e takes the tiles i with i % 2 == e
+//               and always the accumulator e: tcgen05.ld of the accumulator row (one
+//               key per thread), sign bits -> packed words (four independent
+//               funnel-shift chains per word), the key norm from the tile still in
+//               shared memory, 16-byte stores.
+// The epilogue computes the tile's norms from shared memory as soon as the tile has
+// landed (while the MMA runs), returns the stage to the producer as soon as the MMA is
+// done, then packs the sign bits.  The epilogue of tile i overlaps the MMA of tile i+1
+// (double-buffered accumulator) and the TMA loads of tiles i+1..i+5 (five stages); each
+// warpgroup has two tiles' time for one.
 //
-// Norms: the sum of squares is formed in fp64 in index order (each square of an fp16
-// value is exact), square-rooted with IEEE rounding and converted to fp16 with one
-// rounding, so the stored norm is the correctly rounded fp16 of the fp64 norm.
-// Sign bits: bit = 1 iff the fp32 accumulator is >= 0 (-0 is canonicalised to +0); a
-// zero key (sum of squares 0) has all bits set, since every projection is exactly 0.
+// Norms: the stored norm is the fp16 rounding of the fp64 norm whose sum of squares
+// is accumulated in index order.  The fast path
+// sums the exact fp32 squares (fp16 squares fit in fp32) in a fixed tree, error
+// <= 8 u relative, takes the IEEE root, and checks that n (1 - 2^-19) and
+// n (1 + 2^-19) round to the same fp16 value; then that value is the rounding of the
+// exact norm and of the fp64 one.  Otherwise (about one key in 200) the thread redoes
+// the sum in fp64 in index order and rounds that.
+// Sign bits: bit = 1 iff the fp32 accumulator's sign bit is clear.  An exactly zero
+// projection of a nonzero key lies inside the tolerance band whatever its sign; a zero
+// key (sum of squares 0) gets all bits set, since every projection is exactly 0.
 //
 // Every mbarrier wait is bounded: after kMaxPolls polls the waiting role records an
 // error code in g_kvq_device_error, raises a CTA-wide abort flag and leaves its loop;
@@ -43,10 +53,10 @@ namespace {
 
 constexpr int kBM = 128;                 // keys per tile (MMA M)
 constexpr int kDim = 128;                // head_dim (MMA K in total)
-constexpr int kStages = 4;
+constexpr int kStages = 5;
 constexpr int kHalfBytes = kBM * 64 * 2; // one 64-column box of a key tile: 16 KB
 constexpr int kTileBytes = 2 * kHalfBytes;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;             // producer, MMA, 2 x 4 epilogue warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccStride = 256;     // TMEM columns between the two accumulators
 constexpr uint32_t kMaxPolls = 1u << 24;
@@ -173,6 +183,100 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int n) {
     return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
 }
 
+// Bit i of the result = 1 iff r[i] (an fp32 bit pattern) has its sign bit clear.
+// Four independent chains of eight funnel shifts keep the dependency chain short.
+__device__ __forceinline__ uint32_t pack_nonneg_bits(const uint32_t* r) {
+    uint32_t n0 = 0, n1 = 0, n2 = 0, n3 = 0;
+#pragma unroll
+    for (int j = 7; j >= 0; --j) {
+        n0 = __funnelshift_l(r[j], n0, 1);
+        n1 = __funnelshift_l(r[8 + j], n1, 1);
+        n2 = __funnelshift_l(r[16 + j], n2, 1);
+        n3 = __funnelshift_l(r[24 + j], n3, 1);
+    }
+    return ~(n0 | (n1 << 8) | (n2 << 16) | (n3 << 24));
+}
+
+// fp32 pair arithmetic (sm_100 packed instructions).
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+    float2 f;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
+    return f;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 16-byte chunk c (of 16) of key row `row` in a swizzled [128 x 128] fp16 tile.
+__device__ __forceinline__ uint4 tile_chunk(const uint8_t* st, int row, int c) {
+    const int kb = c >> 3, cc = c & 7;
+    return *reinterpret_cast<const uint4*>(st + kb * kHalfBytes + row * 128 + ((cc ^ (row & 7)) << 4));
+}
+
+// Sum of the 128 squares of a key row in fp32: each square is exact; 16 chunk sums of
+// 8 terms (pairs), then a 4-level tree and one final add: relative error <= 8 u.
+__device__ __forceinline__ float row_sum_squares(const uint8_t* st, int row) {
+    uint64_t s[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        const uint4 v = tile_chunk(st, row, c);
+        const __half2* h = reinterpret_cast<const __half2*>(&v);
+        uint64_t a = 0ull;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 f = __half22float2(h[i]);
+            const uint64_t pr = f2_pack(f.x, f.y);
+            a = i == 0 ? f2_mul(pr, pr) : f2_fma(pr, pr, a);
+        }
+        s[c] = a;
+    }
+#pragma unroll
+    for (int step = 8; step >= 1; step >>= 1)
+#pragma unroll
+        for (int i = 0; i < step; ++i) s[i] = f2_add(s[i], s[i + step]);
+    const float2 t = f2_unpack(s[0]);
+    return __fadd_rn(t.x, t.y);
+}
+
+// fp16 bits of the norm: the fp32 fast path when both ends of n (1 -+ 2^-19) round to
+// the same fp16 value, else the defining sequence (fp64 sum in index order, IEEE root,
+// one rounding to fp16).
+__device__ __forceinline__ uint16_t norm_f16_bits(const uint8_t* st, int row, float ss) {
+    const float n = __fsqrt_rn(ss);
+    const __half lo = __float2half_rn(__fmul_rn(n, 1.0f - 1.9073486328125e-06f));
+    const __half hi = __float2half_rn(__fmul_rn(n, 1.0f + 1.9073486328125e-06f));
+    if (__half_as_ushort(lo) == __half_as_ushort(hi)) return __half_as_ushort(lo);
+    double s64 = 0.0;
+#pragma unroll 1
+    for (int c = 0; c < 16; ++c) {
+        const uint4 v = tile_chunk(st, row, c);
+        const __half* h = reinterpret_cast<const __half*>(&v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const double d = (double)__half2float(h[i]);
+            s64 = __fma_rn(d, d, s64);
+        }
+    }
+    return __half_as_ushort(__double2half(__dsqrt_rn(s64)));
+}
+
 struct Smem {
     uint32_t s_base;      // S: two 64-column halves of m rows x 128 B
     uint32_t stage_base;  // key stages
@@ -293,63 +397,54 @@ qjl_mma_kernel(const __grid_constant__ CUtensorMap tmap_rows,
                 if (mbar_try_wait(done_bar, 0)) break;
         }
     } else {
-        // ---------------- epilogue (warps 2..5) ----------------
+        // ---------------- epilogue (warps 2..9) ----------------
+        const int eg = (warp - 2) >> 2;          // warpgroup: handles tiles it % 2 == eg
         const int quarter = warp & 3;            // TMEM lanes this warp may access
         const int row = quarter * 32 + lane;     // key row within the tile
         const int nw = m / 32;
         int it = 0;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x, ++it) {
+            if ((it & 1) != eg) continue;
             const int stage = it % kStages;
-            const int acc = it & 1;
+            const int acc = eg;
             const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+            const int64_t key = tile * kBM + row;
+            float ss = 0.0f;
+            uint16_t nbits = 0;
+            if constexpr (!kSketchOut) {
+                // The norm needs only the landed tile: compute it while the MMA runs.
+                const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+                const bool okf = mbar_wait(full_bar(stage), ph, abort_flag, kErrEpilogue);
+                if (!__all_sync(0xffffffffu, okf)) break;
+                const uint8_t* st = base_ptr + (stage_base - base) + (size_t)stage * kTileBytes;
+                ss = row_sum_squares(st, row);
+                nbits = norm_f16_bits(st, row, ss);
+            }
             const bool ok = mbar_wait(tfull_bar(acc), aph, abort_flag, kErrEpilogue);
             if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform: tcgen05.ld is .aligned
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)acc * kAccStride;
-            const int64_t key = tile * kBM + row;
             if constexpr (!kSketchOut) {
+                // The MMA has finished reading the stage: hand it back to the producer.
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty_bar(stage));
                 uint32_t wbits[8];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
+                for (int c = 0; c < 8; c += 2) {
                     if (c < nw) {
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(taddr + (uint32_t)c * 32u, r);
+                        uint32_t r0[32], r1[32];
+                        tmem_ld_32x32b_x32(taddr + (uint32_t)c * 32u, r0);
+                        if (c + 1 < nw) tmem_ld_32x32b_x32(taddr + (uint32_t)(c + 1) * 32u, r1);
                         tmem_ld_wait();
-                        uint32_t neg = 0;
-#pragma unroll
-                        for (int j = 31; j >= 0; --j) {
-                            const float v = __fadd_rn(__uint_as_float(r[j]), 0.0f);
-                            neg = __funnelshift_l(__float_as_uint(v), neg, 1);
-                        }
-                        wbits[c] = ~neg;
+                        wbits[c] = pack_nonneg_bits(r0);
+                        if (c + 1 < nw) wbits[c + 1] = pack_nonneg_bits(r1);
                     }
                 }
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(tempty_bar(acc));
-                // Norm from the key tile in shared memory: row `row`, 16-byte chunk c of a
-                // 128-byte swizzled row lives at chunk position c ^ (row & 7).
-                const uint8_t* st = base_ptr + (stage_base - base) + (size_t)stage * kTileBytes;
-                double ss = 0.0;
-#pragma unroll
-                for (int kb = 0; kb < 2; ++kb) {
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const uint4 v = *reinterpret_cast<const uint4*>(
-                            st + kb * kHalfBytes + row * 128 + ((c ^ (row & 7)) << 4));
-                        const __half2* h = reinterpret_cast<const __half2*>(&v);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float2 f = __half22float2(h[i]);
-                            ss = __fma_rn((double)f.x, (double)f.x, ss);
-                            ss = __fma_rn((double)f.y, (double)f.y, ss);
-                        }
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(stage));
                 if (key < n_rows) {
-                    if (ss == 0.0) {
+                    if (ss == 0.0f) {
 #pragma unroll
                         for (int c = 0; c < 8; ++c) wbits[c] = 0xFFFFFFFFu;
                     }
@@ -365,8 +460,7 @@ qjl_mma_kernel(const __grid_constant__ CUtensorMap tmap_rows,
                         for (int c = 0; c < 8; ++c)
                             if (c < nw) dst[c] = wbits[c];
                     }
-                    const __half hn = __double2half(__dsqrt_rn(ss));
-                    norms[key] = __half_as_ushort(hn);
+                    norms[key] = nbits;
                 }
             } else {
                 float* dst = sketch_out + key * m;

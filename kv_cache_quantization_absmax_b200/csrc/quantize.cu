@@ -12,11 +12,15 @@
 //
 // Bit-exactness of the codes.  The code is rint_even(fl32(x / s)) with s the stored
 // fp32 scale.  Instead of one IEEE division per element, the fast path multiplies by
-// r = fl32(1 / s) and rounds with the 1.5 * 2^23 addition (for |q| < 2^22 the sum's
+// a reciprocal r of s and rounds with the 1.5 * 2^23 addition (for |q| < 2^22 the sum's
 // ulp is 1, so round-to-nearest-even of the addition is rint_even(q), and the code is
-// the low byte of the sum's bit pattern).  |x r - x / s| <= 2^-23 |x / s| <= 1.6e-5 and
+// the low byte of the sum's bit pattern).  r comes from the hardware reciprocal
+// approximation refined by one Newton-Raphson step, r1 = r0 + r0 (1 - s r0) (two
+// FMAs): its relative error is the square of the approximation's plus one rounding,
+// below 2^-23.  Then |x r - x / s| <= 2^-22 |x / s| <= 3.1e-5 and
 // |fl32(x / s) - x / s| <= 3.9e-6 for |x / s| <= 127.00002, so whenever q = x r is
-// more than 2^-14 away from a half-integer both quotients round to the same integer.
+// more than 2^-14 (6.1e-5) away from a half-integer both quotients round to the same
+// integer.
 // A thread whose elements come closer than that (about one element in 8000), or
 // whose scale is subnormal (1 / s would overflow), recomputes its codes with the IEEE
 // division __fdiv_rn and __float2int_rn, plus the page's clamp.
@@ -53,6 +57,20 @@ __device__ __forceinline__ void unpack(const uint4& v, float* f, float) {
     f[3] = __uint_as_float(v.w);
 }
 
+// max |x| over one 16-byte vector (exact: max of magnitudes).
+__device__ __forceinline__ float vec_absmax(const uint4& v, __half) {
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+    __half2 m = __habs2(h[0]);
+    m = __hmax2(m, __habs2(h[1]));
+    m = __hmax2(m, __habs2(h[2]));
+    m = __hmax2(m, __habs2(h[3]));
+    return fmaxf(__low2float(m), __high2float(m));
+}
+__device__ __forceinline__ float vec_absmax(const uint4& v, float) {
+    return fmaxf(fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
+                 fmaxf(fabsf(__uint_as_float(v.z)), fabsf(__uint_as_float(v.w))));
+}
+
 // Low bytes of four words -> one word (byte i of the result = low byte of w_i).
 __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t w0, uint32_t w1, uint32_t w2,
                                                    uint32_t w3) {
@@ -62,10 +80,22 @@ __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t w0, uint32_t w1, uin
 }
 
 // Quantize N (multiple of 4) values sharing scale s into N/4 packed words.
+// 1/s for a normal s: hardware approximation + one Newton-Raphson step.
+__device__ __forceinline__ float reciprocal_nr(float s) {
+    float r0;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(s));
+    const float e = __fmaf_rn(-s, r0, 1.0f);
+    return __fmaf_rn(r0, e, r0);
+}
+
+// Reciprocal used by the fast path (0 for a zero scale, which makes every code 0).
+__device__ __forceinline__ float scale_reciprocal(float s) {
+    return (s >= kFltMinNormal) ? reciprocal_nr(s) : 0.0f;
+}
+
 template <int N>
-__device__ __forceinline__ void quantize_values(const float* f, float s, uint32_t* out) {
+__device__ __forceinline__ void quantize_values(const float* f, float s, float rinv, uint32_t* out) {
     const bool s_zero = (s == 0.0f);
-    const float rinv = s_zero ? 0.0f : __fdiv_rn(1.0f, s);
     const bool fast_ok = s_zero || (s >= kFltMinNormal);
     uint32_t y[N];
     float tmax = 0.0f;
@@ -129,22 +159,22 @@ quantize_rows_warp(const T* __restrict__ x, int64_t n_rows, int8_t* __restrict__
 #pragma unroll
         for (int r = 0; r < RPT; ++r) {
             const int64_t row = base + r * GROUPS + group;
-            float f[VPT * PV];
-#pragma unroll
-            for (int i = 0; i < VPT; ++i) unpack(v[r][i], f + i * PV, T());
             float a = 0.0f;
 #pragma unroll
-            for (int e = 0; e < VPT * PV; ++e) a = fmaxf(a, fabsf(f[e]));
+            for (int i = 0; i < VPT; ++i) a = fmaxf(a, vec_absmax(v[r][i], T()));
 #pragma unroll
             for (int off = TPR / 2; off > 0; off >>= 1)
                 a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
             const float s = __fdiv_rn(a, 127.0f);
+            const float rinv = scale_reciprocal(s);
             if (row < n_rows) {
                 if (lane == 0) scales[row] = s;
 #pragma unroll
                 for (int i = 0; i < VPT; ++i) {
+                    float f[PV];
+                    unpack(v[r][i], f, T());
                     uint32_t w[PV / 4];
-                    quantize_values<PV>(f + i * PV, s, w);
+                    quantize_values<PV>(f, s, rinv, w);
                     store_codes<PV>(codes + row * D + (int64_t)(i * TPR + lane) * PV, w);
                 }
             }
@@ -166,12 +196,9 @@ quantize_rows_cta(const T* __restrict__ x, int64_t n_rows, int8_t* __restrict__ 
         uint4 v[VPT];
 #pragma unroll
         for (int i = 0; i < VPT; ++i) v[i] = __ldcs(src + i * 256 + tid);
-        float f[VPT * PV];
-#pragma unroll
-        for (int i = 0; i < VPT; ++i) unpack(v[i], f + i * PV, T());
         float a = 0.0f;
 #pragma unroll
-        for (int e = 0; e < VPT * PV; ++e) a = fmaxf(a, fabsf(f[e]));
+        for (int i = 0; i < VPT; ++i) a = fmaxf(a, vec_absmax(v[i], T()));
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
         if ((tid & 31) == 0) red[tid >> 5] = a;
@@ -180,11 +207,14 @@ quantize_rows_cta(const T* __restrict__ x, int64_t n_rows, int8_t* __restrict__ 
 #pragma unroll
         for (int w = 1; w < 8; ++w) a = fmaxf(a, red[w]);
         const float s = __fdiv_rn(a, 127.0f);
+        const float rinv = scale_reciprocal(s);
         if (tid == 0) scales[row] = s;
 #pragma unroll
         for (int i = 0; i < VPT; ++i) {
+            float f[PV];
+            unpack(v[i], f, T());
             uint32_t w[PV / 4];
-            quantize_values<PV>(f + i * PV, s, w);
+            quantize_values<PV>(f, s, rinv, w);
             store_codes<PV>(codes + row * D + (int64_t)(i * 256 + tid) * PV, w);
         }
         __syncthreads();  // red[] is reused by the next row
@@ -214,12 +244,13 @@ quantize_rows_generic(const T* __restrict__ x, int64_t n_rows, int64_t d,
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
         const float s = __fdiv_rn(a, 127.0f);
+        const float rinv = scale_reciprocal(s);
         if (lane == 0) scales[row] = s;
         for (int64_t i = lane; i < nvec; i += 32) {
             float f[PV];
             unpack(src[i], f, T());
             uint32_t w[PV / 4];
-            quantize_values<PV>(f, s, w);
+            quantize_values<PV>(f, s, rinv, w);
             store_codes<PV>(codes + row * d + i * PV, w);
         }
     }
@@ -366,14 +397,16 @@ cudaError_t run_generic(const void* x, int64_t n, int64_t d, int8_t* c, float* s
 
 cudaError_t launch_quantize_int8(const void* x, bool f16, int64_t n, int64_t d, int8_t* c,
                                  float* s, cudaStream_t st) {
+    // Row mappings: each lane holds up to four 16-byte vectors of its row (fewer lanes
+    // per row amortise the per-row reduction, scale and reciprocal over more elements).
     if (f16) {
         switch (d) {  // 8 halves per 16-byte vector
             case 16: return run_warp<__half, 2, 1, 4>(x, n, c, s, st);
-            case 32: return run_warp<__half, 4, 1, 4>(x, n, c, s, st);
-            case 64: return run_warp<__half, 8, 1, 4>(x, n, c, s, st);
-            case 128: return run_warp<__half, 16, 1, 4>(x, n, c, s, st);
-            case 256: return run_warp<__half, 32, 1, 4>(x, n, c, s, st);
-            case 512: return run_warp<__half, 32, 2, 2>(x, n, c, s, st);
+            case 32: return run_warp<__half, 2, 2, 2>(x, n, c, s, st);
+            case 64: return run_warp<__half, 2, 4, 1>(x, n, c, s, st);
+            case 128: return run_warp<__half, 4, 4, 1>(x, n, c, s, st);
+            case 256: return run_warp<__half, 8, 4, 1>(x, n, c, s, st);
+            case 512: return run_warp<__half, 16, 4, 1>(x, n, c, s, st);
             case 1024: return run_warp<__half, 32, 4, 1>(x, n, c, s, st);
             case 2048: return run_cta<__half, 1>(x, n, c, s, st);
             case 4096: return run_cta<__half, 2>(x, n, c, s, st);
@@ -382,11 +415,11 @@ cudaError_t launch_quantize_int8(const void* x, bool f16, int64_t n, int64_t d, 
         }
     }
     switch (d) {  // 4 floats per 16-byte vector
-        case 16: return run_warp<float, 4, 1, 4>(x, n, c, s, st);
-        case 32: return run_warp<float, 8, 1, 4>(x, n, c, s, st);
-        case 64: return run_warp<float, 16, 1, 4>(x, n, c, s, st);
-        case 128: return run_warp<float, 16, 2, 2>(x, n, c, s, st);
-        case 256: return run_warp<float, 32, 2, 2>(x, n, c, s, st);
+        case 16: return run_warp<float, 2, 2, 2>(x, n, c, s, st);
+        case 32: return run_warp<float, 2, 4, 1>(x, n, c, s, st);
+        case 64: return run_warp<float, 4, 4, 1>(x, n, c, s, st);
+        case 128: return run_warp<float, 8, 4, 1>(x, n, c, s, st);
+        case 256: return run_warp<float, 16, 4, 1>(x, n, c, s, st);
         case 512: return run_warp<float, 32, 4, 1>(x, n, c, s, st);
         case 1024: return run_warp<float, 32, 8, 1>(x, n, c, s, st);
         case 2048: return run_cta<float, 2>(x, n, c, s, st);

@@ -125,3 +125,28 @@ def gaussian_queries_device(seed: int, shape, device):
     g = torch.Generator(device=device)
     g.manual_seed(seed)
     return torch.randn(tuple(shape), generator=g, device=device).to(torch.float16)
+
+
+def sweep_matrix_device(total: int, d: int, dtype, sweep_index: int, device):
+    """The throughput-sweep recipe drawn on the device (for the 1e9-element points): the
+    scaled columns and the fp32 query come from numpy (seed 2000 + sweep index), the
+    matrix from torch's seeded generator."""
+    import torch
+
+    rng = np.random.default_rng(2000 + sweep_index)
+    n = sweep_rows(total, d)
+    k = max(1, int(round(0.01 * d)))
+    cols = np.sort(rng.choice(d, k, replace=False))
+    q = rng.standard_normal((d,), dtype=np.float32)
+    g = torch.Generator(device=device)
+    g.manual_seed(2000 + sweep_index)
+    tdt = torch.float16 if dtype == np.float16 else torch.float32
+    x = torch.empty((n, d), dtype=tdt, device=device)
+    factor = torch.ones(d, dtype=torch.float32, device=device)
+    factor[torch.from_numpy(cols).to(device)] = 20.0
+    step = max(1, (1 << 28) // d)
+    for r0 in range(0, n, step):
+        r1 = min(n, r0 + step)
+        chunk = torch.randn((r1 - r0, d), generator=g, device=device, dtype=torch.float32)
+        x[r0:r1].copy_(chunk.mul_(factor))
+    return x, q, cols
