@@ -7,7 +7,18 @@
 namespace kvq {
 namespace dev {
 
-constexpr uint32_t kMaxPolls = 1u << 24;  // bound on every mbarrier wait
+// Every mbarrier wait gives up after this much wall time (nanoseconds of the global
+// timer); a healthy wait lasts microseconds.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// Suspend-time hint of each try_wait: the thread sleeps until the phase completes or
+// this many nanoseconds pass, instead of spinning and taking issue slots.
+constexpr uint32_t kSuspendHintNs = 1000000u;
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -30,10 +41,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -41,18 +52,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // raising *abort_flag) or as soon as another thread of the CTA has raised *abort_flag.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned int* err_word, unsigned int err) {
-    for (uint32_t i = 0; i < kMaxPolls; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 1023u) == 1023u && *abort_flag) return false;
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kWaitLimitNs) break;
     }
     atomicCAS(err_word, 0u, err);
     *abort_flag = 1;
     return false;
 }
-// Waits for a phase with a bound and no side effects (used to drain in-flight copies).
+// Waits for a phase with the same bound and no side effects (used to drain in-flight
+// copies before a CTA exits).
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kMaxPolls; ++i)
-        if (mbar_try_wait(bar, parity)) return;
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > kWaitLimitNs) return;
 }
 
 // Untiled bulk copy global -> shared; completes `bytes` of transaction on `bar`.

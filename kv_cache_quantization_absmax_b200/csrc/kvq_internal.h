@@ -30,9 +30,10 @@ cudaError_t read_and_clear_device_error(uint32_t* code);
 // decode.cu
 struct DecodePlan {
     int64_t units;        // B * Hkv
-    int splits;           // token chunks per unit
-    int64_t chunk;        // tokens per chunk
-    size_t partial_bytes; // per-split softmax states
+    int ctas;             // CTAs of the partial kernel (one contiguous token range each)
+    int64_t W;            // tokens per CTA range
+    int maxj;             // unit segments one range can touch
+    size_t partial_bytes; // per-segment softmax states
     size_t sketch_bytes;  // query sketches (QJL)
     size_t total_bytes;
 };

@@ -26,7 +26,7 @@
 // Norms: the stored norm is the fp16 rounding of the fp64 norm whose sum of squares
 // is accumulated in index order.  The fast path
 // sums the exact fp32 squares (fp16 squares fit in fp32) in a fixed tree, error
-// <= 8 u relative, takes the IEEE root, and checks that n (1 - 2^-19) and
+// <= 12 u relative, takes the IEEE root, and checks that n (1 - 2^-19) and
 // n (1 + 2^-19) round to the same fp16 value; then that value is the rounding of the
 // exact norm and of the fp64 one.  Otherwise (about one key in 200) the thread redoes
 // the sum in fp64 in index order and rounds that.
@@ -34,7 +34,7 @@
 // projection of a nonzero key lies inside the tolerance band whatever its sign; a zero
 // key (sum of squares 0) gets all bits set, since every projection is exactly 0.
 //
-// Every mbarrier wait is bounded: after kMaxPolls polls the waiting role records an
+// Every mbarrier wait is bounded: after 2 s of global time the waiting role records an
 // error code in g_kvq_device_error, raises a CTA-wide abort flag and leaves its loop;
 // the producer then waits (bounded) for its own TMA loads still in flight, the MMA
 // thread for its own MMAs, and TMEM is freed before the CTA exits.
@@ -43,6 +43,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "kvq_device.cuh"
 #include "kvq_internal.h"
 
 namespace kvq {
@@ -59,7 +60,6 @@ constexpr int kTileBytes = 2 * kHalfBytes;
 constexpr int kThreads = 320;             // producer, MMA, 2 x 4 epilogue warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccStride = 256;     // TMEM columns between the two accumulators
-constexpr uint32_t kMaxPolls = 1u << 24;
 
 enum : unsigned int {
     kErrProducer = 0x101,
@@ -71,41 +71,16 @@ enum : unsigned int {
 // --------------------------------------------------------------------------------
 // PTX wrappers
 // --------------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait.  Returns false (after recording `err`) on timeout or when another
-// role has already aborted the CTA.
+using dev::mbar_arrive;
+using dev::mbar_arrive_expect_tx;
+using dev::mbar_drain;
+using dev::mbar_init;
+using dev::mbar_try_wait;
+using dev::smem_u32;
+
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned int err) {
-    for (uint32_t i = 0; i < kMaxPolls; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 1023u) == 1023u && *abort_flag) return false;
-    }
-    atomicCAS(&g_kvq_device_error, 0u, err);
-    *abort_flag = 1;
-    return false;
+    return dev::mbar_wait(bar, parity, abort_flag, &g_kvq_device_error, err);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
@@ -197,62 +172,41 @@ __device__ __forceinline__ uint32_t pack_nonneg_bits(const uint32_t* r) {
     return ~(n0 | (n1 << 8) | (n2 << 16) | (n3 << 24));
 }
 
-// fp32 pair arithmetic (sm_100 packed instructions).
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
-    float2 f;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
-    return f;
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
 // 16-byte chunk c (of 16) of key row `row` in a swizzled [128 x 128] fp16 tile.
 __device__ __forceinline__ uint4 tile_chunk(const uint8_t* st, int row, int c) {
     const int kb = c >> 3, cc = c & 7;
     return *reinterpret_cast<const uint4*>(st + kb * kHalfBytes + row * 128 + ((cc ^ (row & 7)) << 4));
 }
 
+// acc + h * h with an fp16 h: the product is exact in fp32 (11-bit significands) and the
+// sum is rounded once (mixed-precision FMA, no conversion instruction).
+__device__ __forceinline__ float fma_sq_f16(uint16_t h, float acc) {
+    float d;
+    asm("fma.rn.f32.f16 %0, %1, %1, %2;" : "=f"(d) : "h"(h), "f"(acc));
+    return d;
+}
+
 // Sum of the 128 squares of a key row in fp32: each square is exact; 16 chunk sums of
-// 8 terms (pairs), then a 4-level tree and one final add: relative error <= 8 u.
+// 8 terms (8 sequential FMAs), then a 4-level tree: relative error <= 12 u.
 __device__ __forceinline__ float row_sum_squares(const uint8_t* st, int row) {
-    uint64_t s[16];
+    float s[16];
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
         const uint4 v = tile_chunk(st, row, c);
-        const __half2* h = reinterpret_cast<const __half2*>(&v);
-        uint64_t a = 0ull;
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        float a = 0.0f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float2 f = __half22float2(h[i]);
-            const uint64_t pr = f2_pack(f.x, f.y);
-            a = i == 0 ? f2_mul(pr, pr) : f2_fma(pr, pr, a);
+            a = fma_sq_f16((uint16_t)(w[i] & 0xFFFFu), a);
+            a = fma_sq_f16((uint16_t)(w[i] >> 16), a);
         }
         s[c] = a;
     }
 #pragma unroll
     for (int step = 8; step >= 1; step >>= 1)
 #pragma unroll
-        for (int i = 0; i < step; ++i) s[i] = f2_add(s[i], s[i + step]);
-    const float2 t = f2_unpack(s[0]);
-    return __fadd_rn(t.x, t.y);
+        for (int i = 0; i < step; ++i) s[i] = __fadd_rn(s[i], s[i + step]);
+    return s[0];
 }
 
 // fp16 bits of the norm: the fp32 fast path when both ends of n (1 -+ 2^-19) round to
@@ -324,8 +278,7 @@ qjl_mma_kernel(const __grid_constant__ CUtensorMap tmap_rows,
         }
         mbar_init(s_bar, 1);
         mbar_init(done_bar, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        dev::mbar_init_fence();
     }
     if (warp == 1) tmem_alloc(smem_u32(&tmem_slot), kTmemCols);
     tc_fence_before();
@@ -357,12 +310,9 @@ qjl_mma_kernel(const __grid_constant__ CUtensorMap tmap_rows,
                 issued_parity[stage] = ph;
             }
             // Never leave the CTA with a TMA write in flight.
-            mbar_wait(s_bar, 0, abort_flag, kErrDrain);
+            mbar_drain(s_bar, 0);
             for (int s = 0; s < kStages; ++s)
-                if (issued[s]) {
-                    for (uint32_t i = 0; i < kMaxPolls; ++i)
-                        if (mbar_try_wait(full_bar(s), issued_parity[s])) break;
-                }
+                if (issued[s]) mbar_drain(full_bar(s), issued_parity[s]);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -393,8 +343,7 @@ qjl_mma_kernel(const __grid_constant__ CUtensorMap tmap_rows,
             }
             // Wait for every MMA this thread issued before TMEM can be released.
             tc_commit(done_bar);
-            for (uint32_t i = 0; i < kMaxPolls; ++i)
-                if (mbar_try_wait(done_bar, 0)) break;
+            mbar_drain(done_bar, 0);
         }
     } else {
         // ---------------- epilogue (warps 2..9) ----------------

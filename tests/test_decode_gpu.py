@@ -38,7 +38,8 @@ def _cuda(*arrs):
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,T", [(1, 1, 1, 1), (1, 4, 4, 5), (2, 8, 2, 33), (1, 8, 1, 1000),
-                                        (2, 16, 4, 4097), (1, 8, 8, 300), (1, 16, 2, 2500)])
+                                        (2, 16, 4, 4097), (1, 8, 8, 300), (1, 16, 2, 2500),
+                                        (16, 16, 8, 3), (4, 8, 8, 100), (3, 24, 3, 70)])
 def test_decode_int8_parity(kvq, B, Hq, Hkv, T):
     q, kc, ks, vc, vs = _int8_cache(10 + T, B, Hkv, T, Hq)
     ref = oracle.decode_attention(q, k_codes=kc, k_scales=ks, v_codes=vc, v_scales=vs,
@@ -81,7 +82,8 @@ def _qjl_cache(seed, B, Hkv, T, Hq, m=256):
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,T,m", [(1, 1, 1, 1, 256), (1, 4, 1, 7, 256), (2, 8, 2, 1500, 256),
-                                          (1, 32, 8, 2049, 256), (1, 4, 4, 700, 128), (1, 2, 1, 333, 32)])
+                                          (1, 32, 8, 2049, 256), (1, 4, 4, 700, 128), (1, 2, 1, 333, 32),
+                                          (16, 32, 8, 3, 256), (4, 8, 4, 100, 256)])
 def test_decode_qjl_parity(kvq, B, Hq, Hkv, T, m):
     q, S, w, n, vc, vs = _qjl_cache(100 + T, B, Hkv, T, Hq, m)
     ref = oracle.decode_attention(q, k_words=w, k_norms=n, S=S, v_codes=vc, v_scales=vs,
