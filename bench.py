@@ -511,14 +511,19 @@ def run_gpu(args):
 
 
 def load_traffic(kernel_row: str):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if its
-    recorded source hash matches the current kernels (else null)."""
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if the
+    kernel's source file is unchanged since the counters were taken (else null)."""
+    import hashlib
+
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             tr = json.load(f)
-        from kv_cache_quantization_absmax_b200 import build as kb
-        if tr.get("source_hash") != kb.source_hash():
+        h = hashlib.sha256()
+        for rel in tr["kernel_sources"]:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
+        if tr.get("sources_hash") != h.hexdigest():
             return None
         v = tr.get("rows", {}).get(kernel_row)
         return None if v is None else float(v)

@@ -471,12 +471,12 @@ decode_int8_kernel(const DecodeParams p) {
 //    partial sums in packed fp32x2 registers, so each fp32x2 FMA consumes a weight pair
 //    and a code pair as they come.
 // -----------------------------------------------------------------------------------
-template <int G>
-__global__ void __launch_bounds__(512, 1)
+template <int G, int THREADS>
+__global__ void __launch_bounds__(THREADS, 1)
 decode_qjl_kernel(const DecodeParams p) {
     extern __shared__ float4 dsmem4[];
     float* dsmem = reinterpret_cast<float*>(dsmem4);
-    constexpr int THREADS = 512;
+    static_assert(THREADS >= 512 && THREADS % 32 == 0, "the table build uses 512 threads");
     constexpr int WARPS = THREADS / 32;
     constexpr int TOK_PER_STEP = WARPS * 32;
     constexpr int HALF_FLOATS = 256 * 16 * 4;        // one table half: 64 KB
@@ -511,45 +511,44 @@ decode_qjl_kernel(const DecodeParams p) {
         const int64_t b = sg.u / p.Hkv;
         const int kvh = (int)(sg.u % p.Hkv);
         __syncthreads();  // the previous segment's merge no longer reads red[]
-    // ---- byte tables ----
-    {
-        const int pos = threadIdx.x & 31;
-        const int c = threadIdx.x >> 5;               // high nibble of the byte value
-        float v[G][8];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float* src = p.sketch_v + (b * p.Hq + (int64_t)kvh * G + g) * p.m + pos * 8;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) v[g][k] = pos < npos ? __ldg(src + k) : 0.0f;
-        }
-        float val[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            float s = 0.0f;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) s -= v[g][k];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) s += ((c >> k) & 1) ? v[g][4 + k] : -v[g][4 + k];
-            val[g] = s;
-        }
-        float* base = lut + (pos >> 4) * HALF_FLOATS + (c * 16 * 16 + (pos & 15)) * 4;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int gray = i ^ (i >> 1);
-            if (i > 0) {
-                const int k = __ffs(i) - 1;               // the bit that flips at step i
-                const bool on = (gray >> k) & 1;
-#pragma unroll
-                for (int g = 0; g < G; ++g) val[g] += on ? 2.0f * v[g][k] : -2.0f * v[g][k];
+        // ---- byte tables ----
+        if (threadIdx.x < 512) {
+            const int pos = threadIdx.x & 31;
+            const int c = threadIdx.x >> 5;               // high nibble of the byte value
+            float v[G][8];
+    #pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float* src = p.sketch_v + (b * p.Hq + (int64_t)kvh * G + g) * p.m + pos * 8;
+    #pragma unroll
+                for (int k = 0; k < 8; ++k) v[g][k] = pos < npos ? __ldg(src + k) : 0.0f;
             }
-            float* e = base + gray * 16 * 4;              // byte 16c + gray: +gray*256 B
-            *reinterpret_cast<float4*>(e) = make_float4(val[0], G > 1 ? val[G > 1 ? 1 : 0] : 0.0f,
-                                                        G > 2 ? val[G > 2 ? 2 : 0] : 0.0f,
-                                                        G > 3 ? val[G > 3 ? 3 : 0] : 0.0f);
+            float val[G];
+    #pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float s = 0.0f;
+    #pragma unroll
+                for (int k = 0; k < 4; ++k) s -= v[g][k];
+    #pragma unroll
+                for (int k = 0; k < 4; ++k) s += ((c >> k) & 1) ? v[g][4 + k] : -v[g][4 + k];
+                val[g] = s;
+            }
+            float* base = lut + (pos >> 4) * HALF_FLOATS + (c * 16 * 16 + (pos & 15)) * 4;
+    #pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int gray = i ^ (i >> 1);
+                if (i > 0) {
+                    const int k = __ffs(i) - 1;               // the bit that flips at step i
+                    const bool on = (gray >> k) & 1;
+    #pragma unroll
+                    for (int g = 0; g < G; ++g) val[g] += on ? 2.0f * v[g][k] : -2.0f * v[g][k];
+                }
+                float* e = base + gray * 16 * 4;              // byte 16c + gray: +gray*256 B
+                *reinterpret_cast<float4*>(e) = make_float4(val[0], G > 1 ? val[G > 1 ? 1 : 0] : 0.0f,
+                                                            G > 2 ? val[G > 2 ? 2 : 0] : 0.0f,
+                                                            G > 3 ? val[G > 3 ? 3 : 0] : 0.0f);
+            }
         }
-    }
-    __syncthreads();
-
+        __syncthreads();
 
         float mrun[G], lsum[G];
         uint64_t acc[G][4];                               // (even, odd) token partial sums, 4 dims
@@ -753,11 +752,13 @@ template <int G>
 size_t int8_smem() {
     return (size_t)kI8Stages * kI8StageBytes + (size_t)kI8Consumers * G * (2 + kD) * sizeof(float);
 }
-template <int G>
+constexpr int kQjlThreads = 512;
+
+template <int G, int THREADS = kQjlThreads>
 size_t qjl_smem() {
     const size_t tables = (size_t)2 * 256 * 16 * 4 * sizeof(float);   // entries padded to 16 B
-    const size_t wbuf = (size_t)16 * 32 * G * sizeof(float);
-    const size_t red = (size_t)16 * G * (2 + kD) * sizeof(float);
+    const size_t wbuf = (size_t)(THREADS / 32) * 32 * G * sizeof(float);
+    const size_t red = (size_t)(THREADS / 32) * G * (2 + kD) * sizeof(float);
     const size_t a = tables + wbuf;
     return a > red ? a : red;
 }
@@ -774,11 +775,11 @@ cudaError_t run_int8(const DecodeParams& p, int ctas, cudaStream_t st) {
 
 template <int G>
 cudaError_t run_qjl(const DecodeParams& p, int ctas, cudaStream_t st) {
-    auto kern = decode_qjl_kernel<G>;
+    auto kern = decode_qjl_kernel<G, kQjlThreads>;
     const size_t smem = qjl_smem<G>();
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<ctas, 512, smem, st>>>(p);
+    kern<<<ctas, kQjlThreads, smem, st>>>(p);
     return cudaGetLastError();
 }
 
