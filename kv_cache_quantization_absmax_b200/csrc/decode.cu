@@ -163,18 +163,24 @@ __device__ __forceinline__ void merge_warps_and_store(const float* red, const De
 }
 
 // -----------------------------------------------------------------------------------
-// INT8 keys.  The CTA's range streams through a 4-stage shared-memory ring of stages of
-// up to 64 tokens of one unit (K rows, V rows, and the scales when they are 16-byte
+// INT8 keys.  The CTA's range streams through a shared-memory ring of stages of up to
+// 64 or 128 tokens of one unit (K rows, V rows, and the scales when they are 16-byte
 // aligned) filled by bulk asynchronous copies that one producer thread issues; eight
 // consumer warps read the stage from shared memory.  8 lanes share a token (lane `sub`
-// owns dims 16 sub .. 16 sub + 15 of K and V); each 8-lane group takes 2 consecutive
+// owns dims 16 sub .. 16 sub + 15 of K and V); each 8-lane group takes U consecutive
 // tokens of a stage and keeps its own online-softmax state; at the end of each unit
 // segment the states are merged across groups (shuffles) and warps (shared memory)
 // into the segment's slot while the producer already streams the next segment.
 // -----------------------------------------------------------------------------------
-constexpr int kI8StageTok = 64;
-constexpr int kI8Stages = 4;
-constexpr int kI8StageBytes = 2 * kI8StageTok * kD + 2 * kI8StageTok * 4;  // K rows, V rows, K scales, V scales
+// Ring geometry per group size G (measured on B200: for G = 1, two 128-token stages
+// with three CTAs per SM beat four 64-token stages, the per-stage bookkeeping being
+// spread over 4 tokens per lane group instead of 2).
+template <int G>
+struct I8Ring {
+    static constexpr int tok = G == 1 ? 128 : 64;             // tokens per stage
+    static constexpr int stages = G == 1 ? 2 : 4;
+    static constexpr int bytes = 2 * tok * kD + 2 * tok * 4;  // K rows, V rows, K scales, V scales
+};
 constexpr int kI8Consumers = 8;                          // consumer warps; warp 8 produces
 constexpr int kI8Threads = 32 * (kI8Consumers + 1);
 
@@ -189,6 +195,10 @@ __host__ __device__ constexpr int int8_ctas_per_sm(int G) { return G == 1 ? 3 : 
 template <int G>
 __global__ void __launch_bounds__(kI8Threads, int8_ctas_per_sm(G))
 decode_int8_kernel(const DecodeParams p) {
+    constexpr int kI8StageTok = I8Ring<G>::tok;
+    constexpr int kI8Stages = I8Ring<G>::stages;
+    constexpr int kI8StageBytes = I8Ring<G>::bytes;
+    static_assert(kI8StageTok % (4 * kI8Consumers) == 0, "each 8-lane group takes whole tokens");
     extern __shared__ __align__(128) unsigned char smem_raw[];
     __shared__ uint64_t bars[2 * kI8Stages];
     __shared__ int abort_storage;
@@ -214,12 +224,14 @@ decode_int8_kernel(const DecodeParams p) {
         dev::mbar_init_fence();
     }
     __syncthreads();
+    dev::griddep_launch_dependents();  // the combine kernel may be scheduled (it waits)
 
     if (warp == kI8Consumers) {
         // ---------------- producer ----------------
         if (lane == 0) {
-            bool issued[kI8Stages] = {false, false, false, false};
-            uint32_t ph_issued[kI8Stages] = {0, 0, 0, 0};
+            bool issued[kI8Stages];
+            uint32_t ph_issued[kI8Stages];
+            for (int s = 0; s < kI8Stages; ++s) issued[s] = false, ph_issued[s] = 0;
             int i = 0;
             bool run = true;
             for (int jj = 0; run && jj < nseg; ++jj) {
@@ -502,6 +514,7 @@ decode_qjl_kernel(const DecodeParams p) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) sel[e] = 0x6504u | ((uint32_t)((e ^ x) & 3) << 4);
     const uint32_t lut_s = (uint32_t)__cvta_generic_to_shared(lut);
+    dev::griddep_launch_dependents();  // the combine kernel may be scheduled (it waits)
     float* mybuf = wbuf + warp * 32 * G;
     const uint64_t magic = pack2(-kCodeMagic, -kCodeMagic);
 
@@ -721,6 +734,9 @@ decode_qjl_kernel(const DecodeParams p) {
 __global__ void __launch_bounds__(kD)
 decode_combine_kernel(const float* __restrict__ ws, int64_t T, int64_t W, int maxj, int Hq, int Hkv,
                       float* __restrict__ out) {
+    // Launched as a programmatic dependent of the decode kernel: nothing is read before
+    // that kernel has completed and its partial states are visible.
+    dev::griddep_wait();
     const int64_t bh = blockIdx.x;
     const int64_t b = bh / Hq;
     const int h = (int)(bh % Hq);
@@ -750,7 +766,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 template <int G>
 size_t int8_smem() {
-    return (size_t)kI8Stages * kI8StageBytes + (size_t)kI8Consumers * G * (2 + kD) * sizeof(float);
+    return (size_t)I8Ring<G>::stages * I8Ring<G>::bytes + (size_t)kI8Consumers * G * (2 + kD) * sizeof(float);
 }
 constexpr int kQjlThreads = 512;
 
@@ -870,9 +886,21 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
     }
     e = run_partial(qjl, G, p, pl.ctas, st);
     if (e != cudaSuccess || !a->out) return e;
-    decode_combine_kernel<<<(unsigned)(a->batch * a->n_q_heads), kD, 0, st>>>(
-        p.ws, p.T, p.W, p.maxj, p.Hq, p.Hkv, a->out);
-    return cudaGetLastError();
+    // The combine kernel is scheduled as the decode kernel's CTAs retire (programmatic
+    // dependent launch) instead of after it has fully drained, hiding its launch latency;
+    // it waits for the decode kernel before reading the partial states.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a->batch * a->n_q_heads));
+    cfg.blockDim = dim3(kD);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const float* ws_c = p.ws;
+    return cudaLaunchKernelEx(&cfg, decode_combine_kernel, ws_c, p.T, p.W, p.maxj, p.Hq, p.Hkv, a->out);
 }
 
 }  // namespace kvq

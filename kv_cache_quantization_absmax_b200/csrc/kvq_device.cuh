@@ -71,6 +71,16 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
         if (global_ns() - t0 > kWaitLimitNs) return;
 }
 
+// Programmatic dependent launch (sm_90+).  A kernel launched with programmatic stream
+// serialisation may be scheduled before the previous kernel of its stream has ended;
+// launch_dependents (in the earlier kernel) allows that, and wait (in the later kernel)
+// blocks until every earlier kernel it depends on has completed and its memory
+// operations are visible.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Untiled bulk copy global -> shared; completes `bytes` of transaction on `bar`.
 // dst, src and bytes must be multiples of 16.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {

@@ -163,3 +163,51 @@ def test_decode_rejects_bad_workspace(kvq):
     a.workspace_bytes = need
     assert kvq.lib.kvq_decode_attention(ctypes.byref(a), None) == kvq.KVQ_OK
     torch.cuda.synchronize()
+
+
+def test_decode_workspace_reused_across_calls_and_shapes(kvq):
+    """One workspace serves a sequence of calls of different shapes and key formats
+    (units split over several CTAs, units inside one range), twice over: every result
+    matches the oracle, whatever an earlier call left in the workspace."""
+    cases = []
+    for (B, Hq, Hkv, T) in [(1, 8, 1, 1000), (16, 16, 8, 3), (2, 16, 4, 4097)]:
+        q, kc, ks, vc, vs = _int8_cache(200 + T, B, Hkv, T, Hq)
+        ref = oracle.decode_attention(q, k_codes=kc, k_scales=ks, v_codes=vc, v_scales=vs)["out"]
+        qg, kcg, ksg, vcg, vsg = _cuda(q, kc, ks, vc, vs)
+        cases.append((ref, dict(q=qg, k_codes=kcg, k_scales=ksg, v_codes=vcg, v_scales=vsg)))
+    q, S, w, n, vc, vs = _qjl_cache(300, 4, 8, 100, 8)
+    ref = oracle.decode_attention(q, k_words=w, k_norms=n, S=S, v_codes=vc, v_scales=vs)["out"]
+    qg, Sg, wg, ng, vcg, vsg = _cuda(q, S, w.view(np.int32), n, vc, vs)
+    cases.append((ref, dict(q=qg, k_words=wg, k_norms=ng, sketch=Sg, v_codes=vcg, v_scales=vsg)))
+    need = 0
+    for _, c in cases:
+        rest = {k: v for k, v in c.items() if k != "q"}
+        need = max(need, kvq.kvq_decode_workspace_bytes(kvq.make_decode_args(
+            c["q"], out=torch.empty(c["q"].shape, dtype=torch.float32, device="cuda"), **rest)))
+    ws = torch.full((need,), 0xA5, dtype=torch.uint8, device="cuda")
+    for rep in range(2):
+        for ref, c in cases:
+            rest = {k: v for k, v in c.items() if k != "q"}
+            out, _ = kvq.kvq_decode_attention(c["q"], workspace=ws, **rest)
+            assert np.abs(to_np(out) - ref).max() <= OUT_TOL
+    assert kvq.kvq_device_error() == 0
+
+
+def test_decode_qjl_scores_only(kvq):
+    """A QJL scores-only call (no values, no output), twice on one workspace: the
+    estimator scores match the oracle's."""
+    q, S, w, n, vc, vs = _qjl_cache(400, 2, 4, 3000, 8)
+    qg, Sg, wg, ng = _cuda(q, S, w.view(np.int32), n)
+    scores = torch.empty((2, 8, 3000), dtype=torch.float32, device="cuda")
+    a = kvq.make_decode_args(qg, k_words=wg, k_norms=ng, sketch=Sg, scores_out=scores)
+    need = kvq.kvq_decode_workspace_bytes(a)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        _, sc = kvq.kvq_decode_attention(qg, k_words=wg, k_norms=ng, sketch=Sg, want_out=False,
+                                         want_scores=True, workspace=ws)
+        torch.cuda.synchronize()
+    ref = oracle.decode_attention(q, k_words=w, k_norms=n, S=S, want_out=False, want_scores=True)
+    v64, _ = oracle.qjl_query_sketch(q.reshape(-1, 128), S)
+    tol = score_tolerance(ref["scores"].reshape(16, 3000), np.repeat(n, 2, axis=1).reshape(16, 3000), v64, 256)
+    err = np.abs(to_np(sc).astype(np.float64) - ref["scores"]).reshape(16, 3000)
+    assert np.all(err <= tol)
