@@ -256,6 +256,70 @@ ROW_NAMES = ["quantize_cache", "decode_int8", "dequantize_cache", "qjl_encode", 
              "decode_qjl"]
 
 
+def measure_next_rows(wl, stream, reps=3):
+    """Device time of the widened rows (not part of the step): append-on-decode on the
+    same caches, whose last row each call re-appends (the new key / value rows are the
+    cache's own fp16 rows at that position, so the cache does not change)."""
+    import ctypes
+    import torch
+    kvq = wl.kvq
+    lib = kvq.lib
+    L, B, H, T, D = (LLAMA[k] for k in ("layers", "batch", "heads", "seq", "dim"))
+    gb, gq, gk, gt, m = (GQA[k] for k in ("batch", "q_heads", "kv_heads", "seq", "m"))
+    s = ctypes.c_void_p(stream.cuda_stream)
+    knew = wl.cache[:, :, :, :, T - 1].contiguous()          # [L, 2, B, H, D]
+    gnew = wl.gcache[:, :, :, gt - 1].contiguous()            # [2, gb, gk, D]
+    a7 = [kvq.make_decode_append_args(wl.q7[l], knew[l, 0], knew[l, 1], T=T - 1,
+                                      k_codes=wl.codes[l, 0], k_scales=wl.scales[l, 0],
+                                      v_codes=wl.codes[l, 1], v_scales=wl.scales[l, 1],
+                                      out=wl.out7[l], workspace=wl.ws7) for l in range(L)]
+    ag = kvq.make_decode_append_args(wl.qg, gnew[0], gnew[1], T=gt - 1, k_words=wl.words,
+                                     k_norms=wl.norms, sketch=wl.S, v_codes=wl.vcodes,
+                                     v_scales=wl.vscales, out=wl.outg, workspace=wl.wsg)
+    for a in a7 + [ag]:
+        if lib.kvq_decode_append_workspace_bytes(ctypes.byref(a)) > a.base.workspace_bytes:
+            raise RuntimeError("append workspace larger than the decode workspace")
+
+    def run(args_list):
+        for a in args_list:
+            st = lib.kvq_decode_append(ctypes.byref(a), s)
+            if st != kvq.KVQ_OK:
+                raise kvq.KvqError("kvq_decode_append", st)
+
+    out = {}
+    for name, args_list, units, key_bytes, per_new_written in (
+            ("append_int8", a7, B * H, 2 * (D + 4), 2 * (D + 4)),
+            ("append_qjl", [ag], gb * gk, m // 8 + 2 + D + 4, m // 8 + 2 + D + 4)):
+        with torch.cuda.stream(stream):
+            run(args_list)                                    # warm-up
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(reps):
+                run(args_list)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps / len(args_list)
+        seq = T if name == "append_int8" else gt
+        q_heads = H if name == "append_int8" else gq
+        sketch = 0 if name == "append_int8" else m * D * 2
+        per_call = (units * seq * key_bytes            # T - 1 cached rows + the appended row, read
+                    + units * 2 * D * 2                # new fp16 key and value rows, read
+                    + units * per_new_written          # appended encoded rows, written
+                    + (gb if name == "append_qjl" else B) * q_heads * D * (2 + 4) + sketch)
+        out[name] = {"ms_per_call": round(ms, 4), "GB/s": round(per_call / (ms * 1e-3) / 1e9, 1),
+                     "bytes_per_call": int(per_call),
+                     "workload": ("7B-shaped layer: append 1 token to [8, 32, 4095 + 1, 128] INT8 K/V, "
+                                  "decode over 4096 (per layer, 32 layers)") if name == "append_int8" else
+                                 ("GQA [4, 32q/8kv]: append 1 token to 131071 QJL keys (m = 256) + "
+                                  "INT8 V, decode over 131072")}
+    if kvq.kvq_device_error() != 0:
+        raise RuntimeError("device-side error recorded during the widened rows")
+    return out
+
+
 # ---------------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample of the same workload, single thread)
 # ---------------------------------------------------------------------------------
@@ -474,8 +538,13 @@ def run_gpu(args):
         e2e = {"value": None, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
                "unavailable": str(exc)[:200]}
 
+    next_rows = measure_next_rows(wl, stream)
+    barrier()
+
     if rank == 0:
         peak, peak_kind = load_peaks()
+        for v in next_rows.values():
+            v["frac_hbm"] = round(v["GB/s"] / peak, 4)
         dom = max(("quantize_cache", "dequantize_cache"), key=lambda n: row_ms[n])
         achieved = rb[dom] / (row_ms[dom] * 1e-3) / 1e9
         traffic = load_traffic(dom)
@@ -495,6 +564,7 @@ def run_gpu(args):
                          "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs"},
             "e2e": e2e,
+            "next_rows": next_rows,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clocks,
         }

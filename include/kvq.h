@@ -182,6 +182,43 @@ kvq_status kvq_decode_attention(const kvq_decode_args* a, kvq_stream_t stream);
 size_t kvq_decode_workspace_bytes(const kvq_decode_args* a);
 
 /*
+ * kvq_decode_append -- one decode step that first appends the newly generated token to
+ * the compressed cache ("Quantum-Inspired GPU & J-Space VRAM Optimizer" page, section 4,
+ * "Framework Integration": the cache writes are intercepted and the compressed
+ * representation is stored; the INT8 and QJL encodings are those of
+ * kvq_quantize_int8 and kvq_qjl_encode).  For every (batch b, KV head g):
+ *   keys   INT8: k_codes/k_scales row T = the per-row absmax INT8 quantization of
+ *               k_new[b][g] (bit-identical to kvq_quantize_int8 of that row);
+ *          QJL:  k_words row T = sign bits of S k_new[b][g] and k_norms row T =
+ *               fp16(||k_new[b][g]||) (as kvq_qjl_encode: the norm bit-identical, the
+ *               bits computed in fp32, so a bit may differ from an exact computation
+ *               only where |(S k)_i| < 1e-4 ||k||);
+ *   values v_codes/v_scales row T = the INT8 quantization of v_new[b][g];
+ * then the decode step of kvq_decode_attention over the T + 1 tokens 0 .. T, with the
+ * result that step would give on the updated cache.
+ *   base:      the decode arguments, with base.seq_len = T >= 0, the tokens already
+ *              cached, and the cache arrays laid out [B][Hkv][capacity][...] (unit
+ *              stride `capacity` rows instead of seq_len); base.out [B][Hq][D] and/or
+ *              base.scores_out [B][Hq][T + 1].  base.out needs base.v_codes/v_scales.
+ *   capacity:  rows per (b, KV head) in the cache arrays, >= T + 1; rows other than
+ *              0 .. T are neither read nor written.
+ *   k_new_f16, v_new_f16: [B][Hkv][D] fp16, 16-byte aligned; v_new_f16 may be NULL
+ *              when base.out is NULL (the value rows are then not appended).
+ * The appended rows are written by the decode kernel itself, which uses them in the
+ * same launch.  Workspace as kvq_decode_attention, sized by
+ * kvq_decode_append_workspace_bytes.  Errors as kvq_decode_attention.
+ */
+typedef struct kvq_decode_append_args {
+    kvq_decode_args base;
+    int64_t capacity;
+    const uint16_t* k_new_f16;
+    const uint16_t* v_new_f16;
+} kvq_decode_append_args;
+
+kvq_status kvq_decode_append(const kvq_decode_append_args* a, kvq_stream_t stream);
+size_t kvq_decode_append_workspace_bytes(const kvq_decode_append_args* a);
+
+/*
  * kvq_decode_attention_noalloc -- kvq_decode_attention for callers that cannot
  * allocate device memory and cannot lend a workspace (for example code inside a host
  * engine that has already reserved all device memory through its own allocator, or a

@@ -176,6 +176,43 @@ KVQ_API kvq_status kvq_decode_attention(const kvq_decode_args* a, kvq_stream_t s
     return from_cuda(kvq::launch_decode(a, plan, cs(stream)));
 }
 
+namespace {
+
+// The decode arguments of an append call as the kernels see them (T + 1 tokens), after
+// validating the append-specific fields.
+kvq_status check_append(const kvq_decode_append_args* a, kvq_decode_args* view) {
+    if (!a) return KVQ_ERR_INVALID_ARG;
+    const int64_t T = a->base.seq_len;
+    if (T < 0 || a->capacity < T + 1) return KVQ_ERR_INVALID_ARG;
+    *view = a->base;
+    view->seq_len = T + 1;
+    const kvq_status st = check_decode(view);
+    if (st != KVQ_OK || view->batch == 0) return st;
+    if (!a->k_new_f16 || !aligned(a->k_new_f16, 16)) return KVQ_ERR_INVALID_ARG;
+    if (view->out && (!a->v_new_f16 || !aligned(a->v_new_f16, 16))) return KVQ_ERR_INVALID_ARG;
+    return KVQ_OK;
+}
+
+}  // namespace
+
+KVQ_API size_t kvq_decode_append_workspace_bytes(const kvq_decode_append_args* a) {
+    kvq_decode_args view;
+    if (check_append(a, &view) != KVQ_OK) return 0;
+    return kvq::plan_decode(&view, kvq::device_sm_count()).total_bytes;
+}
+
+KVQ_API kvq_status kvq_decode_append(const kvq_decode_append_args* a, kvq_stream_t stream) {
+    kvq_decode_args view;
+    const kvq_status st = check_append(a, &view);
+    if (st != KVQ_OK) return st;
+    if (view.batch == 0) return KVQ_OK;
+    const kvq::DecodePlan plan = kvq::plan_decode(&view, kvq::device_sm_count());
+    if (!view.workspace || !aligned(view.workspace, 256) || view.workspace_bytes < plan.total_bytes)
+        return KVQ_ERR_WORKSPACE;
+    const kvq::AppendSpec app{a->capacity, a->k_new_f16, a->v_new_f16};
+    return from_cuda(kvq::launch_decode(&view, plan, cs(stream), &app));
+}
+
 KVQ_API kvq_status kvq_device_error(uint32_t* code) {
     if (!code) return KVQ_ERR_INVALID_ARG;
     uint32_t a = 0, b = 0;

@@ -24,6 +24,7 @@
 #include <stdint.h>
 
 #include "kvq_device.cuh"
+#include "kvq_int8.cuh"
 #include "kvq_internal.h"
 
 namespace kvq {
@@ -45,7 +46,11 @@ struct DecodeParams {
     const float* sketch_v;  // [B * Hq][m] fp32 (QJL)
     float* scores_out;
     float* ws;              // partial states [ctas][maxj][G][2 + D]
-    int64_t T;
+    int64_t T;              // tokens attended per unit
+    int64_t cap;            // cache rows per unit (row of token t of unit u: u * cap + t)
+    const uint16_t* knew;   // append: new key rows [units][D] fp16, stored at token T - 1
+    const uint16_t* vnew;   // append: new value rows [units][D] fp16 (or null)
+    const uint16_t* S;      // append with QJL keys: the sketch matrix [m][D] fp16
     int64_t W;              // tokens per CTA range
     int64_t total;          // units * T
     int Hq;
@@ -134,6 +139,59 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
+// ---- append of a new token (kvq_decode_append) ----
+// One warp quantizes one fp16 row of D = 128 values (lane l: values 4 l .. 4 l + 3) with
+// the per-row absmax INT8 rule of kvq_quantize_int8, bit for bit (kvq_int8.cuh), and
+// stores the 128 codes and the scale.
+__device__ __forceinline__ void append_int8_row(const uint16_t* src, int8_t* codes, float* scale, int lane) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(src + 4 * lane);
+    const __half2* h = reinterpret_cast<const __half2*>(&raw);
+    const float2 x01 = __half22float2(h[0]), x23 = __half22float2(h[1]);
+    const float f[4] = {x01.x, x01.y, x23.x, x23.y};
+    const float a_lane = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
+    // max of non-negative floats = max of their bit patterns as unsigned integers
+    const float a = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(a_lane)));
+    const float sc = i8::row_scale(a);
+    uint32_t word;
+    i8::quantize_values<4>(f, sc, i8::scale_reciprocal(sc), &word);
+    *reinterpret_cast<uint32_t*>(codes + 4 * lane) = word;
+    if (lane == 0) *scale = sc;
+}
+
+// One warp writes sign word `w` (sketch rows 32 w .. 32 w + 31) of a new key: lane l
+// computes (S k)_{32 w + l} in fp32 from the fp16 S row and key.
+__device__ __forceinline__ uint32_t append_sign_word(const uint16_t* S, const uint16_t* k, int w, int lane) {
+    const uint4* srow = reinterpret_cast<const uint4*>(S + (int64_t)(32 * w + lane) * kD);
+    const uint4* kv = reinterpret_cast<const uint4*>(k);
+    float acc = 0.0f;
+#pragma unroll 4
+    for (int c = 0; c < kD / 8; ++c) {
+        const uint4 sv = __ldg(srow + c);
+        const uint4 kk = __ldg(kv + c);  // the same 16 bytes in every lane
+        const __half2* sh = reinterpret_cast<const __half2*>(&sv);
+        const __half2* kh = reinterpret_cast<const __half2*>(&kk);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 a = __half22float2(sh[i]), b = __half22float2(kh[i]);
+            acc = __fmaf_rn(a.x, b.x, acc);
+            acc = __fmaf_rn(a.y, b.y, acc);
+        }
+    }
+    return __ballot_sync(0xffffffffu, acc >= 0.0f);
+}
+
+// fp16 bits of ||k|| by the defining sequence: squares summed in fp64 in index order,
+// IEEE square root, one rounding to fp16 (one thread).
+__device__ __forceinline__ uint16_t append_norm_bits(const uint16_t* k) {
+    double s64 = 0.0;
+#pragma unroll 1
+    for (int j = 0; j < kD; ++j) {
+        const double d = (double)__half2float(__ushort_as_half(k[j]));
+        s64 = __fma_rn(d, d, s64);
+    }
+    return __half_as_ushort(__double2half(__dsqrt_rn(s64)));
+}
+
 // Merge of per-warp softmax states (m, l, acc[D]) through shared memory into the
 // segment's partial slot.  red: [WARPS][G][2 + kD] floats, already written.
 template <int G, int WARPS>
@@ -200,7 +258,7 @@ decode_int8_kernel(const DecodeParams p) {
     constexpr int kI8StageBytes = I8Ring<G>::bytes;
     static_assert(kI8StageTok % (4 * kI8Consumers) == 0, "each 8-lane group takes whole tokens");
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    __shared__ uint64_t bars[2 * kI8Stages];
+    __shared__ uint64_t bars[2 * kI8Stages + 1];
     __shared__ int abort_storage;
     volatile int* abort_flag = &abort_storage;
     constexpr int U = kI8StageTok / (kI8Consumers * 4);   // tokens per 8-lane group per stage
@@ -214,6 +272,7 @@ decode_int8_kernel(const DecodeParams p) {
     const uint32_t bar0 = dev::smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (kI8Stages + s); };
+    const uint32_t append_bar = bar0 + 8u * (2 * kI8Stages);  // appended rows are in global memory
 
     if (threadIdx.x == 0) {
         abort_storage = 0;
@@ -221,6 +280,7 @@ decode_int8_kernel(const DecodeParams p) {
             dev::mbar_init(full_bar(s), 1);
             dev::mbar_init(empty_bar(s), kI8Consumers);
         }
+        dev::mbar_init(append_bar, kI8Consumers);
         dev::mbar_init_fence();
     }
     __syncthreads();
@@ -234,9 +294,10 @@ decode_int8_kernel(const DecodeParams p) {
             for (int s = 0; s < kI8Stages; ++s) issued[s] = false, ph_issued[s] = 0;
             int i = 0;
             bool run = true;
+            bool appended_visible = false;
             for (int jj = 0; run && jj < nseg; ++jj) {
                 const Segment sg = walk.seg(jj);
-                const int64_t row0 = sg.u * p.T;
+                const int64_t row0 = sg.u * p.cap;
                 for (int64_t t = sg.t0; t < sg.t1; t += kI8StageTok, ++i) {
                     const int s = i % kI8Stages;
                     const uint32_t ph = (uint32_t)(i / kI8Stages) & 1u;
@@ -245,6 +306,16 @@ decode_int8_kernel(const DecodeParams p) {
                         break;
                     }
                     const uint32_t n = (uint32_t)min((int64_t)kI8StageTok, sg.t1 - t);
+                    if (p.knew != nullptr && !appended_visible && sg.t1 == p.T && t + n == sg.t1) {
+                        // this stage holds a token the consumers append: copy it only once
+                        // they have stored it (and made it visible to the async proxy)
+                        if (!dev::mbar_wait(append_bar, 0u, abort_flag, &g_decode_error, kErrI8Producer)) {
+                            run = false;
+                            break;
+                        }
+                        asm volatile("fence.proxy.async.global;" ::: "memory");
+                        appended_visible = true;
+                    }
                     const uint32_t dst = ring + (uint32_t)s * kI8StageBytes;
                     // Values are copied only when the output is wanted (scores-only calls
                     // pass no value pointers); scales only when their rows start 16-byte
@@ -273,13 +344,37 @@ decode_int8_kernel(const DecodeParams p) {
     }
 
     // ---------------- consumers (warps 0 .. kI8Consumers-1) ----------------
+    if (p.knew != nullptr) {
+        // Append: the new token of every unit whose last token lies in this range is
+        // quantized here (one warp per unit and row) and stored at token T - 1 before the
+        // producer copies the stage holding it.
+        int k = 0;
+        for (int jj = 0; jj < nseg; ++jj) {
+            const Segment sg = walk.seg(jj);
+            if (sg.t1 != p.T) continue;
+            if ((k++ % kI8Consumers) != warp) continue;
+            const int64_t row = sg.u * p.cap + p.T - 1;
+            append_int8_row(p.knew + sg.u * kD, const_cast<int8_t*>(p.kc) + row * kD,
+                            const_cast<float*>(p.ks) + row, lane);
+            if (p.vnew != nullptr)
+                append_int8_row(p.vnew + sg.u * kD, const_cast<int8_t*>(p.vc) + row * kD,
+                                const_cast<float*>(p.vs) + row, lane);
+        }
+        // visible to the producer's bulk copies (async proxy) and, through the barrier
+        // below, to the other consumer warps' direct scale loads
+        __threadfence();
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) dev::mbar_arrive(append_bar);
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kI8Consumers) : "memory");
+    }
     const int tg = lane >> 3;
     const int sub = lane & 7;
     int i = 0;
     bool aborted = false;
     for (int jj = 0; jj < nseg; ++jj) {
         const Segment sg = walk.seg(jj);
-        const int64_t row0 = sg.u * p.T;
+        const int64_t row0 = sg.u * p.cap;
         const int64_t b = sg.u / p.Hkv;
         const int kvh = (int)(sg.u % p.Hkv);
         uint64_t qp[G][8];
@@ -319,9 +414,10 @@ decode_int8_kernel(const DecodeParams p) {
                 const int64_t t = tstage + tok0 + u;
                 valid[u] = t < sg.t1;
                 if (!p.scales_bulk) {
+                    // coherent loads: an appended row's scales were stored by this kernel
                     const int64_t r = row0 + (valid[u] ? t : sg.t0);
-                    ksc[u] = __ldg(p.ks + r);
-                    vsc[u] = p.want_out ? __ldg(p.vs + r) : 0.0f;
+                    ksc[u] = __ldcg(p.ks + r);
+                    vsc[u] = p.want_out ? __ldcg(p.vs + r) : 0.0f;
                 }
             }
             // After an abort a warp keeps walking the same stages and barriers (so every
@@ -515,12 +611,36 @@ decode_qjl_kernel(const DecodeParams p) {
     for (int e = 0; e < 4; ++e) sel[e] = 0x6504u | ((uint32_t)((e ^ x) & 3) << 4);
     const uint32_t lut_s = (uint32_t)__cvta_generic_to_shared(lut);
     dev::griddep_launch_dependents();  // the combine kernel may be scheduled (it waits)
+
+    if (p.knew != nullptr) {
+        // Append: the new token of every unit whose last token lies in this range is
+        // encoded here (warps 0 .. m/32 - 1: one sign word each; warp m/32: the norm;
+        // warp m/32 + 1: the INT8 value row) and stored at token T - 1; the barrier
+        // below orders these stores before the loads of the segment loop.
+        for (int jj = 0; jj < nseg; ++jj) {
+            const Segment sg = walk.seg(jj);
+            if (sg.t1 != p.T) continue;
+            const int64_t row = sg.u * p.cap + p.T - 1;
+            const uint16_t* kn = p.knew + sg.u * kD;
+            if (warp < nw) {
+                const uint32_t word = append_sign_word(p.S, kn, warp, lane);
+                if (lane == 0) const_cast<uint32_t*>(p.kw)[row * nw + warp] = word;
+            } else if (warp == nw) {
+                if (lane == 0) const_cast<uint16_t*>(p.kn)[row] = append_norm_bits(kn);
+            } else if (warp == nw + 1 && p.vnew != nullptr) {
+                append_int8_row(p.vnew + sg.u * kD, const_cast<int8_t*>(p.vc) + row * kD,
+                                const_cast<float*>(p.vs) + row, lane);
+            }
+        }
+        __threadfence();
+        __syncthreads();
+    }
     float* mybuf = wbuf + warp * 32 * G;
     const uint64_t magic = pack2(-kCodeMagic, -kCodeMagic);
 
     for (int jj = 0; jj < nseg; ++jj) {
         const Segment sg = walk.seg(jj);
-        const int64_t row0 = sg.u * p.T;
+        const int64_t row0 = sg.u * p.cap;
         const int64_t b = sg.u / p.Hkv;
         const int kvh = (int)(sg.u % p.Hkv);
         __syncthreads();  // the previous segment's merge no longer reads red[]
@@ -849,7 +969,8 @@ DecodePlan plan_decode(const kvq_decode_args* a, int sm_count) {
     return pl;
 }
 
-cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaStream_t st) {
+cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaStream_t st,
+                          const AppendSpec* app) {
     const int G = (int)(a->n_q_heads / a->n_kv_heads);
     const bool qjl = a->key_format == KVQ_KEYS_QJL;
     char* ws = static_cast<char*>(a->workspace);
@@ -865,6 +986,10 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
     p.ws = reinterpret_cast<float*>(ws);
     p.sketch_v = qjl ? reinterpret_cast<float*>(ws + pl.partial_bytes) : nullptr;
     p.T = a->seq_len;
+    p.cap = app ? app->capacity : a->seq_len;
+    p.knew = app ? app->k_new : nullptr;
+    p.vnew = (app && a->out) ? app->v_new : nullptr;
+    p.S = a->sketch_f16;
     p.W = pl.W;
     p.total = pl.units * a->seq_len;
     p.Hq = (int)a->n_q_heads;
@@ -875,7 +1000,7 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
     p.scale_log2 = sm * kLog2e;
     p.qjl_c = qjl ? (float)(1.2533141373155002512 / (double)a->sketch_dim) : 0.0f;  // sqrt(pi/2)/m
     p.want_out = a->out != nullptr;
-    p.scales_bulk = !qjl && (a->seq_len % 4 == 0) &&
+    p.scales_bulk = !qjl && (a->seq_len % 4 == 0) && (p.cap % 4 == 0) &&
                     (reinterpret_cast<uintptr_t>(a->k_scales) % 16 == 0) &&
                     (a->out == nullptr || reinterpret_cast<uintptr_t>(a->v_scales) % 16 == 0);
     cudaError_t e;

@@ -39,6 +39,14 @@ struct DecodePlan {
 };
 DecodePlan plan_decode(const kvq_decode_args* a, int sm_count);
 cudaError_t read_and_clear_decode_error(uint32_t* code);
-cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& plan, cudaStream_t st);
+// Append-on-decode: the new token (row T - 1 of every unit, a->seq_len = T) is encoded
+// by the decode kernel itself; the cache arrays have `capacity` rows per unit.
+struct AppendSpec {
+    int64_t capacity;
+    const uint16_t* k_new;
+    const uint16_t* v_new;  // null: values not appended
+};
+cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& plan, cudaStream_t st,
+                          const AppendSpec* app = nullptr);
 
 }  // namespace kvq

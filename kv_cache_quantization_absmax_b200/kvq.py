@@ -36,6 +36,11 @@ class DecodeArgs(ctypes.Structure):
     ]
 
 
+class DecodeAppendArgs(ctypes.Structure):
+    """Mirror of ``kvq_decode_append_args``."""
+    _fields_ = [("base", DecodeArgs), ("capacity", _I64), ("k_new_f16", _P), ("v_new_f16", _P)]
+
+
 class KvqError(RuntimeError):
     def __init__(self, fn, status):
         self.status = status
@@ -61,6 +66,10 @@ def _load():
     so.kvq_decode_attention_noalloc.restype = ctypes.c_int
     so.kvq_decode_noalloc_max_workspace_bytes.argtypes = []
     so.kvq_decode_noalloc_max_workspace_bytes.restype = ctypes.c_size_t
+    so.kvq_decode_append.argtypes = [ctypes.POINTER(DecodeAppendArgs), _P]
+    so.kvq_decode_append.restype = ctypes.c_int
+    so.kvq_decode_append_workspace_bytes.argtypes = [ctypes.POINTER(DecodeAppendArgs)]
+    so.kvq_decode_append_workspace_bytes.restype = ctypes.c_size_t
     for f in ("kvq_quantize_int8", "kvq_dequantize_int8", "kvq_int8_scores", "kvq_qjl_encode",
               "kvq_qjl_query_sketch", "kvq_decode_attention", "kvq_device_error"):
         getattr(so, f).restype = ctypes.c_int
@@ -254,3 +263,47 @@ def kvq_device_error() -> int:
     code = ctypes.c_uint32(0)
     _check("kvq_device_error", lib.kvq_device_error(ctypes.byref(code)))
     return int(code.value)
+
+
+def make_decode_append_args(q, k_new, v_new, *, T, k_codes=None, k_scales=None, k_words=None,
+                            k_norms=None, sketch=None, v_codes=None, v_scales=None, out=None,
+                            scores_out=None, sm_scale=0.0, workspace=None):
+    """Fill a ``kvq_decode_append_args``: cache tensors [B, Hkv, capacity, ...] holding T
+    tokens; k_new / v_new [B, Hkv, D] fp16."""
+    a = DecodeAppendArgs()
+    a.base = make_decode_args(q, k_codes=k_codes, k_scales=k_scales, k_words=k_words,
+                              k_norms=k_norms, sketch=sketch, v_codes=v_codes, v_scales=v_scales,
+                              out=out, scores_out=scores_out, sm_scale=sm_scale, workspace=workspace)
+    ref = k_words if k_words is not None else k_codes
+    a.capacity = ref.shape[2]
+    a.base.seq_len = T
+    a.k_new_f16 = k_new.data_ptr()
+    a.v_new_f16 = v_new.data_ptr() if v_new is not None else None
+    return a
+
+
+def kvq_decode_append(q, k_new, v_new, *, T, k_codes=None, k_scales=None, k_words=None,
+                      k_norms=None, sketch=None, v_codes=None, v_scales=None, want_out=True,
+                      want_scores=False, sm_scale=0.0, workspace=None, out=None, scores_out=None,
+                      stream=None):
+    """Append-on-decode (see include/kvq.h): writes the new token's encoded key / value
+    rows at position T of the cache tensors (in place) and returns the decode step over
+    the T + 1 tokens: (out [B, Hq, D] fp32 or None, scores [B, Hq, T + 1] or None)."""
+    _need_cuda(q, k_new, v_new, k_codes, k_scales, k_words, k_norms, sketch, v_codes, v_scales)
+    B, Hq, D = q.shape
+    if want_out and out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    if want_scores and scores_out is None:
+        scores_out = torch.empty((B, Hq, T + 1), dtype=torch.float32, device=q.device)
+    a = make_decode_append_args(q, k_new, v_new if want_out else None, T=T, k_codes=k_codes,
+                                k_scales=k_scales, k_words=k_words, k_norms=k_norms, sketch=sketch,
+                                v_codes=v_codes if want_out else None,
+                                v_scales=v_scales if want_out else None,
+                                out=out if want_out else None,
+                                scores_out=scores_out if want_scores else None, sm_scale=sm_scale)
+    need = int(lib.kvq_decode_append_workspace_bytes(ctypes.byref(a)))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    _check("kvq_decode_append", lib.kvq_decode_append(ctypes.byref(a), _stream(stream)))
+    return (out if want_out else None), (scores_out if want_scores else None)

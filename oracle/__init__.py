@@ -190,3 +190,47 @@ def decode_attention(q_f16, *, k_codes=None, k_scales=None, k_words=None, k_norm
         float(sm_scale), _ptr(out), _ptr(scores), _ptr(probs))
     _check(rc, "ora_decode_attention")
     return {"out": out, "scores": scores, "probs": probs}
+
+
+def decode_append(q_f16, k_new_f16, v_new_f16, *, T, k_codes=None, k_scales=None, k_words=None,
+                  k_norms=None, S=None, v_codes=None, v_scales=None, sm_scale=0.0,
+                  want_out=True, want_scores=False):
+    """Append-on-decode ("Quantum-Inspired GPU & J-Space VRAM Optimizer" page, section 4:
+    the cache writes are intercepted and the compressed representation stored): the new
+    token's key row [B, Hkv, D] is quantized (INT8 keys: quantize_int8) or sign-sketched
+    (QJL keys: qjl_encode) and its value row INT8-quantized, both stored at token T of
+    copies of the cache arrays ([B, Hkv, capacity, ...], capacity >= T + 1); then one
+    decode step over the T + 1 tokens.  Returns a dict with the decode outputs and the
+    updated cache copies."""
+    kn = np.ascontiguousarray(k_new_f16, np.float16)
+    B, Hkv, D = kn.shape
+    qjl = k_words is not None
+    res = {}
+    if qjl:
+        w, n = qjl_encode(kn.reshape(-1, D), S)
+        kw = np.array(k_words, np.uint32, copy=True)
+        kno = np.array(k_norms, np.float16, copy=True)
+        kw[:, :, T] = w.reshape(B, Hkv, -1)
+        kno[:, :, T] = n.reshape(B, Hkv)
+        res.update(k_words=kw, k_norms=kno)
+        keys = dict(k_words=kw[:, :, :T + 1], k_norms=kno[:, :, :T + 1], S=S)
+    else:
+        c, s = quantize_int8(kn.reshape(-1, D))
+        kc = np.array(k_codes, np.int8, copy=True)
+        ks = np.array(k_scales, np.float32, copy=True)
+        kc[:, :, T] = c.reshape(B, Hkv, D)
+        ks[:, :, T] = s.reshape(B, Hkv)
+        res.update(k_codes=kc, k_scales=ks)
+        keys = dict(k_codes=kc[:, :, :T + 1], k_scales=ks[:, :, :T + 1])
+    vals = {}
+    if want_out:
+        c, s = quantize_int8(np.ascontiguousarray(v_new_f16, np.float16).reshape(-1, D))
+        vc = np.array(v_codes, np.int8, copy=True)
+        vs = np.array(v_scales, np.float32, copy=True)
+        vc[:, :, T] = c.reshape(B, Hkv, D)
+        vs[:, :, T] = s.reshape(B, Hkv)
+        res.update(v_codes=vc, v_scales=vs)
+        vals = dict(v_codes=vc[:, :, :T + 1], v_scales=vs[:, :, :T + 1])
+    res.update(decode_attention(q_f16, sm_scale=sm_scale, want_out=want_out,
+                                want_scores=want_scores, **keys, **vals))
+    return res

@@ -357,3 +357,83 @@ def test_decode_gqa_group_mapping():
     vs = np.ones_like(vs)
     r = oracle.decode_attention(q, k_codes=kc, k_scales=ks, v_codes=vc, v_scales=vs)
     assert np.allclose(r["out"][0, :2], 10) and np.allclose(r["out"][0, 2:], -10)
+
+
+# ---- append-on-decode ----
+
+def _append_case(T, cap, D=8, B=1, Hq=4, Hkv=2, seed=5):
+    """A cache of `cap` rows per head holding T tokens (rows >= T filled with a sentinel)
+    and a new token's key / value rows."""
+    rng = np.random.default_rng(seed)
+    full_k = rng.standard_normal((B, Hkv, T + 1, D)).astype(np.float16)
+    full_v = rng.standard_normal((B, Hkv, T + 1, D)).astype(np.float16)
+    q = rng.standard_normal((B, Hq, D)).astype(np.float16)
+    kc = np.full((B, Hkv, cap, D), 77, np.int8)
+    ks = np.full((B, Hkv, cap), 3.5, np.float32)
+    vc = np.full((B, Hkv, cap, D), -77, np.int8)
+    vs = np.full((B, Hkv, cap), 2.5, np.float32)
+    if T > 0:
+        c, s = oracle.quantize_int8(full_k[:, :, :T].reshape(-1, D))
+        kc[:, :, :T], ks[:, :, :T] = c.reshape(B, Hkv, T, D), s.reshape(B, Hkv, T)
+        c, s = oracle.quantize_int8(full_v[:, :, :T].reshape(-1, D))
+        vc[:, :, :T], vs[:, :, :T] = c.reshape(B, Hkv, T, D), s.reshape(B, Hkv, T)
+    return q, full_k, full_v, kc, ks, vc, vs
+
+
+def test_decode_append_to_empty_cache_returns_the_new_value_row():
+    """T = 0: one token, p = 1 exactly, so every query head returns its KV head's
+    dequantized new value row, bit for bit."""
+    q, fk, fv, kc, ks, vc, vs = _append_case(0, 3)
+    r = oracle.decode_append(q, fk[:, :, 0], fv[:, :, 0], T=0, k_codes=kc, k_scales=ks,
+                             v_codes=vc, v_scales=vs)
+    c, s = oracle.quantize_int8(fv[:, :, 0].reshape(-1, 8))
+    vhat = (c.astype(np.float32) * s[:, None]).reshape(1, 2, 8)
+    assert np.array_equal(r["out"], np.repeat(vhat, 2, axis=1))
+
+
+@pytest.mark.parametrize("T,cap", [(1, 2), (5, 9), (33, 34)])
+def test_decode_append_int8_against_brute_force(T, cap):
+    q, fk, fv, kc, ks, vc, vs = _append_case(T, cap)
+    r = oracle.decode_append(q, fk[:, :, T], fv[:, :, T], T=T, k_codes=kc, k_scales=ks,
+                             v_codes=vc, v_scales=vs, want_scores=True)
+    # the appended rows are the per-row quantization of the new rows; nothing else moves
+    c, s = oracle.quantize_int8(fk[:, :, T].reshape(-1, 8))
+    assert np.array_equal(r["k_codes"][:, :, T], c.reshape(1, 2, 8))
+    assert np.array_equal(r["k_scales"][:, :, T], s.reshape(1, 2))
+    keep = np.ones(cap, bool)
+    keep[T] = False
+    assert np.array_equal(r["k_codes"][:, :, keep], kc[:, :, keep])
+    assert np.array_equal(r["v_scales"][:, :, keep], vs[:, :, keep])
+    # fp64 attention over all T + 1 tokens quantized from scratch
+    kc_all, ks_all = oracle.quantize_int8(fk.reshape(-1, 8))
+    vc_all, vs_all = oracle.quantize_int8(fv.reshape(-1, 8))
+    kdeq = _fl32_product(kc_all.reshape(1, 2, T + 1, 8), ks_all.reshape(1, 2, T + 1))
+    vdeq = _fl32_product(vc_all.reshape(1, 2, T + 1, 8), vs_all.reshape(1, 2, T + 1))
+    sigma = float(np.float32(1.0) / np.sqrt(np.float32(8)))
+    out, sc, _ = _brute_force(q, kdeq, vdeq, 4, sigma)
+    assert np.allclose(r["scores"], sc, rtol=0, atol=1e-5)
+    assert np.allclose(r["out"], out, rtol=0, atol=1e-5)
+
+
+def test_decode_append_qjl_against_brute_force():
+    T, cap = 7, 8
+    q, fk, fv, _, _, vc, vs = _append_case(T, cap, seed=9)
+    S = inputs.sketch_matrix(32, 8, seed=3)
+    w, n = oracle.qjl_encode(fk[:, :, :T].reshape(-1, 8), S)
+    kw = np.zeros((1, 2, cap, 1), np.uint32)
+    kn = np.zeros((1, 2, cap), np.float16)
+    kw[:, :, :T] = w.reshape(1, 2, T, 1)
+    kn[:, :, :T] = n.reshape(1, 2, T)
+    r = oracle.decode_append(q, fk[:, :, T], fv[:, :, T], T=T, k_words=kw, k_norms=kn, S=S,
+                             v_codes=vc, v_scales=vs, want_scores=True)
+    # estimator scores from the definition over all T + 1 keys, sketched from scratch
+    w_all, n_all = oracle.qjl_encode(fk.reshape(-1, 8), S)
+    assert np.array_equal(r["k_words"][:, :, :T + 1].reshape(-1), w_all.reshape(-1))
+    assert np.array_equal(r["k_norms"][:, :, :T + 1].reshape(-1).view(np.uint16),
+                          n_all.reshape(-1).view(np.uint16))
+    v = (q.astype(np.float64) @ S.astype(np.float64).T).astype(np.float32).astype(np.float64)
+    bits = ((w_all.reshape(1, 2, T + 1)[..., None] >> np.arange(32, dtype=np.uint32)) & 1)
+    sgn = np.repeat(2.0 * bits - 1, 2, axis=1)
+    nrm = np.repeat(n_all.reshape(1, 2, T + 1).astype(np.float64), 2, axis=1)
+    sc = math.sqrt(math.pi / 2) / 32 * nrm * np.einsum("bhm,bhtm->bht", v, sgn)
+    assert np.allclose(r["scores"], sc, rtol=1e-6, atol=1e-6)
