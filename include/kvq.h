@@ -182,6 +182,46 @@ kvq_status kvq_decode_attention(const kvq_decode_args* a, kvq_stream_t stream);
 size_t kvq_decode_workspace_bytes(const kvq_decode_args* a);
 
 /*
+ * kvq_quantize_int8_channelwise / kvq_dequantize_int8_channelwise -- the symmetric INT8
+ * equation of kvq_quantize_int8 with one scale per channel ("Q-TensorFormer" model
+ * card, section 6, Symmetric Channel-Wise INT8: X_hat = clamp(round(X / s8), -128, 127)
+ * * s8, s8 = max|X| / 127).  x holds n_blocks blocks of [rows][d] row-major, one block
+ * after another (for a KV cache [B][H][T][D]: n_blocks = B * H, rows = T); for block b
+ * and column j:
+ *   s[b][j] = fl32(max_r |x[b][r][j]| / 127),
+ *   codes[b][r][j] = clamp(rint_even(fl32(x[b][r][j] / s[b][j])), -128, 127)  (0 if s = 0);
+ *   dequantize: out = fl32(codes * s) (fp16 out: that value rounded to nearest even).
+ * Bit-identical to that definition.  d must be a multiple of 64, rows >= 1; x, codes,
+ * out 16-byte aligned, scales [n_blocks][d] 4-byte aligned (else KVQ_ERR_INVALID_ARG).
+ * n_blocks == 0: no launch.  One launch each; stream-ordered, no synchronisation.
+ */
+kvq_status kvq_quantize_int8_channelwise(const void* x, kvq_dtype x_dtype, int64_t n_blocks, int64_t rows,
+                                         int64_t d, int8_t* codes, float* scales, kvq_stream_t stream);
+kvq_status kvq_dequantize_int8_channelwise(const int8_t* codes, const float* scales, int64_t n_blocks,
+                                           int64_t rows, int64_t d, void* out, kvq_dtype out_dtype,
+                                           kvq_stream_t stream);
+
+/*
+ * kvq_quantize_int4 / kvq_dequantize_int4 -- asymmetric group-wise INT4 ("Q-TensorFormer"
+ * model card, section 6, Asymmetric Group-Wise INT4: X_hat = clamp(round((X - z4) / s4),
+ * 0, 15) * s4 + z4, s4 = (max X - min X) / 15, z4 = min X).  x: [n_rows][d] fp32 or fp16;
+ * each row is cut into groups of `group` consecutive elements (32, 64 or 128; d a
+ * multiple of it).  Per group g of row r, in fp32 with IEEE operations:
+ *   z = min x,  s = fl32(fl32(max x - min x) / 15),
+ *   c = clamp(rint_even(fl32(fl32(x - z) / s)), 0, 15)  (0 if s = 0),
+ *   dequantize: out = fl32(fl32(c * s) + z) (fp16 out: rounded to nearest even).
+ * packed: [n_rows][d/2] bytes, element 2i in bits 0-3 and 2i+1 in bits 4-7;
+ * scales, zeros: [n_rows][d/group] fp32.  Bit-identical to the definition.  x and out
+ * 16-byte aligned, packed 4-byte aligned, scales/zeros 4-byte aligned (else
+ * KVQ_ERR_INVALID_ARG); other group sizes KVQ_ERR_UNSUPPORTED.  One launch each.
+ */
+kvq_status kvq_quantize_int4(const void* x, kvq_dtype x_dtype, int64_t n_rows, int64_t d, int32_t group,
+                             uint8_t* packed, float* scales, float* zeros, kvq_stream_t stream);
+kvq_status kvq_dequantize_int4(const uint8_t* packed, const float* scales, const float* zeros,
+                               int64_t n_rows, int64_t d, int32_t group, void* out, kvq_dtype out_dtype,
+                               kvq_stream_t stream);
+
+/*
  * kvq_decode_append -- one decode step that first appends the newly generated token to
  * the compressed cache ("Quantum-Inspired GPU & J-Space VRAM Optimizer" page, section 4,
  * "Framework Integration": the cache writes are intercepted and the compressed

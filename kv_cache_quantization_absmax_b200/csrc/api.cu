@@ -161,6 +161,59 @@ KVQ_API kvq_status kvq_qjl_query_sketch(const uint16_t* q_f16, int64_t n_q, int3
     return from_cuda(kvq::launch_qjl_query_sketch(q_f16, n_q, sketch_f16, m, v, cs(stream)));
 }
 
+KVQ_API kvq_status kvq_quantize_int8_channelwise(const void* x, kvq_dtype x_dtype, int64_t n_blocks,
+                                                 int64_t rows, int64_t d, int8_t* codes, float* scales,
+                                                 kvq_stream_t stream) {
+    if (!valid_dtype(x_dtype) || n_blocks < 0 || rows <= 0 || d <= 0 || d % 64 != 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (n_blocks == 0) return KVQ_OK;
+    if (n_blocks > 65535) return KVQ_ERR_UNSUPPORTED;
+    if (!x || !codes || !scales || !aligned(x, 16) || !aligned(codes, 16) || !aligned(scales, 4))
+        return KVQ_ERR_INVALID_ARG;
+    return from_cuda(kvq::launch_quantize_int8_channelwise(x, x_dtype == KVQ_F16, n_blocks, rows, d,
+                                                           codes, scales, cs(stream)));
+}
+
+KVQ_API kvq_status kvq_dequantize_int8_channelwise(const int8_t* codes, const float* scales, int64_t n_blocks,
+                                                   int64_t rows, int64_t d, void* out, kvq_dtype out_dtype,
+                                                   kvq_stream_t stream) {
+    if (!valid_dtype(out_dtype) || n_blocks < 0 || rows <= 0 || d <= 0 || d % 64 != 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (n_blocks == 0) return KVQ_OK;
+    if (!codes || !scales || !out || !aligned(codes, 16) || !aligned(scales, 4) || !aligned(out, 16))
+        return KVQ_ERR_INVALID_ARG;
+    return from_cuda(kvq::launch_dequantize_int8_channelwise(codes, scales, n_blocks, rows, d, out,
+                                                             out_dtype == KVQ_F16, cs(stream)));
+}
+
+KVQ_API kvq_status kvq_quantize_int4(const void* x, kvq_dtype x_dtype, int64_t n_rows, int64_t d,
+                                     int32_t group, uint8_t* packed, float* scales, float* zeros,
+                                     kvq_stream_t stream) {
+    if (!valid_dtype(x_dtype) || n_rows < 0 || d <= 0 || group <= 0 || d % group != 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (group != 32 && group != 64 && group != 128) return KVQ_ERR_UNSUPPORTED;
+    if (n_rows == 0) return KVQ_OK;
+    if (!x || !packed || !scales || !zeros || !aligned(x, 16) || !aligned(packed, 4) ||
+        !aligned(scales, 4) || !aligned(zeros, 4))
+        return KVQ_ERR_INVALID_ARG;
+    return from_cuda(kvq::launch_quantize_int4(x, x_dtype == KVQ_F16, n_rows, d, group, packed, scales, zeros,
+                                               cs(stream)));
+}
+
+KVQ_API kvq_status kvq_dequantize_int4(const uint8_t* packed, const float* scales, const float* zeros,
+                                       int64_t n_rows, int64_t d, int32_t group, void* out,
+                                       kvq_dtype out_dtype, kvq_stream_t stream) {
+    if (!valid_dtype(out_dtype) || n_rows < 0 || d <= 0 || group <= 0 || d % group != 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (group != 32 && group != 64 && group != 128) return KVQ_ERR_UNSUPPORTED;
+    if (n_rows == 0) return KVQ_OK;
+    if (!packed || !scales || !zeros || !out || !aligned(packed, 4) || !aligned(scales, 4) ||
+        !aligned(zeros, 4) || !aligned(out, 16))
+        return KVQ_ERR_INVALID_ARG;
+    return from_cuda(kvq::launch_dequantize_int4(packed, scales, zeros, n_rows, d, group, out,
+                                                 out_dtype == KVQ_F16, cs(stream)));
+}
+
 KVQ_API size_t kvq_decode_workspace_bytes(const kvq_decode_args* a) {
     if (check_decode(a) != KVQ_OK) return 0;
     return kvq::plan_decode(a, kvq::device_sm_count()).total_bytes;

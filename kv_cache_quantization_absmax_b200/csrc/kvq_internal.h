@@ -19,6 +19,18 @@ cudaError_t launch_int8_scores(const void* q, bool q_f16, const int8_t* codes,
                                const float* scales, int64_t n_rows, int64_t d, float* scores,
                                cudaStream_t st);
 
+// lowbit.cu
+cudaError_t launch_quantize_int4(const void* x, bool f16, int64_t n_rows, int64_t d, int group,
+                                 uint8_t* packed, float* scales, float* zeros, cudaStream_t st);
+cudaError_t launch_dequantize_int4(const uint8_t* packed, const float* scales, const float* zeros,
+                                   int64_t n_rows, int64_t d, int group, void* out, bool f16,
+                                   cudaStream_t st);
+cudaError_t launch_quantize_int8_channelwise(const void* x, bool f16, int64_t n_blocks, int64_t rows,
+                                             int64_t d, int8_t* codes, float* scales, cudaStream_t st);
+cudaError_t launch_dequantize_int8_channelwise(const int8_t* codes, const float* scales, int64_t n_blocks,
+                                               int64_t rows, int64_t d, void* out, bool f16,
+                                               cudaStream_t st);
+
 // qjl.cu
 // Returns cudaErrorNotSupported when the driver's tensor-map encoder is unavailable.
 cudaError_t launch_qjl_encode(const uint16_t* keys, int64_t n_keys, const uint16_t* S, int m,

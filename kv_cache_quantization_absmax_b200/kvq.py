@@ -66,6 +66,13 @@ def _load():
     so.kvq_decode_attention_noalloc.restype = ctypes.c_int
     so.kvq_decode_noalloc_max_workspace_bytes.argtypes = []
     so.kvq_decode_noalloc_max_workspace_bytes.restype = ctypes.c_size_t
+    so.kvq_quantize_int8_channelwise.argtypes = [_P, ctypes.c_int, _I64, _I64, _I64, _P, _P, _P]
+    so.kvq_dequantize_int8_channelwise.argtypes = [_P, _P, _I64, _I64, _I64, _P, ctypes.c_int, _P]
+    so.kvq_quantize_int4.argtypes = [_P, ctypes.c_int, _I64, _I64, _I32, _P, _P, _P, _P]
+    so.kvq_dequantize_int4.argtypes = [_P, _P, _P, _I64, _I64, _I32, _P, ctypes.c_int, _P]
+    for f in ("kvq_quantize_int8_channelwise", "kvq_dequantize_int8_channelwise", "kvq_quantize_int4",
+              "kvq_dequantize_int4"):
+        getattr(so, f).restype = ctypes.c_int
     so.kvq_decode_append.argtypes = [ctypes.POINTER(DecodeAppendArgs), _P]
     so.kvq_decode_append.restype = ctypes.c_int
     so.kvq_decode_append_workspace_bytes.argtypes = [ctypes.POINTER(DecodeAppendArgs)]
@@ -307,3 +314,61 @@ def kvq_decode_append(q, k_new, v_new, *, T, k_codes=None, k_scales=None, k_word
     a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel()
     _check("kvq_decode_append", lib.kvq_decode_append(ctypes.byref(a), _stream(stream)))
     return (out if want_out else None), (scores_out if want_scores else None)
+
+
+def kvq_quantize_int8_channelwise(x, codes=None, scales=None, stream=None):
+    """Channel-wise INT8 of x [..., rows, d] (fp16/fp32): each leading index is a block
+    with one scale per column; returns (codes int8 like x, scales fp32 [..., d])."""
+    _need_cuda(x)
+    rows, d = x.shape[-2], x.shape[-1]
+    nb = x.numel() // (rows * d)
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-2] + (d,), dtype=torch.float32, device=x.device)
+    _check("kvq_quantize_int8_channelwise",
+           lib.kvq_quantize_int8_channelwise(x.data_ptr(), _dtype_code(x), nb, rows, d, codes.data_ptr(),
+                                             scales.data_ptr(), _stream(stream)))
+    return codes, scales
+
+
+def kvq_dequantize_int8_channelwise(codes, scales, out=None, out_dtype=torch.float16, stream=None):
+    _need_cuda(codes, scales)
+    rows, d = codes.shape[-2], codes.shape[-1]
+    nb = codes.numel() // (rows * d)
+    if out is None:
+        out = torch.empty(codes.shape, dtype=out_dtype, device=codes.device)
+    _check("kvq_dequantize_int8_channelwise",
+           lib.kvq_dequantize_int8_channelwise(codes.data_ptr(), scales.data_ptr(), nb, rows, d,
+                                               out.data_ptr(), _dtype_code(out), _stream(stream)))
+    return out
+
+
+def kvq_quantize_int4(x, group, packed=None, scales=None, zeros=None, stream=None):
+    """Group-wise asymmetric INT4 of x [..., d]: returns (packed uint8 [..., d/2], scales,
+    zeros fp32 [..., d/group])."""
+    _need_cuda(x)
+    d = x.shape[-1]
+    n = x.numel() // d
+    if packed is None:
+        packed = torch.empty(x.shape[:-1] + (d // 2,), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1] + (d // group,), dtype=torch.float32, device=x.device)
+    if zeros is None:
+        zeros = torch.empty(x.shape[:-1] + (d // group,), dtype=torch.float32, device=x.device)
+    _check("kvq_quantize_int4",
+           lib.kvq_quantize_int4(x.data_ptr(), _dtype_code(x), n, d, group, packed.data_ptr(), scales.data_ptr(),
+                                 zeros.data_ptr(), _stream(stream)))
+    return packed, scales, zeros
+
+
+def kvq_dequantize_int4(packed, scales, zeros, group, out=None, out_dtype=torch.float16, stream=None):
+    _need_cuda(packed, scales, zeros)
+    d = packed.shape[-1] * 2
+    n = packed.numel() * 2 // d
+    if out is None:
+        out = torch.empty(packed.shape[:-1] + (d,), dtype=out_dtype, device=packed.device)
+    _check("kvq_dequantize_int4",
+           lib.kvq_dequantize_int4(packed.data_ptr(), scales.data_ptr(), zeros.data_ptr(), n, d, group,
+                                   out.data_ptr(), _dtype_code(out), _stream(stream)))
+    return out

@@ -42,7 +42,14 @@ def _load():
         lib.ora_qjl_estimate.restype = ctypes.c_double
         lib.ora_qjl_scores.argtypes = [P, I64, P, P, I64, I32, P]
         lib.ora_decode_attention.argtypes = [I64, I64, I64, I64, I32, P, I32, P, P, P, P, P,
-                                             I32, P, P, ctypes.c_float, P, P, P]
+                                             I32, P, P, P, P, P, I32, ctypes.c_float, P, P, P]
+        lib.ora_quantize_int8_channelwise.argtypes = [P, I32, I64, I64, I64, P, P]
+        lib.ora_dequantize_int8_channelwise.argtypes = [P, P, I64, I64, I64, P, I32]
+        lib.ora_quantize_int4_group.argtypes = [P, I32, I64, I64, I32, P, P, P]
+        lib.ora_dequantize_int4_group.argtypes = [P, P, P, I64, I64, I32, P, I32]
+        for f in ("ora_quantize_int8_channelwise", "ora_dequantize_int8_channelwise",
+                  "ora_quantize_int4_group", "ora_dequantize_int4_group"):
+            getattr(lib, f).restype = I32
         for f in ("ora_quantize_int8", "ora_dequantize_int8", "ora_int8_scores",
                   "ora_qjl_encode", "ora_qjl_query_sketch", "ora_qjl_scores",
                   "ora_decode_attention"):
@@ -157,10 +164,11 @@ def qjl_scores(v: np.ndarray, words: np.ndarray, norms_f16: np.ndarray):
 
 
 def decode_attention(q_f16, *, k_codes=None, k_scales=None, k_words=None, k_norms=None,
-                     S=None, v_codes=None, v_scales=None, sm_scale=0.0,
+                     S=None, v_codes=None, v_scales=None, v4=None, sm_scale=0.0,
                      want_out=True, want_scores=False, want_probs=False):
     """One decode step.  q [B, Hq, D] fp16; INT8 keys [B, Hkv, T, D] + [B, Hkv, T] or
-    QJL keys words [B, Hkv, T, m/32] + norms [B, Hkv, T] + S [m, D]; INT8 values.
+    QJL keys words [B, Hkv, T, m/32] + norms [B, Hkv, T] + S [m, D]; INT8 values, or
+    group-wise INT4 values v4 = (packed [B, Hkv, T, D/2], scales, zeros [B, Hkv, T, D/g], g).
     Returns a dict with 'out' [B, Hq, D], 'scores' / 'probs' [B, Hq, T] as requested."""
     q = np.ascontiguousarray(q_f16, np.float16)
     B, Hq, D = q.shape
@@ -176,7 +184,14 @@ def decode_attention(q_f16, *, k_codes=None, k_scales=None, k_words=None, k_norm
         k_scales = np.ascontiguousarray(k_scales, np.float32)
         Hkv, T = k_codes.shape[1], k_codes.shape[2]
         S64, m = None, 0
-    if want_out:
+    v4p = v4s = v4z = None
+    v4g = 0
+    if want_out and v4 is not None:
+        v4p = np.ascontiguousarray(v4[0], np.uint8)
+        v4s = np.ascontiguousarray(v4[1], np.float32)
+        v4z = np.ascontiguousarray(v4[2], np.float32)
+        v4g = int(v4[3])
+    elif want_out:
         v_codes = np.ascontiguousarray(v_codes, np.int8)
         v_scales = np.ascontiguousarray(v_scales, np.float32)
     out = np.empty((B, Hq, D), np.float32) if want_out else None
@@ -186,7 +201,9 @@ def decode_attention(q_f16, *, k_codes=None, k_scales=None, k_words=None, k_norm
         B, Hq, Hkv, T, D, _ptr(q), KEYS_QJL if qjl else KEYS_INT8,
         _ptr(k_codes) if not qjl else None, _ptr(k_scales) if not qjl else None,
         _ptr(k_words) if qjl else None, _ptr(k_norms) if qjl else None, _ptr(S64), m,
-        _ptr(v_codes) if want_out else None, _ptr(v_scales) if want_out else None,
+        _ptr(v_codes) if (want_out and v4 is None) else None,
+        _ptr(v_scales) if (want_out and v4 is None) else None,
+        _ptr(v4p), _ptr(v4s), _ptr(v4z), v4g,
         float(sm_scale), _ptr(out), _ptr(scores), _ptr(probs))
     _check(rc, "ora_decode_attention")
     return {"out": out, "scores": scores, "probs": probs}
@@ -234,3 +251,52 @@ def decode_append(q_f16, k_new_f16, v_new_f16, *, T, k_codes=None, k_scales=None
     res.update(decode_attention(q_f16, sm_scale=sm_scale, want_out=want_out,
                                 want_scores=want_scores, **keys, **vals))
     return res
+
+
+def quantize_int8_channelwise(x: np.ndarray):
+    """Channel-wise INT8 of blocks x [n_blocks, rows, d]: returns (codes int8 like x,
+    scales fp32 [n_blocks, d]), one scale per column of each block."""
+    x = np.ascontiguousarray(x)
+    nb, rows, d = x.shape
+    codes = np.empty(x.shape, np.int8)
+    scales = np.empty((nb, d), np.float32)
+    _check(_load().ora_quantize_int8_channelwise(_ptr(x), _dtype_code(x), nb, rows, d, _ptr(codes),
+                                                 _ptr(scales)), "ora_quantize_int8_channelwise")
+    return codes, scales
+
+
+def dequantize_int8_channelwise(codes: np.ndarray, scales: np.ndarray, out_dtype=np.float32):
+    codes = np.ascontiguousarray(codes, np.int8)
+    scales = np.ascontiguousarray(scales, np.float32)
+    nb, rows, d = codes.shape
+    out = np.empty(codes.shape, out_dtype)
+    _check(_load().ora_dequantize_int8_channelwise(_ptr(codes), _ptr(scales), nb, rows, d, _ptr(out),
+                                                   F16 if out_dtype == np.float16 else F32),
+           "ora_dequantize_int8_channelwise")
+    return out
+
+
+def quantize_int4_group(x: np.ndarray, g: int):
+    """Group-wise asymmetric INT4 of rows x [n, d] (fp16 or fp32), groups of g: returns
+    (packed uint8 [n, d/2], scales fp32 [n, d/g], zeros fp32 [n, d/g])."""
+    x = np.ascontiguousarray(x)
+    n, d = x.shape
+    packed = np.zeros((n, d // 2), np.uint8)
+    scales = np.empty((n, d // g), np.float32)
+    zeros = np.empty((n, d // g), np.float32)
+    _check(_load().ora_quantize_int4_group(_ptr(x), _dtype_code(x), n, d, g, _ptr(packed), _ptr(scales),
+                                           _ptr(zeros)), "ora_quantize_int4_group")
+    return packed, scales, zeros
+
+
+def dequantize_int4_group(packed, scales, zeros, g: int, out_dtype=np.float32):
+    packed = np.ascontiguousarray(packed, np.uint8)
+    scales = np.ascontiguousarray(scales, np.float32)
+    zeros = np.ascontiguousarray(zeros, np.float32)
+    n, half = packed.shape
+    d = 2 * half
+    out = np.empty((n, d), out_dtype)
+    _check(_load().ora_dequantize_int4_group(_ptr(packed), _ptr(scales), _ptr(zeros), n, d, g, _ptr(out),
+                                             F16 if out_dtype == np.float16 else F32),
+           "ora_dequantize_int4_group")
+    return out

@@ -22,6 +22,9 @@
  *          asymmetric unbiased inner-product estimator.
  *  [GQA]   "Q-TensorFormer" model card, section 4 "Grouped-Query Attention (GQA) &
  *          Multi-Query Attention (MQA)": KV head broadcast by unsqueeze/expand/reshape.
+ *  [INT4]  "Q-TensorFormer" model card, section 6, Asymmetric Group-Wise INT4 equations:
+ *          X_hat = clamp(round((X - z4) / s4), 0, 15) * s4 + z4,
+ *          s4 = (max X - min X) / 15,  z4 = min X.
  *
  * Readings where the pages are silent (each listed in the design notes):
  *  - granularity is one scale per row of head_dim ("per token");
@@ -139,6 +142,120 @@ int ora_dequantize_int8(const int8_t* codes, const float* scales, int64_t n_rows
     return 0;
 }
 
+/* ---------------------------------------------------------------------------------
+ * [INT8] channel-wise: the same equation with one scale per column.  x holds n_blocks
+ * blocks of [rows][d] (row-major, blocks one after another); for block b and column j:
+ *   a = max_r |x_brj|,  s_bj = fl32(a / 127),
+ *   c_brj = clamp(round_half_even(fl32(x_brj / s_bj)), -128, 127);  s_bj == 0 -> c = 0.
+ * scales: [n_blocks][d].
+ * ------------------------------------------------------------------------------- */
+int ora_quantize_int8_channelwise(const void* x, int dtype, int64_t n_blocks, int64_t rows,
+                                  int64_t d, int8_t* codes, float* scales) {
+    if (n_blocks < 0 || rows <= 0 || d <= 0) return 1;
+    for (int64_t b = 0; b < n_blocks; ++b) {
+        for (int64_t j = 0; j < d; ++j) {
+            float a = 0.0f;
+            for (int64_t r = 0; r < rows; ++r) {
+                float v = fabsf(load_elem(x, dtype, (b * rows + r) * d + j));
+                if (v > a) a = v;
+            }
+            float s = a / 127.0f;
+            scales[b * d + j] = s;
+            for (int64_t r = 0; r < rows; ++r) {
+                int8_t c = 0;
+                if (s != 0.0f) {
+                    float qt = load_elem(x, dtype, (b * rows + r) * d + j) / s;
+                    float rq = nearbyintf(qt);
+                    if (rq < -128.0f) rq = -128.0f;
+                    if (rq > 127.0f) rq = 127.0f;
+                    c = (int8_t)rq;
+                }
+                codes[(b * rows + r) * d + j] = c;
+            }
+        }
+    }
+    return 0;
+}
+
+/* [INT8] channel-wise dequantize: x_hat_brj = fl32(c_brj * s_bj). */
+int ora_dequantize_int8_channelwise(const int8_t* codes, const float* scales, int64_t n_blocks,
+                                    int64_t rows, int64_t d, void* out, int out_dtype) {
+    if (n_blocks < 0 || rows <= 0 || d <= 0) return 1;
+    for (int64_t b = 0; b < n_blocks; ++b)
+        for (int64_t r = 0; r < rows; ++r)
+            for (int64_t j = 0; j < d; ++j) {
+                int64_t i = (b * rows + r) * d + j;
+                float v = (float)codes[i] * scales[b * d + j];
+                if (out_dtype == ORA_F16) ((uint16_t*)out)[i] = ora_double_to_half((double)v);
+                else ((float*)out)[i] = v;
+            }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------------
+ * [INT4] asymmetric group-wise: each row of d is cut into groups of g consecutive
+ * elements.  Per group:  mn = min x,  mx = max x,  s4 = fl32(fl32(mx - mn) / 15),
+ * z4 = mn,  c = clamp(round_half_even(fl32(fl32(x - z4) / s4)), 0, 15)  (s4 == 0 ->
+ * c = 0).  Codes are packed two per byte: element 2i in bits 0-3, element 2i+1 in
+ * bits 4-7 (packed: [n_rows][d/2]); scales and zeros: [n_rows][d/g] fp32.
+ * ------------------------------------------------------------------------------- */
+int ora_quantize_int4_group(const void* x, int dtype, int64_t n_rows, int64_t d, int g,
+                            uint8_t* packed, float* scales, float* zeros) {
+    if (n_rows < 0 || d <= 0 || g <= 0 || (d % g) != 0 || (g % 2) != 0) return 1;
+    int64_t ng = d / g;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        for (int64_t k = 0; k < ng; ++k) {
+            int64_t o = r * d + k * g;
+            float mn = load_elem(x, dtype, o), mx = mn;
+            for (int e = 1; e < g; ++e) {
+                float v = load_elem(x, dtype, o + e);
+                if (v < mn) mn = v;
+                if (v > mx) mx = v;
+            }
+            float s = (mx - mn) / 15.0f;
+            scales[r * ng + k] = s;
+            zeros[r * ng + k] = mn;
+            for (int e = 0; e < g; ++e) {
+                int c = 0;
+                if (s != 0.0f) {
+                    float qt = (load_elem(x, dtype, o + e) - mn) / s;
+                    float rq = nearbyintf(qt);
+                    if (rq < 0.0f) rq = 0.0f;
+                    if (rq > 15.0f) rq = 15.0f;
+                    c = (int)rq;
+                }
+                int64_t i = o + e;
+                uint8_t* byte = &packed[i / 2];
+                if ((i % 2) == 0) *byte = (uint8_t)((*byte & 0xF0) | c);
+                else *byte = (uint8_t)((*byte & 0x0F) | (c << 4));
+            }
+        }
+    }
+    return 0;
+}
+
+/* [INT4] dequantize: x_hat = fl32(fl32(c * s4) + z4). */
+static float int4_value(const uint8_t* packed, const float* scales, const float* zeros,
+                        int64_t r, int64_t d, int g, int64_t j) {
+    int64_t i = r * d + j;
+    int c = (packed[i / 2] >> ((i % 2) * 4)) & 0xF;
+    int64_t k = r * (d / g) + j / g;
+    float cs = (float)c * scales[k];
+    return cs + zeros[k];
+}
+
+int ora_dequantize_int4_group(const uint8_t* packed, const float* scales, const float* zeros,
+                              int64_t n_rows, int64_t d, int g, void* out, int out_dtype) {
+    if (n_rows < 0 || d <= 0 || g <= 0 || (d % g) != 0 || (g % 2) != 0) return 1;
+    for (int64_t r = 0; r < n_rows; ++r)
+        for (int64_t j = 0; j < d; ++j) {
+            float v = int4_value(packed, scales, zeros, r, d, g, j);
+            if (out_dtype == ORA_F16) ((uint16_t*)out)[r * d + j] = ora_double_to_half((double)v);
+            else ((float*)out)[r * d + j] = v;
+        }
+    return 0;
+}
+
 /* [PAPER] attention score against an INT8 row: score = sum_j q_j * x_hat_j, with
  * x_hat_j = fl32(c_j * s), accumulated in fp32 in index order. */
 static float int8_row_score(const float* q, const int8_t* c, float s, int64_t d) {
@@ -245,7 +362,9 @@ int ora_qjl_scores(const double* v, int64_t n_q, const uint32_t* words,
  *   q:        fp16 [B][Hq][D]
  *   keys:     INT8 codes [B][Hkv][T][D] + fp32 scales [B][Hkv][T], or
  *             QJL words [B][Hkv][T][m/32] + fp16 norms [B][Hkv][T] + sketch S (fp64 m x D)
- *   values:   INT8 codes [B][Hkv][T][D] + fp32 scales [B][Hkv][T]
+ *   values:   INT8 codes [B][Hkv][T][D] + fp32 scales [B][Hkv][T], or (when v_packed4
+ *             is given) [INT4] group-wise codes [B][Hkv][T][D/2] + scales and zeros
+ *             [B][Hkv][T][D/v_group], x_hat = fl32(fl32(c * s4) + z4)
  *   [GQA]     query head h reads KV head h / (Hq / Hkv)  (expand along a new group axis
  *             after the KV-head axis, then merge the two axes).
  *   score_t   = INT8: sum_j q_j x_hat_tj (fp32, index order); QJL: the estimator, fp32.
@@ -260,7 +379,9 @@ int ora_decode_attention(int64_t B, int64_t Hq, int64_t Hkv, int64_t T, int D,
                          const int8_t* k_codes, const float* k_scales,
                          const uint32_t* k_words, const uint16_t* k_norms_f16,
                          const double* S, int m,
-                         const int8_t* v_codes, const float* v_scales, float sm_scale,
+                         const int8_t* v_codes, const float* v_scales,
+                         const uint8_t* v_packed4, const float* v_scales4, const float* v_zeros4,
+                         int v_group, float sm_scale,
                          float* out, float* scores_out, float* probs_out) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || T <= 0 || D <= 0 || (Hq % Hkv) != 0) return 1;
     if (key_format == ORA_KEYS_QJL && (m <= 0 || (m % 32) != 0)) return 1;
@@ -317,7 +438,9 @@ int ora_decode_attention(int64_t B, int64_t Hq, int64_t Hkv, int64_t T, int D,
                 for (int j = 0; j < D; ++j) {
                     float acc = 0.0f;
                     for (int64_t t = 0; t < T; ++t) {
-                        float xv = (float)v_codes[(base + t) * D + j] * v_scales[base + t];
+                        float xv = v_packed4
+                                       ? int4_value(v_packed4, v_scales4, v_zeros4, base + t, D, v_group, j)
+                                       : (float)v_codes[(base + t) * D + j] * v_scales[base + t];
                         float prod = e[t] * xv;
                         acc = acc + prod;
                     }

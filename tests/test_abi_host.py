@@ -113,3 +113,17 @@ def test_product_path_has_no_cpu_fallback():
     assert "oracle" not in src.replace("never the oracle", "")
     for f in os.listdir(os.path.join(ROOT, "kv_cache_quantization_absmax_b200", "csrc")):
         assert "oracle" not in open(os.path.join(ROOT, "kv_cache_quantization_absmax_b200", "csrc", f)).read()
+
+
+def test_lowbit_rejects_bad_arguments(kvq):
+    L = kvq.lib
+    E, U = kvq.KVQ_ERR_INVALID_ARG, kvq.KVQ_ERR_UNSUPPORTED
+    assert L.kvq_quantize_int4(_p(A16), 1, 4, 128, 48, _p(A16), _p(A16), _p(A16), None) == E  # d % group
+    assert L.kvq_quantize_int4(_p(A16), 1, 4, 128, 16, _p(A16), _p(A16), _p(A16), None) == U  # group size
+    assert L.kvq_quantize_int4(_p(A16 + 8), 1, 4, 128, 32, _p(A16), _p(A16), _p(A16), None) == E
+    assert L.kvq_quantize_int4(None, 1, 0, 128, 32, None, None, None, None) == kvq.KVQ_OK    # no rows
+    assert L.kvq_dequantize_int4(_p(A16), _p(A16), _p(A16), 4, 128, 32, _p(A16 + 4), 0, None) == E
+    assert L.kvq_quantize_int8_channelwise(_p(A16), 1, 2, 10, 96, _p(A16), _p(A16), None) == E  # d % 64
+    assert L.kvq_quantize_int8_channelwise(_p(A16), 1, 2, 0, 128, _p(A16), _p(A16), None) == E  # rows
+    assert L.kvq_quantize_int8_channelwise(_p(A16), 1, 0, 10, 128, _p(A16), _p(A16), None) == kvq.KVQ_OK
+    assert L.kvq_dequantize_int8_channelwise(_p(A16), _p(A16 + 2), 2, 10, 128, _p(A16), 1, None) == E

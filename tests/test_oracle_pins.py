@@ -437,3 +437,86 @@ def test_decode_append_qjl_against_brute_force():
     nrm = np.repeat(n_all.reshape(1, 2, T + 1).astype(np.float64), 2, axis=1)
     sc = math.sqrt(math.pi / 2) / 32 * nrm * np.einsum("bhm,bhtm->bht", v, sgn)
     assert np.allclose(r["scores"], sc, rtol=1e-6, atol=1e-6)
+
+
+# ---- channel-wise INT8 and group-wise INT4 ----
+
+@pytest.mark.parametrize("dtype", [np.float16, np.float32])
+def test_channelwise_int8_is_the_row_rule_on_the_transpose(dtype):
+    """One scale per column of each block = the pinned per-row rule applied to the
+    block's transpose (codes and scales bit for bit; dequantized values too)."""
+    rng = np.random.default_rng(21)
+    x = (rng.standard_normal((3, 37, 24)) * rng.lognormal(0, 1, (3, 1, 24))).astype(dtype)
+    x[1, :, 5] = 0                                   # an all-zero column: scale 0, codes 0
+    codes, scales = oracle.quantize_int8_channelwise(x)
+    deq = oracle.dequantize_int8_channelwise(codes, scales)
+    for b in range(3):
+        c_t, s_t = oracle.quantize_int8(np.ascontiguousarray(x[b].T))
+        assert np.array_equal(codes[b], c_t.T)
+        assert np.array_equal(scales[b].view(np.uint32), s_t.view(np.uint32))
+        assert np.array_equal(deq[b].view(np.uint32), oracle.dequantize_int8(c_t, s_t).T.view(np.uint32))
+    assert np.all(codes[1, :, 5] == 0) and scales[1, 5] == 0
+
+
+def _hex32(h):
+    return np.float32(float.fromhex(h))
+
+
+def test_int4_worked_examples():
+    spec = json.load(open(os.path.join(GOLDEN, "int4_worked_examples.json")))
+    for ex in spec["examples"]:
+        x = np.array([ex["x"]], np.float32)
+        g = ex["group"]
+        packed, s, z = oracle.quantize_int4_group(x, g)
+        assert s[0, 0] == _hex32(ex["scale_hex"]), ex["name"]
+        assert z[0, 0] == np.float32(ex["zero"]), ex["name"]
+        assert list(packed[0]) == ex["packed"], ex["name"]
+        lo, hi = packed[0] & 0xF, packed[0] >> 4
+        assert list(np.stack([lo, hi], 1).reshape(-1)) == ex["codes"], ex["name"]
+        xh = oracle.dequantize_int4_group(packed, s, z, g)[0]
+        want = ([_hex32(h) for h in ex["x_hat_hex"]] if "x_hat_hex" in ex
+                else [np.float32(v) for v in ex["x_hat"]])
+        assert np.array_equal(xh, np.array(want, np.float32)), ex["name"]
+    # the tie case: the exact quotient 1.5 / s4 is below 7.5, the fp32 one is 7.5
+    s4 = float(_hex32("0x1.99999ap-3"))
+    assert Fraction(3, 2) / Fraction(s4) < Fraction(15, 2)
+    assert np.float32(np.float32(1.5) / np.float32(s4)) == np.float32(7.5)
+
+
+@pytest.mark.parametrize("dtype,g", [(np.float16, 32), (np.float32, 64), (np.float16, 128)])
+def test_int4_invariants(dtype, g):
+    rng = np.random.default_rng(31)
+    x = (rng.standard_normal((50, 256)) * 3 + rng.standard_normal((50, 1))).astype(dtype)
+    packed, s, z = oracle.quantize_int4_group(x, g)
+    codes = np.stack([packed & 0xF, packed >> 4], -1).reshape(50, 256)
+    xg = x.astype(np.float64).reshape(50, -1, g)
+    cg = codes.reshape(50, -1, g)
+    # the minimum maps to 0, the maximum to 15, the zero point is the minimum
+    assert np.all(np.take_along_axis(cg, xg.argmin(-1)[..., None], -1) == 0)
+    assert np.all(np.take_along_axis(cg, xg.argmax(-1)[..., None], -1) == 15)
+    assert np.array_equal(z, xg.min(-1).astype(np.float32))
+    # reconstruction error: half a step, plus the fp32 roundings of the quotient and of
+    # the reconstruction (a few ulps of the group's magnitude)
+    xh = oracle.dequantize_int4_group(packed, s, z, g).astype(np.float64).reshape(50, -1, g)
+    mag = np.abs(xg).max(-1, keepdims=True)
+    slack = s.astype(np.float64)[..., None] * 2.0 ** -19 + 4 * mag * 2.0 ** -23
+    assert np.all(np.abs(xh - xg) <= s.astype(np.float64)[..., None] / 2 + slack)
+    # groups are independent: each group quantized as a row of its own
+    p1, s1, z1 = oracle.quantize_int4_group(np.ascontiguousarray(x.reshape(-1, g)), g)
+    assert np.array_equal(p1.reshape(packed.shape), packed)
+    assert np.array_equal(s1.reshape(s.shape), s) and np.array_equal(z1.reshape(z.shape), z)
+
+
+def test_decode_int4_values_against_brute_force():
+    T, g = 9, 4
+    _, q, kc, ks, _, _ = _tiny_cache(T)
+    rng = np.random.default_rng(12)
+    v = rng.standard_normal((1, 2, T, 8)).astype(np.float16)
+    packed, s, z = oracle.quantize_int4_group(v.reshape(-1, 8), g)
+    v4 = (packed.reshape(1, 2, T, 4), s.reshape(1, 2, T, 2), z.reshape(1, 2, T, 2), g)
+    r = oracle.decode_attention(q, k_codes=kc, k_scales=ks, v4=v4)
+    vdeq = oracle.dequantize_int4_group(packed, s, z, g).astype(np.float64).reshape(1, 2, T, 8)
+    kdeq = _fl32_product(kc, ks)
+    sigma = float(np.float32(1.0) / np.sqrt(np.float32(8)))
+    out, _, _ = _brute_force(q, kdeq, vdeq, 4, sigma)
+    assert np.allclose(r["out"], out, rtol=0, atol=1e-5)
