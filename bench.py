@@ -315,6 +315,57 @@ def measure_next_rows(wl, stream, reps=3):
                                   "decode over 4096 (per layer, 32 layers)") if name == "append_int8" else
                                  ("GQA [4, 32q/8kv]: append 1 token to 131071 QJL keys (m = 256) + "
                                   "INT8 V, decode over 131072")}
+    # ---- group-wise INT4 (groups of 32) and channel-wise INT8 over the 7B-shaped cache ----
+    g = 32
+    elems = L * 2 * B * H * T * D
+    v4p = torch.empty((L, 2, B, H, T, D // 2), dtype=torch.uint8, device=wl.cache.device)
+    v4s = torch.empty((L, 2, B, H, T, D // g), dtype=torch.float32, device=wl.cache.device)
+    v4z = torch.empty_like(v4s)
+    cws = torch.empty((L, 2, B, H, D), dtype=torch.float32, device=wl.cache.device)
+
+    def timed(fn, n=reps):
+        with torch.cuda.stream(stream):
+            fn()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(n):
+                fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    def row(name, ms, nbytes, workload):
+        out[name] = {"ms_per_call": round(ms, 4), "GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                     "bytes_per_call": int(nbytes), "workload": workload}
+
+    cache_desc = "7B-shaped cache, 32 L x {K, V} x [8, 32, 4096, 128] fp16"
+    ms = timed(lambda: kvq.kvq_quantize_int4(wl.cache, g, v4p, v4s, v4z, stream=stream))
+    row("int4_quantize", ms, elems * (2 + 0.5) + elems // g * 8, cache_desc + ", groups of 32")
+    ms = timed(lambda: kvq.kvq_dequantize_int4(v4p, v4s, v4z, g, out=wl.deq, stream=stream))
+    row("int4_dequantize", ms, elems * (0.5 + 2) + elems // g * 8, cache_desc + " -> fp16")
+    a4 = [kvq.make_decode_int4v_args(wl.q7[l], k_codes=wl.codes[l, 0], k_scales=wl.scales[l, 0],
+                                     v_packed=v4p[l, 1], v_scales4=v4s[l, 1], v_zeros4=v4z[l, 1],
+                                     v_group=g, out=wl.out7[l], workspace=wl.ws7) for l in range(L)]
+
+    def dec4():
+        for a in a4:
+            st = lib.kvq_decode_attention_int4v(ctypes.byref(a), s)
+            if st != kvq.KVQ_OK:
+                raise kvq.KvqError("kvq_decode_attention_int4v", st)
+    ms = timed(dec4) / L
+    keys = B * H * T
+    row("decode_int8k_int4v", ms, keys * (D + 4 + D // 2 + (D // g) * 8) + B * H * D * 6,
+        "7B-shaped layer: INT8 K + INT4 V (groups of 32) [8, 32, 4096, 128], one decode step per layer")
+    ms = timed(lambda: kvq.kvq_quantize_int8_channelwise(wl.cache, wl.codes, cws, stream=stream))
+    row("int8_channelwise_quantize", ms, elems * 3 + cws.numel() * 4,
+        cache_desc + ", one scale per (layer, K/V, batch, head, channel)")
+    ms = timed(lambda: kvq.kvq_dequantize_int8_channelwise(wl.codes, cws, out=wl.deq, stream=stream))
+    row("int8_channelwise_dequantize", ms, elems * 3 + cws.numel() * 4, cache_desc + " -> fp16")
+    del v4p, v4s, v4z, cws
+
     if kvq.kvq_device_error() != 0:
         raise RuntimeError("device-side error recorded during the widened rows")
     return out

@@ -259,6 +259,30 @@ kvq_status kvq_decode_append(const kvq_decode_append_args* a, kvq_stream_t strea
 size_t kvq_decode_append_workspace_bytes(const kvq_decode_append_args* a);
 
 /*
+ * kvq_decode_attention_int4v -- the decode step of kvq_decode_attention with INT8 keys
+ * and group-wise INT4 values (the layout kvq_quantize_int4 writes; "Q-TensorFormer" model
+ * card, section 6): the value row of token t is x_hat = fl32(fl32(c * s4) + z4) per group,
+ * out = sum_t p_t x_hat_t.  base as for kvq_decode_attention with INT8 keys, except that
+ * base.v_codes / base.v_scales are ignored:
+ *   v_packed  [B][Hkv][T][D/2] bytes (element 2i in bits 0-3), 16-byte aligned;
+ *   v_scales4, v_zeros4  [B][Hkv][T][D/v_group] fp32, 4-byte aligned;
+ *   v_group   32, 64 or 128 (KVQ_ERR_UNSUPPORTED otherwise, and for QJL keys).
+ * Workspace from kvq_decode_int4v_workspace_bytes; results and errors as
+ * kvq_decode_attention (outputs within fp32 reassociation of the definition: the kernel
+ * accumulates sum_t (p_t s4) c + sum_t p_t z4).
+ */
+typedef struct kvq_decode_int4v_args {
+    kvq_decode_args base;
+    const uint8_t* v_packed;
+    const float* v_scales4;
+    const float* v_zeros4;
+    int32_t v_group;
+} kvq_decode_int4v_args;
+
+kvq_status kvq_decode_attention_int4v(const kvq_decode_int4v_args* a, kvq_stream_t stream);
+size_t kvq_decode_int4v_workspace_bytes(const kvq_decode_int4v_args* a);
+
+/*
  * kvq_decode_attention_noalloc -- kvq_decode_attention for callers that cannot
  * allocate device memory and cannot lend a workspace (for example code inside a host
  * engine that has already reserved all device memory through its own allocator, or a

@@ -266,6 +266,45 @@ KVQ_API kvq_status kvq_decode_append(const kvq_decode_append_args* a, kvq_stream
     return from_cuda(kvq::launch_decode(&view, plan, cs(stream), &app));
 }
 
+namespace {
+
+// The decode arguments of an INT4-value call as the shared checks see them (the INT4
+// arrays stand in for the INT8 value arrays, with the same alignment rules).
+kvq_status check_int4v(const kvq_decode_int4v_args* a, kvq_decode_args* view) {
+    if (!a) return KVQ_ERR_INVALID_ARG;
+    *view = a->base;
+    if (view->key_format != KVQ_KEYS_INT8) return KVQ_ERR_UNSUPPORTED;
+    if (view->out) {
+        view->v_codes = reinterpret_cast<const int8_t*>(a->v_packed);
+        view->v_scales = a->v_scales4;
+    }
+    const kvq_status st = check_decode(view);
+    if (st != KVQ_OK || view->batch == 0 || !view->out) return st;
+    if (a->v_group != 32 && a->v_group != 64 && a->v_group != 128) return KVQ_ERR_UNSUPPORTED;
+    if (!a->v_zeros4 || !aligned(a->v_zeros4, 4)) return KVQ_ERR_INVALID_ARG;
+    return KVQ_OK;
+}
+
+}  // namespace
+
+KVQ_API size_t kvq_decode_int4v_workspace_bytes(const kvq_decode_int4v_args* a) {
+    kvq_decode_args view;
+    if (check_int4v(a, &view) != KVQ_OK) return 0;
+    return kvq::plan_decode(&view, kvq::device_sm_count()).total_bytes;
+}
+
+KVQ_API kvq_status kvq_decode_attention_int4v(const kvq_decode_int4v_args* a, kvq_stream_t stream) {
+    kvq_decode_args view;
+    const kvq_status st = check_int4v(a, &view);
+    if (st != KVQ_OK) return st;
+    if (view.batch == 0) return KVQ_OK;
+    const kvq::DecodePlan plan = kvq::plan_decode(&view, kvq::device_sm_count());
+    if (!view.workspace || !aligned(view.workspace, 256) || view.workspace_bytes < plan.total_bytes)
+        return KVQ_ERR_WORKSPACE;
+    const kvq::Int4Values v4{a->v_packed, a->v_scales4, a->v_zeros4, a->v_group};
+    return from_cuda(kvq::launch_decode(&view, plan, cs(stream), nullptr, &v4));
+}
+
 KVQ_API kvq_status kvq_device_error(uint32_t* code) {
     if (!code) return KVQ_ERR_INVALID_ARG;
     uint32_t a = 0, b = 0;

@@ -34,6 +34,7 @@ constexpr int kD = 128;
 constexpr int kRange = 64;                 // CTA ranges are multiples of this many tokens
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kCodeMagic = 12583040.0f;  // 1.5 * 2^23 + 128
+constexpr float kRoundMagic = 12582912.0f; // 1.5 * 2^23
 
 struct DecodeParams {
     const uint16_t* q;
@@ -51,6 +52,10 @@ struct DecodeParams {
     const uint16_t* knew;   // append: new key rows [units][D] fp16, stored at token T - 1
     const uint16_t* vnew;   // append: new value rows [units][D] fp16 (or null)
     const uint16_t* S;      // append with QJL keys: the sketch matrix [m][D] fp16
+    const uint8_t* v4p;     // INT4 values: packed codes [units * cap][D / 2]
+    const float* v4s;       // INT4 values: group scales [units * cap][D / v4g]
+    const float* v4z;       // INT4 values: group zero points
+    int v4g;                // INT4 values: group size (32, 64 or 128)
     int64_t W;              // tokens per CTA range
     int64_t total;          // units * T
     int Hq;
@@ -233,11 +238,15 @@ __device__ __forceinline__ void merge_warps_and_store(const float* red, const De
 // Ring geometry per group size G (measured on B200: for G = 1, two 128-token stages
 // with three CTAs per SM beat four 64-token stages, the per-stage bookkeeping being
 // spread over 4 tokens per lane group instead of 2).
-template <int G>
+template <int G, bool V4 = false>
 struct I8Ring {
     static constexpr int tok = G == 1 ? 128 : 64;             // tokens per stage
     static constexpr int stages = G == 1 ? 2 : 4;
-    static constexpr int bytes = 2 * tok * kD + 2 * tok * 4;  // K rows, V rows, K scales, V scales
+    static constexpr int vrow = V4 ? kD / 2 : kD;             // bytes of a value row
+    static constexpr int v_off = tok * kD;                    // K rows | V rows | K scales | V scales
+    static constexpr int ks_off = v_off + tok * vrow;
+    static constexpr int vs_off = ks_off + tok * 4;
+    static constexpr int bytes = vs_off + tok * 4;
 };
 constexpr int kI8Consumers = 8;                          // consumer warps; warp 8 produces
 constexpr int kI8Threads = 32 * (kI8Consumers + 1);
@@ -250,12 +259,13 @@ enum : unsigned int { kErrI8Producer = 0x201, kErrI8Consumer = 0x202 };
 // need more registers per thread).
 __host__ __device__ constexpr int int8_ctas_per_sm(int G) { return G == 1 ? 3 : (G == 2 ? 2 : 1); }
 
-template <int G>
+template <int G, bool V4>
 __global__ void __launch_bounds__(kI8Threads, int8_ctas_per_sm(G))
 decode_int8_kernel(const DecodeParams p) {
-    constexpr int kI8StageTok = I8Ring<G>::tok;
-    constexpr int kI8Stages = I8Ring<G>::stages;
-    constexpr int kI8StageBytes = I8Ring<G>::bytes;
+    using Ring = I8Ring<G, V4>;
+    constexpr int kI8StageTok = Ring::tok;
+    constexpr int kI8Stages = Ring::stages;
+    constexpr int kI8StageBytes = Ring::bytes;
     static_assert(kI8StageTok % (4 * kI8Consumers) == 0, "each 8-lane group takes whole tokens");
     extern __shared__ __align__(128) unsigned char smem_raw[];
     __shared__ uint64_t bars[2 * kI8Stages + 1];
@@ -320,16 +330,24 @@ decode_int8_kernel(const DecodeParams p) {
                     // Values are copied only when the output is wanted (scores-only calls
                     // pass no value pointers); scales only when their rows start 16-byte
                     // aligned.
-                    const uint32_t per_tensor = n * kD + (p.scales_bulk ? n * 4u : 0u);
-                    dev::mbar_arrive_expect_tx(full_bar(s), (p.want_out ? 2u : 1u) * per_tensor);
+                    // (INT4 values: packed rows here, group scales and zero points loaded by
+                    // the consumers)
+                    const uint32_t k_bytes = n * kD + (p.scales_bulk ? n * 4u : 0u);
+                    const uint32_t v_bytes = !p.want_out ? 0u
+                                             : n * Ring::vrow + ((!V4 && p.scales_bulk) ? n * 4u : 0u);
+                    dev::mbar_arrive_expect_tx(full_bar(s), k_bytes + v_bytes);
                     dev::bulk_g2s(dst, p.kc + (row0 + t) * kD, n * kD, full_bar(s));
-                    if (p.want_out)
-                        dev::bulk_g2s(dst + kI8StageTok * kD, p.vc + (row0 + t) * kD, n * kD, full_bar(s));
+                    if (p.want_out) {
+                        if constexpr (V4)
+                            dev::bulk_g2s(dst + Ring::v_off, p.v4p + (row0 + t) * Ring::vrow, n * Ring::vrow,
+                                          full_bar(s));
+                        else
+                            dev::bulk_g2s(dst + Ring::v_off, p.vc + (row0 + t) * kD, n * kD, full_bar(s));
+                    }
                     if (p.scales_bulk) {
-                        dev::bulk_g2s(dst + 2 * kI8StageTok * kD, p.ks + row0 + t, n * 4u, full_bar(s));
-                        if (p.want_out)
-                            dev::bulk_g2s(dst + 2 * kI8StageTok * kD + kI8StageTok * 4, p.vs + row0 + t,
-                                          n * 4u, full_bar(s));
+                        dev::bulk_g2s(dst + Ring::ks_off, p.ks + row0 + t, n * 4u, full_bar(s));
+                        if (!V4 && p.want_out)
+                            dev::bulk_g2s(dst + Ring::vs_off, p.vs + row0 + t, n * 4u, full_bar(s));
                     }
                     issued[s] = true;
                     ph_issued[s] = ph;
@@ -395,10 +413,12 @@ decode_int8_kernel(const DecodeParams p) {
         }
         float mrun[G], lrun[G];
         uint64_t acc[G][8];
+        float zacc[G];  // INT4 values: sum over tokens of p * zero point (the same for the lane's dims)
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             mrun[g] = -INFINITY;
             lrun[g] = 0.0f;
+            zacc[g] = 0.0f;
 #pragma unroll
             for (int k = 0; k < 8; ++k) acc[g][k] = 0ull;
         }
@@ -408,16 +428,25 @@ decode_int8_kernel(const DecodeParams p) {
             const uint32_t ph = (uint32_t)(i / kI8Stages) & 1u;
             const int tok0 = warp * (4 * U) + tg * U;        // first token of this group in the stage
             bool valid[U];
-            float ksc[U], vsc[U];
+            float ksc[U], vsc[U], vz[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int64_t t = tstage + tok0 + u;
                 valid[u] = t < sg.t1;
+                const int64_t r = row0 + (valid[u] ? t : sg.t0);
                 if (!p.scales_bulk) {
                     // coherent loads: an appended row's scales were stored by this kernel
-                    const int64_t r = row0 + (valid[u] ? t : sg.t0);
                     ksc[u] = __ldcg(p.ks + r);
-                    vsc[u] = p.want_out ? __ldcg(p.vs + r) : 0.0f;
+                    if constexpr (!V4) vsc[u] = p.want_out ? __ldcg(p.vs + r) : 0.0f;
+                }
+                if constexpr (V4) {
+                    // this lane's 16 dims lie in one group (groups of 32, 64 or 128)
+                    const int ng = kD / p.v4g;
+                    const int64_t gi = r * ng + (sub * 16) / p.v4g;
+                    vsc[u] = p.want_out ? __ldcg(p.v4s + gi) : 0.0f;
+                    vz[u] = p.want_out ? __ldcg(p.v4z + gi) : 0.0f;
+                } else {
+                    vz[u] = 0.0f;
                 }
             }
             // After an abort a warp keeps walking the same stages and barriers (so every
@@ -429,13 +458,14 @@ decode_int8_kernel(const DecodeParams p) {
             }
             if (aborted) continue;
             const unsigned char* kst = smem_raw + (size_t)s * kI8StageBytes;
-            const unsigned char* vst = kst + kI8StageTok * kD;
+            const unsigned char* vst = kst + Ring::v_off;
             if (p.scales_bulk) {
-                const float* kss = reinterpret_cast<const float*>(kst + 2 * kI8StageTok * kD);
+                const float* kss = reinterpret_cast<const float*>(kst + Ring::ks_off);
+                const float* vss = reinterpret_cast<const float*>(kst + Ring::vs_off);
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     ksc[u] = kss[tok0 + u];
-                    vsc[u] = p.want_out ? kss[kI8StageTok + tok0 + u] : 0.0f;
+                    if constexpr (!V4) vsc[u] = p.want_out ? vss[tok0 + u] : 0.0f;
                 }
             }
             float score[U][G];
@@ -483,6 +513,7 @@ decode_int8_kernel(const DecodeParams p) {
                     if (mb > mrun[g]) {
                         const float corr = fast_exp2(mrun[g] - mb);
                         lrun[g] *= corr;
+                        if constexpr (V4) zacc[g] *= corr;
                         const uint64_t c2 = pack2(corr, corr);
 #pragma unroll
                         for (int k = 0; k < 8; ++k) acc[g][k] = mul2(acc[g][k], c2);
@@ -492,17 +523,33 @@ decode_int8_kernel(const DecodeParams p) {
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     if (!valid[u]) continue;
-                    const uint4 vv = *reinterpret_cast<const uint4*>(vst + (tok0 + u) * kD + sub * 16);
                     uint64_t c[8];
-                    const uint32_t w4[4] = {vv.x ^ 0x80808080u, vv.y ^ 0x80808080u, vv.z ^ 0x80808080u,
-                                            vv.w ^ 0x80808080u};
+                    if constexpr (V4) {
+                        // 16 nibbles: byte i holds dims 2i (low) and 2i + 1 (high) -> the pairs
+                        const uint2 vv = *reinterpret_cast<const uint2*>(vst + (tok0 + u) * Ring::vrow + sub * 8);
+                        const uint32_t wds[2] = {vv.x, vv.y};
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) codes4(w4[k], c[2 * k], c[2 * k + 1]);
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t lo = wds[h] & 0x0F0F0F0Fu, hi = (wds[h] >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                c[4 * h + k] = add2(pack2(__uint_as_float(__byte_perm(lo, 0x4B400000u, 0x7650u + k)),
+                                                          __uint_as_float(__byte_perm(hi, 0x4B400000u, 0x7650u + k))),
+                                                    pack2(-kRoundMagic, -kRoundMagic));
+                        }
+                    } else {
+                        const uint4 vv = *reinterpret_cast<const uint4*>(vst + (tok0 + u) * kD + sub * 16);
+                        const uint32_t w4[4] = {vv.x ^ 0x80808080u, vv.y ^ 0x80808080u, vv.z ^ 0x80808080u,
+                                                vv.w ^ 0x80808080u};
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) codes4(w4[k], c[2 * k], c[2 * k + 1]);
+                    }
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
                         const float pe = fast_exp2(score[u][g] * p.scale_log2 - mrun[g]);
                         lrun[g] += pe;
                         const float wv = pe * vsc[u];
+                        if constexpr (V4) zacc[g] = __fmaf_rn(pe, vz[u], zacc[g]);
                         const uint64_t w2 = pack2(wv, wv);
 #pragma unroll
                         for (int k = 0; k < 8; ++k) acc[g][k] = fma2(w2, c[k], acc[g][k]);
@@ -515,6 +562,14 @@ decode_int8_kernel(const DecodeParams p) {
         if (!p.want_out) continue;
 
         // ---- end of the unit segment: merge lane groups, then warps, into slot jj ----
+        if constexpr (V4) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const uint64_t z2 = pack2(zacc[g], zacc[g]);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) acc[g][k] = add2(acc[g][k], z2);
+            }
+        }
 #pragma unroll
         for (int off = 8; off <= 16; off <<= 1) {
 #pragma unroll
@@ -884,9 +939,10 @@ decode_combine_kernel(const float* __restrict__ ws, int64_t T, int64_t W, int ma
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-template <int G>
+template <int G, bool V4>
 size_t int8_smem() {
-    return (size_t)I8Ring<G>::stages * I8Ring<G>::bytes + (size_t)kI8Consumers * G * (2 + kD) * sizeof(float);
+    return (size_t)I8Ring<G, V4>::stages * I8Ring<G, V4>::bytes +
+           (size_t)kI8Consumers * G * (2 + kD) * sizeof(float);
 }
 constexpr int kQjlThreads = 512;
 
@@ -899,10 +955,10 @@ size_t qjl_smem() {
     return a > red ? a : red;
 }
 
-template <int G>
+template <int G, bool V4>
 cudaError_t run_int8(const DecodeParams& p, int ctas, cudaStream_t st) {
-    auto kern = decode_int8_kernel<G>;
-    const size_t smem = int8_smem<G>();
+    auto kern = decode_int8_kernel<G, V4>;
+    const size_t smem = int8_smem<G, V4>();
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<ctas, kI8Threads, smem, st>>>(p);
@@ -928,11 +984,20 @@ cudaError_t run_partial(bool qjl, int G, const DecodeParams& p, int ctas, cudaSt
             default: return cudaErrorNotSupported;
         }
     }
+    if (p.v4p != nullptr) {
+        switch (G) {
+            case 1: return run_int8<1, true>(p, ctas, st);
+            case 2: return run_int8<2, true>(p, ctas, st);
+            case 4: return run_int8<4, true>(p, ctas, st);
+            case 8: return run_int8<8, true>(p, ctas, st);
+            default: return cudaErrorNotSupported;
+        }
+    }
     switch (G) {
-        case 1: return run_int8<1>(p, ctas, st);
-        case 2: return run_int8<2>(p, ctas, st);
-        case 4: return run_int8<4>(p, ctas, st);
-        case 8: return run_int8<8>(p, ctas, st);
+        case 1: return run_int8<1, false>(p, ctas, st);
+        case 2: return run_int8<2, false>(p, ctas, st);
+        case 4: return run_int8<4, false>(p, ctas, st);
+        case 8: return run_int8<8, false>(p, ctas, st);
         default: return cudaErrorNotSupported;
     }
 }
@@ -970,7 +1035,7 @@ DecodePlan plan_decode(const kvq_decode_args* a, int sm_count) {
 }
 
 cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaStream_t st,
-                          const AppendSpec* app) {
+                          const AppendSpec* app, const Int4Values* v4) {
     const int G = (int)(a->n_q_heads / a->n_kv_heads);
     const bool qjl = a->key_format == KVQ_KEYS_QJL;
     char* ws = static_cast<char*>(a->workspace);
@@ -990,6 +1055,12 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
     p.knew = app ? app->k_new : nullptr;
     p.vnew = (app && a->out) ? app->v_new : nullptr;
     p.S = a->sketch_f16;
+    if (v4 != nullptr && a->out != nullptr) {
+        p.v4p = v4->packed;
+        p.v4s = v4->scales;
+        p.v4z = v4->zeros;
+        p.v4g = v4->group;
+    }
     p.W = pl.W;
     p.total = pl.units * a->seq_len;
     p.Hq = (int)a->n_q_heads;

@@ -58,7 +58,14 @@ struct AppendSpec {
     const uint16_t* k_new;
     const uint16_t* v_new;  // null: values not appended
 };
+// INT4 values (group-wise, packed): replace a->v_codes / a->v_scales.
+struct Int4Values {
+    const uint8_t* packed;
+    const float* scales;
+    const float* zeros;
+    int group;
+};
 cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& plan, cudaStream_t st,
-                          const AppendSpec* app = nullptr);
+                          const AppendSpec* app = nullptr, const Int4Values* v4 = nullptr);
 
 }  // namespace kvq

@@ -41,6 +41,12 @@ class DecodeAppendArgs(ctypes.Structure):
     _fields_ = [("base", DecodeArgs), ("capacity", _I64), ("k_new_f16", _P), ("v_new_f16", _P)]
 
 
+class DecodeInt4vArgs(ctypes.Structure):
+    """Mirror of ``kvq_decode_int4v_args``."""
+    _fields_ = [("base", DecodeArgs), ("v_packed", _P), ("v_scales4", _P), ("v_zeros4", _P),
+                ("v_group", _I32)]
+
+
 class KvqError(RuntimeError):
     def __init__(self, fn, status):
         self.status = status
@@ -73,6 +79,10 @@ def _load():
     for f in ("kvq_quantize_int8_channelwise", "kvq_dequantize_int8_channelwise", "kvq_quantize_int4",
               "kvq_dequantize_int4"):
         getattr(so, f).restype = ctypes.c_int
+    so.kvq_decode_attention_int4v.argtypes = [ctypes.POINTER(DecodeInt4vArgs), _P]
+    so.kvq_decode_attention_int4v.restype = ctypes.c_int
+    so.kvq_decode_int4v_workspace_bytes.argtypes = [ctypes.POINTER(DecodeInt4vArgs)]
+    so.kvq_decode_int4v_workspace_bytes.restype = ctypes.c_size_t
     so.kvq_decode_append.argtypes = [ctypes.POINTER(DecodeAppendArgs), _P]
     so.kvq_decode_append.restype = ctypes.c_int
     so.kvq_decode_append_workspace_bytes.argtypes = [ctypes.POINTER(DecodeAppendArgs)]
@@ -372,3 +382,38 @@ def kvq_dequantize_int4(packed, scales, zeros, group, out=None, out_dtype=torch.
            lib.kvq_dequantize_int4(packed.data_ptr(), scales.data_ptr(), zeros.data_ptr(), n, d, group,
                                    out.data_ptr(), _dtype_code(out), _stream(stream)))
     return out
+
+
+def make_decode_int4v_args(q, *, k_codes, k_scales, v_packed, v_scales4, v_zeros4, v_group, out=None,
+                           scores_out=None, sm_scale=0.0, workspace=None):
+    """Fill a ``kvq_decode_int4v_args`` (INT8 keys, group-wise INT4 values)."""
+    a = DecodeInt4vArgs()
+    a.base = make_decode_args(q, k_codes=k_codes, k_scales=k_scales, out=out, scores_out=scores_out,
+                              sm_scale=sm_scale, workspace=workspace)
+    a.v_packed = v_packed.data_ptr() if v_packed is not None else None
+    a.v_scales4 = v_scales4.data_ptr() if v_scales4 is not None else None
+    a.v_zeros4 = v_zeros4.data_ptr() if v_zeros4 is not None else None
+    a.v_group = v_group
+    return a
+
+
+def kvq_decode_attention_int4v(q, *, k_codes, k_scales, v_packed, v_scales4, v_zeros4, v_group,
+                               want_scores=False, sm_scale=0.0, workspace=None, out=None,
+                               scores_out=None, stream=None):
+    """Decode step with INT8 keys and group-wise INT4 values; returns (out, scores or None)."""
+    _need_cuda(q, k_codes, k_scales, v_packed, v_scales4, v_zeros4)
+    B, Hq, D = q.shape
+    T = k_codes.shape[2]
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    if want_scores and scores_out is None:
+        scores_out = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    a = make_decode_int4v_args(q, k_codes=k_codes, k_scales=k_scales, v_packed=v_packed,
+                               v_scales4=v_scales4, v_zeros4=v_zeros4, v_group=v_group, out=out,
+                               scores_out=scores_out if want_scores else None, sm_scale=sm_scale)
+    need = int(lib.kvq_decode_int4v_workspace_bytes(ctypes.byref(a)))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    _check("kvq_decode_attention_int4v", lib.kvq_decode_attention_int4v(ctypes.byref(a), _stream(stream)))
+    return out, (scores_out if want_scores else None)

@@ -76,3 +76,50 @@ def test_channelwise_int8_bit_exact(kvq, dtype, nb, rows, d):
         got = to_np(kvq.kvq_dequantize_int8_channelwise(c, s, out_dtype=tod))
         assert np.array_equal(got.view(np.uint16 if od == np.float16 else np.uint32),
                               ref.view(np.uint16 if od == np.float16 else np.uint32))
+
+
+OUT_TOL = 2e-3
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T,g", [(1, 4, 4, 5, 32), (2, 8, 2, 33, 64), (1, 8, 1, 1000, 128),
+                                          (2, 16, 4, 4097, 32), (16, 16, 8, 3, 32), (1, 8, 8, 1501, 32),
+                                          (4, 8, 8, 100, 64)])
+def test_decode_int4_values(kvq, B, Hq, Hkv, T, g):
+    k, v = inputs.lognormal_cache(60 + T, B, Hkv, T, n_tensors=2)
+    q = inputs.gaussian_queries(61 + T, B, Hq)
+    kc, ks = oracle.quantize_int8(k.reshape(-1, 128))
+    vp, vs4, vz4 = oracle.quantize_int4_group(v.reshape(-1, 128), g)
+    shp = (B, Hkv, T)
+    kc, ks = kc.reshape(shp + (128,)), ks.reshape(shp)
+    vp, vs4, vz4 = vp.reshape(shp + (64,)), vs4.reshape(shp + (-1,)), vz4.reshape(shp + (-1,))
+    ref = oracle.decode_attention(q, k_codes=kc, k_scales=ks, v4=(vp, vs4, vz4, g), want_scores=True)
+    qg, kcg, ksg, vpg, vsg, vzg = [torch.from_numpy(np.ascontiguousarray(a)).cuda()
+                                   for a in (q, kc, ks, vp, vs4, vz4)]
+    out, scores = kvq.kvq_decode_attention_int4v(qg, k_codes=kcg, k_scales=ksg, v_packed=vpg,
+                                                 v_scales4=vsg, v_zeros4=vzg, v_group=g, want_scores=True)
+    assert np.abs(to_np(out) - ref["out"]).max() <= OUT_TOL
+    xh = kc.astype(np.float64) * ks.astype(np.float64)[..., None]
+    terms = np.abs(np.repeat(xh, Hq // Hkv, axis=1) * q.astype(np.float64)[:, :, None, :]).sum(-1)
+    assert np.all(np.abs(to_np(scores).astype(np.float64) - ref["scores"]) <= 2 * 128 * 2.0 ** -24 * terms + 1e-30)
+    assert kvq.kvq_device_error() == 0
+
+
+def test_decode_int4_values_7b_layer_sampled(kvq):
+    """One 7B-shaped layer: K INT8 and V INT4 (groups of 32) quantized on the GPU, one
+    decode step; 6 sampled (batch, head) units re-done by the oracle."""
+    B, H, T = 8, 32, 4096
+    kv = inputs.lognormal_cache_device(13, (2, B, H, T, 128), n_sigma_dims=(0, 2, 4), device="cuda")
+    q = inputs.gaussian_queries_device(31, (B, H, 128), "cuda")
+    kc, ks = kvq.kvq_quantize_int8(kv[0])
+    vp, vs4, vz4 = kvq.kvq_quantize_int4(kv[1], 32)
+    out, _ = kvq.kvq_decode_attention_int4v(q, k_codes=kc, k_scales=ks, v_packed=vp, v_scales4=vs4,
+                                            v_zeros4=vz4, v_group=32)
+    out = to_np(out)
+    rng = np.random.default_rng(8)
+    for b, h in zip(rng.integers(0, B, 6), rng.integers(0, H, 6)):
+        kc_r, ks_r = oracle.quantize_int8(to_np(kv[0, b, h]))
+        vp_r, vs_r, vz_r = oracle.quantize_int4_group(to_np(kv[1, b, h]), 32)
+        ref = oracle.decode_attention(to_np(q[b, h])[None, None], k_codes=kc_r[None, None],
+                                      k_scales=ks_r[None, None],
+                                      v4=(vp_r[None, None], vs_r[None, None], vz_r[None, None], 32))
+        assert np.abs(out[b, h] - ref["out"][0, 0]).max() <= OUT_TOL
