@@ -688,6 +688,25 @@ def run_profile_case(case: str, reps: int = 3):
             else:
                 kvq.kvq_decode_attention(q, k_words=words, k_norms=norms, sketch=S, v_codes=vc,
                                          v_scales=vs)
+    elif case in ("int4_quantize", "int4_dequantize", "cw_quantize", "cw_dequantize", "decode_int4v"):
+        kv = inputs.lognormal_cache_device(3, (2, B, H, T, D), n_sigma_dims=(0, 2, 4), device=dev)
+        p4, s4, z4 = kvq.kvq_quantize_int4(kv, 32)
+        cwc, cws = kvq.kvq_quantize_int8_channelwise(kv)
+        out = torch.empty_like(kv)
+        kc, ks = kvq.kvq_quantize_int8(kv[0])
+        q = inputs.gaussian_queries_device(30, (B, H, D), dev)
+        for _ in range(reps):
+            if case == "int4_quantize":
+                kvq.kvq_quantize_int4(kv, 32, p4, s4, z4)
+            elif case == "int4_dequantize":
+                kvq.kvq_dequantize_int4(p4, s4, z4, 32, out=out)
+            elif case == "cw_quantize":
+                kvq.kvq_quantize_int8_channelwise(kv, cwc, cws)
+            elif case == "cw_dequantize":
+                kvq.kvq_dequantize_int8_channelwise(cwc, cws, out=out)
+            else:
+                kvq.kvq_decode_attention_int4v(q, k_codes=kc, k_scales=ks, v_packed=p4[1], v_scales4=s4[1],
+                                               v_zeros4=z4[1], v_group=32)
     else:
         raise SystemExit(f"unknown profile case {case}")
     torch.cuda.synchronize()
@@ -710,7 +729,8 @@ def main(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--profile-case", default=None,
                    help="run one small single-kernel case (quantize, dequantize, decode_int8, "
-                        "qjl_encode, decode_qjl) for an ncu capture, then exit")
+                        "qjl_encode, decode_qjl, int4_quantize, int4_dequantize, cw_quantize, "
+                        "cw_dequantize, decode_int4v) for an ncu capture, then exit")
     args = p.parse_args(argv)
     if args.profile_case:
         return run_profile_case(args.profile_case)

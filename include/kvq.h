@@ -192,7 +192,8 @@ size_t kvq_decode_workspace_bytes(const kvq_decode_args* a);
  *   codes[b][r][j] = clamp(rint_even(fl32(x[b][r][j] / s[b][j])), -128, 127)  (0 if s = 0);
  *   dequantize: out = fl32(codes * s) (fp16 out: that value rounded to nearest even).
  * Bit-identical to that definition.  d must be a multiple of 64, rows >= 1; x, codes,
- * out 16-byte aligned, scales [n_blocks][d] 4-byte aligned (else KVQ_ERR_INVALID_ARG).
+ * out 16-byte aligned, scales [n_blocks][d] 4-byte aligned (else KVQ_ERR_INVALID_ARG);
+ * n_blocks <= 65535 and rows * d < 2^35 (else KVQ_ERR_UNSUPPORTED).
  * n_blocks == 0: no launch.  One launch each; stream-ordered, no synchronisation.
  */
 kvq_status kvq_quantize_int8_channelwise(const void* x, kvq_dtype x_dtype, int64_t n_blocks, int64_t rows,

@@ -180,6 +180,7 @@ KVQ_API kvq_status kvq_dequantize_int8_channelwise(const int8_t* codes, const fl
     if (!valid_dtype(out_dtype) || n_blocks < 0 || rows <= 0 || d <= 0 || d % 64 != 0)
         return KVQ_ERR_INVALID_ARG;
     if (n_blocks == 0) return KVQ_OK;
+    if (n_blocks > 65535 || rows * d >= (int64_t(1) << 35)) return KVQ_ERR_UNSUPPORTED;
     if (!codes || !scales || !out || !aligned(codes, 16) || !aligned(scales, 4) || !aligned(out, 16))
         return KVQ_ERR_INVALID_ARG;
     return from_cuda(kvq::launch_dequantize_int8_channelwise(codes, scales, n_blocks, rows, d, out,

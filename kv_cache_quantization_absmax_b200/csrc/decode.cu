@@ -24,6 +24,7 @@
 #include <stdint.h>
 
 #include "kvq_device.cuh"
+#include "kvq_f32x2.cuh"
 #include "kvq_int8.cuh"
 #include "kvq_internal.h"
 
@@ -56,6 +57,8 @@ struct DecodeParams {
     const float* v4s;       // INT4 values: group scales [units * cap][D / v4g]
     const float* v4z;       // INT4 values: group zero points
     int v4g;                // INT4 values: group size (32, 64 or 128)
+    int v4_bulk;            // INT4 values: groups of 32 with 16-byte aligned parameters ->
+                            // their scales and zero points are staged with the rows
     int64_t W;              // tokens per CTA range
     int64_t total;          // units * T
     int Hq;
@@ -90,32 +93,11 @@ struct RangeWalk {
     }
 };
 
-// ---- packed fp32x2 arithmetic (sm_100): one instruction for two lanes of a pair ----
-__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ float2 unpack2(uint64_t v) {
-    float2 f;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
-    return f;
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
+using x2::add2;
+using x2::fma2;
+using x2::mul2;
+using x2::pack2;
+using x2::unpack2;
 
 // Four int8 codes (one word, each byte biased by 128) -> two exact float pairs.
 __device__ __forceinline__ void codes4(uint32_t biased, uint64_t& c01, uint64_t& c23) {
@@ -243,10 +225,14 @@ struct I8Ring {
     static constexpr int tok = G == 1 ? 128 : 64;             // tokens per stage
     static constexpr int stages = G == 1 ? 2 : 4;
     static constexpr int vrow = V4 ? kD / 2 : kD;             // bytes of a value row
-    static constexpr int v_off = tok * kD;                    // K rows | V rows | K scales | V scales
+    // K rows | V rows | K scales | V scales | (INT4 values in groups of 32: the 4 group
+    // scales, then the 4 zero points of each token)
+    static constexpr int v_off = tok * kD;
     static constexpr int ks_off = v_off + tok * vrow;
     static constexpr int vs_off = ks_off + tok * 4;
-    static constexpr int bytes = vs_off + tok * 4;
+    static constexpr int s4_off = vs_off + tok * 4;
+    static constexpr int z4_off = s4_off + (V4 ? tok * 16 : 0);
+    static constexpr int bytes = z4_off + (V4 ? tok * 16 : 0);
 };
 constexpr int kI8Consumers = 8;                          // consumer warps; warp 8 produces
 constexpr int kI8Threads = 32 * (kI8Consumers + 1);
@@ -332,12 +318,18 @@ decode_int8_kernel(const DecodeParams p) {
                     // aligned.
                     // (INT4 values: packed rows here, group scales and zero points loaded by
                     // the consumers)
+                    const bool g32 = V4 && p.v4_bulk && p.want_out;  // group params staged too
                     const uint32_t k_bytes = n * kD + (p.scales_bulk ? n * 4u : 0u);
                     const uint32_t v_bytes = !p.want_out ? 0u
-                                             : n * Ring::vrow + ((!V4 && p.scales_bulk) ? n * 4u : 0u);
+                                             : n * Ring::vrow + ((!V4 && p.scales_bulk) ? n * 4u : 0u) +
+                                                   (g32 ? 2u * n * 16u : 0u);
                     dev::mbar_arrive_expect_tx(full_bar(s), k_bytes + v_bytes);
                     dev::bulk_g2s(dst, p.kc + (row0 + t) * kD, n * kD, full_bar(s));
                     if (p.want_out) {
+                        if (g32) {
+                            dev::bulk_g2s(dst + Ring::s4_off, p.v4s + (row0 + t) * 4, n * 16u, full_bar(s));
+                            dev::bulk_g2s(dst + Ring::z4_off, p.v4z + (row0 + t) * 4, n * 16u, full_bar(s));
+                        }
                         if constexpr (V4)
                             dev::bulk_g2s(dst + Ring::v_off, p.v4p + (row0 + t) * Ring::vrow, n * Ring::vrow,
                                           full_bar(s));
@@ -440,11 +432,17 @@ decode_int8_kernel(const DecodeParams p) {
                     if constexpr (!V4) vsc[u] = p.want_out ? __ldcg(p.vs + r) : 0.0f;
                 }
                 if constexpr (V4) {
-                    // this lane's 16 dims lie in one group (groups of 32, 64 or 128)
-                    const int ng = kD / p.v4g;
-                    const int64_t gi = r * ng + (sub * 16) / p.v4g;
-                    vsc[u] = p.want_out ? __ldcg(p.v4s + gi) : 0.0f;
-                    vz[u] = p.want_out ? __ldcg(p.v4z + gi) : 0.0f;
+                    // this lane's 16 dims lie in one group (groups of 32, 64 or 128); groups
+                    // of 32 come with the stage, the others are loaded here
+                    if (!p.v4_bulk && p.want_out) {
+                        const int ng = kD / p.v4g;
+                        const int64_t gi = r * ng + (sub * 16) / p.v4g;
+                        vsc[u] = __ldcg(p.v4s + gi);
+                        vz[u] = __ldcg(p.v4z + gi);
+                    } else {
+                        vsc[u] = 0.0f;
+                        vz[u] = 0.0f;
+                    }
                 } else {
                     vz[u] = 0.0f;
                 }
@@ -459,6 +457,17 @@ decode_int8_kernel(const DecodeParams p) {
             if (aborted) continue;
             const unsigned char* kst = smem_raw + (size_t)s * kI8StageBytes;
             const unsigned char* vst = kst + Ring::v_off;
+            if constexpr (V4) {
+                if (p.v4_bulk && p.want_out) {
+                    const float* s4s = reinterpret_cast<const float*>(kst + Ring::s4_off);
+                    const float* z4s = reinterpret_cast<const float*>(kst + Ring::z4_off);
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        vsc[u] = s4s[(tok0 + u) * 4 + (sub >> 1)];
+                        vz[u] = z4s[(tok0 + u) * 4 + (sub >> 1)];
+                    }
+                }
+            }
             if (p.scales_bulk) {
                 const float* kss = reinterpret_cast<const float*>(kst + Ring::ks_off);
                 const float* vss = reinterpret_cast<const float*>(kst + Ring::vs_off);
@@ -1060,6 +1069,8 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
         p.v4s = v4->scales;
         p.v4z = v4->zeros;
         p.v4g = v4->group;
+        p.v4_bulk = v4->group == 32 && reinterpret_cast<uintptr_t>(v4->scales) % 16 == 0 &&
+                    reinterpret_cast<uintptr_t>(v4->zeros) % 16 == 0;
     }
     p.W = pl.W;
     p.total = pl.units * a->seq_len;

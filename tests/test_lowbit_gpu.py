@@ -123,3 +123,25 @@ def test_decode_int4_values_7b_layer_sampled(kvq):
                                       k_scales=ks_r[None, None],
                                       v4=(vp_r[None, None], vs_r[None, None], vz_r[None, None], 32))
         assert np.abs(out[b, h] - ref["out"][0, 0]).max() <= OUT_TOL
+
+
+def test_decode_int4_values_unaligned_group_params(kvq):
+    """Group parameters that are only 4-byte aligned take the direct-load path."""
+    B, Hq, Hkv, T, g = 2, 8, 4, 257, 32
+    k, v = inputs.lognormal_cache(77, B, Hkv, T, n_tensors=2)
+    q = inputs.gaussian_queries(78, B, Hq)
+    kc, ks = oracle.quantize_int8(k.reshape(-1, 128))
+    vp, vs4, vz4 = oracle.quantize_int4_group(v.reshape(-1, 128), g)
+    shp = (B, Hkv, T)
+    ref = oracle.decode_attention(q, k_codes=kc.reshape(shp + (128,)), k_scales=ks.reshape(shp),
+                                  v4=(vp.reshape(shp + (64,)), vs4.reshape(shp + (4,)), vz4.reshape(shp + (4,)), g))
+    # copy the parameters into buffers offset by one float
+    sbuf = torch.zeros(vs4.size + 1, dtype=torch.float32, device="cuda")
+    zbuf = torch.zeros(vz4.size + 1, dtype=torch.float32, device="cuda")
+    sbuf[1:] = torch.from_numpy(vs4.reshape(-1)).cuda()
+    zbuf[1:] = torch.from_numpy(vz4.reshape(-1)).cuda()
+    qg, kcg, ksg, vpg = [torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in
+                         (q, kc.reshape(shp + (128,)), ks.reshape(shp), vp.reshape(shp + (64,)))]
+    out, _ = kvq.kvq_decode_attention_int4v(qg, k_codes=kcg, k_scales=ksg, v_packed=vpg,
+                                            v_scales4=sbuf[1:], v_zeros4=zbuf[1:], v_group=g)
+    assert np.abs(to_np(out) - ref["out"]).max() <= OUT_TOL
