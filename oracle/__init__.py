@@ -300,3 +300,37 @@ def dequantize_int4_group(packed, scales, zeros, g: int, out_dtype=np.float32):
                                              F16 if out_dtype == np.float16 else F32),
            "ora_dequantize_int4_group")
     return out
+
+
+def attention_mass(q_f16, **decode_kwargs):
+    """Attention mass of one decode step ("Q-TensorFormer" model card, section 6,
+    Attention-Sink Dynamic Eviction: sum over heads h of alpha_{h,j}): the oracle's
+    softmax probabilities [B, Hq, T] summed over the query heads -> [B, T] (fp64 sum of
+    the fp32 probabilities)."""
+    r = decode_attention(q_f16, want_out=False, want_probs=True, **decode_kwargs)
+    return r["probs"].astype(np.float64).sum(axis=1)
+
+
+def evict_select(mass, n_sink: int, n_keep: int):
+    """Tokens retained per batch row of mass [B, T] (same section): the first n_sink
+    tokens, plus the n_keep - n_sink tokens of largest mass among the others (equal
+    masses: the smaller token index first); returned in token order, int32 [B, n_keep]."""
+    mass = np.asarray(mass)
+    B, T = mass.shape
+    assert 0 <= n_sink <= n_keep <= T
+    out = np.empty((B, n_keep), np.int32)
+    for b in range(B):
+        rest = np.arange(n_sink, T)
+        # primary key: larger mass first; secondary: smaller index first
+        order = rest[np.lexsort((rest, -mass[b, n_sink:]))]
+        kept = np.concatenate([np.arange(n_sink), order[: n_keep - n_sink]])
+        out[b] = np.sort(kept)
+    return out
+
+
+def gather_rows(cache, kept):
+    """Compaction of a cache [B, H, T, ...] to the kept tokens [B, n_keep] (in order):
+    out[b, h, j] = cache[b, h, kept[b, j]]."""
+    cache = np.asarray(cache)
+    B = cache.shape[0]
+    return np.stack([cache[b][:, kept[b]] for b in range(B)])

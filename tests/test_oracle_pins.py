@@ -520,3 +520,50 @@ def test_decode_int4_values_against_brute_force():
     sigma = float(np.float32(1.0) / np.sqrt(np.float32(8)))
     out, _, _ = _brute_force(q, kdeq, vdeq, 4, sigma)
     assert np.allclose(r["out"], out, rtol=0, atol=1e-5)
+
+
+# ---- attention-sink eviction ----
+
+def test_eviction_worked_examples():
+    spec = json.load(open(os.path.join(GOLDEN, "eviction_example.json")))
+    for ex in spec["examples"]:
+        mass = np.array([ex["mass"]], np.float32)
+        kept = oracle.evict_select(mass, ex["n_sink"], ex["n_keep"])
+        assert list(kept[0]) == ex["kept"], ex["name"]
+
+
+def test_eviction_invariants():
+    rng = np.random.default_rng(41)
+    mass = rng.exponential(1.0, (5, 300)).astype(np.float32)
+    mass[:, 100:110] = mass[:, 100:101]            # runs of equal masses
+    kept = oracle.evict_select(mass, 4, 120)
+    for b in range(5):
+        k = kept[b]
+        assert np.all(np.diff(k) > 0) and list(k[:4]) == [0, 1, 2, 3]
+        evicted = np.setdiff1d(np.arange(4, 300), k)
+        assert mass[b, k[4:]].min() >= mass[b, evicted].max()
+        # at the cut, the kept equal masses are the smallest indices
+        cut = mass[b, k[4:]].min()
+        eq_kept = k[4:][mass[b, k[4:]] == cut]
+        eq_evicted = evicted[mass[b, evicted] == cut]
+        assert eq_evicted.size == 0 or eq_kept.max() < eq_evicted.min()
+
+
+def test_attention_mass_sums_to_heads():
+    """Each query head's probabilities sum to one, so one step's mass sums to Hq."""
+    T = 33
+    _, q, kc, ks, vc, vs = _tiny_cache(T)
+    m = oracle.attention_mass(q, k_codes=kc, k_scales=ks)
+    assert m.shape == (1, T)
+    assert abs(m.sum() - 4) <= 4 * T * 2.0 ** -23
+    # equal logits: every token gets Hq / T
+    m0 = oracle.attention_mass(np.zeros_like(q), k_codes=kc, k_scales=ks)
+    assert np.allclose(m0, 4.0 / T, rtol=1e-6)
+
+
+def test_gather_rows_keeps_order():
+    cache = np.arange(2 * 3 * 8 * 2).reshape(2, 3, 8, 2)
+    kept = np.array([[0, 1, 5], [2, 3, 7]], np.int32)
+    g = oracle.gather_rows(cache, kept)
+    assert g.shape == (2, 3, 3, 2)
+    assert np.array_equal(g[1, 2, 2], cache[1, 2, 7])
