@@ -366,6 +366,54 @@ def measure_next_rows(wl, stream, reps=3):
     row("int8_channelwise_dequantize", ms, elems * 3 + cws.numel() * 4, cache_desc + " -> fp16")
     del v4p, v4s, v4z, cws
 
+    # ---- attention-sink eviction over one 7B-shaped layer: 4 sinks + 2044 of 4096 kept ----
+    n_sink, n_keep = 4, T // 2
+    mass = torch.zeros((B, T), dtype=torch.float32, device=wl.cache.device)
+    am = [kvq.make_decode_mass_args(wl.q7[l], mass, k_codes=wl.codes[l, 0], k_scales=wl.scales[l, 0],
+                                    v_codes=wl.codes[l, 1], v_scales=wl.scales[l, 1], out=wl.out7[l])
+          for l in range(L)]
+    mws = torch.empty(int(lib.kvq_decode_mass_workspace_bytes(ctypes.byref(am[0]))), dtype=torch.uint8,
+                      device=wl.cache.device)
+    for a in am:
+        a.base.workspace, a.base.workspace_bytes = mws.data_ptr(), mws.numel()
+
+    def dec_mass():
+        for a in am:
+            st = lib.kvq_decode_attention_mass(ctypes.byref(a), s)
+            if st != kvq.KVQ_OK:
+                raise kvq.KvqError("kvq_decode_attention_mass", st)
+    ms = timed(dec_mass) / L
+    row("decode_int8_mass", ms, keys * 2 * (D + 4) + B * H * D * 6 + keys * 4 * 2 + B * T * 8,
+        "7B-shaped layer: INT8 K/V [8, 32, 4096, 128] decode step that also adds its attention mass "
+        "(scores written and re-read, [8, 4096] mass updated)")
+    kept = torch.empty((B, n_keep), dtype=torch.int32, device=wl.cache.device)
+    P = ctypes.c_void_p
+
+    def select():  # direct C-ABI call: the Python wrapper's checks would dominate a 10 us launch
+        st = lib.kvq_evict_select(P(mass.data_ptr()), B, T, n_sink, n_keep, P(kept.data_ptr()), s)
+        if st != kvq.KVQ_OK:
+            raise kvq.KvqError("kvq_evict_select", st)
+    ms = timed(select)
+    row("evict_select", ms, B * T * 4 + B * n_keep * 4,
+        "mass [8, 4096] fp32 -> 4 sinks + top 2044 per batch row (int32 [8, 2048])")
+    kdst = torch.empty((2, B, H, n_keep, D), dtype=torch.int8, device=wl.cache.device)
+    sdst = torch.empty((2, B, H, n_keep), dtype=torch.float32, device=wl.cache.device)
+
+    gathers = []
+    for t in range(2):
+        gathers.append((P(wl.codes[0, t].data_ptr()), P(kdst[t].data_ptr()), D))
+        gathers.append((P(wl.scales[0, t].data_ptr()), P(sdst[t].data_ptr()), 4))
+
+    def compact():
+        for src, dst, row_bytes in gathers:
+            st = lib.kvq_gather_rows(src, dst, B, H, T, n_keep, row_bytes, P(kept.data_ptr()), n_keep, s)
+            if st != kvq.KVQ_OK:
+                raise kvq.KvqError("kvq_gather_rows", st)
+    ms = timed(compact)
+    row("evict_compact", ms, 2 * 2 * B * H * n_keep * (D + 4) + 4 * B * n_keep * 4,
+        "7B-shaped layer: INT8 K/V codes + scales [8, 32, 4096] -> the 2048 kept tokens (4 launches)")
+    del mass, mws, kdst, sdst
+
     if kvq.kvq_device_error() != 0:
         raise RuntimeError("device-side error recorded during the widened rows")
     return out

@@ -284,6 +284,66 @@ kvq_status kvq_decode_attention_int4v(const kvq_decode_int4v_args* a, kvq_stream
 size_t kvq_decode_int4v_workspace_bytes(const kvq_decode_int4v_args* a);
 
 /*
+ * Attention-sink eviction ("Q-TensorFormer" model card, section 6, Attention-Sink
+ * Dynamic Eviction): once the context outgrows the memory budget, the cache keeps the
+ * first |K_sink| tokens (the sinks) and the tokens with the largest attention mass,
+ * the probability alpha_{h,i,j} that query head h gave token j at decode step i,
+ * summed over heads and steps.  Three calls make it: a decode step that also adds its
+ * mass to a running sum, the selection of the tokens to keep, and the compaction of
+ * each cache array to them.  Readings: the mass is kept per batch row (summed over
+ * all query heads); equal masses are ordered by the smaller token index; kept tokens
+ * keep their relative order.
+ *
+ * kvq_decode_attention_mass -- kvq_decode_attention (same results) plus
+ *   attn_mass[b][t] += sum_h p[b][h][t],  p[b][h][t] = 2^(s[b][h][t] * sm_scale * log2(e) - M) / L,
+ * s the step's scores, M and L that head's softmax max (log2 domain) and sum.
+ *   base:      as kvq_decode_attention, with base.out required (the merge of the partial
+ *              results yields M and L).  base.scores_out may be NULL: the scores then
+ *              go to the workspace.
+ *   attn_mass: [batch][seq_len] fp32, 4-byte aligned, read and written (start it at 0).
+ * Workspace from kvq_decode_mass_workspace_bytes.  Three launches; errors as
+ * kvq_decode_attention, KVQ_ERR_INVALID_ARG for a missing base.out or attn_mass.
+ */
+typedef struct kvq_decode_mass_args {
+    kvq_decode_args base;
+    float* attn_mass;
+} kvq_decode_mass_args;
+
+kvq_status kvq_decode_attention_mass(const kvq_decode_mass_args* a, kvq_stream_t stream);
+size_t kvq_decode_mass_workspace_bytes(const kvq_decode_mass_args* a);
+
+/*
+ * kvq_evict_select -- the tokens a batch row keeps.
+ *   mass: [batch][seq_len] fp32 (no NaN), device; kept: [batch][n_keep] int32, device,
+ *   written with: tokens 0 .. n_sink-1, then the n_keep - n_sink tokens t >= n_sink of
+ *   largest mass[b][t] (equal values, -0 and +0 included: the smaller t first), all in
+ *   increasing token order.  Exact: the comparison is on the fp32 values.
+ * 0 <= n_sink <= n_keep <= seq_len < 2^31, batch <= 2^31 - 1 (else KVQ_ERR_INVALID_ARG);
+ * mass and kept 4-byte aligned.  batch == 0 or n_keep == 0: no launch.  One launch,
+ * one CTA per batch row.
+ */
+kvq_status kvq_evict_select(const float* mass, int64_t batch, int64_t seq_len, int64_t n_sink, int64_t n_keep,
+                            int32_t* kept, kvq_stream_t stream);
+
+/*
+ * kvq_gather_rows -- compacts one cache array to the kept tokens:
+ *   dst[b][h][j][:] = src[b][h][kept[b][j]][:],  j < n_keep,
+ * src: [batch][n_heads][src_rows][row_bytes] bytes, dst: [batch][n_heads][dst_rows]
+ * [row_bytes] (n_keep <= dst_rows; rows from n_keep on are left as they are), kept:
+ * [batch][n_keep] int32 (as kvq_evict_select writes it).  Works on any per-token array
+ * of the cache: codes (row_bytes = head_dim), per-token scales (4), sign words
+ * (sketch_dim / 8), norms (2), INT4 groups.  src and dst must not overlap (the
+ * compaction is not in place).  A kept index outside [0, src_rows) skips that row and
+ * records code 0x301 for kvq_device_error.
+ * batch, n_heads, n_keep >= 0, row_bytes >= 1, src_rows >= 1 and dst_rows >= n_keep,
+ * n_keep * row_bytes < 2^31 (else KVQ_ERR_INVALID_ARG).  Any alignment (the widest
+ * access that divides row_bytes and both addresses is used).  One launch.
+ */
+kvq_status kvq_gather_rows(const void* src, void* dst, int64_t batch, int64_t n_heads, int64_t src_rows,
+                           int64_t dst_rows, int64_t row_bytes, const int32_t* kept, int64_t n_keep,
+                           kvq_stream_t stream);
+
+/*
  * kvq_decode_attention_noalloc -- kvq_decode_attention for callers that cannot
  * allocate device memory and cannot lend a workspace (for example code inside a host
  * engine that has already reserved all device memory through its own allocator, or a

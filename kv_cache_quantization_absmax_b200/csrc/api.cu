@@ -306,11 +306,86 @@ KVQ_API kvq_status kvq_decode_attention_int4v(const kvq_decode_int4v_args* a, kv
     return from_cuda(kvq::launch_decode(&view, plan, cs(stream), nullptr, &v4));
 }
 
+namespace {
+
+// Workspace of a mass decode: the decode's own, then [B * Hq][2] fp32 final max/sum, then
+// (when the caller passes no scores buffer) the [B][Hq][T] fp32 scores.
+struct MassLayout {
+    kvq::DecodePlan plan;
+    size_t ml_off, scores_off, total;
+};
+
+MassLayout mass_layout(const kvq_decode_args* a) {
+    MassLayout l;
+    l.plan = kvq::plan_decode(a, kvq::device_sm_count());
+    const auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    l.ml_off = up(l.plan.total_bytes);
+    l.scores_off = up(l.ml_off + (size_t)a->batch * a->n_q_heads * 2 * sizeof(float));
+    l.total = l.scores_off + (a->scores_out ? 0 : (size_t)a->batch * a->n_q_heads * a->seq_len * sizeof(float));
+    return l;
+}
+
+kvq_status check_mass(const kvq_decode_mass_args* a) {
+    if (!a) return KVQ_ERR_INVALID_ARG;
+    if (!a->base.out) return KVQ_ERR_INVALID_ARG;
+    const kvq_status st = check_decode(&a->base);
+    if (st != KVQ_OK || a->base.batch == 0) return st;
+    if (!a->attn_mass || !aligned(a->attn_mass, 4)) return KVQ_ERR_INVALID_ARG;
+    return KVQ_OK;
+}
+
+}  // namespace
+
+KVQ_API size_t kvq_decode_mass_workspace_bytes(const kvq_decode_mass_args* a) {
+    if (check_mass(a) != KVQ_OK || a->base.batch == 0) return 0;
+    return mass_layout(&a->base).total;
+}
+
+KVQ_API kvq_status kvq_decode_attention_mass(const kvq_decode_mass_args* a, kvq_stream_t stream) {
+    const kvq_status st = check_mass(a);
+    if (st != KVQ_OK) return st;
+    if (a->base.batch == 0) return KVQ_OK;
+    const MassLayout l = mass_layout(&a->base);
+    if (!a->base.workspace || !aligned(a->base.workspace, 256) || a->base.workspace_bytes < l.total)
+        return KVQ_ERR_WORKSPACE;
+    kvq_decode_args view = a->base;
+    char* ws = static_cast<char*>(a->base.workspace);
+    float* fin_ml = reinterpret_cast<float*>(ws + l.ml_off);
+    if (!view.scores_out) view.scores_out = reinterpret_cast<float*>(ws + l.scores_off);
+    cudaStream_t s = cs(stream);
+    cudaError_t e = kvq::launch_decode(&view, l.plan, s, nullptr, nullptr, fin_ml);
+    if (e != cudaSuccess) return from_cuda(e);
+    return from_cuda(kvq::launch_attention_mass(view.scores_out, fin_ml, view.batch, view.n_q_heads,
+                                                view.seq_len, kvq::decode_scale_log2(&view), a->attn_mass, s));
+}
+
+KVQ_API kvq_status kvq_evict_select(const float* mass, int64_t batch, int64_t seq_len, int64_t n_sink,
+                                    int64_t n_keep, int32_t* kept, kvq_stream_t stream) {
+    if (batch < 0 || batch > INT32_MAX || n_sink < 0 || n_keep < n_sink || seq_len < n_keep || seq_len > INT32_MAX)
+        return KVQ_ERR_INVALID_ARG;
+    if (batch == 0 || n_keep == 0) return KVQ_OK;
+    if (!mass || !kept || !aligned(mass, 4) || !aligned(kept, 4)) return KVQ_ERR_INVALID_ARG;
+    return from_cuda(kvq::launch_evict_select(mass, batch, seq_len, n_sink, n_keep, kept, cs(stream)));
+}
+
+KVQ_API kvq_status kvq_gather_rows(const void* src, void* dst, int64_t batch, int64_t n_heads, int64_t src_rows,
+                                   int64_t dst_rows, int64_t row_bytes, const int32_t* kept, int64_t n_keep,
+                                   kvq_stream_t stream) {
+    if (batch < 0 || n_heads < 0 || n_keep < 0 || row_bytes < 1 || src_rows < 1 || dst_rows < n_keep ||
+        n_keep * row_bytes >= ((int64_t)1 << 31) || n_heads > INT32_MAX)
+        return KVQ_ERR_INVALID_ARG;
+    if (batch == 0 || n_heads == 0 || n_keep == 0) return KVQ_OK;
+    if (!src || !dst || !kept || !aligned(kept, 4)) return KVQ_ERR_INVALID_ARG;
+    return from_cuda(kvq::launch_gather_rows(src, dst, batch, n_heads, src_rows, dst_rows, row_bytes, kept, n_keep,
+                                             cs(stream)));
+}
+
 KVQ_API kvq_status kvq_device_error(uint32_t* code) {
     if (!code) return KVQ_ERR_INVALID_ARG;
-    uint32_t a = 0, b = 0;
+    uint32_t a = 0, b = 0, c = 0;
     if (kvq::read_and_clear_device_error(&a) != cudaSuccess) return KVQ_ERR_CUDA;
     if (kvq::read_and_clear_decode_error(&b) != cudaSuccess) return KVQ_ERR_CUDA;
-    *code = a ? a : b;
+    if (kvq::read_and_clear_evict_error(&c) != cudaSuccess) return KVQ_ERR_CUDA;
+    *code = a ? a : (b ? b : c);
     return KVQ_OK;
 }

@@ -917,7 +917,7 @@ decode_qjl_kernel(const DecodeParams p) {
 // acc_s[d] 2^(m_s - M) / sum_s l_s 2^(m_s - M).
 __global__ void __launch_bounds__(kD)
 decode_combine_kernel(const float* __restrict__ ws, int64_t T, int64_t W, int maxj, int Hq, int Hkv,
-                      float* __restrict__ out) {
+                      float* __restrict__ out, float* __restrict__ fin_ml) {
     // Launched as a programmatic dependent of the decode kernel: nothing is read before
     // that kernel has completed and its partial states are visible.
     dev::griddep_wait();
@@ -944,6 +944,10 @@ decode_combine_kernel(const float* __restrict__ ws, int64_t T, int64_t W, int ma
         a += sl[2 + d] * f;
     }
     out[bh * kD + d] = a / l;
+    if (fin_ml != nullptr && d == 0) {  // the head's final softmax max (log2 domain) and sum
+        fin_ml[2 * bh] = mx;
+        fin_ml[2 * bh + 1] = l;
+    }
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -1043,8 +1047,13 @@ DecodePlan plan_decode(const kvq_decode_args* a, int sm_count) {
     return pl;
 }
 
+float decode_scale_log2(const kvq_decode_args* a) {
+    const float sm = a->sm_scale != 0.0f ? a->sm_scale : 1.0f / sqrtf((float)a->head_dim);
+    return sm * kLog2e;
+}
+
 cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaStream_t st,
-                          const AppendSpec* app, const Int4Values* v4) {
+                          const AppendSpec* app, const Int4Values* v4, float* fin_ml) {
     const int G = (int)(a->n_q_heads / a->n_kv_heads);
     const bool qjl = a->key_format == KVQ_KEYS_QJL;
     char* ws = static_cast<char*>(a->workspace);
@@ -1078,8 +1087,7 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
     p.Hkv = (int)a->n_kv_heads;
     p.maxj = pl.maxj;
     p.m = qjl ? a->sketch_dim : 0;
-    const float sm = a->sm_scale != 0.0f ? a->sm_scale : 1.0f / sqrtf((float)a->head_dim);
-    p.scale_log2 = sm * kLog2e;
+    p.scale_log2 = decode_scale_log2(a);
     p.qjl_c = qjl ? (float)(1.2533141373155002512 / (double)a->sketch_dim) : 0.0f;  // sqrt(pi/2)/m
     p.want_out = a->out != nullptr;
     p.scales_bulk = !qjl && (a->seq_len % 4 == 0) && (p.cap % 4 == 0) &&
@@ -1107,7 +1115,7 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const float* ws_c = p.ws;
-    return cudaLaunchKernelEx(&cfg, decode_combine_kernel, ws_c, p.T, p.W, p.maxj, p.Hq, p.Hkv, a->out);
+    return cudaLaunchKernelEx(&cfg, decode_combine_kernel, ws_c, p.T, p.W, p.maxj, p.Hq, p.Hkv, a->out, fin_ml);
 }
 
 }  // namespace kvq

@@ -65,7 +65,22 @@ struct Int4Values {
     const float* zeros;
     int group;
 };
+// sm_scale * log2(e), the factor the decode kernels apply to a score before exp2.
+float decode_scale_log2(const kvq_decode_args* a);
+// fin_ml (optional, [B * Hq][2]): each query head's final softmax max (log2 domain) and
+// sum, written by the combine kernel (needs a->out).
 cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& plan, cudaStream_t st,
-                          const AppendSpec* app = nullptr, const Int4Values* v4 = nullptr);
+                          const AppendSpec* app = nullptr, const Int4Values* v4 = nullptr,
+                          float* fin_ml = nullptr);
+
+// evict.cu
+cudaError_t launch_attention_mass(const float* scores, const float* fin_ml, int64_t B, int64_t Hq,
+                                  int64_t T, float scale_log2, float* mass, cudaStream_t st);
+cudaError_t launch_evict_select(const float* mass, int64_t B, int64_t T, int64_t n_sink, int64_t n_keep,
+                                int32_t* kept, cudaStream_t st);
+cudaError_t launch_gather_rows(const void* src, void* dst, int64_t B, int64_t H, int64_t src_rows,
+                               int64_t dst_rows, int64_t row_bytes, const int32_t* kept, int64_t n_keep,
+                               cudaStream_t st);
+cudaError_t read_and_clear_evict_error(uint32_t* code);
 
 }  // namespace kvq

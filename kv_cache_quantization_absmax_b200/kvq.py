@@ -47,6 +47,11 @@ class DecodeInt4vArgs(ctypes.Structure):
                 ("v_group", _I32)]
 
 
+class DecodeMassArgs(ctypes.Structure):
+    """Mirror of ``kvq_decode_mass_args``."""
+    _fields_ = [("base", DecodeArgs), ("attn_mass", _P)]
+
+
 class KvqError(RuntimeError):
     def __init__(self, fn, status):
         self.status = status
@@ -87,6 +92,14 @@ def _load():
     so.kvq_decode_append.restype = ctypes.c_int
     so.kvq_decode_append_workspace_bytes.argtypes = [ctypes.POINTER(DecodeAppendArgs)]
     so.kvq_decode_append_workspace_bytes.restype = ctypes.c_size_t
+    so.kvq_decode_attention_mass.argtypes = [ctypes.POINTER(DecodeMassArgs), _P]
+    so.kvq_decode_attention_mass.restype = ctypes.c_int
+    so.kvq_decode_mass_workspace_bytes.argtypes = [ctypes.POINTER(DecodeMassArgs)]
+    so.kvq_decode_mass_workspace_bytes.restype = ctypes.c_size_t
+    so.kvq_evict_select.argtypes = [_P, _I64, _I64, _I64, _I64, _P, _P]
+    so.kvq_evict_select.restype = ctypes.c_int
+    so.kvq_gather_rows.argtypes = [_P, _P, _I64, _I64, _I64, _I64, _I64, _P, _I64, _P]
+    so.kvq_gather_rows.restype = ctypes.c_int
     for f in ("kvq_quantize_int8", "kvq_dequantize_int8", "kvq_int8_scores", "kvq_qjl_encode",
               "kvq_qjl_query_sketch", "kvq_decode_attention", "kvq_device_error"):
         getattr(so, f).restype = ctypes.c_int
@@ -417,3 +430,72 @@ def kvq_decode_attention_int4v(q, *, k_codes, k_scales, v_packed, v_scales4, v_z
     a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel()
     _check("kvq_decode_attention_int4v", lib.kvq_decode_attention_int4v(ctypes.byref(a), _stream(stream)))
     return out, (scores_out if want_scores else None)
+
+
+def make_decode_mass_args(q, attn_mass, *, k_codes=None, k_scales=None, k_words=None, k_norms=None,
+                          sketch=None, v_codes, v_scales, out, scores_out=None, sm_scale=0.0,
+                          workspace=None):
+    """Fill a ``kvq_decode_mass_args``."""
+    a = DecodeMassArgs()
+    a.base = make_decode_args(q, k_codes=k_codes, k_scales=k_scales, k_words=k_words, k_norms=k_norms,
+                              sketch=sketch, v_codes=v_codes, v_scales=v_scales, out=out,
+                              scores_out=scores_out, sm_scale=sm_scale, workspace=workspace)
+    a.attn_mass = attn_mass.data_ptr() if attn_mass is not None else None
+    return a
+
+
+def kvq_decode_attention_mass(q, attn_mass, *, k_codes=None, k_scales=None, k_words=None, k_norms=None,
+                              sketch=None, v_codes, v_scales, want_scores=False, sm_scale=0.0,
+                              workspace=None, out=None, scores_out=None, stream=None):
+    """Decode step that also adds its attention mass (summed over query heads) into
+    ``attn_mass`` [B, T] fp32 in place; returns (out, scores or None)."""
+    _need_cuda(q, attn_mass, k_codes, k_scales, k_words, k_norms, sketch, v_codes, v_scales)
+    B, Hq, D = q.shape
+    ref = k_words if k_words is not None else k_codes
+    T = ref.shape[2]
+    if attn_mass.dtype != torch.float32 or tuple(attn_mass.shape) != (B, T):
+        raise ValueError("attn_mass must be fp32 [batch, seq_len]")
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    if want_scores and scores_out is None:
+        scores_out = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    a = make_decode_mass_args(q, attn_mass, k_codes=k_codes, k_scales=k_scales, k_words=k_words,
+                              k_norms=k_norms, sketch=sketch, v_codes=v_codes, v_scales=v_scales, out=out,
+                              scores_out=scores_out if want_scores else None, sm_scale=sm_scale)
+    need = int(lib.kvq_decode_mass_workspace_bytes(ctypes.byref(a)))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    _check("kvq_decode_attention_mass", lib.kvq_decode_attention_mass(ctypes.byref(a), _stream(stream)))
+    return out, (scores_out if want_scores else None)
+
+
+def kvq_evict_select(mass, n_sink, n_keep, kept=None, stream=None):
+    """Tokens to keep per batch row of ``mass`` [B, T] fp32: int32 [B, n_keep], increasing."""
+    _need_cuda(mass, kept)
+    if mass.dtype != torch.float32 or mass.dim() != 2:
+        raise ValueError("mass must be fp32 [batch, seq_len]")
+    B, T = mass.shape
+    if kept is None:
+        kept = torch.empty((B, max(int(n_keep), 0)), dtype=torch.int32, device=mass.device)
+    _check("kvq_evict_select", lib.kvq_evict_select(_ptr(mass), B, T, int(n_sink), int(n_keep), _ptr(kept),
+                                                    _stream(stream)))
+    return kept
+
+
+def kvq_gather_rows(src, kept, dst=None, stream=None):
+    """Compact ``src`` [B, H, T, ...] to the kept tokens (int32 [B, n_keep]):
+    dst[b, h, j] = src[b, h, kept[b, j]]; ``dst`` [B, H, R >= n_keep, ...] if given."""
+    _need_cuda(src, kept, dst)
+    if kept.dtype != torch.int32:
+        raise ValueError("kept must be int32")
+    B, H, T = src.shape[:3]
+    n_keep = kept.shape[1]
+    row_bytes = src[0, 0, 0].numel() * src.element_size() if src.numel() else 0
+    if dst is None:
+        dst = torch.empty((B, H, n_keep) + tuple(src.shape[3:]), dtype=src.dtype, device=src.device)
+    if dst.dtype != src.dtype or dst.shape[:2] != src.shape[:2] or dst.shape[3:] != src.shape[3:]:
+        raise ValueError("dst must match src except along the token axis")
+    _check("kvq_gather_rows", lib.kvq_gather_rows(_ptr(src), _ptr(dst), B, H, T, dst.shape[2], row_bytes,
+                                                  _ptr(kept), n_keep, _stream(stream)))
+    return dst

@@ -127,3 +127,35 @@ def test_lowbit_rejects_bad_arguments(kvq):
     assert L.kvq_quantize_int8_channelwise(_p(A16), 1, 2, 0, 128, _p(A16), _p(A16), None) == E  # rows
     assert L.kvq_quantize_int8_channelwise(_p(A16), 1, 0, 10, 128, _p(A16), _p(A16), None) == kvq.KVQ_OK
     assert L.kvq_dequantize_int8_channelwise(_p(A16), _p(A16 + 2), 2, 10, 128, _p(A16), 1, None) == E
+
+
+def test_eviction_rejects_bad_arguments(kvq):
+    L = kvq.lib
+    E = kvq.KVQ_ERR_INVALID_ARG
+    sel = L.kvq_evict_select
+    assert sel(_p(A16), 2, 100, 5, 4, _p(A16), None) == E          # n_keep < n_sink
+    assert sel(_p(A16), 2, 100, 0, 101, _p(A16), None) == E        # n_keep > seq_len
+    assert sel(_p(A16), 2, 100, -1, 4, _p(A16), None) == E
+    assert sel(_p(A16), 2, 1 << 31, 4, 8, _p(A16), None) == E      # seq_len >= 2^31
+    assert sel(_p(A16 + 2), 2, 100, 4, 8, _p(A16), None) == E      # misaligned mass
+    assert sel(None, 2, 100, 4, 8, _p(A16), None) == E
+    assert sel(None, 0, 100, 4, 8, None, None) == kvq.KVQ_OK        # no rows
+    assert sel(None, 2, 100, 0, 0, None, None) == kvq.KVQ_OK        # nothing kept
+    g = L.kvq_gather_rows
+    assert g(_p(A16), _p(A16), 2, 4, 100, 10, 0, _p(A16), 10, None) == E          # row_bytes
+    assert g(_p(A16), _p(A16), 2, 4, 100, 9, 128, _p(A16), 10, None) == E         # dst_rows < n_keep
+    assert g(_p(A16), _p(A16), 2, 4, 100, 1 << 25, 128, _p(A16), 1 << 24, None) == E  # too many bytes
+    assert g(_p(A16), _p(A16), 2, 4, 100, 10, 128, _p(A16 + 1), 10, None) == E    # kept alignment
+    assert g(None, _p(A16), 2, 4, 100, 10, 128, _p(A16), 10, None) == E
+    assert g(None, None, 2, 4, 100, 10, 128, None, 0, None) == kvq.KVQ_OK         # nothing kept
+    m = kvq.DecodeMassArgs()
+    m.base = _args(kvq)
+    assert L.kvq_decode_attention_mass(ctypes.byref(m), None) == E   # no attn_mass
+    m.attn_mass = A16 + 2
+    assert L.kvq_decode_attention_mass(ctypes.byref(m), None) == E   # misaligned
+    m.attn_mass = A16
+    m.base = _args(kvq, out=None, scores_out=A16)
+    assert L.kvq_decode_attention_mass(ctypes.byref(m), None) == E   # no output
+    m.base = _args(kvq)
+    assert L.kvq_decode_attention_mass(ctypes.byref(m), None) == kvq.KVQ_ERR_WORKSPACE
+    assert L.kvq_decode_mass_workspace_bytes(ctypes.byref(m)) > L.kvq_decode_workspace_bytes(ctypes.byref(m.base))
