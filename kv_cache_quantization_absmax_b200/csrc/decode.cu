@@ -419,13 +419,13 @@ decode_int8_kernel(const DecodeParams p) {
             const int s = i % kI8Stages;
             const uint32_t ph = (uint32_t)(i / kI8Stages) & 1u;
             const int tok0 = warp * (4 * U) + tg * U;        // first token of this group in the stage
+            const int rem = (int)min((int64_t)kI8StageTok, sg.t1 - tstage);  // tokens of the stage in range
             bool valid[U];
             float ksc[U], vsc[U], vz[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int64_t t = tstage + tok0 + u;
-                valid[u] = t < sg.t1;
-                const int64_t r = row0 + (valid[u] ? t : sg.t0);
+                valid[u] = tok0 + u < rem;
+                const int64_t r = row0 + tstage + (valid[u] ? tok0 + u : 0);
                 if (!p.scales_bulk) {
                     // coherent loads: an appended row's scales were stored by this kernel
                     ksc[u] = __ldcg(p.ks + r);
@@ -469,12 +469,27 @@ decode_int8_kernel(const DecodeParams p) {
                 }
             }
             if (p.scales_bulk) {
-                const float* kss = reinterpret_cast<const float*>(kst + Ring::ks_off);
-                const float* vss = reinterpret_cast<const float*>(kst + Ring::vs_off);
+                // the group's U consecutive scales in one 8- or 16-byte load (tok0 is a
+                // multiple of U and the scale arrays start 16-byte aligned in the stage)
+                const float* kss = reinterpret_cast<const float*>(kst + Ring::ks_off) + tok0;
+                const float* vss = reinterpret_cast<const float*>(kst + Ring::vs_off) + tok0;
+                if constexpr (U == 4) {
+                    const float4 k4 = *reinterpret_cast<const float4*>(kss);
+                    ksc[0] = k4.x, ksc[1] = k4.y, ksc[2] = k4.z, ksc[3] = k4.w;
+                    if constexpr (!V4) {
+                        const float4 v4 = p.want_out ? *reinterpret_cast<const float4*>(vss) : make_float4(0, 0, 0, 0);
+                        vsc[0] = v4.x, vsc[1] = v4.y, vsc[2] = v4.z, vsc[3] = v4.w;
+                    }
+                } else {
 #pragma unroll
-                for (int u = 0; u < U; ++u) {
-                    ksc[u] = kss[tok0 + u];
-                    if constexpr (!V4) vsc[u] = p.want_out ? vss[tok0 + u] : 0.0f;
+                    for (int u = 0; u < U; u += 2) {
+                        const float2 k2 = *reinterpret_cast<const float2*>(kss + u);
+                        ksc[u] = k2.x, ksc[u + 1] = k2.y;
+                        if constexpr (!V4) {
+                            const float2 v2 = p.want_out ? *reinterpret_cast<const float2*>(vss + u) : make_float2(0, 0);
+                            vsc[u] = v2.x, vsc[u + 1] = v2.y;
+                        }
+                    }
                 }
             }
             float score[U][G];
