@@ -755,6 +755,24 @@ def run_profile_case(case: str, reps: int = 3):
             else:
                 kvq.kvq_decode_attention_int4v(q, k_codes=kc, k_scales=ks, v_packed=p4[1], v_scales4=s4[1],
                                                v_zeros4=z4[1], v_group=32)
+    elif case in ("decode_mass", "evict_select", "evict_compact"):
+        kv = inputs.lognormal_cache_device(3, (2, B, H, T, D), n_sigma_dims=(0, 2, 4), device=dev)
+        codes, scales = kvq.kvq_quantize_int8(kv)
+        del kv
+        q = inputs.gaussian_queries_device(30, (B, H, D), dev)
+        mass = torch.zeros((B, T), dtype=torch.float32, device=dev)
+        kvq.kvq_decode_attention_mass(q, mass, k_codes=codes[0], k_scales=scales[0], v_codes=codes[1],
+                                      v_scales=scales[1])
+        kept = kvq.kvq_evict_select(mass, 4, T // 2)
+        dst = torch.empty((B, H, T // 2, D), dtype=torch.int8, device=dev)
+        for _ in range(reps):
+            if case == "decode_mass":
+                kvq.kvq_decode_attention_mass(q, mass, k_codes=codes[0], k_scales=scales[0], v_codes=codes[1],
+                                              v_scales=scales[1])
+            elif case == "evict_select":
+                kvq.kvq_evict_select(mass, 4, T // 2, kept=kept)
+            else:
+                kvq.kvq_gather_rows(codes[0], kept, dst=dst)
     else:
         raise SystemExit(f"unknown profile case {case}")
     torch.cuda.synchronize()
@@ -778,7 +796,8 @@ def main(argv=None):
     p.add_argument("--profile-case", default=None,
                    help="run one small single-kernel case (quantize, dequantize, decode_int8, "
                         "qjl_encode, decode_qjl, int4_quantize, int4_dequantize, cw_quantize, "
-                        "cw_dequantize, decode_int4v) for an ncu capture, then exit")
+                        "cw_dequantize, decode_int4v, decode_mass, evict_select, evict_compact) for an ncu "
+                        "capture, then exit")
     args = p.parse_args(argv)
     if args.profile_case:
         return run_profile_case(args.profile_case)
