@@ -16,7 +16,7 @@ import numpy as np
 from . import build as _build
 
 F32, F16 = 0, 1
-KEYS_INT8, KEYS_QJL = 0, 1
+KEYS_INT8, KEYS_QJL, KEYS_QJLRES = 0, 1, 2
 
 _lib = None
 
@@ -42,7 +42,10 @@ def _load():
         lib.ora_qjl_estimate.restype = ctypes.c_double
         lib.ora_qjl_scores.argtypes = [P, I64, P, P, I64, I32, P]
         lib.ora_decode_attention.argtypes = [I64, I64, I64, I64, I32, P, I32, P, P, P, P, P,
-                                             I32, P, P, P, P, P, I32, ctypes.c_float, P, P, P]
+                                             I32, P, P, P, I32, P, P, P, P, P, I32, ctypes.c_float,
+                                             P, P, P]
+        lib.ora_qjlres_encode.argtypes = [P, I64, I32, I32, P, I32, P, P, P, P, P, P, P]
+        lib.ora_qjlres_encode.restype = I32
         lib.ora_quantize_int8_channelwise.argtypes = [P, I32, I64, I64, I64, P, P]
         lib.ora_dequantize_int8_channelwise.argtypes = [P, P, I64, I64, I64, P, I32]
         lib.ora_quantize_int4_group.argtypes = [P, I32, I64, I64, I32, P, P, P]
@@ -163,16 +166,53 @@ def qjl_scores(v: np.ndarray, words: np.ndarray, norms_f16: np.ndarray):
     return out
 
 
+def qjl_residual_encode(keys_f16: np.ndarray, group: int, S: np.ndarray, want_r: bool = False,
+                        want_u: bool = False):
+    """QJL as the 1-bit residual of group-wise INT4 (the "TurboQuant" news page: a first
+    quantizer, then a 1-bit QJL correction of its residual error).  keys fp16 [n, d];
+    returns a dict: packed uint8 [n, d/2], scales, zeros fp32 [n, d/group] (the INT4
+    stage, as quantize_int4_group), words uint32 [n, m/32] and rnorms fp16 [n] (the QJL
+    sketch of r = fp16(fl32(k - k_hat)), k_hat the INT4 reconstruction), and optionally
+    r fp16 [n, d] and u fp64 [n, m] = S r."""
+    keys = np.ascontiguousarray(keys_f16, np.float16)
+    S64 = np.ascontiguousarray(S, np.float64)
+    n, d = keys.shape
+    m = S64.shape[0]
+    assert S64.shape[1] == d
+    out = dict(packed=np.zeros((n, d // 2), np.uint8), scales=np.empty((n, d // group), np.float32),
+               zeros=np.empty((n, d // group), np.float32), words=np.empty((n, m // 32), np.uint32),
+               rnorms=np.empty((n,), np.float16))
+    r = np.empty((n, d), np.float16) if want_r else None
+    u = np.empty((n, m), np.float64) if want_u else None
+    _check(_load().ora_qjlres_encode(_ptr(keys), n, d, group, _ptr(S64), m, _ptr(out["packed"]),
+                                     _ptr(out["scales"]), _ptr(out["zeros"]), _ptr(out["words"]),
+                                     _ptr(out["rnorms"]), _ptr(r), _ptr(u)), "ora_qjlres_encode")
+    if want_r:
+        out["r"] = r
+    if want_u:
+        out["u"] = u
+    return out
+
+
 def decode_attention(q_f16, *, k_codes=None, k_scales=None, k_words=None, k_norms=None,
-                     S=None, v_codes=None, v_scales=None, v4=None, sm_scale=0.0,
+                     S=None, k4=None, v_codes=None, v_scales=None, v4=None, sm_scale=0.0,
                      want_out=True, want_scores=False, want_probs=False):
     """One decode step.  q [B, Hq, D] fp16; INT8 keys [B, Hkv, T, D] + [B, Hkv, T] or
-    QJL keys words [B, Hkv, T, m/32] + norms [B, Hkv, T] + S [m, D]; INT8 values, or
-    group-wise INT4 values v4 = (packed [B, Hkv, T, D/2], scales, zeros [B, Hkv, T, D/g], g).
+    QJL keys words [B, Hkv, T, m/32] + norms [B, Hkv, T] + S [m, D], or residual keys:
+    k4 = (packed [B, Hkv, T, D/2], scales, zeros [B, Hkv, T, D/g], g) with the residual's
+    words and norms in k_words / k_norms; INT8 values, or group-wise INT4 values
+    v4 = (packed [B, Hkv, T, D/2], scales, zeros [B, Hkv, T, D/g], g).
     Returns a dict with 'out' [B, Hq, D], 'scores' / 'probs' [B, Hq, T] as requested."""
     q = np.ascontiguousarray(q_f16, np.float16)
     B, Hq, D = q.shape
     qjl = k_words is not None
+    k4p = k4s = k4z = None
+    k4g = 0
+    if k4 is not None:
+        k4p = np.ascontiguousarray(k4[0], np.uint8)
+        k4s = np.ascontiguousarray(k4[1], np.float32)
+        k4z = np.ascontiguousarray(k4[2], np.float32)
+        k4g = int(k4[3])
     if qjl:
         k_words = np.ascontiguousarray(k_words, np.uint32)
         k_norms = np.ascontiguousarray(k_norms, np.float16)
@@ -198,9 +238,10 @@ def decode_attention(q_f16, *, k_codes=None, k_scales=None, k_words=None, k_norm
     scores = np.empty((B, Hq, T), np.float32) if want_scores else None
     probs = np.empty((B, Hq, T), np.float32) if want_probs else None
     rc = _load().ora_decode_attention(
-        B, Hq, Hkv, T, D, _ptr(q), KEYS_QJL if qjl else KEYS_INT8,
+        B, Hq, Hkv, T, D, _ptr(q), (KEYS_QJLRES if k4 is not None else KEYS_QJL) if qjl else KEYS_INT8,
         _ptr(k_codes) if not qjl else None, _ptr(k_scales) if not qjl else None,
         _ptr(k_words) if qjl else None, _ptr(k_norms) if qjl else None, _ptr(S64), m,
+        _ptr(k4p), _ptr(k4s), _ptr(k4z), k4g,
         _ptr(v_codes) if (want_out and v4 is None) else None,
         _ptr(v_scales) if (want_out and v4 is None) else None,
         _ptr(v4p), _ptr(v4s), _ptr(v4z), v4g,

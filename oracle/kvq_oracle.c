@@ -25,6 +25,12 @@
  *  [INT4]  "Q-TensorFormer" model card, section 6, Asymmetric Group-Wise INT4 equations:
  *          X_hat = clamp(round((X - z4) / s4), 0, 15) * s4 + z4,
  *          s4 = (max X - min X) / 15,  z4 = min X.
+ *  [RES]   "TurboQuant" news report (ArsTechnica, via amp.my.ua): a first quantizer does
+ *          most of the compression and a 1-bit QJL layer then corrects its residual
+ *          error, one sign bit per sketch coordinate, for better attention scores.  The
+ *          first stage here is [INT4]; the residual is the key minus its INT4
+ *          reconstruction, and the score is the reconstruction's dot product plus the
+ *          [QJL] estimate of the residual's.
  *
  * Readings where the pages are silent (each listed in the design notes):
  *  - granularity is one scale per row of head_dim ("per token");
@@ -50,6 +56,7 @@
 #define ORA_F16 1
 #define ORA_KEYS_INT8 0
 #define ORA_KEYS_QJL 1
+#define ORA_KEYS_QJLRES 2
 
 /* ---------------------------------------------------------------------------------
  * IEEE-754 binary16 <-> binary64, written from the format's definition
@@ -358,16 +365,70 @@ int ora_qjl_scores(const double* v, int64_t n_q, const uint32_t* words,
 }
 
 /* ---------------------------------------------------------------------------------
+ * [RES] encode of keys (fp16, [n_keys][d]) as INT4 groups of g plus the 1-bit QJL sketch
+ * of the residual.  Per key:
+ *   packed, scales, zeros = [INT4] of the key (groups of g);
+ *   k_hat_j = fl32(fl32(c_j * s4) + z4), the INT4 reconstruction;
+ *   r_j     = fp16(fl32(k_j - k_hat_j)), the residual in the key's own precision;
+ *   words, rnorm = [QJL] encode of r (sign bits of S r in fp64; fp16 of the fp64 norm).
+ * r_out_f16 ([n_keys][d]) and u_out ([n_keys][m], the fp64 projections of r) are
+ * optional.
+ * ------------------------------------------------------------------------------- */
+int ora_qjlres_encode(const uint16_t* keys_f16, int64_t n_keys, int d, int g, const double* S, int m,
+                      uint8_t* packed, float* scales, float* zeros, uint32_t* words,
+                      uint16_t* rnorms_f16, uint16_t* r_out_f16, double* u_out) {
+    if (n_keys < 0 || d <= 0 || g <= 0 || (d % g) != 0 || (g % 2) != 0 || (d % 2) != 0) return 1;
+    if (m <= 0 || (m % 32) != 0) return 1;
+    int nw = m / 32, ng = d / g;
+    uint16_t* r16 = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)d);
+    if (!r16) return 2;
+    for (int64_t n = 0; n < n_keys; ++n) {
+        const uint16_t* k = keys_f16 + n * d;
+        uint8_t* pk = packed + n * (d / 2);
+        float* sc = scales + n * ng;
+        float* zr = zeros + n * ng;
+        int rc = ora_quantize_int4_group(k, ORA_F16, 1, d, g, pk, sc, zr);
+        if (rc) { free(r16); return rc; }
+        for (int j = 0; j < d; ++j) {
+            float k_hat = int4_value(pk, sc, zr, 0, d, g, j);
+            float kj = (float)ora_half_to_double(k[j]);
+            float diff = kj - k_hat;
+            r16[j] = ora_double_to_half((double)diff);
+            if (r_out_f16) r_out_f16[n * d + j] = r16[j];
+        }
+        rc = ora_qjl_encode(r16, 1, d, S, m, words + n * nw, rnorms_f16 + n, u_out ? u_out + n * m : NULL);
+        if (rc) { free(r16); return rc; }
+    }
+    free(r16);
+    return 0;
+}
+
+/* [RES] score of a query against key `row` of a residual-format cache:
+ *   sum_j q_j k_hat_j (fp64, the INT4 reconstruction) + the [QJL] estimate with the
+ *   residual's sign bits and stored norm, from the fp32 stored query sketch vst. */
+static double qjlres_score(const float* qf, const uint8_t* packed, const float* s4, const float* z4,
+                           int64_t row, int d, int g, const double* vst, const uint32_t* words,
+                           double rnorm, int m) {
+    double base = 0.0;
+    for (int j = 0; j < d; ++j)
+        base += (double)qf[j] * (double)int4_value(packed, s4, z4, row, d, g, j);
+    return base + ora_qjl_estimate(vst, words + row * (m / 32), rnorm, m);
+}
+
+/* ---------------------------------------------------------------------------------
  * One decode step over a compressed cache.
  *   q:        fp16 [B][Hq][D]
  *   keys:     INT8 codes [B][Hkv][T][D] + fp32 scales [B][Hkv][T], or
- *             QJL words [B][Hkv][T][m/32] + fp16 norms [B][Hkv][T] + sketch S (fp64 m x D)
+ *             QJL words [B][Hkv][T][m/32] + fp16 norms [B][Hkv][T] + sketch S (fp64 m x D), or
+ *             [RES] INT4 codes [B][Hkv][T][D/2] + scales, zeros [B][Hkv][T][D/k_group] and
+ *             the residual's words and fp16 norms (k_words, k_norms_f16) + S
  *   values:   INT8 codes [B][Hkv][T][D] + fp32 scales [B][Hkv][T], or (when v_packed4
  *             is given) [INT4] group-wise codes [B][Hkv][T][D/2] + scales and zeros
  *             [B][Hkv][T][D/v_group], x_hat = fl32(fl32(c * s4) + z4)
  *   [GQA]     query head h reads KV head h / (Hq / Hkv)  (expand along a new group axis
  *             after the KV-head axis, then merge the two axes).
- *   score_t   = INT8: sum_j q_j x_hat_tj (fp32, index order); QJL: the estimator, fp32.
+ *   score_t   = INT8: sum_j q_j x_hat_tj (fp32, index order); QJL: the estimator, fp32;
+ *               RES: qjlres_score, rounded to fp32.
  *   logit_t   = fl32(sm_scale * score_t), sm_scale = fl32(1/sqrt(D)) when 0 is given.
  *   p_t       = expf(logit_t - max logit) / sum_t expf(...), fp32 in token order.
  *   out_j     = sum_t p_t * x_hat_v_tj, fp32 accumulation in token order.
@@ -379,12 +440,16 @@ int ora_decode_attention(int64_t B, int64_t Hq, int64_t Hkv, int64_t T, int D,
                          const int8_t* k_codes, const float* k_scales,
                          const uint32_t* k_words, const uint16_t* k_norms_f16,
                          const double* S, int m,
+                         const uint8_t* k_packed4, const float* k_scales4, const float* k_zeros4,
+                         int k_group,
                          const int8_t* v_codes, const float* v_scales,
                          const uint8_t* v_packed4, const float* v_scales4, const float* v_zeros4,
                          int v_group, float sm_scale,
                          float* out, float* scores_out, float* probs_out) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || T <= 0 || D <= 0 || (Hq % Hkv) != 0) return 1;
-    if (key_format == ORA_KEYS_QJL && (m <= 0 || (m % 32) != 0)) return 1;
+    int sketched = key_format == ORA_KEYS_QJL || key_format == ORA_KEYS_QJLRES;
+    if (sketched && (m <= 0 || (m % 32) != 0)) return 1;
+    if (key_format == ORA_KEYS_QJLRES && (k_group <= 0 || (D % k_group) != 0)) return 1;
     int64_t G = Hq / Hkv;
     int nw = m / 32;
     float sigma = sm_scale != 0.0f ? sm_scale : 1.0f / sqrtf((float)D);
@@ -403,7 +468,7 @@ int ora_decode_attention(int64_t B, int64_t Hq, int64_t Hkv, int64_t T, int D,
             int64_t qo = (b * Hq + h) * D;
             int64_t base = (b * Hkv + kvh) * T;   /* first token row of this KV head */
             for (int j = 0; j < D; ++j) qf[j] = (float)ora_half_to_double(q_f16[qo + j]);
-            if (key_format == ORA_KEYS_QJL) {
+            if (sketched) {
                 for (int i = 0; i < m; ++i) {
                     double v = 0.0;
                     for (int j = 0; j < D; ++j) v += S[(int64_t)i * D + j] * (double)qf[j];
@@ -415,6 +480,9 @@ int ora_decode_attention(int64_t B, int64_t Hq, int64_t Hkv, int64_t T, int D,
                 if (key_format == ORA_KEYS_QJL)
                     score[t] = (float)ora_qjl_estimate(vst, k_words + (base + t) * nw,
                                                        ora_half_to_double(k_norms_f16[base + t]), m);
+                else if (key_format == ORA_KEYS_QJLRES)
+                    score[t] = (float)qjlres_score(qf, k_packed4, k_scales4, k_zeros4, base + t, D, k_group,
+                                                   vst, k_words, ora_half_to_double(k_norms_f16[base + t]), m);
                 else
                     score[t] = int8_row_score(qf, k_codes + (base + t) * D, k_scales[base + t], D);
             }

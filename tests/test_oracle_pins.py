@@ -567,3 +567,95 @@ def test_gather_rows_keeps_order():
     g = oracle.gather_rows(cache, kept)
     assert g.shape == (2, 3, 3, 2)
     assert np.array_equal(g[1, 2, 2], cache[1, 2, 7])
+
+
+# ---- QJL as the 1-bit residual of group-wise INT4 ("TurboQuant" news page) ----
+
+def _grid_keys(n, d=128, g=32, seed=0):
+    """Keys exactly on an INT4 grid: per group z + c * s with s a power of two, codes
+    0..15 and both ends present, all representable in fp16."""
+    rng = np.random.default_rng(seed)
+    keys = np.empty((n, d), np.float64)
+    for r in range(n):
+        for k in range(d // g):
+            z = rng.integers(-64, 64) / 16.0
+            s = 2.0 ** rng.integers(-5, 0)
+            c = rng.integers(0, 16, g)
+            c[rng.integers(0, g)] = 0
+            c[(rng.integers(1, g) + np.argmin(c)) % g] = 15
+            keys[r, k * g:(k + 1) * g] = z + c * s
+    k16 = keys.astype(np.float16)
+    assert np.array_equal(k16.astype(np.float64), keys)
+    return k16
+
+
+def test_qjlres_zero_residual_closed_form():
+    """Keys on the INT4 grid: the residual is exactly 0, its norm is 0, every sign bit is
+    set (bit = [u >= 0]) and the score is the exact dot product <q, k> in fp32."""
+    k = _grid_keys(6)
+    S = inputs.sketch_matrix(256, 128)
+    e = oracle.qjl_residual_encode(k, 32, S, want_r=True)
+    assert not np.any(e["r"].astype(np.float64))
+    assert not np.any(e["rnorms"].astype(np.float64))
+    assert np.all(e["words"] == 0xFFFFFFFF)
+    q = inputs.gaussian_queries(9, 1, 2)
+    k4 = (e["packed"].reshape(1, 1, 6, 64), e["scales"].reshape(1, 1, 6, 4), e["zeros"].reshape(1, 1, 6, 4), 32)
+    r = oracle.decode_attention(q, k4=k4, k_words=e["words"].reshape(1, 1, 6, 8), k_norms=e["rnorms"].reshape(1, 1, 6),
+                                S=S, want_out=False, want_scores=True)
+    exact = (q.astype(np.float64)[0] @ k.astype(np.float64).T).astype(np.float32)
+    assert np.array_equal(r["scores"][0], exact)
+
+
+@pytest.mark.parametrize("g", [32, 64, 128])
+def test_qjlres_decomposition(g):
+    """The INT4 stage is the standalone group-wise INT4 quantizer; k_hat + r reproduces k
+    to within half an fp16 ulp of r; the stored norm is fp16 of numpy's norm of r; the
+    sign bits are those of numpy's S @ r away from zero."""
+    k, = inputs.lognormal_cache(21, 1, 2, 40, n_tensors=1)
+    k = k.reshape(-1, 128)
+    S = inputs.sketch_matrix(256, 128)
+    e = oracle.qjl_residual_encode(k, g, S, want_r=True)
+    p, s, z = oracle.quantize_int4_group(k, g)
+    assert np.array_equal(e["packed"], p) and np.array_equal(e["scales"], s) and np.array_equal(e["zeros"], z)
+    khat = oracle.dequantize_int4_group(p, s, z, g).astype(np.float64)
+    r = e["r"].astype(np.float64)
+    half_ulp = np.spacing(np.abs(e["r"]).astype(np.float16)).astype(np.float64) / 2
+    assert np.all(np.abs(k.astype(np.float64) - khat - r) <= half_ulp + 2.0 ** -24 * np.abs(k.astype(np.float64)))
+    assert np.any(r)
+    assert np.array_equal(e["rnorms"], np.linalg.norm(r, axis=1).astype(np.float16))
+    u = r @ S.astype(np.float64).T
+    bits = ((e["words"][:, :, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(len(k), -1).astype(bool)
+    far = np.abs(u) > 1e-9 * np.linalg.norm(r, axis=1, keepdims=True)
+    assert np.array_equal(bits[far], (u >= 0)[far])
+
+
+def test_qjlres_unbiased_and_tighter_than_plain_qjl():
+    """Over 1000 independent Gaussian sketches the residual score's mean lies within 3
+    standard errors of <q, k_hat + r> (about <q, k>), and its spread is at most
+    1.3 * ||r|| / ||k|| of the plain QJL estimator's on the same sketches."""
+    k, = inputs.lognormal_cache(31, 1, 1, 1, n_tensors=1)
+    k = k.reshape(1, 128)
+    q = inputs.gaussian_queries(41, 1, 1)
+    e0 = oracle.qjl_residual_encode(k, 32, inputs.sketch_matrix(256, 128), want_r=True)
+    khat = oracle.dequantize_int4_group(e0["packed"], e0["scales"], e0["zeros"], 32).astype(np.float64)
+    r = e0["r"].astype(np.float64)
+    target = float(q[0, 0].astype(np.float64) @ (khat[0] + r[0]))
+    exact = float(q[0, 0].astype(np.float64) @ k[0].astype(np.float64))
+    assert abs(target - exact) <= 1e-3 * np.abs(q[0, 0].astype(np.float64) * k[0]).sum()
+    res, plain = [], []
+    for seed in range(20000, 21000):
+        S = inputs.sketch_matrix_f64(256, 128, seed)
+        e = oracle.qjl_residual_encode(k, 32, S)
+        k4 = (e["packed"].reshape(1, 1, 1, 64), e["scales"].reshape(1, 1, 1, 4), e["zeros"].reshape(1, 1, 1, 4), 32)
+        sc = oracle.decode_attention(q, k4=k4, k_words=e["words"].reshape(1, 1, 1, 8),
+                                     k_norms=e["rnorms"].reshape(1, 1, 1), S=S, want_out=False, want_scores=True)
+        res.append(float(sc["scores"][0, 0, 0]))
+        w, n = oracle.qjl_encode(k, S)
+        v64, _ = oracle.qjl_query_sketch(q[0], S)
+        plain.append(oracle.qjl_estimate(v64[0], w[0], float(n[0])))
+    res, plain = np.array(res), np.array(plain)
+    se = res.std(ddof=1) / math.sqrt(len(res))
+    assert abs(res.mean() - target) <= 3 * se, (res.mean(), target, se)
+    ratio = np.linalg.norm(r[0]) / np.linalg.norm(k[0].astype(np.float64))
+    assert ratio < 0.5
+    assert res.std() <= 1.3 * ratio * plain.std(), (res.std(), plain.std(), ratio)
