@@ -414,6 +414,44 @@ def measure_next_rows(wl, stream, reps=3):
         "7B-shaped layer: INT8 K/V codes + scales [8, 32, 4096] -> the 2048 kept tokens (4 launches)")
     del mass, mws, kdst, sdst
 
+    # ---- QJL as the 1-bit residual of group-wise INT4 (groups of 32), GQA cache keys ----
+    dev = wl.cache.device
+    n_keys = gb * gk * gt
+    kshape = (gb, gk, gt)
+    rp = torch.empty(kshape + (D // 2,), dtype=torch.uint8, device=dev)
+    rs = torch.empty(kshape + (D // 32,), dtype=torch.float32, device=dev)
+    rz = torch.empty_like(rs)
+    rr = torch.empty(kshape + (D,), dtype=torch.float16, device=dev)
+    rw = torch.empty(kshape + (m // 32,), dtype=torch.int32, device=dev)
+    rn = torch.empty(kshape, dtype=torch.float16, device=dev)
+    enc_args = [P(wl.gcache[0].data_ptr()), n_keys, D, 32, P(wl.S.data_ptr()), m, P(rp.data_ptr()),
+                P(rs.data_ptr()), P(rz.data_ptr()), P(rr.data_ptr()), P(rw.data_ptr()), P(rn.data_ptr()), s]
+
+    def res_encode():
+        st = lib.kvq_qjl_residual_encode(*enc_args)
+        if st != kvq.KVQ_OK:
+            raise kvq.KvqError("kvq_qjl_residual_encode", st)
+    ms = timed(res_encode)
+    # algorithmic: fp16 keys read; INT4 codes, group scales and zeros, the fp16 residual
+    # (an output), sign words and norms written (the residual's re-read by the sketch
+    # stage is not counted)
+    row("qjlres_encode", ms, n_keys * (2 * D + D // 2 + 8 * (D // 32) + 2 * D + m // 8 + 2),
+        "GQA cache keys [4, 8, 131072, 128] fp16 -> INT4 (groups of 32) + residual sign sketch (m = 256)")
+    ar = kvq.make_decode_qjlres_args(wl.qg, k_packed4=rp, k_scales4=rs, k_zeros4=rz, k_group=32, k_words=rw,
+                                     k_norms=rn, sketch=wl.S, v_codes=wl.vcodes, v_scales=wl.vscales,
+                                     out=wl.outg)
+    rws = torch.empty(int(lib.kvq_decode_qjlres_workspace_bytes(ctypes.byref(ar))), dtype=torch.uint8, device=dev)
+    ar.base.workspace, ar.base.workspace_bytes = rws.data_ptr(), rws.numel()
+
+    def dec_res():
+        st = lib.kvq_decode_attention_qjlres(ctypes.byref(ar), s)
+        if st != kvq.KVQ_OK:
+            raise kvq.KvqError("kvq_decode_attention_qjlres", st)
+    ms = timed(dec_res)
+    row("decode_qjlres", ms, n_keys * (D // 2 + 8 * (D // 32) + m // 8 + 2 + D + 4) + gb * gq * D * (2 + 4) + m * D * 2,
+        "GQA [4, 32q/8kv, 131072]: INT4 keys + residual sign sketch (m = 256) + INT8 V, one fused decode step")
+    del rp, rs, rz, rr, rw, rn, rws
+
     if kvq.kvq_device_error() != 0:
         raise RuntimeError("device-side error recorded during the widened rows")
     return out
@@ -755,6 +793,22 @@ def run_profile_case(case: str, reps: int = 3):
             else:
                 kvq.kvq_decode_attention_int4v(q, k_codes=kc, k_scales=ks, v_packed=p4[1], v_scales4=s4[1],
                                                v_zeros4=z4[1], v_group=32)
+    elif case in ("qjlres_encode", "decode_qjlres"):
+        gb, gq, gk, gt, m = (GQA[k] for k in ("batch", "q_heads", "kv_heads", "seq", "m"))
+        if case == "qjlres_encode":
+            gb = 1
+        kv = inputs.lognormal_cache_device(5, (2, gb, gk, gt, D), n_sigma_dims=(0, 2, 4), device=dev)
+        S = torch.from_numpy(inputs.sketch_matrix(m, D)).to(dev)
+        e = kvq.kvq_qjl_residual_encode(kv[0], 32, S)
+        vc, vs = kvq.kvq_quantize_int8(kv[1])
+        q = inputs.gaussian_queries_device(50, (gb, gq, D), dev)
+        for _ in range(reps):
+            if case == "qjlres_encode":
+                kvq.kvq_qjl_residual_encode(kv[0], 32, S)
+            else:
+                kvq.kvq_decode_attention_qjlres(q, k_packed4=e["packed"], k_scales4=e["scales"],
+                                                k_zeros4=e["zeros"], k_group=32, k_words=e["words"],
+                                                k_norms=e["rnorms"], sketch=S, v_codes=vc, v_scales=vs)
     elif case in ("decode_mass", "evict_select", "evict_compact"):
         kv = inputs.lognormal_cache_device(3, (2, B, H, T, D), n_sigma_dims=(0, 2, 4), device=dev)
         codes, scales = kvq.kvq_quantize_int8(kv)
@@ -796,7 +850,8 @@ def main(argv=None):
     p.add_argument("--profile-case", default=None,
                    help="run one small single-kernel case (quantize, dequantize, decode_int8, "
                         "qjl_encode, decode_qjl, int4_quantize, int4_dequantize, cw_quantize, "
-                        "cw_dequantize, decode_int4v, decode_mass, evict_select, evict_compact) for an ncu "
+                        "cw_dequantize, decode_int4v, decode_mass, evict_select, evict_compact, qjlres_encode, "
+                        "decode_qjlres) for an ncu "
                         "capture, then exit")
     args = p.parse_args(argv)
     if args.profile_case:

@@ -213,14 +213,39 @@ kvq_status kvq_dequantize_int8_channelwise(const int8_t* codes, const float* sca
  *   dequantize: out = fl32(fl32(c * s) + z) (fp16 out: rounded to nearest even).
  * packed: [n_rows][d/2] bytes, element 2i in bits 0-3 and 2i+1 in bits 4-7;
  * scales, zeros: [n_rows][d/group] fp32.  Bit-identical to the definition.  x and out
- * 16-byte aligned, packed 4-byte aligned, scales/zeros 4-byte aligned (else
- * KVQ_ERR_INVALID_ARG); other group sizes KVQ_ERR_UNSUPPORTED.  One launch each.
+ * 16-byte aligned, packed 16-byte aligned (quantize) or 4-byte aligned (dequantize),
+ * scales/zeros 4-byte aligned (else KVQ_ERR_INVALID_ARG); other group sizes
+ * KVQ_ERR_UNSUPPORTED.  One launch each.
  */
 kvq_status kvq_quantize_int4(const void* x, kvq_dtype x_dtype, int64_t n_rows, int64_t d, int32_t group,
                              uint8_t* packed, float* scales, float* zeros, kvq_stream_t stream);
 kvq_status kvq_dequantize_int4(const uint8_t* packed, const float* scales, const float* zeros,
                                int64_t n_rows, int64_t d, int32_t group, void* out, kvq_dtype out_dtype,
                                kvq_stream_t stream);
+
+/*
+ * kvq_qjl_residual_encode -- keys as group-wise INT4 plus a 1-bit QJL sketch of the INT4
+ * residual: a first quantizer takes most of the bits and a 1-bit Johnson-Lindenstrauss
+ * layer corrects its error (the "TurboQuant" news page, "Кризис отменяется: Google
+ * изобрел квантовый алгоритм сокращения объема памяти для ИИ в 6 раз", on its two
+ * stages; the 1-bit stage is the QJL sketch of kvq_qjl_encode, the first stage the
+ * asymmetric group-wise INT4 of kvq_quantize_int4).  Per key k (fp16, d = 128):
+ *   packed, scales, zeros = kvq_quantize_int4 of k (groups of `group`), bit-identical;
+ *   residual_f16 = fp16(fl32(k - k_hat)), k_hat = fl32(fl32(c * s) + z) (the INT4
+ *                  reconstruction), RN; an output, and the input of the sketch stage;
+ *   sign_words, rnorms_f16 = kvq_qjl_encode of the residual rows (bits of S r, fp16 of
+ *                  ||r||), with the same exactness as kvq_qjl_encode.
+ * Scores against such a key (see kvq_decode_attention_qjlres): <q, k_hat> +
+ * sqrt(pi/2)/m * ||r|| * sum_i (S q)_i (2 b_i - 1).
+ * keys, packed, residual_f16 16-byte aligned, scales/zeros 4-byte, sign_words as in
+ * kvq_qjl_encode, rnorms 2-byte (else KVQ_ERR_INVALID_ARG); d and m as kvq_qjl_encode,
+ * group 32/64/128 (else KVQ_ERR_UNSUPPORTED).  Two launches (INT4 + residual, then the
+ * tensor-core sketch); stream-ordered.
+ */
+kvq_status kvq_qjl_residual_encode(const uint16_t* keys_f16, int64_t n_keys, int32_t d, int32_t group,
+                                   const uint16_t* sketch_f16, int32_t m, uint8_t* packed, float* scales,
+                                   float* zeros, uint16_t* residual_f16, uint32_t* sign_words,
+                                   uint16_t* rnorms_f16, kvq_stream_t stream);
 
 /*
  * kvq_decode_append -- one decode step that first appends the newly generated token to
@@ -342,6 +367,34 @@ kvq_status kvq_evict_select(const float* mass, int64_t batch, int64_t seq_len, i
 kvq_status kvq_gather_rows(const void* src, void* dst, int64_t batch, int64_t n_heads, int64_t src_rows,
                            int64_t dst_rows, int64_t row_bytes, const int32_t* kept, int64_t n_keep,
                            kvq_stream_t stream);
+
+/*
+ * kvq_decode_attention_qjlres -- the decode step of kvq_decode_attention over keys
+ * stored by kvq_qjl_residual_encode (group-wise INT4 + the 1-bit QJL sketch of the INT4
+ * residual), INT8 values.  Per cached token t and query head h (KV head h / G):
+ *   score = sum_g s_g * sum_{j in g} q_j c_j + z_g * sum_{j in g} q_j          (<q, k_hat>)
+ *           + sqrt(pi/2)/m * ||r||_fp16 * sum_i (S q)_i (2 b_i - 1),          (residual)
+ * the INT4 part in fp32 in that factored form, the residual part with the fp32 query
+ * sketch (kvq_qjl_query_sketch) through per-CTA byte tables; then softmax and the
+ * INT8-value sum exactly as kvq_decode_attention.
+ *   base:      key_format = KVQ_KEYS_QJL with k_words / k_norms_f16 = the residual's
+ *              sign words and fp16 norms, sketch_f16 / sketch_dim = S and m (128 or
+ *              256, else KVQ_ERR_UNSUPPORTED); everything else as kvq_decode_attention
+ *              (G = Hq / Hkv in {1, 2, 4}).
+ *   k_packed4: [B][Hkv][T][D/2] INT4 codes (16-byte aligned); k_scales4, k_zeros4:
+ *              [B][Hkv][T][D/k_group] fp32 (4-byte aligned); k_group 32, 64 or 128.
+ * Workspace from kvq_decode_qjlres_workspace_bytes.  Errors as kvq_decode_attention.
+ */
+typedef struct kvq_decode_qjlres_args {
+    kvq_decode_args base;
+    const uint8_t* k_packed4;
+    const float* k_scales4;
+    const float* k_zeros4;
+    int32_t k_group;
+} kvq_decode_qjlres_args;
+
+kvq_status kvq_decode_attention_qjlres(const kvq_decode_qjlres_args* a, kvq_stream_t stream);
+size_t kvq_decode_qjlres_workspace_bytes(const kvq_decode_qjlres_args* a);
 
 /*
  * kvq_decode_attention_noalloc -- kvq_decode_attention for callers that cannot

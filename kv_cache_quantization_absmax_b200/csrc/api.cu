@@ -194,11 +194,33 @@ KVQ_API kvq_status kvq_quantize_int4(const void* x, kvq_dtype x_dtype, int64_t n
         return KVQ_ERR_INVALID_ARG;
     if (group != 32 && group != 64 && group != 128) return KVQ_ERR_UNSUPPORTED;
     if (n_rows == 0) return KVQ_OK;
-    if (!x || !packed || !scales || !zeros || !aligned(x, 16) || !aligned(packed, 4) ||
+    if (!x || !packed || !scales || !zeros || !aligned(x, 16) || !aligned(packed, 16) ||
         !aligned(scales, 4) || !aligned(zeros, 4))
         return KVQ_ERR_INVALID_ARG;
     return from_cuda(kvq::launch_quantize_int4(x, x_dtype == KVQ_F16, n_rows, d, group, packed, scales, zeros,
                                                cs(stream)));
+}
+
+KVQ_API kvq_status kvq_qjl_residual_encode(const uint16_t* keys_f16, int64_t n_keys, int32_t d, int32_t group,
+                                           const uint16_t* sketch_f16, int32_t m, uint8_t* packed, float* scales,
+                                           float* zeros, uint16_t* residual_f16, uint32_t* sign_words,
+                                           uint16_t* rnorms_f16, kvq_stream_t stream) {
+    if (n_keys < 0 || d <= 0 || d % 16 != 0 || group <= 0 || d % group != 0 || m <= 0 || m % 32 != 0)
+        return KVQ_ERR_INVALID_ARG;
+    if (group != 32 && group != 64 && group != 128) return KVQ_ERR_UNSUPPORTED;
+    if (!qjl_dims_ok(d, m)) return KVQ_ERR_UNSUPPORTED;
+    if (n_keys == 0) return KVQ_OK;
+    const uintptr_t wa = ((m / 32) % 4 == 0) ? 16 : 4;
+    if (!keys_f16 || !sketch_f16 || !packed || !scales || !zeros || !residual_f16 || !sign_words ||
+        !rnorms_f16 || !aligned(keys_f16, 16) || !aligned(sketch_f16, 16) || !aligned(packed, 16) ||
+        !aligned(scales, 4) || !aligned(zeros, 4) || !aligned(residual_f16, 16) || !aligned(sign_words, wa) ||
+        !aligned(rnorms_f16, 2))
+        return KVQ_ERR_INVALID_ARG;
+    cudaStream_t s = cs(stream);
+    const cudaError_t e = kvq::launch_quantize_int4_residual(keys_f16, n_keys, d, group, packed, scales, zeros,
+                                                             residual_f16, s);
+    if (e != cudaSuccess) return from_cuda(e);
+    return from_cuda(kvq::launch_qjl_encode(residual_f16, n_keys, sketch_f16, m, sign_words, rnorms_f16, s));
 }
 
 KVQ_API kvq_status kvq_dequantize_int4(const uint8_t* packed, const float* scales, const float* zeros,
@@ -378,6 +400,42 @@ KVQ_API kvq_status kvq_gather_rows(const void* src, void* dst, int64_t batch, in
     if (!src || !dst || !kept || !aligned(kept, 4)) return KVQ_ERR_INVALID_ARG;
     return from_cuda(kvq::launch_gather_rows(src, dst, batch, n_heads, src_rows, dst_rows, row_bytes, kept, n_keep,
                                              cs(stream)));
+}
+
+namespace {
+
+// Residual keys: the decode arguments carry the residual's sign words, norms and the
+// sketch as QJL keys; the INT4 stage comes in the extra fields.
+kvq_status check_qjlres(const kvq_decode_qjlres_args* a) {
+    if (!a) return KVQ_ERR_INVALID_ARG;
+    if (a->base.key_format != KVQ_KEYS_QJL) return KVQ_ERR_INVALID_ARG;
+    const kvq_status st = check_decode(&a->base);
+    if (st != KVQ_OK) return st;
+    if (a->k_group != 32 && a->k_group != 64 && a->k_group != 128) return KVQ_ERR_UNSUPPORTED;
+    if (a->base.sketch_dim != 128 && a->base.sketch_dim != 256) return KVQ_ERR_UNSUPPORTED;
+    if (a->base.batch == 0) return KVQ_OK;
+    if (!a->k_packed4 || !a->k_scales4 || !a->k_zeros4 || !aligned(a->k_packed4, 16) ||
+        !aligned(a->k_scales4, 4) || !aligned(a->k_zeros4, 4) || !aligned(a->base.k_words, 16))
+        return KVQ_ERR_INVALID_ARG;
+    return KVQ_OK;
+}
+
+}  // namespace
+
+KVQ_API size_t kvq_decode_qjlres_workspace_bytes(const kvq_decode_qjlres_args* a) {
+    if (check_qjlres(a) != KVQ_OK || a->base.batch == 0) return 0;
+    return kvq::plan_decode(&a->base, kvq::device_sm_count(), true).total_bytes;
+}
+
+KVQ_API kvq_status kvq_decode_attention_qjlres(const kvq_decode_qjlres_args* a, kvq_stream_t stream) {
+    const kvq_status st = check_qjlres(a);
+    if (st != KVQ_OK) return st;
+    if (a->base.batch == 0) return KVQ_OK;
+    const kvq::DecodePlan plan = kvq::plan_decode(&a->base, kvq::device_sm_count(), true);
+    if (!a->base.workspace || !aligned(a->base.workspace, 256) || a->base.workspace_bytes < plan.total_bytes)
+        return KVQ_ERR_WORKSPACE;
+    const kvq::Int4Keys k4{a->k_packed4, a->k_scales4, a->k_zeros4, a->k_group};
+    return from_cuda(kvq::launch_decode(&a->base, plan, cs(stream), nullptr, nullptr, nullptr, &k4));
 }
 
 KVQ_API kvq_status kvq_device_error(uint32_t* code) {

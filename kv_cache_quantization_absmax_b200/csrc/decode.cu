@@ -59,6 +59,12 @@ struct DecodeParams {
     int v4g;                // INT4 values: group size (32, 64 or 128)
     int v4_bulk;            // INT4 values: groups of 32 with 16-byte aligned parameters ->
                             // their scales and zero points are staged with the rows
+    const uint8_t* k4p;     // residual keys: INT4 codes [units * cap][D / 2]
+    const float* k4s;       // residual keys: group scales [units * cap][D / k4g]
+    const float* k4z;       // residual keys: group zero points
+    int k4_ng_shift;        // residual keys: log2(D / k4g)
+    int k4_g_shift;         // residual keys: log2(k4g)
+    int k4_bulk;            // residual keys: group parameters and norms staged with the rows
     int64_t W;              // tokens per CTA range
     int64_t total;          // units * T
     int Hq;
@@ -220,19 +226,25 @@ __device__ __forceinline__ void merge_warps_and_store(const float* red, const De
 // Ring geometry per group size G (measured on B200: for G = 1, two 128-token stages
 // with three CTAs per SM beat four 64-token stages, the per-stage bookkeeping being
 // spread over 4 tokens per lane group instead of 2).
-template <int G, bool V4 = false>
+template <int G, bool V4 = false, bool RES = false>
 struct I8Ring {
     static constexpr int tok = G == 1 ? 128 : 64;             // tokens per stage
     static constexpr int stages = G == 1 ? 2 : 4;
     static constexpr int vrow = V4 ? kD / 2 : kD;             // bytes of a value row
-    // K rows | V rows | K scales | V scales | (INT4 values in groups of 32: the 4 group
-    // scales, then the 4 zero points of each token)
-    static constexpr int v_off = tok * kD;
+    static constexpr int krow = RES ? kD / 2 : kD;            // bytes of a key row (INT4 or INT8)
+    static constexpr int kside = RES ? 32 : 4;                // per-token key side data: residual
+                                                              // sign words (m <= 256) or the scale
+    // K rows | V rows | K scales (residual keys: sign words) | V scales | (INT4 values in
+    // groups of 32: the 4 group scales, then the 4 zero points of each token)
+    static constexpr int v_off = tok * krow;
     static constexpr int ks_off = v_off + tok * vrow;
-    static constexpr int vs_off = ks_off + tok * 4;
+    static constexpr int vs_off = ks_off + tok * kside;
     static constexpr int s4_off = vs_off + tok * 4;
-    static constexpr int z4_off = s4_off + (V4 ? tok * 16 : 0);
-    static constexpr int bytes = z4_off + (V4 ? tok * 16 : 0);
+    static constexpr int z4_off = s4_off + ((V4 || RES) ? tok * 16 : 0);
+    // residual keys: the key group scales and zero points (up to 16 B each per token)
+    // at s4_off / z4_off, then the fp16 residual norms
+    static constexpr int rn_off = z4_off + ((V4 || RES) ? tok * 16 : 0);
+    static constexpr int bytes = rn_off + (RES ? tok * 2 : 0);
 };
 constexpr int kI8Consumers = 8;                          // consumer warps; warp 8 produces
 constexpr int kI8Threads = 32 * (kI8Consumers + 1);
@@ -242,13 +254,61 @@ __device__ unsigned int g_decode_error = 0;
 enum : unsigned int { kErrI8Producer = 0x201, kErrI8Consumer = 0x202 };
 
 // Resident INT8 CTAs per SM the register budget is shaped for (more heads per group
-// need more registers per thread).
-__host__ __device__ constexpr int int8_ctas_per_sm(int G) { return G == 1 ? 3 : (G == 2 ? 2 : 1); }
+// need more registers per thread).  Residual keys: one (the byte tables take 128 KB).
+__host__ __device__ constexpr int int8_ctas_per_sm(int G, bool res = false) {
+    return res ? 1 : (G == 1 ? 3 : (G == 2 ? 2 : 1));
+}
 
-template <int G, bool V4>
-__global__ void __launch_bounds__(kI8Threads, int8_ctas_per_sm(G))
+// Residual keys: the byte tables of the sign-sketch estimator (the layout of the QJL
+// decode kernel's tables, described there): entry (pos, b) holds, for each of the G
+// heads, sum_{k<8} v[8 pos + k] * (bit k of b ? +1 : -1), at byte offset
+// (pos / 16) * 64 KB + b * 256 + (pos % 16) * 16.  Built by `nthr` threads.
+template <int G>
+__device__ __forceinline__ void build_sign_tables(float* lut, const float* v, int m, int64_t vstride, int tid,
+                                                  int nthr) {
+    constexpr int HALF_FLOATS = 256 * 16 * 4;
+    const int npos = m / 8;
+    for (int item = tid; item < 512; item += nthr) {
+        const int pos = item & 31;
+        const int c = item >> 5;                       // high nibble of the byte value
+        float vv[G][8];
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) vv[g][k] = pos < npos ? __ldg(v + g * vstride + pos * 8 + k) : 0.0f;
+        float val[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float sacc = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sacc -= vv[g][k];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) sacc += ((c >> k) & 1) ? vv[g][4 + k] : -vv[g][4 + k];
+            val[g] = sacc;
+        }
+        float* base = lut + (pos >> 4) * HALF_FLOATS + (c * 16 * 16 + (pos & 15)) * 4;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int gray = i ^ (i >> 1);
+            if (i > 0) {
+                const int k = __ffs(i) - 1;           // the bit that flips at step i
+                const bool on = (gray >> k) & 1;
+#pragma unroll
+                for (int g = 0; g < G; ++g) val[g] += on ? 2.0f * vv[g][k] : -2.0f * vv[g][k];
+            }
+            *reinterpret_cast<float4*>(base + gray * 16 * 4) =
+                make_float4(val[0], G > 1 ? val[G > 1 ? 1 : 0] : 0.0f, G > 2 ? val[G > 2 ? 2 : 0] : 0.0f,
+                            G > 3 ? val[G > 3 ? 3 : 0] : 0.0f);
+        }
+    }
+}
+constexpr int kSignTableBytes = 2 * 256 * 16 * 16;      // 128 KB
+
+template <int G, bool V4, bool RES = false>
+__global__ void __launch_bounds__(kI8Threads, int8_ctas_per_sm(G, RES))
 decode_int8_kernel(const DecodeParams p) {
-    using Ring = I8Ring<G, V4>;
+    static_assert(!(RES && V4), "residual keys come with INT8 values");
+    using Ring = I8Ring<G, V4, RES>;
     constexpr int kI8StageTok = Ring::tok;
     constexpr int kI8Stages = Ring::stages;
     constexpr int kI8StageBytes = Ring::bytes;
@@ -265,6 +325,7 @@ decode_int8_kernel(const DecodeParams p) {
     const int nseg = walk.count();
     const uint32_t ring = dev::smem_u32(smem_raw);
     float* red = reinterpret_cast<float*>(smem_raw + kI8Stages * kI8StageBytes);  // [warps][G][2+D]
+    float* lut = red + kI8Consumers * G * (2 + kD);                                 // residual keys
     const uint32_t bar0 = dev::smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (kI8Stages + s); };
@@ -319,12 +380,29 @@ decode_int8_kernel(const DecodeParams p) {
                     // (INT4 values: packed rows here, group scales and zero points loaded by
                     // the consumers)
                     const bool g32 = V4 && p.v4_bulk && p.want_out;  // group params staged too
-                    const uint32_t k_bytes = n * kD + (p.scales_bulk ? n * 4u : 0u);
+                    const uint32_t wrow = (uint32_t)p.m / 8u;        // residual keys: sign bytes per token
+                    const uint32_t gpb = 4u << (RES ? p.k4_ng_shift : 0);   // group parameter bytes per token
+                    const uint32_t k_bytes = RES ? n * (uint32_t)Ring::krow + n * wrow +
+                                                       (p.k4_bulk ? n * (2u * gpb + 2u) : 0u)
+                                                 : n * kD + (p.scales_bulk ? n * 4u : 0u);
                     const uint32_t v_bytes = !p.want_out ? 0u
                                              : n * Ring::vrow + ((!V4 && p.scales_bulk) ? n * 4u : 0u) +
                                                    (g32 ? 2u * n * 16u : 0u);
                     dev::mbar_arrive_expect_tx(full_bar(s), k_bytes + v_bytes);
-                    dev::bulk_g2s(dst, p.kc + (row0 + t) * kD, n * kD, full_bar(s));
+                    if constexpr (RES) {
+                        dev::bulk_g2s(dst, p.k4p + (row0 + t) * Ring::krow, n * Ring::krow, full_bar(s));
+                        dev::bulk_g2s(dst + Ring::ks_off, reinterpret_cast<const unsigned char*>(p.kw) + (row0 + t) * wrow,
+                                      n * wrow, full_bar(s));
+                        if (p.k4_bulk) {
+                            dev::bulk_g2s(dst + Ring::s4_off, reinterpret_cast<const unsigned char*>(p.k4s) + (row0 + t) * gpb,
+                                          n * gpb, full_bar(s));
+                            dev::bulk_g2s(dst + Ring::z4_off, reinterpret_cast<const unsigned char*>(p.k4z) + (row0 + t) * gpb,
+                                          n * gpb, full_bar(s));
+                            dev::bulk_g2s(dst + Ring::rn_off, p.kn + row0 + t, n * 2u, full_bar(s));
+                        }
+                    } else {
+                        dev::bulk_g2s(dst, p.kc + (row0 + t) * kD, n * kD, full_bar(s));
+                    }
                     if (p.want_out) {
                         if (g32) {
                             dev::bulk_g2s(dst + Ring::s4_off, p.v4s + (row0 + t) * 4, n * 16u, full_bar(s));
@@ -337,7 +415,7 @@ decode_int8_kernel(const DecodeParams p) {
                             dev::bulk_g2s(dst + Ring::v_off, p.vc + (row0 + t) * kD, n * kD, full_bar(s));
                     }
                     if (p.scales_bulk) {
-                        dev::bulk_g2s(dst + Ring::ks_off, p.ks + row0 + t, n * 4u, full_bar(s));
+                        if constexpr (!RES) dev::bulk_g2s(dst + Ring::ks_off, p.ks + row0 + t, n * 4u, full_bar(s));
                         if (!V4 && p.want_out)
                             dev::bulk_g2s(dst + Ring::vs_off, p.vs + row0 + t, n * 4u, full_bar(s));
                     }
@@ -403,6 +481,25 @@ decode_int8_kernel(const DecodeParams p) {
                 qp[g][4 + k] = pack2(f1.x, f1.y);
             }
         }
+        float qsum[G];  // residual keys: the sum of the lane's 16 query values, per head
+        if constexpr (RES) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float a = 0.0f;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const float2 q2 = unpack2(qp[g][k]);
+                    a += q2.x + q2.y;
+                }
+                qsum[g] = a;
+            }
+            // the unit's sign tables, from its heads' query sketches (the barrier before
+            // the build: every consumer is done with the previous unit's tables)
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * kI8Consumers) : "memory");
+            build_sign_tables<G>(lut, p.sketch_v + (b * p.Hq + (int64_t)kvh * G) * p.m, p.m, p.m, threadIdx.x,
+                                 32 * kI8Consumers);
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * kI8Consumers) : "memory");
+        }
         float mrun[G], lrun[G];
         uint64_t acc[G][8];
         float zacc[G];  // INT4 values: sum over tokens of p * zero point (the same for the lane's dims)
@@ -422,13 +519,22 @@ decode_int8_kernel(const DecodeParams p) {
             const int rem = (int)min((int64_t)kI8StageTok, sg.t1 - tstage);  // tokens of the stage in range
             bool valid[U];
             float ksc[U], vsc[U], vz[U];
+            float k4sc[U], k4zc[U], rnrm[U];   // residual keys: group scale, zero point, residual norm
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 valid[u] = tok0 + u < rem;
                 const int64_t r = row0 + tstage + (valid[u] ? tok0 + u : 0);
+                if constexpr (RES) {
+                    if (!p.k4_bulk) {
+                        const int64_t gi = (r << p.k4_ng_shift) + ((sub * 16) >> p.k4_g_shift);
+                        k4sc[u] = __ldg(p.k4s + gi);
+                        k4zc[u] = __ldg(p.k4z + gi);
+                        rnrm[u] = __half2float(__ushort_as_half(__ldg(p.kn + r)));
+                    }
+                }
                 if (!p.scales_bulk) {
                     // coherent loads: an appended row's scales were stored by this kernel
-                    ksc[u] = __ldcg(p.ks + r);
+                    if constexpr (!RES) ksc[u] = __ldcg(p.ks + r);
                     if constexpr (!V4) vsc[u] = p.want_out ? __ldcg(p.vs + r) : 0.0f;
                 }
                 if constexpr (V4) {
@@ -457,6 +563,21 @@ decode_int8_kernel(const DecodeParams p) {
             if (aborted) continue;
             const unsigned char* kst = smem_raw + (size_t)s * kI8StageBytes;
             const unsigned char* vst = kst + Ring::v_off;
+            if constexpr (RES) {
+                if (p.k4_bulk) {
+                    const float* s4s = reinterpret_cast<const float*>(kst + Ring::s4_off);
+                    const float* z4s = reinterpret_cast<const float*>(kst + Ring::z4_off);
+                    const __half* rns = reinterpret_cast<const __half*>(kst + Ring::rn_off);
+                    const int gsub = (sub * 16) >> p.k4_g_shift;
+#pragma unroll
+                    for (int u = 0; u < U; ++u) {
+                        const int gi = ((tok0 + u) << p.k4_ng_shift) + gsub;
+                        k4sc[u] = s4s[gi];
+                        k4zc[u] = z4s[gi];
+                        rnrm[u] = __half2float(rns[tok0 + u]);
+                    }
+                }
+            }
             if constexpr (V4) {
                 if (p.v4_bulk && p.want_out) {
                     const float* s4s = reinterpret_cast<const float*>(kst + Ring::s4_off);
@@ -474,8 +595,10 @@ decode_int8_kernel(const DecodeParams p) {
                 const float* kss = reinterpret_cast<const float*>(kst + Ring::ks_off) + tok0;
                 const float* vss = reinterpret_cast<const float*>(kst + Ring::vs_off) + tok0;
                 if constexpr (U == 4) {
-                    const float4 k4 = *reinterpret_cast<const float4*>(kss);
-                    ksc[0] = k4.x, ksc[1] = k4.y, ksc[2] = k4.z, ksc[3] = k4.w;
+                    if constexpr (!RES) {
+                        const float4 k4 = *reinterpret_cast<const float4*>(kss);
+                        ksc[0] = k4.x, ksc[1] = k4.y, ksc[2] = k4.z, ksc[3] = k4.w;
+                    }
                     if constexpr (!V4) {
                         const float4 v4 = p.want_out ? *reinterpret_cast<const float4*>(vss) : make_float4(0, 0, 0, 0);
                         vsc[0] = v4.x, vsc[1] = v4.y, vsc[2] = v4.z, vsc[3] = v4.w;
@@ -483,8 +606,10 @@ decode_int8_kernel(const DecodeParams p) {
                 } else {
 #pragma unroll
                     for (int u = 0; u < U; u += 2) {
-                        const float2 k2 = *reinterpret_cast<const float2*>(kss + u);
-                        ksc[u] = k2.x, ksc[u + 1] = k2.y;
+                        if constexpr (!RES) {
+                            const float2 k2 = *reinterpret_cast<const float2*>(kss + u);
+                            ksc[u] = k2.x, ksc[u + 1] = k2.y;
+                        }
                         if constexpr (!V4) {
                             const float2 v2 = p.want_out ? *reinterpret_cast<const float2*>(vss + u) : make_float2(0, 0);
                             vsc[u] = v2.x, vsc[u + 1] = v2.y;
@@ -495,6 +620,78 @@ decode_int8_kernel(const DecodeParams p) {
             float score[U][G];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
+                if constexpr (RES) {
+                    // INT4 key dims 16 sub .. 16 sub + 15: s * <q, c> + z * sum q, plus this
+                    // lane's 4 (m = 256) or 2 (m = 128) byte lookups of the residual's sign
+                    // sketch (byte positions sub + 8 e: a quarter-warp reads 8 distinct
+                    // 16-byte bank groups), then one 8-lane reduction
+                    const uint2 kv = *reinterpret_cast<const uint2*>(kst + (tok0 + u) * Ring::krow + sub * 8);
+                    uint64_t c[8];
+                    const uint32_t wds[2] = {kv.x, kv.y};
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t lo = wds[h] & 0x0F0F0F0Fu, hi = (wds[h] >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            c[4 * h + k] = add2(pack2(__uint_as_float(__byte_perm(lo, 0x4B400000u, 0x7650u + k)),
+                                                      __uint_as_float(__byte_perm(hi, 0x4B400000u, 0x7650u + k))),
+                                                pack2(-kRoundMagic, -kRoundMagic));
+                    }
+                    const unsigned char* wrow = kst + Ring::ks_off + (tok0 + u) * (p.m / 8);
+                    uint32_t wsel[4];
+                    const uint4 w0 = *reinterpret_cast<const uint4*>(wrow);
+                    wsel[0] = (sub & 4) ? w0.y : w0.x;
+                    wsel[1] = (sub & 4) ? w0.w : w0.z;
+                    const bool m256 = p.m == 256;
+                    if (m256) {
+                        const uint4 w1 = *reinterpret_cast<const uint4*>(wrow + 16);
+                        wsel[2] = (sub & 4) ? w1.y : w1.x;
+                        wsel[3] = (sub & 4) ? w1.w : w1.z;
+                    } else {
+                        wsel[2] = wsel[3] = 0u;
+                    }
+                    float la[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                    const uint32_t lut_s = dev::smem_u32(lut);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        if (e >= 2 && !m256) break;
+                        const uint32_t byte = (wsel[e] >> (8 * (sub & 3))) & 0xFFu;
+                        const uint32_t addr = lut_s + (uint32_t)(e >> 1) * 65536u + byte * 256u +
+                                              (uint32_t)(sub + 8 * (e & 1)) * 16u;
+                        if constexpr (G == 4) {
+                            float4 f;
+                            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                         : "=f"(f.x), "=f"(f.y), "=f"(f.z), "=f"(f.w) : "r"(addr));
+                            la[0] += f.x, la[1] += f.y, la[2] += f.z, la[3] += f.w;
+                        } else if constexpr (G == 2) {
+                            float2 f;
+                            asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(f.x), "=f"(f.y) : "r"(addr));
+                            la[0] += f.x, la[1] += f.y;
+                        } else {
+                            float f;
+                            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(f) : "r"(addr));
+                            la[0] += f;
+                        }
+                    }
+                    const float cr = p.qjl_c * rnrm[u];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        uint64_t dp0 = 0ull, dp1 = 0ull;
+#pragma unroll
+                        for (int k = 0; k < 8; k += 2) {
+                            dp0 = fma2(qp[g][k], c[k], dp0);
+                            dp1 = fma2(qp[g][k + 1], c[k + 1], dp1);
+                        }
+                        const float2 d2 = unpack2(add2(dp0, dp1));
+                        float d = __fmaf_rn(d2.x + d2.y, k4sc[u], __fmul_rn(k4zc[u], qsum[g]));
+                        d = __fmaf_rn(cr, la[g < 4 ? g : 0], d);
+                        d += __shfl_xor_sync(0xffffffffu, d, 1);
+                        d += __shfl_xor_sync(0xffffffffu, d, 2);
+                        d += __shfl_xor_sync(0xffffffffu, d, 4);
+                        score[u][g] = d;
+                    }
+                    continue;
+                }
                 const uint4 kv = *reinterpret_cast<const uint4*>(kst + (tok0 + u) * kD + sub * 16);
                 uint64_t c[8];
                 const uint32_t w4[4] = {kv.x ^ 0x80808080u, kv.y ^ 0x80808080u, kv.z ^ 0x80808080u,
@@ -967,10 +1164,10 @@ decode_combine_kernel(const float* __restrict__ ws, int64_t T, int64_t W, int ma
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-template <int G, bool V4>
+template <int G, bool V4, bool RES = false>
 size_t int8_smem() {
-    return (size_t)I8Ring<G, V4>::stages * I8Ring<G, V4>::bytes +
-           (size_t)kI8Consumers * G * (2 + kD) * sizeof(float);
+    return (size_t)I8Ring<G, V4, RES>::stages * I8Ring<G, V4, RES>::bytes +
+           (size_t)kI8Consumers * G * (2 + kD) * sizeof(float) + (RES ? (size_t)kSignTableBytes : 0);
 }
 constexpr int kQjlThreads = 512;
 
@@ -983,10 +1180,10 @@ size_t qjl_smem() {
     return a > red ? a : red;
 }
 
-template <int G, bool V4>
+template <int G, bool V4, bool RES = false>
 cudaError_t run_int8(const DecodeParams& p, int ctas, cudaStream_t st) {
-    auto kern = decode_int8_kernel<G, V4>;
-    const size_t smem = int8_smem<G, V4>();
+    auto kern = decode_int8_kernel<G, V4, RES>;
+    const size_t smem = int8_smem<G, V4, RES>();
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<ctas, kI8Threads, smem, st>>>(p);
@@ -1004,6 +1201,14 @@ cudaError_t run_qjl(const DecodeParams& p, int ctas, cudaStream_t st) {
 }
 
 cudaError_t run_partial(bool qjl, int G, const DecodeParams& p, int ctas, cudaStream_t st) {
+    if (p.k4p != nullptr) {
+        switch (G) {
+            case 1: return run_int8<1, false, true>(p, ctas, st);
+            case 2: return run_int8<2, false, true>(p, ctas, st);
+            case 4: return run_int8<4, false, true>(p, ctas, st);
+            default: return cudaErrorNotSupported;
+        }
+    }
     if (qjl) {
         switch (G) {
             case 1: return run_qjl<1>(p, ctas, st);
@@ -1041,7 +1246,7 @@ cudaError_t read_and_clear_decode_error(uint32_t* code) {
     return e;
 }
 
-DecodePlan plan_decode(const kvq_decode_args* a, int sm_count) {
+DecodePlan plan_decode(const kvq_decode_args* a, int sm_count, bool residual_keys) {
     DecodePlan pl{};
     const int64_t G = a->n_q_heads / a->n_kv_heads;
     const bool qjl = a->key_format == KVQ_KEYS_QJL;
@@ -1050,7 +1255,7 @@ DecodePlan plan_decode(const kvq_decode_args* a, int sm_count) {
     const int64_t total = pl.units * T;
     // As many CTAs as can be resident at once: up to three 68 KB-ring INT8 CTAs per SM,
     // or one 512-thread QJL CTA per SM (its byte tables fill shared memory).
-    const int64_t resident = (int64_t)sm_count * (qjl ? 1 : int8_ctas_per_sm((int)G));
+    const int64_t resident = (int64_t)sm_count * (qjl && !residual_keys ? 1 : int8_ctas_per_sm((int)G, residual_keys));
     int64_t W = total > 0 ? (total + resident - 1) / resident : kRange;
     W = (W + kRange - 1) / kRange * kRange;
     pl.W = W;
@@ -1068,7 +1273,7 @@ float decode_scale_log2(const kvq_decode_args* a) {
 }
 
 cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaStream_t st,
-                          const AppendSpec* app, const Int4Values* v4, float* fin_ml) {
+                          const AppendSpec* app, const Int4Values* v4, float* fin_ml, const Int4Keys* k4) {
     const int G = (int)(a->n_q_heads / a->n_kv_heads);
     const bool qjl = a->key_format == KVQ_KEYS_QJL;
     char* ws = static_cast<char*>(a->workspace);
@@ -1105,8 +1310,21 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
     p.scale_log2 = decode_scale_log2(a);
     p.qjl_c = qjl ? (float)(1.2533141373155002512 / (double)a->sketch_dim) : 0.0f;  // sqrt(pi/2)/m
     p.want_out = a->out != nullptr;
-    p.scales_bulk = !qjl && (a->seq_len % 4 == 0) && (p.cap % 4 == 0) &&
-                    (reinterpret_cast<uintptr_t>(a->k_scales) % 16 == 0) &&
+    if (k4 != nullptr) {
+        p.k4p = k4->packed;
+        p.k4s = k4->scales;
+        p.k4z = k4->zeros;
+        p.k4_g_shift = k4->group == 32 ? 5 : (k4->group == 64 ? 6 : 7);
+        p.k4_ng_shift = 7 - p.k4_g_shift;
+        // every stage then starts and ends on a multiple of 8 tokens, so the group
+        // parameters (4-16 B per token) and norms (2 B) move in 16-byte multiples
+        p.k4_bulk = (a->seq_len % 8 == 0) && (p.cap % 8 == 0) &&
+                    reinterpret_cast<uintptr_t>(k4->scales) % 16 == 0 &&
+                    reinterpret_cast<uintptr_t>(k4->zeros) % 16 == 0 &&
+                    reinterpret_cast<uintptr_t>(a->k_norms_f16) % 16 == 0;
+    }
+    p.scales_bulk = (!qjl || k4 != nullptr) && (a->seq_len % 4 == 0) && (p.cap % 4 == 0) &&
+                    (k4 != nullptr || reinterpret_cast<uintptr_t>(a->k_scales) % 16 == 0) &&
                     (a->out == nullptr || reinterpret_cast<uintptr_t>(a->v_scales) % 16 == 0);
     cudaError_t e;
     if (qjl) {

@@ -22,6 +22,9 @@ cudaError_t launch_int8_scores(const void* q, bool q_f16, const int8_t* codes,
 // lowbit.cu
 cudaError_t launch_quantize_int4(const void* x, bool f16, int64_t n_rows, int64_t d, int group,
                                  uint8_t* packed, float* scales, float* zeros, cudaStream_t st);
+cudaError_t launch_quantize_int4_residual(const uint16_t* x, int64_t n_rows, int64_t d, int group,
+                                          uint8_t* packed, float* scales, float* zeros, uint16_t* resid,
+                                          cudaStream_t st);
 cudaError_t launch_dequantize_int4(const uint8_t* packed, const float* scales, const float* zeros,
                                    int64_t n_rows, int64_t d, int group, void* out, bool f16,
                                    cudaStream_t st);
@@ -49,7 +52,8 @@ struct DecodePlan {
     size_t sketch_bytes;  // query sketches (QJL)
     size_t total_bytes;
 };
-DecodePlan plan_decode(const kvq_decode_args* a, int sm_count);
+// residual_keys: keys as group-wise INT4 + the residual's sign sketch (one CTA per SM)
+DecodePlan plan_decode(const kvq_decode_args* a, int sm_count, bool residual_keys = false);
 cudaError_t read_and_clear_decode_error(uint32_t* code);
 // Append-on-decode: the new token (row T - 1 of every unit, a->seq_len = T) is encoded
 // by the decode kernel itself; the cache arrays have `capacity` rows per unit.
@@ -69,9 +73,18 @@ struct Int4Values {
 float decode_scale_log2(const kvq_decode_args* a);
 // fin_ml (optional, [B * Hq][2]): each query head's final softmax max (log2 domain) and
 // sum, written by the combine kernel (needs a->out).
+// Residual keys: group-wise INT4 codes [units * T][D / 2], scales and zero points
+// [units * T][D / group]; the residual's sign words and norms come in k_words /
+// k_norms_f16 of the decode arguments (key_format QJL).
+struct Int4Keys {
+    const uint8_t* packed;
+    const float* scales;
+    const float* zeros;
+    int group;
+};
 cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& plan, cudaStream_t st,
                           const AppendSpec* app = nullptr, const Int4Values* v4 = nullptr,
-                          float* fin_ml = nullptr);
+                          float* fin_ml = nullptr, const Int4Keys* k4 = nullptr);
 
 // evict.cu
 cudaError_t launch_attention_mass(const float* scores, const float* fin_ml, int64_t B, int64_t Hq,

@@ -165,11 +165,14 @@ __device__ __forceinline__ void load32(const void* x, int64_t e0, float* f, floa
     }
 }
 
-template <bool F16, int LPG>
+// RES: also write the residual of each element against its INT4 reconstruction,
+// fp16(fl32(x - fl32(fl32(c * s) + z))), to resid (same layout as x; fp16 x only).
+template <bool F16, int LPG, bool RES = false>
 __global__ void __launch_bounds__(256) int4_quantize_kernel(const void* __restrict__ x, int64_t n32,
                                                             uint8_t* __restrict__ packed,
                                                             float* __restrict__ scales,
-                                                            float* __restrict__ zeros) {
+                                                            float* __restrict__ zeros,
+                                                            __half* __restrict__ resid = nullptr) {
     const int lane = threadIdx.x & 31;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     // the loop bound is warp-uniform (n32 is a multiple of LPG and every warp starts on a
@@ -202,6 +205,25 @@ __global__ void __launch_bounds__(256) int4_quantize_kernel(const void* __restri
             word[c] = quant8_u4(t, s, r);
         }
         *reinterpret_cast<uint4*>(packed + i * 16) = make_uint4(word[0], word[1], word[2], word[3]);
+        if constexpr (RES) {
+            // k_hat = fl32(fl32(c * s) + z), r = fp16(fl32(x - k_hat)): scalar IEEE
+            // operations, each rounded on its own (never contracted into an fma)
+            uint4 out[4];
+            uint32_t* o = reinterpret_cast<uint32_t*>(out);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+                const uint32_t w = word[e >> 3];
+                const float c0 = (float)((w >> (4 * (e & 7))) & 0xFu);
+                const float c1 = (float)((w >> (4 * ((e & 7) + 1))) & 0xFu);
+                const float r0 = __fsub_rn(f[e], __fadd_rn(__fmul_rn(c0, s), mn));
+                const float r1 = __fsub_rn(f[e + 1], __fadd_rn(__fmul_rn(c1, s), mn));
+                const __half2 h = __floats2half2_rn(r0, r1);
+                o[e >> 1] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(resid + i * 32);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dst[k] = out[k];
+        }
         if ((lane & (LPG - 1)) == 0) {
             const int64_t gi = i / LPG;   // group index: 32 LPG elements per group
             scales[gi] = s;
@@ -379,6 +401,22 @@ cudaError_t launch_quantize_int4(const void* x, bool f16, int64_t n_rows, int64_
         case 129: int4_quantize_kernel<true, 2><<<grid, 256, 0, st>>>(x, n32, packed, scales, zeros); break;
         case 256: int4_quantize_kernel<false, 4><<<grid, 256, 0, st>>>(x, n32, packed, scales, zeros); break;
         case 257: int4_quantize_kernel<true, 4><<<grid, 256, 0, st>>>(x, n32, packed, scales, zeros); break;
+        default: return cudaErrorNotSupported;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_int4_residual(const uint16_t* x, int64_t n_rows, int64_t d, int group,
+                                          uint8_t* packed, float* scales, float* zeros, uint16_t* resid,
+                                          cudaStream_t st) {
+    const int64_t n32 = n_rows * d / 32;
+    if (n32 == 0) return cudaSuccess;
+    const unsigned grid = grid_for(n32, 256);
+    __half* r = reinterpret_cast<__half*>(resid);
+    switch (group) {
+        case 32: int4_quantize_kernel<true, 1, true><<<grid, 256, 0, st>>>(x, n32, packed, scales, zeros, r); break;
+        case 64: int4_quantize_kernel<true, 2, true><<<grid, 256, 0, st>>>(x, n32, packed, scales, zeros, r); break;
+        case 128: int4_quantize_kernel<true, 4, true><<<grid, 256, 0, st>>>(x, n32, packed, scales, zeros, r); break;
         default: return cudaErrorNotSupported;
     }
     return cudaGetLastError();

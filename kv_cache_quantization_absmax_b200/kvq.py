@@ -47,6 +47,12 @@ class DecodeInt4vArgs(ctypes.Structure):
                 ("v_group", _I32)]
 
 
+class DecodeQjlresArgs(ctypes.Structure):
+    """Mirror of ``kvq_decode_qjlres_args``."""
+    _fields_ = [("base", DecodeArgs), ("k_packed4", _P), ("k_scales4", _P), ("k_zeros4", _P),
+                ("k_group", _I32)]
+
+
 class DecodeMassArgs(ctypes.Structure):
     """Mirror of ``kvq_decode_mass_args``."""
     _fields_ = [("base", DecodeArgs), ("attn_mass", _P)]
@@ -100,6 +106,12 @@ def _load():
     so.kvq_evict_select.restype = ctypes.c_int
     so.kvq_gather_rows.argtypes = [_P, _P, _I64, _I64, _I64, _I64, _I64, _P, _I64, _P]
     so.kvq_gather_rows.restype = ctypes.c_int
+    so.kvq_decode_attention_qjlres.argtypes = [ctypes.POINTER(DecodeQjlresArgs), _P]
+    so.kvq_decode_attention_qjlres.restype = ctypes.c_int
+    so.kvq_decode_qjlres_workspace_bytes.argtypes = [ctypes.POINTER(DecodeQjlresArgs)]
+    so.kvq_decode_qjlres_workspace_bytes.restype = ctypes.c_size_t
+    so.kvq_qjl_residual_encode.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _P, _P, _P, _P, _P, _P, _P]
+    so.kvq_qjl_residual_encode.restype = ctypes.c_int
     for f in ("kvq_quantize_int8", "kvq_dequantize_int8", "kvq_int8_scores", "kvq_qjl_encode",
               "kvq_qjl_query_sketch", "kvq_decode_attention", "kvq_device_error"):
         getattr(so, f).restype = ctypes.c_int
@@ -499,3 +511,67 @@ def kvq_gather_rows(src, kept, dst=None, stream=None):
     _check("kvq_gather_rows", lib.kvq_gather_rows(_ptr(src), _ptr(dst), B, H, T, dst.shape[2], row_bytes,
                                                   _ptr(kept), n_keep, _stream(stream)))
     return dst
+
+
+def kvq_qjl_residual_encode(keys, group, sketch, stream=None):
+    """Keys fp16 [..., D] -> group-wise INT4 + the residual's 1-bit QJL sketch: a dict of
+    packed [..., D/2] uint8, scales / zeros [..., D/group] fp32, residual [..., D] fp16,
+    words [..., m/32] (int32 view of uint32) and rnorms [...] fp16."""
+    _need_cuda(keys, sketch)
+    if keys.dtype != torch.float16:
+        raise ValueError("keys must be fp16")
+    D = keys.shape[-1]
+    lead = tuple(keys.shape[:-1])
+    n = keys.numel() // D
+    m = sketch.shape[0]
+    dev = keys.device
+    o = dict(packed=torch.empty(lead + (D // 2,), dtype=torch.uint8, device=dev),
+             scales=torch.empty(lead + (D // group,), dtype=torch.float32, device=dev),
+             zeros=torch.empty(lead + (D // group,), dtype=torch.float32, device=dev),
+             residual=torch.empty(lead + (D,), dtype=torch.float16, device=dev),
+             words=torch.empty(lead + (m // 32,), dtype=torch.int32, device=dev),
+             rnorms=torch.empty(lead, dtype=torch.float16, device=dev))
+    _check("kvq_qjl_residual_encode", lib.kvq_qjl_residual_encode(
+        _ptr(keys), n, D, int(group), _ptr(sketch), m, _ptr(o["packed"]), _ptr(o["scales"]), _ptr(o["zeros"]),
+        _ptr(o["residual"]), _ptr(o["words"]), _ptr(o["rnorms"]), _stream(stream)))
+    return o
+
+
+def make_decode_qjlres_args(q, *, k_packed4, k_scales4, k_zeros4, k_group, k_words, k_norms, sketch,
+                            v_codes=None, v_scales=None, out=None, scores_out=None, sm_scale=0.0,
+                            workspace=None):
+    """Fill a ``kvq_decode_qjlres_args`` (residual keys, INT8 values)."""
+    a = DecodeQjlresArgs()
+    a.base = make_decode_args(q, k_words=k_words, k_norms=k_norms, sketch=sketch, v_codes=v_codes,
+                              v_scales=v_scales, out=out, scores_out=scores_out, sm_scale=sm_scale,
+                              workspace=workspace)
+    a.k_packed4 = k_packed4.data_ptr() if k_packed4 is not None else None
+    a.k_scales4 = k_scales4.data_ptr() if k_scales4 is not None else None
+    a.k_zeros4 = k_zeros4.data_ptr() if k_zeros4 is not None else None
+    a.k_group = int(k_group)
+    return a
+
+
+def kvq_decode_attention_qjlres(q, *, k_packed4, k_scales4, k_zeros4, k_group, k_words, k_norms, sketch,
+                                v_codes=None, v_scales=None, want_out=True, want_scores=False,
+                                sm_scale=0.0, workspace=None, out=None, scores_out=None, stream=None):
+    """Decode step over residual keys (kvq_qjl_residual_encode) and INT8 values; returns
+    (out [B, Hq, D] fp32 or None, scores [B, Hq, T] or None)."""
+    _need_cuda(q, k_packed4, k_scales4, k_zeros4, k_words, k_norms, sketch, v_codes, v_scales)
+    B, Hq, D = q.shape
+    T = k_words.shape[2]
+    if want_out and out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    if want_scores and scores_out is None:
+        scores_out = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    a = make_decode_qjlres_args(q, k_packed4=k_packed4, k_scales4=k_scales4, k_zeros4=k_zeros4,
+                                k_group=k_group, k_words=k_words, k_norms=k_norms, sketch=sketch,
+                                v_codes=v_codes if want_out else None,
+                                v_scales=v_scales if want_out else None, out=out if want_out else None,
+                                scores_out=scores_out if want_scores else None, sm_scale=sm_scale)
+    need = int(lib.kvq_decode_qjlres_workspace_bytes(ctypes.byref(a)))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    _check("kvq_decode_attention_qjlres", lib.kvq_decode_attention_qjlres(ctypes.byref(a), _stream(stream)))
+    return (out if want_out else None), (scores_out if want_scores else None)

@@ -25,7 +25,8 @@
  *  [INT4]  "Q-TensorFormer" model card, section 6, Asymmetric Group-Wise INT4 equations:
  *          X_hat = clamp(round((X - z4) / s4), 0, 15) * s4 + z4,
  *          s4 = (max X - min X) / 15,  z4 = min X.
- *  [RES]   "TurboQuant" news report (ArsTechnica, via amp.my.ua): a first quantizer does
+ *  [RES]   "Кризис отменяется: Google изобрел квантовый алгоритм сокращения объема памяти
+ *          для ИИ в 6 раз" (news page on TurboQuant): a first quantizer does
  *          most of the compression and a 1-bit QJL layer then corrects its residual
  *          error, one sign bit per sketch coordinate, for better attention scores.  The
  *          first stage here is [INT4]; the residual is the key minus its INT4

@@ -159,3 +159,39 @@ def test_eviction_rejects_bad_arguments(kvq):
     m.base = _args(kvq)
     assert L.kvq_decode_attention_mass(ctypes.byref(m), None) == kvq.KVQ_ERR_WORKSPACE
     assert L.kvq_decode_mass_workspace_bytes(ctypes.byref(m)) > L.kvq_decode_workspace_bytes(ctypes.byref(m.base))
+
+
+def test_qjlres_rejects_bad_arguments(kvq):
+    L = kvq.lib
+    E, U = kvq.KVQ_ERR_INVALID_ARG, kvq.KVQ_ERR_UNSUPPORTED
+    enc = L.kvq_qjl_residual_encode
+    ok = [_p(A16)] * 0
+    args = lambda **kw: [kw.get("keys", _p(A16)), kw.get("n", 10), kw.get("d", 128), kw.get("g", 32),
+                         kw.get("S", _p(A16)), kw.get("m", 256), kw.get("packed", _p(A16)), _p(A16), _p(A16),
+                         kw.get("resid", _p(A16)), _p(A16), _p(A16), None]
+    assert enc(*args(g=16)) == U
+    assert enc(*args(g=48)) == E                     # d % group
+    assert enc(*args(d=64, g=32)) == U               # d != 128
+    assert enc(*args(m=100)) == E
+    assert enc(*args(packed=_p(A16 + 4))) == E       # packed must be 16-byte aligned
+    assert enc(*args(resid=_p(A16 + 2))) == E
+    assert enc(*args(keys=None)) == E
+    assert enc(*args(n=0, keys=None)) == kvq.KVQ_OK
+    assert L.kvq_quantize_int4(_p(A16), 1, 4, 128, 32, _p(A16 + 4), _p(A16), _p(A16), None) == E
+    r = kvq.DecodeQjlresArgs()
+    r.base = _args(kvq, key_format=kvq.KVQ_KEYS_QJL, k_words=A16, k_norms_f16=A16, sketch_f16=A16, sketch_dim=256)
+    r.k_packed4, r.k_scales4, r.k_zeros4, r.k_group = A16, A16, A16, 32
+    call = lambda: L.kvq_decode_attention_qjlres(ctypes.byref(r), None)
+    assert call() == kvq.KVQ_ERR_WORKSPACE
+    assert L.kvq_decode_qjlres_workspace_bytes(ctypes.byref(r)) > 0
+    r.k_group = 16
+    assert call() == U
+    r.k_group = 32
+    r.k_packed4 = A16 + 8
+    assert call() == E
+    r.k_packed4 = A16
+    r.base.sketch_dim = 64
+    assert call() == U
+    r.base.sketch_dim = 256
+    r.base.key_format = kvq.KVQ_KEYS_INT8
+    assert call() == E
