@@ -217,9 +217,10 @@ __device__ __forceinline__ void merge_warps_and_store(const float* red, const De
 // INT8 keys.  The CTA's range streams through a shared-memory ring of stages of up to
 // 64 or 128 tokens of one unit (K rows, V rows, and the scales when they are 16-byte
 // aligned) filled by bulk asynchronous copies that one producer thread issues; eight
-// consumer warps read the stage from shared memory.  8 lanes share a token (lane `sub`
-// owns dims 16 sub .. 16 sub + 15 of K and V); each 8-lane group takes U consecutive
-// tokens of a stage and keeps its own online-softmax state; at the end of each unit
+// consumer warps read the stage from shared memory.  LPT lanes share a token (8 lanes of
+// 16 dims for up to two query heads per KV head, 16 lanes of 8 dims for four or eight;
+// lane `sub` owns dims DPL sub .. DPL sub + DPL - 1 of K and V); each lane group takes U
+// consecutive tokens of a stage and keeps its own online-softmax state; at the end of each unit
 // segment the states are merged across groups (shuffles) and warps (shared memory)
 // into the segment's slot while the producer already streams the next segment.
 // -----------------------------------------------------------------------------------
@@ -304,6 +305,31 @@ __device__ __forceinline__ void build_sign_tables(float* lut, const float* v, in
 }
 constexpr int kSignTableBytes = 2 * 256 * 16 * 16;      // 128 KB
 
+// A lane's BYTES consecutive bytes of a shared-memory row (16, 8 or 4) as 32-bit words.
+template <int BYTES>
+__device__ __forceinline__ void load_row_words(const unsigned char* src, uint32_t* w) {
+    if constexpr (BYTES == 16) {
+        const uint4 v = *reinterpret_cast<const uint4*>(src);
+        w[0] = v.x, w[1] = v.y, w[2] = v.z, w[3] = v.w;
+    } else if constexpr (BYTES == 8) {
+        const uint2 v = *reinterpret_cast<const uint2*>(src);
+        w[0] = v.x, w[1] = v.y;
+    } else {
+        w[0] = *reinterpret_cast<const uint32_t*>(src);
+    }
+}
+
+// Eight 4-bit codes (one word: element 2i in the low nibble of byte i) -> four exact
+// float pairs (elements 2k, 2k + 1).
+__device__ __forceinline__ void nibbles8(uint32_t w, uint64_t* c) {
+    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        c[k] = add2(pack2(__uint_as_float(__byte_perm(lo, 0x4B400000u, 0x7650u + k)),
+                          __uint_as_float(__byte_perm(hi, 0x4B400000u, 0x7650u + k))),
+                    pack2(-kRoundMagic, -kRoundMagic));
+}
+
 template <int G, bool V4, bool RES = false>
 __global__ void __launch_bounds__(kI8Threads, int8_ctas_per_sm(G, RES))
 decode_int8_kernel(const DecodeParams p) {
@@ -312,12 +338,18 @@ decode_int8_kernel(const DecodeParams p) {
     constexpr int kI8StageTok = Ring::tok;
     constexpr int kI8Stages = Ring::stages;
     constexpr int kI8StageBytes = Ring::bytes;
-    static_assert(kI8StageTok % (4 * kI8Consumers) == 0, "each 8-lane group takes whole tokens");
+    // Lanes per token: 8 (16 dims each) up to two heads per KV head, 16 (8 dims each) for
+    // more, which halves the per-lane query and accumulator state.
+    constexpr int LPT = G >= 4 ? 16 : 8;
+    constexpr int DPL = kD / LPT;          // dims per lane
+    constexpr int NP = DPL / 2;            // packed fp32 pairs per lane
+    constexpr int GPW = 32 / LPT;          // lane groups per warp
+    static_assert(kI8StageTok % (GPW * kI8Consumers) == 0, "each lane group takes whole tokens");
     extern __shared__ __align__(128) unsigned char smem_raw[];
     __shared__ uint64_t bars[2 * kI8Stages + 1];
     __shared__ int abort_storage;
     volatile int* abort_flag = &abort_storage;
-    constexpr int U = kI8StageTok / (kI8Consumers * 4);   // tokens per 8-lane group per stage
+    constexpr int U = kI8StageTok / (kI8Consumers * GPW);  // tokens per lane group per stage
     const int cta = blockIdx.x;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -456,8 +488,8 @@ decode_int8_kernel(const DecodeParams p) {
         if (lane == 0) dev::mbar_arrive(append_bar);
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kI8Consumers) : "memory");
     }
-    const int tg = lane >> 3;
-    const int sub = lane & 7;
+    const int tg = lane / LPT;
+    const int sub = lane % LPT;
     int i = 0;
     bool aborted = false;
     for (int jj = 0; jj < nseg; ++jj) {
@@ -465,29 +497,29 @@ decode_int8_kernel(const DecodeParams p) {
         const int64_t row0 = sg.u * p.cap;
         const int64_t b = sg.u / p.Hkv;
         const int kvh = (int)(sg.u % p.Hkv);
-        uint64_t qp[G][8];
+        uint64_t qp[G][NP];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
             const int64_t h = (int64_t)kvh * G + g;
-            const uint4* src = reinterpret_cast<const uint4*>(p.q + (b * p.Hq + h) * kD + sub * 16);
-            const uint4 a = __ldg(src), c = __ldg(src + 1);
-            const __half2* ha = reinterpret_cast<const __half2*>(&a);
-            const __half2* hc = reinterpret_cast<const __half2*>(&c);
+            const uint4* src = reinterpret_cast<const uint4*>(p.q + (b * p.Hq + h) * kD + sub * DPL);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 f0 = __half22float2(ha[k]);
-                const float2 f1 = __half22float2(hc[k]);
-                qp[g][k] = pack2(f0.x, f0.y);
-                qp[g][4 + k] = pack2(f1.x, f1.y);
+            for (int v = 0; v < DPL / 8; ++v) {
+                const uint4 a = __ldg(src + v);
+                const __half2* ha = reinterpret_cast<const __half2*>(&a);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float2 f0 = __half22float2(ha[k]);
+                    qp[g][4 * v + k] = pack2(f0.x, f0.y);
+                }
             }
         }
-        float qsum[G];  // residual keys: the sum of the lane's 16 query values, per head
+        float qsum[G];  // residual keys: the sum of the lane's query values, per head
         if constexpr (RES) {
 #pragma unroll
             for (int g = 0; g < G; ++g) {
                 float a = 0.0f;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
+                for (int k = 0; k < NP; ++k) {
                     const float2 q2 = unpack2(qp[g][k]);
                     a += q2.x + q2.y;
                 }
@@ -501,7 +533,7 @@ decode_int8_kernel(const DecodeParams p) {
             asm volatile("bar.sync 1, %0;" ::"n"(32 * kI8Consumers) : "memory");
         }
         float mrun[G], lrun[G];
-        uint64_t acc[G][8];
+        uint64_t acc[G][NP];
         float zacc[G];  // INT4 values: sum over tokens of p * zero point (the same for the lane's dims)
 #pragma unroll
         for (int g = 0; g < G; ++g) {
@@ -509,13 +541,13 @@ decode_int8_kernel(const DecodeParams p) {
             lrun[g] = 0.0f;
             zacc[g] = 0.0f;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) acc[g][k] = 0ull;
+            for (int k = 0; k < NP; ++k) acc[g][k] = 0ull;
         }
 
         for (int64_t tstage = sg.t0; tstage < sg.t1; tstage += kI8StageTok, ++i) {
             const int s = i % kI8Stages;
             const uint32_t ph = (uint32_t)(i / kI8Stages) & 1u;
-            const int tok0 = warp * (4 * U) + tg * U;        // first token of this group in the stage
+            const int tok0 = warp * (GPW * U) + tg * U;      // first token of this group in the stage
             const int rem = (int)min((int64_t)kI8StageTok, sg.t1 - tstage);  // tokens of the stage in range
             bool valid[U];
             float ksc[U], vsc[U], vz[U];
@@ -526,7 +558,7 @@ decode_int8_kernel(const DecodeParams p) {
                 const int64_t r = row0 + tstage + (valid[u] ? tok0 + u : 0);
                 if constexpr (RES) {
                     if (!p.k4_bulk) {
-                        const int64_t gi = (r << p.k4_ng_shift) + ((sub * 16) >> p.k4_g_shift);
+                        const int64_t gi = (r << p.k4_ng_shift) + ((sub * DPL) >> p.k4_g_shift);
                         k4sc[u] = __ldg(p.k4s + gi);
                         k4zc[u] = __ldg(p.k4z + gi);
                         rnrm[u] = __half2float(__ushort_as_half(__ldg(p.kn + r)));
@@ -538,11 +570,11 @@ decode_int8_kernel(const DecodeParams p) {
                     if constexpr (!V4) vsc[u] = p.want_out ? __ldcg(p.vs + r) : 0.0f;
                 }
                 if constexpr (V4) {
-                    // this lane's 16 dims lie in one group (groups of 32, 64 or 128); groups
+                    // this lane's dims lie in one group (groups of 32, 64 or 128); groups
                     // of 32 come with the stage, the others are loaded here
                     if (!p.v4_bulk && p.want_out) {
                         const int ng = kD / p.v4g;
-                        const int64_t gi = r * ng + (sub * 16) / p.v4g;
+                        const int64_t gi = r * ng + (sub * DPL) / p.v4g;
                         vsc[u] = __ldcg(p.v4s + gi);
                         vz[u] = __ldcg(p.v4z + gi);
                     } else {
@@ -568,7 +600,7 @@ decode_int8_kernel(const DecodeParams p) {
                     const float* s4s = reinterpret_cast<const float*>(kst + Ring::s4_off);
                     const float* z4s = reinterpret_cast<const float*>(kst + Ring::z4_off);
                     const __half* rns = reinterpret_cast<const __half*>(kst + Ring::rn_off);
-                    const int gsub = (sub * 16) >> p.k4_g_shift;
+                    const int gsub = (sub * DPL) >> p.k4_g_shift;
 #pragma unroll
                     for (int u = 0; u < U; ++u) {
                         const int gi = ((tok0 + u) << p.k4_ng_shift) + gsub;
@@ -584,8 +616,8 @@ decode_int8_kernel(const DecodeParams p) {
                     const float* z4s = reinterpret_cast<const float*>(kst + Ring::z4_off);
 #pragma unroll
                     for (int u = 0; u < U; ++u) {
-                        vsc[u] = s4s[(tok0 + u) * 4 + (sub >> 1)];
-                        vz[u] = z4s[(tok0 + u) * 4 + (sub >> 1)];
+                        vsc[u] = s4s[(tok0 + u) * 4 + ((sub * DPL) >> 5)];
+                        vz[u] = z4s[(tok0 + u) * 4 + ((sub * DPL) >> 5)];
                     }
                 }
             }
@@ -621,43 +653,32 @@ decode_int8_kernel(const DecodeParams p) {
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 if constexpr (RES) {
-                    // INT4 key dims 16 sub .. 16 sub + 15: s * <q, c> + z * sum q, plus this
-                    // lane's 4 (m = 256) or 2 (m = 128) byte lookups of the residual's sign
-                    // sketch (byte positions sub + 8 e: a quarter-warp reads 8 distinct
-                    // 16-byte bank groups), then one 8-lane reduction
-                    const uint2 kv = *reinterpret_cast<const uint2*>(kst + (tok0 + u) * Ring::krow + sub * 8);
-                    uint64_t c[8];
-                    const uint32_t wds[2] = {kv.x, kv.y};
+                    // INT4 key dims DPL sub .. DPL sub + DPL - 1: s * <q, c> + z * sum q, plus
+                    // this lane's byte lookups of the residual's sign sketch (positions
+                    // sub + LPT e, e < m / (8 LPT): a quarter-warp reads 8 distinct 16-byte
+                    // bank groups), then one LPT-lane reduction
+                    uint32_t kw4[DPL / 8];
+                    load_row_words<DPL / 2>(kst + (tok0 + u) * Ring::krow + sub * (DPL / 2), kw4);
+                    uint64_t c[NP];
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint32_t lo = wds[h] & 0x0F0F0F0Fu, hi = (wds[h] >> 4) & 0x0F0F0F0Fu;
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            c[4 * h + k] = add2(pack2(__uint_as_float(__byte_perm(lo, 0x4B400000u, 0x7650u + k)),
-                                                      __uint_as_float(__byte_perm(hi, 0x4B400000u, 0x7650u + k))),
-                                                pack2(-kRoundMagic, -kRoundMagic));
-                    }
+                    for (int h = 0; h < DPL / 8; ++h) nibbles8(kw4[h], c + 4 * h);
                     const unsigned char* wrow = kst + Ring::ks_off + (tok0 + u) * (p.m / 8);
-                    uint32_t wsel[4];
-                    const uint4 w0 = *reinterpret_cast<const uint4*>(wrow);
-                    wsel[0] = (sub & 4) ? w0.y : w0.x;
-                    wsel[1] = (sub & 4) ? w0.w : w0.z;
                     const bool m256 = p.m == 256;
-                    if (m256) {
-                        const uint4 w1 = *reinterpret_cast<const uint4*>(wrow + 16);
-                        wsel[2] = (sub & 4) ? w1.y : w1.x;
-                        wsel[3] = (sub & 4) ? w1.w : w1.z;
-                    } else {
-                        wsel[2] = wsel[3] = 0u;
-                    }
+                    const uint4 w0 = *reinterpret_cast<const uint4*>(wrow);
+                    const uint4 w1 = m256 ? *reinterpret_cast<const uint4*>(wrow + 16) : make_uint4(0, 0, 0, 0);
+                    constexpr int NE = 32 / LPT;                  // lookups per lane at m = 256
                     float la[4] = {0.0f, 0.0f, 0.0f, 0.0f};
                     const uint32_t lut_s = dev::smem_u32(lut);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        if (e >= 2 && !m256) break;
-                        const uint32_t byte = (wsel[e] >> (8 * (sub & 3))) & 0xFFu;
-                        const uint32_t addr = lut_s + (uint32_t)(e >> 1) * 65536u + byte * 256u +
-                                              (uint32_t)(sub + 8 * (e & 1)) * 16u;
+                    for (int e = 0; e < NE; ++e) {
+                        if (e >= NE / 2 && !m256) break;
+                        const int pos = sub + LPT * e;            // byte position in the sketch
+                        const int wi = pos >> 2;                  // its word, 0..7
+                        const uint4 wv = (wi & 4) ? w1 : w0;
+                        const uint32_t word = (wi & 2) ? ((wi & 1) ? wv.w : wv.z) : ((wi & 1) ? wv.y : wv.x);
+                        const uint32_t byte = (word >> (8 * (pos & 3))) & 0xFFu;
+                        const uint32_t addr = lut_s + (uint32_t)(pos >> 4) * 65536u + byte * 256u +
+                                              (uint32_t)(pos & 15) * 16u;
                         if constexpr (G == 4) {
                             float4 f;
                             asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
@@ -678,39 +699,36 @@ decode_int8_kernel(const DecodeParams p) {
                     for (int g = 0; g < G; ++g) {
                         uint64_t dp0 = 0ull, dp1 = 0ull;
 #pragma unroll
-                        for (int k = 0; k < 8; k += 2) {
+                        for (int k = 0; k < NP; k += 2) {
                             dp0 = fma2(qp[g][k], c[k], dp0);
                             dp1 = fma2(qp[g][k + 1], c[k + 1], dp1);
                         }
                         const float2 d2 = unpack2(add2(dp0, dp1));
                         float d = __fmaf_rn(d2.x + d2.y, k4sc[u], __fmul_rn(k4zc[u], qsum[g]));
                         d = __fmaf_rn(cr, la[g < 4 ? g : 0], d);
-                        d += __shfl_xor_sync(0xffffffffu, d, 1);
-                        d += __shfl_xor_sync(0xffffffffu, d, 2);
-                        d += __shfl_xor_sync(0xffffffffu, d, 4);
+#pragma unroll
+                        for (int off = 1; off < LPT; off <<= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
                         score[u][g] = d;
                     }
                     continue;
                 }
-                const uint4 kv = *reinterpret_cast<const uint4*>(kst + (tok0 + u) * kD + sub * 16);
-                uint64_t c[8];
-                const uint32_t w4[4] = {kv.x ^ 0x80808080u, kv.y ^ 0x80808080u, kv.z ^ 0x80808080u,
-                                        kv.w ^ 0x80808080u};
+                uint32_t w4[DPL / 4];
+                load_row_words<DPL>(kst + (tok0 + u) * kD + sub * DPL, w4);
+                uint64_t c[NP];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) codes4(w4[k], c[2 * k], c[2 * k + 1]);
+                for (int k = 0; k < DPL / 4; ++k) codes4(w4[k] ^ 0x80808080u, c[2 * k], c[2 * k + 1]);
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
                     uint64_t dp0 = 0ull, dp1 = 0ull;
 #pragma unroll
-                    for (int k = 0; k < 8; k += 2) {
+                    for (int k = 0; k < NP; k += 2) {
                         dp0 = fma2(qp[g][k], c[k], dp0);
                         dp1 = fma2(qp[g][k + 1], c[k + 1], dp1);
                     }
                     const float2 d2 = unpack2(add2(dp0, dp1));
                     float d = d2.x + d2.y;
-                    d += __shfl_xor_sync(0xffffffffu, d, 1);
-                    d += __shfl_xor_sync(0xffffffffu, d, 2);
-                    d += __shfl_xor_sync(0xffffffffu, d, 4);
+#pragma unroll
+                    for (int off = 1; off < LPT; off <<= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
                     score[u][g] = d * ksc[u];
                 }
             }
@@ -737,33 +755,25 @@ decode_int8_kernel(const DecodeParams p) {
                         if constexpr (V4) zacc[g] *= corr;
                         const uint64_t c2 = pack2(corr, corr);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) acc[g][k] = mul2(acc[g][k], c2);
+                        for (int k = 0; k < NP; ++k) acc[g][k] = mul2(acc[g][k], c2);
                         mrun[g] = mb;
                     }
                 }
 #pragma unroll
                 for (int u = 0; u < U; ++u) {
                     if (!valid[u]) continue;
-                    uint64_t c[8];
+                    uint64_t c[NP];
                     if constexpr (V4) {
-                        // 16 nibbles: byte i holds dims 2i (low) and 2i + 1 (high) -> the pairs
-                        const uint2 vv = *reinterpret_cast<const uint2*>(vst + (tok0 + u) * Ring::vrow + sub * 8);
-                        const uint32_t wds[2] = {vv.x, vv.y};
+                        // DPL nibbles: byte i holds dims 2i (low) and 2i + 1 (high) -> the pairs
+                        uint32_t wds[DPL / 8];
+                        load_row_words<DPL / 2>(vst + (tok0 + u) * Ring::vrow + sub * (DPL / 2), wds);
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const uint32_t lo = wds[h] & 0x0F0F0F0Fu, hi = (wds[h] >> 4) & 0x0F0F0F0Fu;
-#pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                c[4 * h + k] = add2(pack2(__uint_as_float(__byte_perm(lo, 0x4B400000u, 0x7650u + k)),
-                                                          __uint_as_float(__byte_perm(hi, 0x4B400000u, 0x7650u + k))),
-                                                    pack2(-kRoundMagic, -kRoundMagic));
-                        }
+                        for (int h = 0; h < DPL / 8; ++h) nibbles8(wds[h], c + 4 * h);
                     } else {
-                        const uint4 vv = *reinterpret_cast<const uint4*>(vst + (tok0 + u) * kD + sub * 16);
-                        const uint32_t w4[4] = {vv.x ^ 0x80808080u, vv.y ^ 0x80808080u, vv.z ^ 0x80808080u,
-                                                vv.w ^ 0x80808080u};
+                        uint32_t w4[DPL / 4];
+                        load_row_words<DPL>(vst + (tok0 + u) * kD + sub * DPL, w4);
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) codes4(w4[k], c[2 * k], c[2 * k + 1]);
+                        for (int k = 0; k < DPL / 4; ++k) codes4(w4[k] ^ 0x80808080u, c[2 * k], c[2 * k + 1]);
                     }
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
@@ -773,7 +783,7 @@ decode_int8_kernel(const DecodeParams p) {
                         if constexpr (V4) zacc[g] = __fmaf_rn(pe, vz[u], zacc[g]);
                         const uint64_t w2 = pack2(wv, wv);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) acc[g][k] = fma2(w2, c[k], acc[g][k]);
+                        for (int k = 0; k < NP; ++k) acc[g][k] = fma2(w2, c[k], acc[g][k]);
                     }
                 }
             }
@@ -788,11 +798,11 @@ decode_int8_kernel(const DecodeParams p) {
             for (int g = 0; g < G; ++g) {
                 const uint64_t z2 = pack2(zacc[g], zacc[g]);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) acc[g][k] = add2(acc[g][k], z2);
+                for (int k = 0; k < NP; ++k) acc[g][k] = add2(acc[g][k], z2);
             }
         }
 #pragma unroll
-        for (int off = 8; off <= 16; off <<= 1) {
+        for (int off = LPT; off <= 16; off <<= 1) {
 #pragma unroll
             for (int g = 0; g < G; ++g) {
                 const float mo = __shfl_xor_sync(0xffffffffu, mrun[g], off);
@@ -802,7 +812,7 @@ decode_int8_kernel(const DecodeParams p) {
                 const float f2 = mn == -INFINITY ? 0.0f : exp2f(mo - mn);
                 lrun[g] = lrun[g] * f1 + lo * f2;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
+                for (int k = 0; k < NP; ++k) {
                     const float2 a = unpack2(acc[g][k]);
                     const float ax = __shfl_xor_sync(0xffffffffu, a.x, off);
                     const float ay = __shfl_xor_sync(0xffffffffu, a.y, off);
@@ -821,10 +831,10 @@ decode_int8_kernel(const DecodeParams p) {
                     r[1] = lrun[g];
                 }
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
+                for (int k = 0; k < NP; ++k) {
                     const float2 a = unpack2(acc[g][k]);
-                    r[2 + sub * 16 + 2 * k] = a.x;
-                    r[2 + sub * 16 + 2 * k + 1] = a.y;
+                    r[2 + sub * DPL + 2 * k] = a.x;
+                    r[2 + sub * DPL + 2 * k + 1] = a.y;
                 }
             }
         }
