@@ -75,6 +75,8 @@ struct DecodeParams {
     float qjl_c;            // sqrt(pi/2) / m
     int want_out;
     int scales_bulk;        // INT8: scales 16-byte aligned per stage -> bulk-copied too
+    int qjl_bulk;           // QJL: value rows 16-byte aligned -> each warp's next 32 value
+                            // rows come by one bulk copy
 };
 
 // The unit segments of CTA `cta`'s range: unit u, tokens [t0, t1) of that unit, slot j.
@@ -252,7 +254,7 @@ constexpr int kI8Threads = 32 * (kI8Consumers + 1);
 
 __device__ unsigned int g_decode_error = 0;
 
-enum : unsigned int { kErrI8Producer = 0x201, kErrI8Consumer = 0x202 };
+enum : unsigned int { kErrI8Producer = 0x201, kErrI8Consumer = 0x202, kErrQjlStep = 0x203 };
 
 // Resident INT8 CTAs per SM the register budget is shaped for (more heads per group
 // need more registers per thread).  Residual keys: one (the byte tables take 128 KB).
@@ -1135,6 +1137,286 @@ decode_qjl_kernel(const DecodeParams p) {
     }
 }
 
+
+// -----------------------------------------------------------------------------------
+// QJL keys, prefetching variant (16 warps, one CTA per SM).  The byte tables, the
+// estimator lookups, the warp-level online softmax and the value pass are those of
+// decode_qjl_kernel above; the difference is when a step's data is requested.  Each warp
+// has the next step's sign words, norm and value scale loaded into registers while it
+// computes the current step, and a 4 KB value buffer in shared memory that its lane 0
+// refills with one bulk asynchronous copy (32 value rows) as soon as the value pass has
+// read it, so the copy overlaps the next step's lookups and softmax (the wait on the
+// buffer's mbarrier is bounded).  A step of fewer than 32 tokens (a range's tail) is
+// staged into the buffer with ordinary loads.  The value codes no longer sit in 32
+// registers per lane.
+// -----------------------------------------------------------------------------------
+constexpr int kQpfWarps = 16;
+constexpr int kQpfThreads = 32 * kQpfWarps;
+constexpr int kQpfSlot = 32 * kD;                       // 32 value rows
+
+template <int G>
+__global__ void __launch_bounds__(kQpfThreads, 1)
+decode_qjl_pf_kernel(const DecodeParams p) {
+    extern __shared__ float4 dsmem4[];
+    float* dsmem = reinterpret_cast<float*>(dsmem4);
+    constexpr int WARPS = kQpfWarps;
+    constexpr int TOK_PER_STEP = WARPS * 32;
+    constexpr int HALF_FLOATS = 256 * 16 * 4;        // one table half: 64 KB
+    __shared__ uint64_t bars[WARPS];
+    __shared__ int abort_storage;
+    volatile int* abort_flag = &abort_storage;
+    const int cta = blockIdx.x;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const RangeWalk walk(p, cta);
+    const int nseg = walk.count();
+    const int nw = p.m / 32;
+    float* lut = dsmem;                              // 2 halves x [256][16] x 4 floats
+    float* wbuf = dsmem + 2 * HALF_FLOATS;           // [WARPS][16 pairs][G][2]
+    float* red = dsmem;                              // [WARPS][G][2 + kD], reuses the tables
+    unsigned char* vbuf = reinterpret_cast<unsigned char*>(wbuf + WARPS * 32 * G) + (size_t)warp * kQpfSlot;
+    const uint32_t bar = dev::smem_u32(bars) + 8u * warp;
+
+    const int x = lane & 7;
+    const bool swap_words = (x & 4) != 0;
+    uint32_t off16[8];
+    uint32_t sel[4];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) off16[e] = (uint32_t)((e ^ x) * 16);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sel[e] = 0x6504u | ((uint32_t)((e ^ x) & 3) << 4);
+    const uint32_t lut_s = (uint32_t)__cvta_generic_to_shared(lut);
+
+    if (threadIdx.x == 0) {
+        abort_storage = 0;
+        for (int b2 = 0; b2 < WARPS; ++b2) dev::mbar_init(dev::smem_u32(bars) + 8u * b2, 1);
+        dev::mbar_init_fence();
+    }
+    __syncthreads();
+    dev::griddep_launch_dependents();  // the combine kernel may be scheduled (it waits)
+
+    float* mybuf = wbuf + warp * 32 * G;
+    const uint64_t magic = pack2(-kCodeMagic, -kCodeMagic);
+    int nissue = 0, ndone = 0;
+    bool aborted = false;
+
+    for (int jj = 0; jj < nseg; ++jj) {
+        const Segment sg = walk.seg(jj);
+        const int64_t row0 = sg.u * p.cap;
+        const int64_t b = sg.u / p.Hkv;
+        const int kvh = (int)(sg.u % p.Hkv);
+        __syncthreads();  // the previous segment's merge no longer reads red[]
+        build_sign_tables<G>(lut, p.sketch_v + (b * p.Hq + (int64_t)kvh * G) * p.m, p.m, p.m, threadIdx.x,
+                             kQpfThreads);
+        __syncthreads();
+
+        float mrun[G], lsum[G];
+        uint64_t acc[G][4];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            mrun[g] = -INFINITY;
+            lsum[g] = 0.0f;
+#pragma unroll
+            for (int d = 0; d < 4; ++d) acc[g][d] = 0ull;
+        }
+        // a whole block of 32 tokens: its value rows arrive by one bulk copy
+        auto bulk_step = [&](int64_t t0) { return p.qjl_bulk && p.want_out && t0 + 32 <= sg.t1; };
+        auto issue = [&](int64_t t0) {
+            __syncwarp();   // every lane is done reading the buffer
+            if (lane == 0) {
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                dev::mbar_arrive_expect_tx(bar, (uint32_t)kQpfSlot);
+                dev::bulk_g2s(dev::smem_u32(vbuf), p.vc + (row0 + t0) * kD, (uint32_t)kQpfSlot, bar);
+            }
+            ++nissue;
+        };
+        // this lane's token of a step: sign words, norm, value scale (registers)
+        auto load_small = [&](int64_t t0, uint32_t* w, float& nrm, float& vsc) {
+            const bool v = t0 + lane < sg.t1;
+            const int64_t r = row0 + t0 + (v ? lane : 0);
+            if (nw == 8) {
+                const uint4 a = __ldcs(reinterpret_cast<const uint4*>(p.kw + r * 8));
+                const uint4 c = __ldcs(reinterpret_cast<const uint4*>(p.kw + r * 8) + 1);
+                w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+                w[4] = c.x; w[5] = c.y; w[6] = c.z; w[7] = c.w;
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) w[k] = k < nw ? __ldcs(p.kw + r * nw + k) : 0u;
+            }
+            nrm = __half2float(__ushort_as_half(__ldcs(p.kn + r)));
+            vsc = p.want_out ? __ldcs(p.vs + r) : 0.0f;
+        };
+        int64_t t0 = sg.t0 + (int64_t)warp * 32;
+        uint32_t w[8];
+        float nrm = 0.0f, vsc = 0.0f;
+        if (t0 < sg.t1) {
+            load_small(t0, w, nrm, vsc);
+            if (!aborted && bulk_step(t0)) issue(t0);
+        }
+        for (; t0 < sg.t1; t0 += TOK_PER_STEP) {
+            const int64_t tn = t0 + TOK_PER_STEP;
+            uint32_t wn[8];
+            float nrmn = 0.0f, vscn = 0.0f;
+            if (tn < sg.t1) load_small(tn, wn, nrmn, vscn);     // the next step, in flight
+            const int nvalid = (int)min((int64_t)32, sg.t1 - t0);
+            const bool valid = lane < nvalid;
+            if (!aborted) {
+                // ---- estimator: 32 byte-table lookups ----
+                float sc[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) sc[g] = 0.0f;
+                uint64_t s01 = 0ull, s23 = 0ull, t01 = 0ull, t23 = 0ull;
+#pragma unroll
+                for (int pr = 0; pr < 4; ++pr) {
+                    const uint32_t wa = swap_words ? w[2 * pr + 1] : w[2 * pr];
+                    const uint32_t wb = swap_words ? w[2 * pr] : w[2 * pr + 1];
+                    const uint32_t half_off = (uint32_t)((pr >> 1) * HALF_FLOATS * 4 + (pr & 1) * 128);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const uint32_t o = __byte_perm(e < 4 ? wa : wb, off16[e], sel[e & 3]);
+                        const uint32_t addr = lut_s + half_off + o;
+                        if constexpr (G == 4) {
+                            float4 f;
+                            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                         : "=f"(f.x), "=f"(f.y), "=f"(f.z), "=f"(f.w) : "r"(addr));
+                            if (e & 1) {
+                                t01 = add2(t01, pack2(f.x, f.y));
+                                t23 = add2(t23, pack2(f.z, f.w));
+                            } else {
+                                s01 = add2(s01, pack2(f.x, f.y));
+                                s23 = add2(s23, pack2(f.z, f.w));
+                            }
+                        } else if constexpr (G == 2) {
+                            float2 f;
+                            asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(f.x), "=f"(f.y) : "r"(addr));
+                            if (e & 1) t01 = add2(t01, pack2(f.x, f.y));
+                            else s01 = add2(s01, pack2(f.x, f.y));
+                        } else {
+                            float f;
+                            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(f) : "r"(addr));
+                            sc[0] += f;
+                        }
+                    }
+                }
+                if constexpr (G >= 2) {
+                    const float2 a = unpack2(add2(s01, t01));
+                    sc[0] = a.x;
+                    sc[1] = a.y;
+                }
+                if constexpr (G == 4) {
+                    const float2 a = unpack2(add2(s23, t23));
+                    sc[2] = a.x;
+                    sc[3] = a.y;
+                }
+                float score[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) score[g] = p.qjl_c * nrm * sc[g];
+                if (p.scores_out != nullptr && valid) {
+#pragma unroll
+                    for (int g = 0; g < G; ++g)
+                        p.scores_out[(b * p.Hq + (int64_t)kvh * G + g) * p.T + t0 + lane] = score[g];
+                }
+                if (p.want_out) {
+                    // ---- online softmax at warp granularity ----
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const float lg = valid ? score[g] * p.scale_log2 : -INFINITY;
+                        const float mb = warp_max(lg);
+                        if (mb > mrun[g]) {
+                            const float corr = fast_exp2(mrun[g] - mb);
+                            lsum[g] *= corr;
+                            const uint64_t c2 = pack2(corr, corr);
+#pragma unroll
+                            for (int d = 0; d < 4; ++d) acc[g][d] = mul2(acc[g][d], c2);
+                            mrun[g] = mb;
+                        }
+                        const float pe = fast_exp2(lg - mrun[g]);
+                        lsum[g] += pe;
+                        mybuf[(lane >> 1) * (2 * G) + g * 2 + (lane & 1)] = pe * vsc;
+                    }
+                    // ---- this step's value rows ----
+                    if (bulk_step(t0)) {
+                        const bool ok = dev::mbar_wait(bar, (uint32_t)(ndone & 1), abort_flag, &g_decode_error,
+                                                       kErrQjlStep);
+                        aborted = !__all_sync(0xffffffffu, ok);
+                        if (!aborted) ++ndone;
+                    } else {
+                        const unsigned int* vrow = reinterpret_cast<const unsigned int*>(p.vc + (row0 + t0) * kD) + lane;
+                        for (int j = 0; j < 32; ++j)
+                            reinterpret_cast<uint32_t*>(vbuf + j * kD)[lane] = j < nvalid ? __ldcs(vrow + j * (kD / 4))
+                                                                                          : 0x80808080u;
+                    }
+                    __syncwarp();
+                    if (!aborted) {
+                        // ---- values: dims 4 lane .. 4 lane + 3, token pairs (2 jp, 2 jp + 1) ----
+                        const uint32_t* vals = reinterpret_cast<const uint32_t*>(vbuf) + lane;
+#pragma unroll
+                        for (int jp = 0; jp < 16; ++jp) {
+                            const uint32_t ce = vals[(2 * jp) * (kD / 4)] ^ 0x80808080u;
+                            const uint32_t co = vals[(2 * jp + 1) * (kD / 4)] ^ 0x80808080u;
+                            uint64_t cp[4];
+#pragma unroll
+                            for (int d = 0; d < 4; ++d)
+                                cp[d] = add2(pack2(__uint_as_float(__byte_perm(ce, 0x4B400000u, 0x7650u + d)),
+                                                   __uint_as_float(__byte_perm(co, 0x4B400000u, 0x7650u + d))),
+                                             magic);
+                            uint64_t wp[G];
+                            if constexpr (G == 4) {
+                                const float4 a = reinterpret_cast<const float4*>(mybuf)[jp * 2];
+                                const float4 c = reinterpret_cast<const float4*>(mybuf)[jp * 2 + 1];
+                                wp[0] = pack2(a.x, a.y); wp[1] = pack2(a.z, a.w);
+                                wp[2] = pack2(c.x, c.y); wp[3] = pack2(c.z, c.w);
+                            } else if constexpr (G == 2) {
+                                const float4 a = reinterpret_cast<const float4*>(mybuf)[jp];
+                                wp[0] = pack2(a.x, a.y); wp[1] = pack2(a.z, a.w);
+                            } else {
+                                const float2 a = reinterpret_cast<const float2*>(mybuf)[jp];
+                                wp[0] = pack2(a.x, a.y);
+                            }
+#pragma unroll
+                            for (int g = 0; g < G; ++g)
+#pragma unroll
+                                for (int d = 0; d < 4; ++d) acc[g][d] = fma2(wp[g], cp[d], acc[g][d]);
+                        }
+                        // the buffer is read: the next step's value rows may come in
+                        if (tn < sg.t1 && bulk_step(tn)) issue(tn);
+                    }
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) w[k] = wn[k];
+            nrm = nrmn;
+            vsc = vscn;
+        }
+        if (!p.want_out) continue;
+
+        // ---- end of the unit segment: per-warp state -> shared memory -> slot jj ----
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) lsum[g] += __shfl_xor_sync(0xffffffffu, lsum[g], off);
+        __syncthreads();  // the byte tables are no longer read
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float* rr = red + (warp * G + g) * (2 + kD);
+            if (lane == 0) {
+                rr[0] = mrun[g];
+                rr[1] = lsum[g];
+            }
+#pragma unroll
+            for (int d = 0; d < 4; ++d) {
+                const float2 a = unpack2(acc[g][d]);
+                rr[2 + 4 * lane + d] = a.x + a.y;
+            }
+        }
+        __syncthreads();
+        merge_warps_and_store<G, WARPS>(red, p, cta, jj, threadIdx.x, kQpfThreads);
+    }
+    // a copy still in flight after an abort completes before the CTA exits
+    if (lane == 0 && nissue > ndone) dev::mbar_drain(bar, (uint32_t)((nissue - 1) & 1));
+    __syncwarp();
+}
+
 // out[b][h][d]: merge, over the CTAs whose ranges covered unit u = b * Hkv + h / G,
 // acc_s[d] 2^(m_s - M) / sum_s l_s 2^(m_s - M).
 __global__ void __launch_bounds__(kD)
@@ -1201,7 +1483,23 @@ cudaError_t run_int8(const DecodeParams& p, int ctas, cudaStream_t st) {
 }
 
 template <int G>
+size_t qjl_pf_smem() {
+    const size_t tables = (size_t)2 * 256 * 16 * 4 * sizeof(float);
+    const size_t red = (size_t)kQpfWarps * G * (2 + kD) * sizeof(float);
+    const size_t a = (tables > red ? tables : red) + (size_t)kQpfWarps * 32 * G * sizeof(float);
+    return a + (size_t)kQpfWarps * kQpfSlot;
+}
+
+template <int G>
 cudaError_t run_qjl(const DecodeParams& p, int ctas, cudaStream_t st) {
+    if (p.knew == nullptr && p.m <= 256) {
+        auto kern = decode_qjl_pf_kernel<G>;
+        const size_t smem = qjl_pf_smem<G>();
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<ctas, kQpfThreads, smem, st>>>(p);
+        return cudaGetLastError();
+    }
     auto kern = decode_qjl_kernel<G, kQjlThreads>;
     const size_t smem = qjl_smem<G>();
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -1333,6 +1631,9 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
                     reinterpret_cast<uintptr_t>(k4->zeros) % 16 == 0 &&
                     reinterpret_cast<uintptr_t>(a->k_norms_f16) % 16 == 0;
     }
+    // QJL: value rows are 128 B, so a step's 32 rows start 16-byte aligned whenever the
+    // array does
+    p.qjl_bulk = qjl && a->out != nullptr && reinterpret_cast<uintptr_t>(a->v_codes) % 16 == 0;
     p.scales_bulk = (!qjl || k4 != nullptr) && (a->seq_len % 4 == 0) && (p.cap % 4 == 0) &&
                     (k4 != nullptr || reinterpret_cast<uintptr_t>(a->k_scales) % 16 == 0) &&
                     (a->out == nullptr || reinterpret_cast<uintptr_t>(a->v_scales) % 16 == 0);
