@@ -276,6 +276,8 @@ __global__ void __launch_bounds__(256) int4_dequantize_kernel(const uint8_t* __r
 constexpr int kCwCols = 64;
 constexpr int kCwThreads = 512;
 constexpr int kCwRowGroups = kCwThreads / 8;
+constexpr int kCwP1 = 4;
+constexpr int kCwP2 = 2;
 
 template <bool F16>
 __global__ void __launch_bounds__(kCwThreads, 1) int8_cw_quantize_kernel(const void* __restrict__ x,
@@ -293,17 +295,18 @@ __global__ void __launch_bounds__(kCwThreads, 1) int8_cw_quantize_kernel(const v
         float a[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) a[e] = 0.0f;
-        for (int64_t r = rg; r < rows; r += 4 * kCwRowGroups) {
-            float f[4][8];
+        // kCwP1 rows per thread in flight in the column-max pass, kCwP2 in the code pass
+        for (int64_t r = rg; r < rows; r += kCwP1 * kCwRowGroups) {
+            float f[kCwP1][8];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < kCwP1; ++k) {
                 if (r + k * kCwRowGroups < rows) load8<F16>(x, base + (r + k * kCwRowGroups) * d, f[k]);
                 else
 #pragma unroll
                     for (int e = 0; e < 8; ++e) f[k][e] = 0.0f;
             }
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
+            for (int k = 0; k < kCwP1; ++k)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) a[e] = fmaxf(a[e], fabsf(f[k][e]));
         }
@@ -325,13 +328,13 @@ __global__ void __launch_bounds__(kCwThreads, 1) int8_cw_quantize_kernel(const v
             sc[e] = s_sh[8 * cg + e];
             rc[e] = r_sh[8 * cg + e];
         }
-        for (int64_t r = rg; r < rows; r += 2 * kCwRowGroups) {
-            float f[2][8];
+        for (int64_t r = rg; r < rows; r += kCwP2 * kCwRowGroups) {
+            float f[kCwP2][8];
 #pragma unroll
-            for (int k = 0; k < 2; ++k)
+            for (int k = 0; k < kCwP2; ++k)
                 if (r + k * kCwRowGroups < rows) load8<F16>(x, base + (r + k * kCwRowGroups) * d, f[k]);
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
+            for (int k = 0; k < kCwP2; ++k) {
                 if (r + k * kCwRowGroups >= rows) continue;
                 *reinterpret_cast<uint2*>(codes + base + (r + k * kCwRowGroups) * d) = quant8_i8(f[k], sc, rc);
             }
