@@ -256,6 +256,86 @@ ROW_NAMES = ["quantize_cache", "decode_int8", "dequantize_cache", "qjl_encode", 
              "decode_qjl"]
 
 
+SWEEP_D = (128, 1024, 8192)
+SWEEP_TOTALS = (10 ** 6, 10 ** 7, 10 ** 8, 10 ** 9)
+
+
+def measure_sweep(stream, reps=3):
+    """The INT8 quantize/dequantize throughput sweep (fp32 and fp16 [N x D] tensors, D in
+    {128, 1024, 8192}, N = total // D for total in {1e6 .. 1e9}; N(0,1) values with 1% of
+    the columns x20): per point the device time of each kernel (the L2 flushed before
+    every timed launch), the reconstruction error max |x - x_hat| and mean |x - x_hat|,
+    and the attention-score error of one fp32 N(0,1) query, |q.x - q.x_hat| over all rows
+    (scores of the codes by kvq_int8_scores against the fp32 dot product of x)."""
+    import numpy as np
+    import torch
+    from kv_cache_quantization_absmax_b200 import inputs, kvq
+    dev = torch.device("cuda", torch.cuda.current_device())
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peak, _ = load_peaks()
+    out = []
+    idx = 0
+    for dtype in (np.float32, np.float16):
+        for d in SWEEP_D:
+            for total in SWEEP_TOTALS:
+                idx += 1
+                x, q, _ = inputs.sweep_matrix_device(total, d, dtype, 100 + idx, dev)
+                n = x.shape[0]
+                codes = torch.empty((n, d), dtype=torch.int8, device=dev)
+                scales = torch.empty((n,), dtype=torch.float32, device=dev)
+                xh = torch.empty_like(x)
+                # x is drawn on torch's current stream, whose freed temporaries the
+                # outputs above may reuse: the kernels on `stream` start after it is done
+                torch.cuda.synchronize()
+
+                def timed(fn):
+                    with torch.cuda.stream(stream):
+                        fn()                                   # warm-up
+                    ms = 0.0
+                    for _ in range(reps):
+                        with torch.cuda.stream(stream):
+                            flush.fill_(idx & 0xFF)
+                            e0 = torch.cuda.Event(enable_timing=True)
+                            e1 = torch.cuda.Event(enable_timing=True)
+                            e0.record(stream)
+                            fn()
+                            e1.record(stream)
+                        torch.cuda.synchronize()
+                        ms += e0.elapsed_time(e1)
+                    return ms / reps
+                b = x.element_size()
+                qms = timed(lambda: kvq.kvq_quantize_int8(x, codes, scales, stream=stream))
+                dms = timed(lambda: kvq.kvq_dequantize_int8(codes, scales, out=xh, stream=stream))
+                bytes_q = n * d * (b + 1) + 4 * n
+                # errors, in row chunks of at most 2^26 elements
+                qd = torch.from_numpy(q).to(dev)
+                sc = kvq.kvq_int8_scores(qd, codes, scales)
+                rmax = rsum = smax = ssum = 0.0
+                step = max(1, (1 << 26) // d)
+                for r0 in range(0, n, step):
+                    xs = x[r0:r0 + step].float()
+                    e = (xs - xh[r0:r0 + step].float()).abs_()
+                    rmax = max(rmax, float(e.max()))
+                    rsum += float(e.double().sum())
+                    se = (xs @ qd - sc[r0:r0 + step]).abs_()
+                    smax = max(smax, float(se.max()))
+                    ssum += float(se.double().sum())
+                torch.cuda.synchronize()
+                out.append({"dtype": "f16" if dtype == np.float16 else "f32", "d": d, "total": total, "rows": n,
+                            "quantize_ms": round(qms, 4), "quantize_GBps": round(bytes_q / (qms * 1e-3) / 1e9, 1),
+                            "quantize_frac": round(bytes_q / (qms * 1e-3) / 1e9 / peak, 4),
+                            "dequantize_ms": round(dms, 4), "dequantize_GBps": round(bytes_q / (dms * 1e-3) / 1e9, 1),
+                            "dequantize_frac": round(bytes_q / (dms * 1e-3) / 1e9 / peak, 4),
+                            "recon_max_abs": round(rmax, 6), "recon_mean_abs": round(rsum / (n * d), 7),
+                            "score_max_abs": round(smax, 6), "score_mean_abs": round(ssum / n, 7)})
+                del x, codes, scales, xh, sc
+    del flush
+    torch.cuda.empty_cache()
+    if kvq.kvq_device_error() != 0:
+        raise RuntimeError("device-side error recorded during the sweep")
+    return out
+
+
 def measure_next_rows(wl, stream, reps=3):
     """Device time of the widened rows (not part of the step): append-on-decode on the
     same caches, whose last row each call re-appends (the new key / value rows are the
@@ -269,6 +349,7 @@ def measure_next_rows(wl, stream, reps=3):
     s = ctypes.c_void_p(stream.cuda_stream)
     knew = wl.cache[:, :, :, :, T - 1].contiguous()          # [L, 2, B, H, D]
     gnew = wl.gcache[:, :, :, gt - 1].contiguous()            # [2, gb, gk, D]
+    torch.cuda.synchronize()   # made on torch's current stream, used on `stream`
     a7 = [kvq.make_decode_append_args(wl.q7[l], knew[l, 0], knew[l, 1], T=T - 1,
                                       k_codes=wl.codes[l, 0], k_scales=wl.scales[l, 0],
                                       v_codes=wl.codes[l, 1], v_scales=wl.scales[l, 1],
@@ -369,6 +450,7 @@ def measure_next_rows(wl, stream, reps=3):
     # ---- attention-sink eviction over one 7B-shaped layer: 4 sinks + 2044 of 4096 kept ----
     n_sink, n_keep = 4, T // 2
     mass = torch.zeros((B, T), dtype=torch.float32, device=wl.cache.device)
+    torch.cuda.synchronize()   # zero-filled on torch's current stream, used on `stream`
     am = [kvq.make_decode_mass_args(wl.q7[l], mass, k_codes=wl.codes[l, 0], k_scales=wl.scales[l, 0],
                                     v_codes=wl.codes[l, 1], v_scales=wl.scales[l, 1], out=wl.out7[l])
           for l in range(L)]
@@ -676,6 +758,7 @@ def run_gpu(args):
                "unavailable": str(exc)[:200]}
 
     next_rows = measure_next_rows(wl, stream)
+    sweep = measure_sweep(stream) if not args.no_sweep else None
     barrier()
 
     if rank == 0:
@@ -702,6 +785,7 @@ def run_gpu(args):
                          "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs"},
             "e2e": e2e,
             "next_rows": next_rows,
+            "sweep": sweep,
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clocks,
         }
@@ -847,6 +931,7 @@ def main(argv=None):
     p.add_argument("--cpu-scale", type=float, default=8.0,
                    help="size of the oracle sample for the cpu_baseline key")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-sweep", action="store_true", help="skip the quantize/dequantize throughput sweep")
     p.add_argument("--profile-case", default=None,
                    help="run one small single-kernel case (quantize, dequantize, decode_int8, "
                         "qjl_encode, decode_qjl, int4_quantize, int4_dequantize, cw_quantize, "
