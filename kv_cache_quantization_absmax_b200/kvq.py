@@ -134,8 +134,16 @@ def _ptr(t):
 
 
 def _stream(stream=None):
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes.c_void_p(s.cuda_stream)
+    """The stream to enqueue on: torch's current stream, or the one given.  A given stream
+    first waits for the current one, where the inputs were made and the outputs
+    allocated (torch may hand an output a block that work on the current stream still
+    touches)."""
+    cur = torch.cuda.current_stream()
+    if stream is None:
+        return ctypes.c_void_p(cur.cuda_stream)
+    if stream.cuda_stream != cur.cuda_stream:
+        stream.wait_stream(cur)
+    return ctypes.c_void_p(stream.cuda_stream)
 
 
 def _dtype_code(t):
