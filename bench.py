@@ -612,6 +612,84 @@ class CpuSample:
         return r
 
 
+def cpu_next_rates():
+    """The single-threaded C oracle on a bounded sample of each widened row (a few seconds
+    in all), as GB/s by the same byte counts per unit as the GPU rows in `next_rows`."""
+    import numpy as np
+
+    import oracle
+    from kv_cache_quantization_absmax_b200 import inputs
+
+    D, m, T = 128, GQA["m"], LLAMA["seq"]
+    r = {}
+
+    def timed(fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    # INT8 cache of 2 units x 4096 tokens; appended token at T - 1
+    k, v = inputs.lognormal_cache(61, 2, 1, T, n_tensors=2)
+    kc, ks = oracle.quantize_int8(k.reshape(-1, D))
+    vc, vs = oracle.quantize_int8(v.reshape(-1, D))
+    shp = (2, 1, T)
+    c8 = dict(k_codes=kc.reshape(shp + (D,)), k_scales=ks.reshape(shp), v_codes=vc.reshape(shp + (D,)),
+              v_scales=vs.reshape(shp))
+    q = inputs.gaussian_queries(62, 2, 1)
+    kn = k[:, :, T - 1].copy()
+    vn = v[:, :, T - 1].copy()
+    dt = timed(lambda: oracle.decode_append(q, kn, vn, T=T - 1, **c8))
+    r["append_int8"] = 2 * T * 2 * (D + 4) / dt / 1e9
+    dt = timed(lambda: (oracle.decode_attention(q, **c8), oracle.attention_mass(q, **c8)))
+    r["decode_int8_mass"] = 2 * T * (2 * (D + 4) + 12) / dt / 1e9
+    mass = oracle.attention_mass(q, **c8).astype(np.float32)
+    dt = timed(lambda: oracle.evict_select(mass, 4, T // 2))
+    r["evict_select"] = 2 * (T * 4 + (T // 2) * 4) / dt / 1e9
+    kept = oracle.evict_select(mass, 4, T // 2)
+    cache = kc.reshape(2, 1, T, D)
+    dt = timed(lambda: oracle.gather_rows(cache, kept))
+    r["evict_compact"] = 2 * (T // 2) * D * 2 / dt / 1e9
+    # group-wise INT4 and channel-wise INT8 on 65536 rows of 128 fp16
+    x = inputs.lognormal_cache(63, 1, 16, 4096)[0].reshape(-1, D)
+    n = x.shape[0]
+    dt = timed(lambda: oracle.quantize_int4_group(x, 32))
+    r["int4_quantize"] = n * (D * 2.5 + 32) / dt / 1e9
+    p4, s4, z4 = oracle.quantize_int4_group(x, 32)
+    dt = timed(lambda: oracle.dequantize_int4_group(p4, s4, z4, 32, np.float16))
+    r["int4_dequantize"] = n * (D * 2.5 + 32) / dt / 1e9
+    blocks = x.reshape(16, 4096, D)
+    dt = timed(lambda: oracle.quantize_int8_channelwise(blocks))
+    r["int8_channelwise_quantize"] = n * D * 3 / dt / 1e9
+    cwc, cws = oracle.quantize_int8_channelwise(blocks)
+    dt = timed(lambda: oracle.dequantize_int8_channelwise(cwc, cws, np.float16))
+    r["int8_channelwise_dequantize"] = n * D * 3 / dt / 1e9
+    pv, sv, zv = oracle.quantize_int4_group(v.reshape(-1, D), 32)
+    v4 = (pv.reshape(shp + (D // 2,)), sv.reshape(shp + (4,)), zv.reshape(shp + (4,)), 32)
+    dt = timed(lambda: oracle.decode_attention(q, k_codes=c8["k_codes"], k_scales=c8["k_scales"], v4=v4))
+    r["decode_int8k_int4v"] = 2 * T * (D + 4 + D // 2 + 32) / dt / 1e9
+    # QJL-family rows on 8192 keys of one GQA unit (4 query heads)
+    gt = 8192
+    kg, vg = inputs.lognormal_cache(64, 1, 1, gt, n_tensors=2)
+    S = inputs.sketch_matrix(m, D)
+    w, nr = oracle.qjl_encode(kg.reshape(-1, D), S)
+    vgc, vgs = oracle.quantize_int8(vg.reshape(-1, D))
+    gs = (1, 1, gt)
+    cq = dict(k_words=w.reshape(gs + (m // 32,)), k_norms=nr.reshape(gs), S=S, v_codes=vgc.reshape(gs + (D,)),
+              v_scales=vgs.reshape(gs))
+    qg = inputs.gaussian_queries(65, 1, 4)
+    dt = timed(lambda: oracle.decode_append(qg, kg[:, :, gt - 1].copy(), vg[:, :, gt - 1].copy(), T=gt - 1, **cq))
+    r["append_qjl"] = gt * (m // 8 + 2 + D + 4) / dt / 1e9
+    dt = timed(lambda: oracle.qjl_residual_encode(kg.reshape(-1, D), 32, S))
+    r["qjlres_encode"] = gt * (2 * D + D // 2 + 32 + 2 * D + m // 8 + 2) / dt / 1e9
+    e = oracle.qjl_residual_encode(kg.reshape(-1, D), 32, S)
+    cr = dict(k4=(e["packed"].reshape(gs + (D // 2,)), e["scales"].reshape(gs + (4,)), e["zeros"].reshape(gs + (4,)), 32),
+              k_words=e["words"].reshape(gs + (m // 32,)), k_norms=e["rnorms"].reshape(gs), S=S,
+              v_codes=cq["v_codes"], v_scales=cq["v_scales"])
+    dt = timed(lambda: oracle.decode_attention(qg, **cr))
+    r["decode_qjlres"] = gt * (D // 2 + 32 + m // 8 + 2 + D + 4) / dt / 1e9
+    return r
+
+
 def cpu_step_gbs(rates):
     rb = row_bytes()
     t = sum(rb[k] / 1e9 / rates[k] for k in rb)
@@ -794,6 +872,10 @@ def run_gpu(args):
             v, _ = cpu_step_gbs(smp.rates())
             line["cpu_baseline"] = {"value": round(v, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                                     "sample": smp.description}
+            # the widened rows: the same oracle on small samples of each
+            for k, g in cpu_next_rates().items():
+                if k in next_rows:
+                    next_rows[k]["cpu_oracle_GBps"] = round(g, 5)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
