@@ -481,19 +481,18 @@ def measure_next_rows(wl, stream, reps=3):
     kdst = torch.empty((2, B, H, n_keep, D), dtype=torch.int8, device=wl.cache.device)
     sdst = torch.empty((2, B, H, n_keep), dtype=torch.float32, device=wl.cache.device)
 
-    gathers = []
+    garr = (kvq.GatherArray * 4)()
     for t in range(2):
-        gathers.append((P(wl.codes[0, t].data_ptr()), P(kdst[t].data_ptr()), D))
-        gathers.append((P(wl.scales[0, t].data_ptr()), P(sdst[t].data_ptr()), 4))
+        garr[2 * t] = kvq.GatherArray(wl.codes[0, t].data_ptr(), kdst[t].data_ptr(), T, n_keep, D)
+        garr[2 * t + 1] = kvq.GatherArray(wl.scales[0, t].data_ptr(), sdst[t].data_ptr(), T, n_keep, 4)
 
     def compact():
-        for src, dst, row_bytes in gathers:
-            st = lib.kvq_gather_rows(src, dst, B, H, T, n_keep, row_bytes, P(kept.data_ptr()), n_keep, s)
-            if st != kvq.KVQ_OK:
-                raise kvq.KvqError("kvq_gather_rows", st)
+        st = lib.kvq_gather_rows_multi(garr, 4, B, H, P(kept.data_ptr()), n_keep, s)
+        if st != kvq.KVQ_OK:
+            raise kvq.KvqError("kvq_gather_rows_multi", st)
     ms = timed(compact)
-    row("evict_compact", ms, 2 * 2 * B * H * n_keep * (D + 4) + 4 * B * n_keep * 4,
-        "7B-shaped layer: INT8 K/V codes + scales [8, 32, 4096] -> the 2048 kept tokens (4 launches)")
+    row("evict_compact", ms, 2 * 2 * B * H * n_keep * (D + 4) + B * n_keep * 4,
+        "7B-shaped layer: INT8 K/V codes + scales [8, 32, 4096] -> the 2048 kept tokens (one launch)")
     del mass, mws, kdst, sdst
 
     # ---- QJL as the 1-bit residual of group-wise INT4 (groups of 32), GQA cache keys ----

@@ -369,6 +369,25 @@ kvq_status kvq_gather_rows(const void* src, void* dst, int64_t batch, int64_t n_
                            kvq_stream_t stream);
 
 /*
+ * kvq_gather_rows_multi -- kvq_gather_rows for up to 8 arrays of the same cache (for
+ * example K codes, K scales, V codes, V scales) in one launch, all compacted to the
+ * same kept tokens.  arrays[i] gives src, dst, src_rows, dst_rows and row_bytes of one
+ * array, with the rules of kvq_gather_rows for each (the array list itself is read on
+ * the host before the launch).  n_arrays in 1..8 (else KVQ_ERR_INVALID_ARG; 0 with
+ * nothing to do: KVQ_OK).  A bad kept index: code 0x301 as kvq_gather_rows.
+ */
+typedef struct kvq_gather_array {
+    const void* src;
+    void* dst;
+    int64_t src_rows;
+    int64_t dst_rows;
+    int64_t row_bytes;
+} kvq_gather_array;
+
+kvq_status kvq_gather_rows_multi(const kvq_gather_array* arrays, int32_t n_arrays, int64_t batch, int64_t n_heads,
+                                 const int32_t* kept, int64_t n_keep, kvq_stream_t stream);
+
+/*
  * kvq_decode_attention_qjlres -- the decode step of kvq_decode_attention over keys
  * stored by kvq_qjl_residual_encode (group-wise INT4 + the 1-bit QJL sketch of the INT4
  * residual), INT8 values.  Per cached token t and query head h (KV head h / G):

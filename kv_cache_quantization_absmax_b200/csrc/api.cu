@@ -402,6 +402,25 @@ KVQ_API kvq_status kvq_gather_rows(const void* src, void* dst, int64_t batch, in
                                              cs(stream)));
 }
 
+KVQ_API kvq_status kvq_gather_rows_multi(const kvq_gather_array* arrays, int32_t n_arrays, int64_t batch,
+                                         int64_t n_heads, const int32_t* kept, int64_t n_keep, kvq_stream_t stream) {
+    if (n_arrays < 0 || n_arrays > 8 || batch < 0 || n_heads < 0 || n_keep < 0 || n_heads > INT32_MAX)
+        return KVQ_ERR_INVALID_ARG;
+    if (n_arrays > 0 && !arrays) return KVQ_ERR_INVALID_ARG;
+    kvq::GatherArray ga[8];
+    for (int i = 0; i < n_arrays; ++i) {
+        const kvq_gather_array& g = arrays[i];
+        if (g.row_bytes < 1 || g.src_rows < 1 || g.dst_rows < n_keep || n_keep * g.row_bytes >= ((int64_t)1 << 31))
+            return KVQ_ERR_INVALID_ARG;
+        ga[i] = kvq::GatherArray{g.src, g.dst, g.src_rows, g.dst_rows, g.row_bytes};
+    }
+    if (n_arrays == 0 || batch == 0 || n_heads == 0 || n_keep == 0) return KVQ_OK;
+    if (!kept || !aligned(kept, 4)) return KVQ_ERR_INVALID_ARG;
+    for (int i = 0; i < n_arrays; ++i)
+        if (!ga[i].src || !ga[i].dst) return KVQ_ERR_INVALID_ARG;
+    return from_cuda(kvq::launch_gather_rows_multi(ga, n_arrays, batch, n_heads, kept, n_keep, cs(stream)));
+}
+
 namespace {
 
 // Residual keys: the decode arguments carry the residual's sign words, norms and the

@@ -208,48 +208,168 @@ __global__ void __launch_bounds__(kSelThreads) evict_select_kernel(const float* 
 constexpr int kGatherThreads = 256;
 constexpr int kGatherUnroll = 8;  // pieces in flight per lane
 
-// dst[bh][j] = src[bh][kept[b][j]] for rows of `units` UNITs, j < n_keep (bh = b * H + h).
-// A warp moves 32 consecutive kept rows of one (b, h) at a time: one coalesced load of
-// their 32 indices, then the rows' pieces in lane order, kGatherUnroll loads in flight
-// per lane before the stores (which are contiguous in dst).  A kept index outside
-// [0, src_rows) is recorded in g_evict_error and that row is skipped.
+// Warp-level copy of kGatherRows (32) consecutive kept rows (from j0) of one (b, h): one
+// coalesced load of their indices, then the rows' UNIT pieces in lane order,
+// kGatherUnroll loads in flight per lane before the stores (contiguous in dst).  A kept
+// index outside [0, src_rows) is recorded in g_evict_error and that row is skipped.
+// (64-row items with 16 pieces in flight measured slower on B200.)
+constexpr int kGatherRows = 32;
+
+template <typename UNIT>
+__device__ __forceinline__ void gather_group(const UNIT* __restrict__ src, UNIT* __restrict__ dst, int64_t bh,
+                                             int H, int64_t src_rows, int64_t dst_rows, int units, int ushift,
+                                             const int32_t* __restrict__ kept, int n_keep, int j0, int lane) {
+    const int nrows = min(kGatherRows, n_keep - j0);
+    int32_t r_lane = -1;
+    if (lane < nrows) {
+        r_lane = __ldg(kept + (bh / H) * n_keep + j0 + lane);
+        if (r_lane < 0 || r_lane >= src_rows) {
+            atomicCAS(&g_evict_error, 0u, kErrGatherIndex);
+            r_lane = -1;
+        }
+    }
+    const UNIT* s = src + bh * src_rows * units;
+    UNIT* d = dst + (bh * dst_rows + j0) * units;
+    const int pieces = nrows * units;
+    for (int p0 = 0; p0 < pieces; p0 += 32 * kGatherUnroll) {
+        UNIT v[kGatherUnroll];
+        bool ok[kGatherUnroll];
+#pragma unroll
+        for (int k = 0; k < kGatherUnroll; ++k) {
+            const int p = p0 + k * 32 + lane;
+            const int jj = p < pieces ? (ushift >= 0 ? (p >> ushift) : p / units) : 0;
+            const int32_t r = __shfl_sync(0xffffffffu, r_lane, jj);
+            ok[k] = p < pieces && r >= 0;
+            if (ok[k]) v[k] = __ldcs(s + (int64_t)r * units + (p - jj * units));
+        }
+#pragma unroll
+        for (int k = 0; k < kGatherUnroll; ++k)
+            if (ok[k]) d[p0 + k * 32 + lane] = v[k];
+    }
+}
+
+// Rows of a single UNIT (4-16 B): a warp item covers kGatherSmallRows (256) kept rows,
+// a lane takes rows j0 + lane + 32 k with their 8 indices and 8 data loads in flight.
+constexpr int kGatherSmallRows = 256;
+
+template <typename UNIT>
+__device__ __forceinline__ void gather_group_small(const UNIT* __restrict__ src, UNIT* __restrict__ dst, int64_t bh,
+                                                   int H, int64_t src_rows, int64_t dst_rows,
+                                                   const int32_t* __restrict__ kept, int n_keep, int j0, int lane) {
+    constexpr int K = kGatherSmallRows / 32;
+    const int32_t* kb = kept + (bh / H) * n_keep;
+    const UNIT* s = src + bh * src_rows;
+    UNIT* d = dst + bh * dst_rows;
+    int32_t r[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        const int j = j0 + lane + 32 * k;
+        r[k] = j < n_keep ? __ldg(kb + j) : -1;
+        if (j < n_keep && (r[k] < 0 || r[k] >= src_rows)) {
+            atomicCAS(&g_evict_error, 0u, kErrGatherIndex);
+            r[k] = -1;
+        }
+    }
+    UNIT v[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+        if (r[k] >= 0) v[k] = __ldcs(s + r[k]);
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+        if (r[k] >= 0) d[j0 + lane + 32 * k] = v[k];
+}
+
+// dst[bh][j] = src[bh][kept[b][j]] for rows of `units` UNITs, j < n_keep (bh = b * H + h):
+// a warp per 32 kept rows of one (b, h).
 template <typename UNIT>
 __global__ void __launch_bounds__(kGatherThreads) gather_rows_kernel(
     const UNIT* __restrict__ src, UNIT* __restrict__ dst, int64_t BH, int H, int64_t src_rows, int64_t dst_rows,
     int units, int ushift, const int32_t* __restrict__ kept, int n_keep) {
     const int lane = threadIdx.x & 31;
-    const int groups = (n_keep + 31) >> 5;
+    const int rows_item = units == 1 ? kGatherSmallRows : kGatherRows;
+    const int groups = (n_keep + rows_item - 1) / rows_item;
     const int64_t n_work = BH * groups;
     const int64_t n_warps = (int64_t)gridDim.x * (kGatherThreads / 32);
     for (int64_t w = (int64_t)blockIdx.x * (kGatherThreads / 32) + (threadIdx.x >> 5); w < n_work; w += n_warps) {
         const int64_t bh = w / groups;
-        const int j0 = (int)(w - bh * groups) << 5;
-        const int nrows = min(32, n_keep - j0);
-        int32_t r_lane = -1;
-        if (lane < nrows) {
-            r_lane = __ldg(kept + (bh / H) * n_keep + j0 + lane);
-            if (r_lane < 0 || r_lane >= src_rows) {
-                atomicCAS(&g_evict_error, 0u, kErrGatherIndex);
-                r_lane = -1;
+        const int j0 = (int)(w - bh * groups) * rows_item;
+        if (units == 1)
+            gather_group_small<UNIT>(src, dst, bh, H, src_rows, dst_rows, kept, n_keep, j0, lane);
+        else
+            gather_group<UNIT>(src, dst, bh, H, src_rows, dst_rows, units, ushift, kept, n_keep, j0, lane);
+    }
+}
+
+// Several arrays compacted in one launch: the warps walk the arrays' work items one
+// array after another; each array moves in the widest unit its rows and bases allow.
+constexpr int kMaxGatherArrays = 8;
+struct GatherSet {
+    const void* src[kMaxGatherArrays];
+    void* dst[kMaxGatherArrays];
+    int64_t src_rows[kMaxGatherArrays];
+    int64_t dst_rows[kMaxGatherArrays];
+    int64_t work_end[kMaxGatherArrays];   // cumulative warp work items
+    int units[kMaxGatherArrays];
+    int ushift[kMaxGatherArrays];
+    int unit_bytes[kMaxGatherArrays];
+    int rows_item[kMaxGatherArrays];      // kept rows per warp item
+    int n;
+};
+
+__global__ void __launch_bounds__(kGatherThreads, 2) gather_multi_kernel(const GatherSet gs, int H,
+                                                                      const int32_t* __restrict__ kept, int n_keep) {
+    const int lane = threadIdx.x & 31;
+    const int64_t n_work = gs.work_end[gs.n - 1];
+    const int64_t n_warps = (int64_t)gridDim.x * (kGatherThreads / 32);
+    for (int64_t w = (int64_t)blockIdx.x * (kGatherThreads / 32) + (threadIdx.x >> 5); w < n_work; w += n_warps) {
+        int a = 0;
+        while (a + 1 < gs.n && w >= gs.work_end[a]) ++a;
+        const int64_t local = w - (a > 0 ? gs.work_end[a - 1] : 0);
+        const int rows_item = gs.rows_item[a];
+        const int groups = (n_keep + rows_item - 1) / rows_item;
+        const int64_t bh = local / groups;
+        const int j0 = (int)(local - bh * groups) * rows_item;
+        if (gs.units[a] == 1) {
+            switch (gs.unit_bytes[a]) {
+                case 16:
+                    gather_group_small<uint4>(static_cast<const uint4*>(gs.src[a]), static_cast<uint4*>(gs.dst[a]), bh,
+                                              H, gs.src_rows[a], gs.dst_rows[a], kept, n_keep, j0, lane);
+                    break;
+                case 4:
+                    gather_group_small<uint32_t>(static_cast<const uint32_t*>(gs.src[a]),
+                                                 static_cast<uint32_t*>(gs.dst[a]), bh, H, gs.src_rows[a],
+                                                 gs.dst_rows[a], kept, n_keep, j0, lane);
+                    break;
+                case 2:
+                    gather_group_small<uint16_t>(static_cast<const uint16_t*>(gs.src[a]),
+                                                 static_cast<uint16_t*>(gs.dst[a]), bh, H, gs.src_rows[a],
+                                                 gs.dst_rows[a], kept, n_keep, j0, lane);
+                    break;
+                default:
+                    gather_group_small<uint8_t>(static_cast<const uint8_t*>(gs.src[a]), static_cast<uint8_t*>(gs.dst[a]),
+                                                bh, H, gs.src_rows[a], gs.dst_rows[a], kept, n_keep, j0, lane);
             }
+            continue;
         }
-        const UNIT* s = src + bh * src_rows * units;
-        UNIT* d = dst + (bh * dst_rows + j0) * units;
-        const int pieces = nrows * units;
-        for (int p0 = 0; p0 < pieces; p0 += 32 * kGatherUnroll) {
-            UNIT v[kGatherUnroll];
-            bool ok[kGatherUnroll];
-#pragma unroll
-            for (int k = 0; k < kGatherUnroll; ++k) {
-                const int p = p0 + k * 32 + lane;
-                const int jj = p < pieces ? (ushift >= 0 ? (p >> ushift) : p / units) : 0;
-                const int32_t r = __shfl_sync(0xffffffffu, r_lane, jj);
-                ok[k] = p < pieces && r >= 0;
-                if (ok[k]) v[k] = __ldcs(s + (int64_t)r * units + (p - jj * units));
-            }
-#pragma unroll
-            for (int k = 0; k < kGatherUnroll; ++k)
-                if (ok[k]) d[p0 + k * 32 + lane] = v[k];
+        switch (gs.unit_bytes[a]) {
+            case 16:
+                gather_group<uint4>(static_cast<const uint4*>(gs.src[a]), static_cast<uint4*>(gs.dst[a]), bh, H,
+                                    gs.src_rows[a], gs.dst_rows[a], gs.units[a], gs.ushift[a], kept, n_keep, j0, lane);
+                break;
+            case 4:
+                gather_group<uint32_t>(static_cast<const uint32_t*>(gs.src[a]), static_cast<uint32_t*>(gs.dst[a]), bh,
+                                       H, gs.src_rows[a], gs.dst_rows[a], gs.units[a], gs.ushift[a], kept, n_keep, j0,
+                                       lane);
+                break;
+            case 2:
+                gather_group<uint16_t>(static_cast<const uint16_t*>(gs.src[a]), static_cast<uint16_t*>(gs.dst[a]), bh,
+                                       H, gs.src_rows[a], gs.dst_rows[a], gs.units[a], gs.ushift[a], kept, n_keep, j0,
+                                       lane);
+                break;
+            default:
+                gather_group<uint8_t>(static_cast<const uint8_t*>(gs.src[a]), static_cast<uint8_t*>(gs.dst[a]), bh, H,
+                                      gs.src_rows[a], gs.dst_rows[a], gs.units[a], gs.ushift[a], kept, n_keep, j0,
+                                      lane);
         }
     }
 }
@@ -299,7 +419,8 @@ cudaError_t launch_gather_rows(const void* src, void* dst, int64_t B, int64_t H,
     const int ub = (al % 16 == 0) ? 16 : (al % 4 == 0) ? 4 : (al % 2 == 0) ? 2 : 1;
     const int units = (int)(row_bytes / ub);
     const int ushift = (units & (units - 1)) == 0 ? __builtin_ctz((unsigned)units) : -1;
-    const int64_t work = BH * ((n_keep + 31) / 32);  // warps' units of work
+    const int64_t rows_item = (row_bytes / ub == 1) ? kGatherSmallRows : kGatherRows;
+    const int64_t work = BH * ((n_keep + rows_item - 1) / rows_item);  // warps' units of work
     const int64_t want = (work + kGatherThreads / 32 - 1) / (kGatherThreads / 32);
     const int64_t cap = (int64_t)device_sm_count() * 16;  // about 4 waves of 4 resident CTAs
     dim3 grid((unsigned)(want < cap ? want : cap));
@@ -325,6 +446,47 @@ cudaError_t launch_gather_rows(const void* src, void* dst, int64_t B, int64_t H,
                 static_cast<const uint8_t*>(src), static_cast<uint8_t*>(dst), BH, Hi, src_rows, dst_rows, units,
                 ushift, kept, nk);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows_multi(const GatherArray* arrays, int n_arrays, int64_t B, int64_t H,
+                                     const int32_t* kept, int64_t n_keep, cudaStream_t st) {
+    const int64_t BH = B * H;
+    if (BH == 0 || n_keep == 0 || n_arrays == 0) return cudaSuccess;
+    if (n_arrays > kMaxGatherArrays) return cudaErrorInvalidValue;
+    GatherSet gs{};
+    gs.n = n_arrays;
+    // arrays with short rows first: their warps wait mostly on the index and data
+    // latency, which the long-row arrays' streaming then overlaps
+    int order[kMaxGatherArrays];
+    for (int a = 0; a < n_arrays; ++a) order[a] = a;
+    for (int a = 1; a < n_arrays; ++a)
+        for (int b = a; b > 0 && arrays[order[b]].row_bytes < arrays[order[b - 1]].row_bytes; --b) {
+            const int t = order[b];
+            order[b] = order[b - 1];
+            order[b - 1] = t;
+        }
+    int64_t acc = 0;
+    for (int a = 0; a < n_arrays; ++a) {
+        const GatherArray& g = arrays[order[a]];
+        const uintptr_t al = reinterpret_cast<uintptr_t>(g.src) | reinterpret_cast<uintptr_t>(g.dst) |
+                             (uintptr_t)g.row_bytes;
+        const int ub = (al % 16 == 0) ? 16 : (al % 4 == 0) ? 4 : (al % 2 == 0) ? 2 : 1;
+        const int units = (int)(g.row_bytes / ub);
+        gs.src[a] = g.src;
+        gs.dst[a] = g.dst;
+        gs.src_rows[a] = g.src_rows;
+        gs.dst_rows[a] = g.dst_rows;
+        gs.units[a] = units;
+        gs.ushift[a] = (units & (units - 1)) == 0 ? __builtin_ctz((unsigned)units) : -1;
+        gs.unit_bytes[a] = ub;
+        gs.rows_item[a] = units == 1 ? kGatherSmallRows : kGatherRows;
+        acc += BH * ((n_keep + gs.rows_item[a] - 1) / gs.rows_item[a]);
+        gs.work_end[a] = acc;
+    }
+    const int64_t want = (acc + kGatherThreads / 32 - 1) / (kGatherThreads / 32);
+    const int64_t cap = (int64_t)device_sm_count() * 16;
+    gather_multi_kernel<<<(unsigned)(want < cap ? want : cap), kGatherThreads, 0, st>>>(gs, (int)H, kept, (int)n_keep);
     return cudaGetLastError();
 }
 

@@ -94,6 +94,13 @@ cudaError_t launch_evict_select(const float* mass, int64_t B, int64_t T, int64_t
 cudaError_t launch_gather_rows(const void* src, void* dst, int64_t B, int64_t H, int64_t src_rows,
                                int64_t dst_rows, int64_t row_bytes, const int32_t* kept, int64_t n_keep,
                                cudaStream_t st);
+struct GatherArray {
+    const void* src;
+    void* dst;
+    int64_t src_rows, dst_rows, row_bytes;
+};
+cudaError_t launch_gather_rows_multi(const GatherArray* arrays, int n_arrays, int64_t B, int64_t H,
+                                     const int32_t* kept, int64_t n_keep, cudaStream_t st);
 cudaError_t read_and_clear_evict_error(uint32_t* code);
 
 }  // namespace kvq

@@ -47,6 +47,11 @@ class DecodeInt4vArgs(ctypes.Structure):
                 ("v_group", _I32)]
 
 
+class GatherArray(ctypes.Structure):
+    """Mirror of ``kvq_gather_array``."""
+    _fields_ = [("src", _P), ("dst", _P), ("src_rows", _I64), ("dst_rows", _I64), ("row_bytes", _I64)]
+
+
 class DecodeQjlresArgs(ctypes.Structure):
     """Mirror of ``kvq_decode_qjlres_args``."""
     _fields_ = [("base", DecodeArgs), ("k_packed4", _P), ("k_scales4", _P), ("k_zeros4", _P),
@@ -106,6 +111,8 @@ def _load():
     so.kvq_evict_select.restype = ctypes.c_int
     so.kvq_gather_rows.argtypes = [_P, _P, _I64, _I64, _I64, _I64, _I64, _P, _I64, _P]
     so.kvq_gather_rows.restype = ctypes.c_int
+    so.kvq_gather_rows_multi.argtypes = [ctypes.POINTER(GatherArray), _I32, _I64, _I64, _P, _I64, _P]
+    so.kvq_gather_rows_multi.restype = ctypes.c_int
     so.kvq_decode_attention_qjlres.argtypes = [ctypes.POINTER(DecodeQjlresArgs), _P]
     so.kvq_decode_attention_qjlres.restype = ctypes.c_int
     so.kvq_decode_qjlres_workspace_bytes.argtypes = [ctypes.POINTER(DecodeQjlresArgs)]
@@ -583,3 +590,25 @@ def kvq_decode_attention_qjlres(q, *, k_packed4, k_scales4, k_zeros4, k_group, k
     a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel()
     _check("kvq_decode_attention_qjlres", lib.kvq_decode_attention_qjlres(ctypes.byref(a), _stream(stream)))
     return (out if want_out else None), (scores_out if want_scores else None)
+
+
+def kvq_gather_rows_multi(srcs, kept, dsts=None, stream=None):
+    """kvq_gather_rows for several arrays [B, H, T, ...] of one cache in one launch;
+    returns the list of compacted arrays."""
+    _need_cuda(kept, *srcs)
+    if kept.dtype != torch.int32:
+        raise ValueError("kept must be int32")
+    B, H = srcs[0].shape[:2]
+    n_keep = kept.shape[1]
+    if dsts is None:
+        dsts = [torch.empty((B, H, n_keep) + tuple(x.shape[3:]), dtype=x.dtype, device=x.device) for x in srcs]
+    arr = (GatherArray * max(1, len(srcs)))()
+    for i, (x, y) in enumerate(zip(srcs, dsts)):
+        _need_cuda(y)
+        if tuple(x.shape[:2]) != (B, H) or y.dtype != x.dtype or y.shape[:2] != x.shape[:2] or y.shape[3:] != x.shape[3:]:
+            raise ValueError("every array is [B, H, T, ...] with dst matching src except along the token axis")
+        arr[i] = GatherArray(x.data_ptr(), y.data_ptr(), x.shape[2], y.shape[2],
+                             x[0, 0, 0].numel() * x.element_size())
+    _check("kvq_gather_rows_multi", lib.kvq_gather_rows_multi(arr, len(srcs), B, H, _ptr(kept), n_keep,
+                                                              _stream(stream)))
+    return dsts

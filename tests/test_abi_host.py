@@ -195,3 +195,21 @@ def test_qjlres_rejects_bad_arguments(kvq):
     r.base.sketch_dim = 256
     r.base.key_format = kvq.KVQ_KEYS_INT8
     assert call() == E
+
+
+def test_gather_multi_rejects_bad_arguments(kvq):
+    L = kvq.lib
+    E = kvq.KVQ_ERR_INVALID_ARG
+    arr = (kvq.GatherArray * 9)()
+    for i in range(9):
+        arr[i] = kvq.GatherArray(A16, A16, 100, 10, 128)
+    assert L.kvq_gather_rows_multi(arr, 9, 2, 4, _p(A16), 10, None) == E          # too many arrays
+    assert L.kvq_gather_rows_multi(None, 2, 2, 4, _p(A16), 10, None) == E
+    arr[1] = kvq.GatherArray(A16, A16, 100, 9, 128)                             # dst_rows < n_keep
+    assert L.kvq_gather_rows_multi(arr, 2, 2, 4, _p(A16), 10, None) == E
+    arr[1] = kvq.GatherArray(A16, A16, 100, 10, 0)                              # row_bytes
+    assert L.kvq_gather_rows_multi(arr, 2, 2, 4, _p(A16), 10, None) == E
+    arr[1] = kvq.GatherArray(A16, A16, 100, 10, 4)
+    assert L.kvq_gather_rows_multi(arr, 2, 2, 4, _p(A16 + 2), 10, None) == E    # kept alignment
+    assert L.kvq_gather_rows_multi(arr, 0, 2, 4, None, 10, None) == kvq.KVQ_OK
+    assert L.kvq_gather_rows_multi(arr, 2, 2, 4, None, 0, None) == kvq.KVQ_OK

@@ -269,3 +269,38 @@ def test_evict_llama7b_layer_sampled(kvq):
         assert np.array_equal(to_np(kc2[b, h]), to_np(kc[b, h])[k_np[b]])
         assert np.array_equal(to_np(ks2[b, h]), to_np(ks[b, h])[k_np[b]])
     assert kvq.kvq_device_error() == 0
+
+
+def test_gather_rows_multi_exact(kvq):
+    """One launch compacts arrays of different row sizes and alignments (INT8 codes,
+    fp32 scales, int32 sign words, fp16 norms, odd-byte rows at an odd offset) exactly as
+    the oracle's compaction of each."""
+    B, H, T = 3, 4, 700
+    g = torch.Generator().manual_seed(5)
+    shapes = [((B, H, T, 128), torch.int8), ((B, H, T), torch.float32), ((B, H, T, 8), torch.int32),
+              ((B, H, T), torch.float16), ((B, H, T, 3), torch.uint8)]
+    srcs = [torch.randint(-100, 100, sh, generator=g).to(dt).cuda() for sh, dt in shapes]
+    raw = torch.randint(0, 255, (B * H * T * 5 + 1,), dtype=torch.uint8).cuda()
+    srcs.append(raw[1:].view(B, H, T, 5))                                  # 1-byte aligned rows
+    mass = np.random.default_rng(11).random((B, T), dtype=np.float32)
+    kept = oracle.evict_select(mass, 4, 333)
+    dsts = kvq.kvq_gather_rows_multi(srcs, _cuda(kept)[0])
+    for x, y in zip(srcs, dsts):
+        assert np.array_equal(to_np(y), oracle.gather_rows(to_np(x), kept))
+    assert kvq.kvq_device_error() == 0
+
+
+def test_gather_rows_multi_matches_single_calls_at_layer_size(kvq):
+    """The 7B-shaped layer's K/V codes and scales [8, 32, 4096] compacted to 2048 tokens:
+    one multi-array launch equals four single-array launches, byte for byte."""
+    B, H, T = 8, 32, 4096
+    g = torch.Generator(device="cuda").manual_seed(3)
+    codes = [torch.randint(-127, 128, (B, H, T, 128), generator=g, device="cuda", dtype=torch.int32).to(torch.int8)
+             for _ in range(2)]
+    scales = [torch.rand((B, H, T), generator=g, device="cuda") for _ in range(2)]
+    mass = torch.rand((B, T), generator=g, device="cuda")
+    kept = kvq.kvq_evict_select(mass, 4, 2048)
+    multi = kvq.kvq_gather_rows_multi(codes + scales, kept)
+    for x, y in zip(codes + scales, multi):
+        assert torch.equal(y, kvq.kvq_gather_rows(x, kept))
+    assert kvq.kvq_device_error() == 0
