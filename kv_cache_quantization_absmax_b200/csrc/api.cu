@@ -443,14 +443,14 @@ kvq_status check_qjlres(const kvq_decode_qjlres_args* a) {
 
 KVQ_API size_t kvq_decode_qjlres_workspace_bytes(const kvq_decode_qjlres_args* a) {
     if (check_qjlres(a) != KVQ_OK || a->base.batch == 0) return 0;
-    return kvq::plan_decode(&a->base, kvq::device_sm_count(), true).total_bytes;
+    return kvq::plan_decode(&a->base, kvq::device_sm_count()).total_bytes;
 }
 
 KVQ_API kvq_status kvq_decode_attention_qjlres(const kvq_decode_qjlres_args* a, kvq_stream_t stream) {
     const kvq_status st = check_qjlres(a);
     if (st != KVQ_OK) return st;
     if (a->base.batch == 0) return KVQ_OK;
-    const kvq::DecodePlan plan = kvq::plan_decode(&a->base, kvq::device_sm_count(), true);
+    const kvq::DecodePlan plan = kvq::plan_decode(&a->base, kvq::device_sm_count());
     if (!a->base.workspace || !aligned(a->base.workspace, 256) || a->base.workspace_bytes < plan.total_bytes)
         return KVQ_ERR_WORKSPACE;
     const kvq::Int4Keys k4{a->k_packed4, a->k_scales4, a->k_zeros4, a->k_group};

@@ -64,7 +64,6 @@ struct DecodeParams {
     const float* k4z;       // residual keys: group zero points
     int k4_ng_shift;        // residual keys: log2(D / k4g)
     int k4_g_shift;         // residual keys: log2(k4g)
-    int k4_bulk;            // residual keys: group parameters and norms staged with the rows
     int64_t W;              // tokens per CTA range
     int64_t total;          // units * T
     int Hq;
@@ -229,25 +228,19 @@ __device__ __forceinline__ void merge_warps_and_store(const float* red, const De
 // Ring geometry per group size G (measured on B200: for G = 1, two 128-token stages
 // with three CTAs per SM beat four 64-token stages, the per-stage bookkeeping being
 // spread over 4 tokens per lane group instead of 2).
-template <int G, bool V4 = false, bool RES = false>
+template <int G, bool V4 = false>
 struct I8Ring {
     static constexpr int tok = G == 1 ? 128 : 64;             // tokens per stage
     static constexpr int stages = G == 1 ? 2 : 4;
     static constexpr int vrow = V4 ? kD / 2 : kD;             // bytes of a value row
-    static constexpr int krow = RES ? kD / 2 : kD;            // bytes of a key row (INT4 or INT8)
-    static constexpr int kside = RES ? 32 : 4;                // per-token key side data: residual
-                                                              // sign words (m <= 256) or the scale
-    // K rows | V rows | K scales (residual keys: sign words) | V scales | (INT4 values in
-    // groups of 32: the 4 group scales, then the 4 zero points of each token)
-    static constexpr int v_off = tok * krow;
+    // K rows | V rows | K scales | V scales | (INT4 values in groups of 32: the 4 group
+    // scales, then the 4 zero points of each token)
+    static constexpr int v_off = tok * kD;
     static constexpr int ks_off = v_off + tok * vrow;
-    static constexpr int vs_off = ks_off + tok * kside;
+    static constexpr int vs_off = ks_off + tok * 4;
     static constexpr int s4_off = vs_off + tok * 4;
-    static constexpr int z4_off = s4_off + ((V4 || RES) ? tok * 16 : 0);
-    // residual keys: the key group scales and zero points (up to 16 B each per token)
-    // at s4_off / z4_off, then the fp16 residual norms
-    static constexpr int rn_off = z4_off + ((V4 || RES) ? tok * 16 : 0);
-    static constexpr int bytes = rn_off + (RES ? tok * 2 : 0);
+    static constexpr int z4_off = s4_off + (V4 ? tok * 16 : 0);
+    static constexpr int bytes = z4_off + (V4 ? tok * 16 : 0);
 };
 constexpr int kI8Consumers = 8;                          // consumer warps; warp 8 produces
 constexpr int kI8Threads = 32 * (kI8Consumers + 1);
@@ -257,13 +250,11 @@ __device__ unsigned int g_decode_error = 0;
 enum : unsigned int { kErrI8Producer = 0x201, kErrI8Consumer = 0x202, kErrQjlStep = 0x203 };
 
 // Resident INT8 CTAs per SM the register budget is shaped for (more heads per group
-// need more registers per thread).  Residual keys: one (the byte tables take 128 KB).
-__host__ __device__ constexpr int int8_ctas_per_sm(int G, bool res = false) {
-    return res ? 1 : (G == 1 ? 3 : (G == 2 ? 2 : 1));
-}
+// need more registers per thread).
+__host__ __device__ constexpr int int8_ctas_per_sm(int G) { return G == 1 ? 3 : (G == 2 ? 2 : 1); }
 
-// Residual keys: the byte tables of the sign-sketch estimator (the layout of the QJL
-// decode kernel's tables, described there): entry (pos, b) holds, for each of the G
+// The byte tables of the sign-sketch estimator (the layout of the QJL decode kernel's
+// tables, described there): entry (pos, b) holds, for each of the G
 // heads, sum_{k<8} v[8 pos + k] * (bit k of b ? +1 : -1), at byte offset
 // (pos / 16) * 64 KB + b * 256 + (pos % 16) * 16.  Built by `nthr` threads.
 template <int G>
@@ -305,7 +296,6 @@ __device__ __forceinline__ void build_sign_tables(float* lut, const float* v, in
         }
     }
 }
-constexpr int kSignTableBytes = 2 * 256 * 16 * 16;      // 128 KB
 
 // A lane's BYTES consecutive bytes of a shared-memory row (16, 8 or 4) as 32-bit words.
 template <int BYTES>
@@ -332,11 +322,10 @@ __device__ __forceinline__ void nibbles8(uint32_t w, uint64_t* c) {
                     pack2(-kRoundMagic, -kRoundMagic));
 }
 
-template <int G, bool V4, bool RES = false>
-__global__ void __launch_bounds__(kI8Threads, int8_ctas_per_sm(G, RES))
+template <int G, bool V4>
+__global__ void __launch_bounds__(kI8Threads, int8_ctas_per_sm(G))
 decode_int8_kernel(const DecodeParams p) {
-    static_assert(!(RES && V4), "residual keys come with INT8 values");
-    using Ring = I8Ring<G, V4, RES>;
+    using Ring = I8Ring<G, V4>;
     constexpr int kI8StageTok = Ring::tok;
     constexpr int kI8Stages = Ring::stages;
     constexpr int kI8StageBytes = Ring::bytes;
@@ -359,7 +348,6 @@ decode_int8_kernel(const DecodeParams p) {
     const int nseg = walk.count();
     const uint32_t ring = dev::smem_u32(smem_raw);
     float* red = reinterpret_cast<float*>(smem_raw + kI8Stages * kI8StageBytes);  // [warps][G][2+D]
-    float* lut = red + kI8Consumers * G * (2 + kD);                                 // residual keys
     const uint32_t bar0 = dev::smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (kI8Stages + s); };
@@ -414,29 +402,12 @@ decode_int8_kernel(const DecodeParams p) {
                     // (INT4 values: packed rows here, group scales and zero points loaded by
                     // the consumers)
                     const bool g32 = V4 && p.v4_bulk && p.want_out;  // group params staged too
-                    const uint32_t wrow = (uint32_t)p.m / 8u;        // residual keys: sign bytes per token
-                    const uint32_t gpb = 4u << (RES ? p.k4_ng_shift : 0);   // group parameter bytes per token
-                    const uint32_t k_bytes = RES ? n * (uint32_t)Ring::krow + n * wrow +
-                                                       (p.k4_bulk ? n * (2u * gpb + 2u) : 0u)
-                                                 : n * kD + (p.scales_bulk ? n * 4u : 0u);
+                    const uint32_t k_bytes = n * kD + (p.scales_bulk ? n * 4u : 0u);
                     const uint32_t v_bytes = !p.want_out ? 0u
                                              : n * Ring::vrow + ((!V4 && p.scales_bulk) ? n * 4u : 0u) +
                                                    (g32 ? 2u * n * 16u : 0u);
                     dev::mbar_arrive_expect_tx(full_bar(s), k_bytes + v_bytes);
-                    if constexpr (RES) {
-                        dev::bulk_g2s(dst, p.k4p + (row0 + t) * Ring::krow, n * Ring::krow, full_bar(s));
-                        dev::bulk_g2s(dst + Ring::ks_off, reinterpret_cast<const unsigned char*>(p.kw) + (row0 + t) * wrow,
-                                      n * wrow, full_bar(s));
-                        if (p.k4_bulk) {
-                            dev::bulk_g2s(dst + Ring::s4_off, reinterpret_cast<const unsigned char*>(p.k4s) + (row0 + t) * gpb,
-                                          n * gpb, full_bar(s));
-                            dev::bulk_g2s(dst + Ring::z4_off, reinterpret_cast<const unsigned char*>(p.k4z) + (row0 + t) * gpb,
-                                          n * gpb, full_bar(s));
-                            dev::bulk_g2s(dst + Ring::rn_off, p.kn + row0 + t, n * 2u, full_bar(s));
-                        }
-                    } else {
-                        dev::bulk_g2s(dst, p.kc + (row0 + t) * kD, n * kD, full_bar(s));
-                    }
+                    dev::bulk_g2s(dst, p.kc + (row0 + t) * kD, n * kD, full_bar(s));
                     if (p.want_out) {
                         if (g32) {
                             dev::bulk_g2s(dst + Ring::s4_off, p.v4s + (row0 + t) * 4, n * 16u, full_bar(s));
@@ -449,7 +420,7 @@ decode_int8_kernel(const DecodeParams p) {
                             dev::bulk_g2s(dst + Ring::v_off, p.vc + (row0 + t) * kD, n * kD, full_bar(s));
                     }
                     if (p.scales_bulk) {
-                        if constexpr (!RES) dev::bulk_g2s(dst + Ring::ks_off, p.ks + row0 + t, n * 4u, full_bar(s));
+                        dev::bulk_g2s(dst + Ring::ks_off, p.ks + row0 + t, n * 4u, full_bar(s));
                         if (!V4 && p.want_out)
                             dev::bulk_g2s(dst + Ring::vs_off, p.vs + row0 + t, n * 4u, full_bar(s));
                     }
@@ -515,25 +486,6 @@ decode_int8_kernel(const DecodeParams p) {
                 }
             }
         }
-        float qsum[G];  // residual keys: the sum of the lane's query values, per head
-        if constexpr (RES) {
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                float a = 0.0f;
-#pragma unroll
-                for (int k = 0; k < NP; ++k) {
-                    const float2 q2 = unpack2(qp[g][k]);
-                    a += q2.x + q2.y;
-                }
-                qsum[g] = a;
-            }
-            // the unit's sign tables, from its heads' query sketches (the barrier before
-            // the build: every consumer is done with the previous unit's tables)
-            asm volatile("bar.sync 1, %0;" ::"n"(32 * kI8Consumers) : "memory");
-            build_sign_tables<G>(lut, p.sketch_v + (b * p.Hq + (int64_t)kvh * G) * p.m, p.m, p.m, threadIdx.x,
-                                 32 * kI8Consumers);
-            asm volatile("bar.sync 1, %0;" ::"n"(32 * kI8Consumers) : "memory");
-        }
         float mrun[G], lrun[G];
         uint64_t acc[G][NP];
         float zacc[G];  // INT4 values: sum over tokens of p * zero point (the same for the lane's dims)
@@ -553,22 +505,13 @@ decode_int8_kernel(const DecodeParams p) {
             const int rem = (int)min((int64_t)kI8StageTok, sg.t1 - tstage);  // tokens of the stage in range
             bool valid[U];
             float ksc[U], vsc[U], vz[U];
-            float k4sc[U], k4zc[U], rnrm[U];   // residual keys: group scale, zero point, residual norm
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 valid[u] = tok0 + u < rem;
                 const int64_t r = row0 + tstage + (valid[u] ? tok0 + u : 0);
-                if constexpr (RES) {
-                    if (!p.k4_bulk) {
-                        const int64_t gi = (r << p.k4_ng_shift) + ((sub * DPL) >> p.k4_g_shift);
-                        k4sc[u] = __ldg(p.k4s + gi);
-                        k4zc[u] = __ldg(p.k4z + gi);
-                        rnrm[u] = __half2float(__ushort_as_half(__ldg(p.kn + r)));
-                    }
-                }
                 if (!p.scales_bulk) {
                     // coherent loads: an appended row's scales were stored by this kernel
-                    if constexpr (!RES) ksc[u] = __ldcg(p.ks + r);
+                    ksc[u] = __ldcg(p.ks + r);
                     if constexpr (!V4) vsc[u] = p.want_out ? __ldcg(p.vs + r) : 0.0f;
                 }
                 if constexpr (V4) {
@@ -597,21 +540,6 @@ decode_int8_kernel(const DecodeParams p) {
             if (aborted) continue;
             const unsigned char* kst = smem_raw + (size_t)s * kI8StageBytes;
             const unsigned char* vst = kst + Ring::v_off;
-            if constexpr (RES) {
-                if (p.k4_bulk) {
-                    const float* s4s = reinterpret_cast<const float*>(kst + Ring::s4_off);
-                    const float* z4s = reinterpret_cast<const float*>(kst + Ring::z4_off);
-                    const __half* rns = reinterpret_cast<const __half*>(kst + Ring::rn_off);
-                    const int gsub = (sub * DPL) >> p.k4_g_shift;
-#pragma unroll
-                    for (int u = 0; u < U; ++u) {
-                        const int gi = ((tok0 + u) << p.k4_ng_shift) + gsub;
-                        k4sc[u] = s4s[gi];
-                        k4zc[u] = z4s[gi];
-                        rnrm[u] = __half2float(rns[tok0 + u]);
-                    }
-                }
-            }
             if constexpr (V4) {
                 if (p.v4_bulk && p.want_out) {
                     const float* s4s = reinterpret_cast<const float*>(kst + Ring::s4_off);
@@ -629,10 +557,8 @@ decode_int8_kernel(const DecodeParams p) {
                 const float* kss = reinterpret_cast<const float*>(kst + Ring::ks_off) + tok0;
                 const float* vss = reinterpret_cast<const float*>(kst + Ring::vs_off) + tok0;
                 if constexpr (U == 4) {
-                    if constexpr (!RES) {
-                        const float4 k4 = *reinterpret_cast<const float4*>(kss);
-                        ksc[0] = k4.x, ksc[1] = k4.y, ksc[2] = k4.z, ksc[3] = k4.w;
-                    }
+                    const float4 k4 = *reinterpret_cast<const float4*>(kss);
+                    ksc[0] = k4.x, ksc[1] = k4.y, ksc[2] = k4.z, ksc[3] = k4.w;
                     if constexpr (!V4) {
                         const float4 v4 = p.want_out ? *reinterpret_cast<const float4*>(vss) : make_float4(0, 0, 0, 0);
                         vsc[0] = v4.x, vsc[1] = v4.y, vsc[2] = v4.z, vsc[3] = v4.w;
@@ -640,10 +566,8 @@ decode_int8_kernel(const DecodeParams p) {
                 } else {
 #pragma unroll
                     for (int u = 0; u < U; u += 2) {
-                        if constexpr (!RES) {
-                            const float2 k2 = *reinterpret_cast<const float2*>(kss + u);
-                            ksc[u] = k2.x, ksc[u + 1] = k2.y;
-                        }
+                        const float2 k2 = *reinterpret_cast<const float2*>(kss + u);
+                        ksc[u] = k2.x, ksc[u + 1] = k2.y;
                         if constexpr (!V4) {
                             const float2 v2 = p.want_out ? *reinterpret_cast<const float2*>(vss + u) : make_float2(0, 0);
                             vsc[u] = v2.x, vsc[u + 1] = v2.y;
@@ -654,66 +578,6 @@ decode_int8_kernel(const DecodeParams p) {
             float score[U][G];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                if constexpr (RES) {
-                    // INT4 key dims DPL sub .. DPL sub + DPL - 1: s * <q, c> + z * sum q, plus
-                    // this lane's byte lookups of the residual's sign sketch (positions
-                    // sub + LPT e, e < m / (8 LPT): a quarter-warp reads 8 distinct 16-byte
-                    // bank groups), then one LPT-lane reduction
-                    uint32_t kw4[DPL / 8];
-                    load_row_words<DPL / 2>(kst + (tok0 + u) * Ring::krow + sub * (DPL / 2), kw4);
-                    uint64_t c[NP];
-#pragma unroll
-                    for (int h = 0; h < DPL / 8; ++h) nibbles8(kw4[h], c + 4 * h);
-                    const unsigned char* wrow = kst + Ring::ks_off + (tok0 + u) * (p.m / 8);
-                    const bool m256 = p.m == 256;
-                    const uint4 w0 = *reinterpret_cast<const uint4*>(wrow);
-                    const uint4 w1 = m256 ? *reinterpret_cast<const uint4*>(wrow + 16) : make_uint4(0, 0, 0, 0);
-                    constexpr int NE = 32 / LPT;                  // lookups per lane at m = 256
-                    float la[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                    const uint32_t lut_s = dev::smem_u32(lut);
-#pragma unroll
-                    for (int e = 0; e < NE; ++e) {
-                        if (e >= NE / 2 && !m256) break;
-                        const int pos = sub + LPT * e;            // byte position in the sketch
-                        const int wi = pos >> 2;                  // its word, 0..7
-                        const uint4 wv = (wi & 4) ? w1 : w0;
-                        const uint32_t word = (wi & 2) ? ((wi & 1) ? wv.w : wv.z) : ((wi & 1) ? wv.y : wv.x);
-                        const uint32_t byte = (word >> (8 * (pos & 3))) & 0xFFu;
-                        const uint32_t addr = lut_s + (uint32_t)(pos >> 4) * 65536u + byte * 256u +
-                                              (uint32_t)(pos & 15) * 16u;
-                        if constexpr (G == 4) {
-                            float4 f;
-                            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                                         : "=f"(f.x), "=f"(f.y), "=f"(f.z), "=f"(f.w) : "r"(addr));
-                            la[0] += f.x, la[1] += f.y, la[2] += f.z, la[3] += f.w;
-                        } else if constexpr (G == 2) {
-                            float2 f;
-                            asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(f.x), "=f"(f.y) : "r"(addr));
-                            la[0] += f.x, la[1] += f.y;
-                        } else {
-                            float f;
-                            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(f) : "r"(addr));
-                            la[0] += f;
-                        }
-                    }
-                    const float cr = p.qjl_c * rnrm[u];
-#pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        uint64_t dp0 = 0ull, dp1 = 0ull;
-#pragma unroll
-                        for (int k = 0; k < NP; k += 2) {
-                            dp0 = fma2(qp[g][k], c[k], dp0);
-                            dp1 = fma2(qp[g][k + 1], c[k + 1], dp1);
-                        }
-                        const float2 d2 = unpack2(add2(dp0, dp1));
-                        float d = __fmaf_rn(d2.x + d2.y, k4sc[u], __fmul_rn(k4zc[u], qsum[g]));
-                        d = __fmaf_rn(cr, la[g < 4 ? g : 0], d);
-#pragma unroll
-                        for (int off = 1; off < LPT; off <<= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-                        score[u][g] = d;
-                    }
-                    continue;
-                }
                 uint32_t w4[DPL / 4];
                 load_row_words<DPL>(kst + (tok0 + u) * kD + sub * DPL, w4);
                 uint64_t c[NP];
@@ -1154,7 +1018,12 @@ constexpr int kQpfWarps = 16;
 constexpr int kQpfThreads = 32 * kQpfWarps;
 constexpr int kQpfSlot = 32 * kD;                       // 32 value rows
 
-template <int G>
+// RES: keys stored as group-wise INT4 plus the residual's sign sketch.  The lane of a
+// token then also forms <q, k_hat> = sum_g s_g <q, c>_g + z_g sum_g q for its G heads
+// from its 64 code bytes (direct loads) and the unit's queries, which sit in shared
+// memory as fp32 and are read by broadcast; the sign words are the residual's and the
+// estimator is scaled by the residual's norm.
+template <int G, bool RES = false>
 __global__ void __launch_bounds__(kQpfThreads, 1)
 decode_qjl_pf_kernel(const DecodeParams p) {
     extern __shared__ float4 dsmem4[];
@@ -1175,6 +1044,10 @@ decode_qjl_pf_kernel(const DecodeParams p) {
     float* wbuf = dsmem + 2 * HALF_FLOATS;           // [WARPS][16 pairs][G][2]
     float* red = dsmem;                              // [WARPS][G][2 + kD], reuses the tables
     unsigned char* vbuf = reinterpret_cast<unsigned char*>(wbuf + WARPS * 32 * G) + (size_t)warp * kQpfSlot;
+    // residual keys: the unit's queries [G][D] fp32 and their group sums [G][4]
+    float* qs = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(wbuf + WARPS * 32 * G) +
+                                         (size_t)WARPS * kQpfSlot);
+    float* qgs = qs + G * kD;
     const uint32_t bar = dev::smem_u32(bars) + 8u * warp;
 
     const int x = lane & 7;
@@ -1208,7 +1081,22 @@ decode_qjl_pf_kernel(const DecodeParams p) {
         __syncthreads();  // the previous segment's merge no longer reads red[]
         build_sign_tables<G>(lut, p.sketch_v + (b * p.Hq + (int64_t)kvh * G) * p.m, p.m, p.m, threadIdx.x,
                              kQpfThreads);
+        if constexpr (RES) {
+            for (int i = threadIdx.x; i < G * kD; i += kQpfThreads)
+                qs[i] = __half2float(__ushort_as_half(p.q[(b * p.Hq + (int64_t)kvh * G) * kD + i]));
+        }
         __syncthreads();
+        if constexpr (RES) {
+            const int ng = 1 << p.k4_ng_shift;
+            if (threadIdx.x < G * ng) {
+                const int g = threadIdx.x >> p.k4_ng_shift, gi = threadIdx.x & (ng - 1);
+                const int len = 1 << p.k4_g_shift;
+                float a = 0.0f;
+                for (int j = 0; j < len; ++j) a += qs[g * kD + gi * len + j];
+                qgs[g * 4 + gi] = a;
+            }
+            __syncthreads();
+        }
 
         float mrun[G], lsum[G];
         uint64_t acc[G][4];
@@ -1311,6 +1199,60 @@ decode_qjl_pf_kernel(const DecodeParams p) {
                 float score[G];
 #pragma unroll
                 for (int g = 0; g < G; ++g) score[g] = p.qjl_c * nrm * sc[g];
+                if constexpr (RES) {
+                    // ---- <q, k_hat> of this lane's token from its INT4 codes ----
+                    const int64_t r = row0 + t0 + (valid ? lane : 0);
+                    const uint4* crow = reinterpret_cast<const uint4*>(p.k4p + r * (kD / 2));
+                    uint4 cw[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) cw[k] = __ldcs(crow + k);   // dims 32 k .. 32 k + 31
+                    const int ng = 1 << p.k4_ng_shift;
+                    const float* s4 = p.k4s + (r << p.k4_ng_shift);
+                    const float* z4 = p.k4z + (r << p.k4_ng_shift);
+                    float kdot[G];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) kdot[g] = 0.0f;
+                    // dims in blocks of 32 (one 16-byte code load); a block lies in one group
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int gi = (32 * k) >> p.k4_g_shift;
+                        uint64_t part[G];
+#pragma unroll
+                        for (int g = 0; g < G; ++g) part[g] = 0ull;
+                        const uint32_t wds[4] = {cw[k].x, cw[k].y, cw[k].z, cw[k].w};
+#pragma unroll
+                        for (int w8 = 0; w8 < 4; ++w8) {
+                            uint64_t c[4];
+                            nibbles8(wds[w8], c);
+                            const int d0 = 32 * k + 8 * w8;
+#pragma unroll
+                            for (int g = 0; g < G; ++g) {
+                                const float4 qa = *reinterpret_cast<const float4*>(qs + g * kD + d0);
+                                const float4 qb = *reinterpret_cast<const float4*>(qs + g * kD + d0 + 4);
+                                part[g] = fma2(pack2(qa.x, qa.y), c[0], part[g]);
+                                part[g] = fma2(pack2(qa.z, qa.w), c[1], part[g]);
+                                part[g] = fma2(pack2(qb.x, qb.y), c[2], part[g]);
+                                part[g] = fma2(pack2(qb.z, qb.w), c[3], part[g]);
+                            }
+                        }
+                        // the group's scale and zero point close each group of dims
+                        const bool last = ((32 * (k + 1)) >> p.k4_g_shift) != gi || k == 3;
+#pragma unroll
+                        for (int g = 0; g < G; ++g) {
+                            const float2 pp = unpack2(part[g]);
+                            kdot[g] += pp.x + pp.y;
+                        }
+                        if (last) {
+                            const float sg4 = __ldg(s4 + gi), zg4 = __ldg(z4 + gi);
+#pragma unroll
+                            for (int g = 0; g < G; ++g) {
+                                score[g] = __fmaf_rn(kdot[g], sg4, __fmaf_rn(zg4, qgs[g * 4 + gi], score[g]));
+                                kdot[g] = 0.0f;
+                            }
+                        }
+                        (void)ng;
+                    }
+                }
                 if (p.scores_out != nullptr && valid) {
 #pragma unroll
                     for (int g = 0; g < G; ++g)
@@ -1456,10 +1398,10 @@ decode_combine_kernel(const float* __restrict__ ws, int64_t T, int64_t W, int ma
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-template <int G, bool V4, bool RES = false>
+template <int G, bool V4>
 size_t int8_smem() {
-    return (size_t)I8Ring<G, V4, RES>::stages * I8Ring<G, V4, RES>::bytes +
-           (size_t)kI8Consumers * G * (2 + kD) * sizeof(float) + (RES ? (size_t)kSignTableBytes : 0);
+    return (size_t)I8Ring<G, V4>::stages * I8Ring<G, V4>::bytes +
+           (size_t)kI8Consumers * G * (2 + kD) * sizeof(float);
 }
 constexpr int kQjlThreads = 512;
 
@@ -1472,22 +1414,32 @@ size_t qjl_smem() {
     return a > red ? a : red;
 }
 
-template <int G, bool V4, bool RES = false>
+template <int G, bool V4>
 cudaError_t run_int8(const DecodeParams& p, int ctas, cudaStream_t st) {
-    auto kern = decode_int8_kernel<G, V4, RES>;
-    const size_t smem = int8_smem<G, V4, RES>();
+    auto kern = decode_int8_kernel<G, V4>;
+    const size_t smem = int8_smem<G, V4>();
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     kern<<<ctas, kI8Threads, smem, st>>>(p);
     return cudaGetLastError();
 }
 
-template <int G>
+template <int G, bool RES = false>
 size_t qjl_pf_smem() {
     const size_t tables = (size_t)2 * 256 * 16 * 4 * sizeof(float);
     const size_t red = (size_t)kQpfWarps * G * (2 + kD) * sizeof(float);
     const size_t a = (tables > red ? tables : red) + (size_t)kQpfWarps * 32 * G * sizeof(float);
-    return a + (size_t)kQpfWarps * kQpfSlot;
+    return a + (size_t)kQpfWarps * kQpfSlot + (RES ? (size_t)G * (kD + 4) * sizeof(float) : 0);
+}
+
+template <int G, bool RES = false>
+cudaError_t run_qjl_pf(const DecodeParams& p, int ctas, cudaStream_t st) {
+    auto kern = decode_qjl_pf_kernel<G, RES>;
+    const size_t smem = qjl_pf_smem<G, RES>();
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<ctas, kQpfThreads, smem, st>>>(p);
+    return cudaGetLastError();
 }
 
 template <int G>
@@ -1511,9 +1463,9 @@ cudaError_t run_qjl(const DecodeParams& p, int ctas, cudaStream_t st) {
 cudaError_t run_partial(bool qjl, int G, const DecodeParams& p, int ctas, cudaStream_t st) {
     if (p.k4p != nullptr) {
         switch (G) {
-            case 1: return run_int8<1, false, true>(p, ctas, st);
-            case 2: return run_int8<2, false, true>(p, ctas, st);
-            case 4: return run_int8<4, false, true>(p, ctas, st);
+            case 1: return run_qjl_pf<1, true>(p, ctas, st);
+            case 2: return run_qjl_pf<2, true>(p, ctas, st);
+            case 4: return run_qjl_pf<4, true>(p, ctas, st);
             default: return cudaErrorNotSupported;
         }
     }
@@ -1554,7 +1506,7 @@ cudaError_t read_and_clear_decode_error(uint32_t* code) {
     return e;
 }
 
-DecodePlan plan_decode(const kvq_decode_args* a, int sm_count, bool residual_keys) {
+DecodePlan plan_decode(const kvq_decode_args* a, int sm_count) {
     DecodePlan pl{};
     const int64_t G = a->n_q_heads / a->n_kv_heads;
     const bool qjl = a->key_format == KVQ_KEYS_QJL;
@@ -1563,7 +1515,8 @@ DecodePlan plan_decode(const kvq_decode_args* a, int sm_count, bool residual_key
     const int64_t total = pl.units * T;
     // As many CTAs as can be resident at once: up to three 68 KB-ring INT8 CTAs per SM,
     // or one 512-thread QJL CTA per SM (its byte tables fill shared memory).
-    const int64_t resident = (int64_t)sm_count * (qjl && !residual_keys ? 1 : int8_ctas_per_sm((int)G, residual_keys));
+    // (residual keys run the QJL decode kernel: their key_format is QJL too)
+    const int64_t resident = (int64_t)sm_count * (qjl ? 1 : int8_ctas_per_sm((int)G));
     int64_t W = total > 0 ? (total + resident - 1) / resident : kRange;
     W = (W + kRange - 1) / kRange * kRange;
     pl.W = W;
@@ -1624,18 +1577,12 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
         p.k4z = k4->zeros;
         p.k4_g_shift = k4->group == 32 ? 5 : (k4->group == 64 ? 6 : 7);
         p.k4_ng_shift = 7 - p.k4_g_shift;
-        // every stage then starts and ends on a multiple of 8 tokens, so the group
-        // parameters (4-16 B per token) and norms (2 B) move in 16-byte multiples
-        p.k4_bulk = (a->seq_len % 8 == 0) && (p.cap % 8 == 0) &&
-                    reinterpret_cast<uintptr_t>(k4->scales) % 16 == 0 &&
-                    reinterpret_cast<uintptr_t>(k4->zeros) % 16 == 0 &&
-                    reinterpret_cast<uintptr_t>(a->k_norms_f16) % 16 == 0;
     }
     // QJL: value rows are 128 B, so a step's 32 rows start 16-byte aligned whenever the
     // array does
     p.qjl_bulk = qjl && a->out != nullptr && reinterpret_cast<uintptr_t>(a->v_codes) % 16 == 0;
-    p.scales_bulk = (!qjl || k4 != nullptr) && (a->seq_len % 4 == 0) && (p.cap % 4 == 0) &&
-                    (k4 != nullptr || reinterpret_cast<uintptr_t>(a->k_scales) % 16 == 0) &&
+    p.scales_bulk = !qjl && (a->seq_len % 4 == 0) && (p.cap % 4 == 0) &&
+                    reinterpret_cast<uintptr_t>(a->k_scales) % 16 == 0 &&
                     (a->out == nullptr || reinterpret_cast<uintptr_t>(a->v_scales) % 16 == 0);
     cudaError_t e;
     if (qjl) {

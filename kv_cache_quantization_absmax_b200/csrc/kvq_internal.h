@@ -52,8 +52,7 @@ struct DecodePlan {
     size_t sketch_bytes;  // query sketches (QJL)
     size_t total_bytes;
 };
-// residual_keys: keys as group-wise INT4 + the residual's sign sketch (one CTA per SM)
-DecodePlan plan_decode(const kvq_decode_args* a, int sm_count, bool residual_keys = false);
+DecodePlan plan_decode(const kvq_decode_args* a, int sm_count);
 cudaError_t read_and_clear_decode_error(uint32_t* code);
 // Append-on-decode: the new token (row T - 1 of every unit, a->seq_len = T) is encoded
 // by the decode kernel itself; the cache arrays have `capacity` rows per unit.
