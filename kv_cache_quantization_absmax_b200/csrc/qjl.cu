@@ -24,12 +24,19 @@
 // warpgroup has two tiles' time for one.
 //
 // Norms: the stored norm is the fp16 rounding of the fp64 norm whose sum of squares
-// is accumulated in index order.  The fast path
-// sums the exact fp32 squares (fp16 squares fit in fp32) in a fixed tree, error
-// <= 12 u relative, takes the IEEE root, and checks that n (1 - 2^-19) and
-// n (1 + 2^-19) round to the same fp16 value; then that value is the rounding of the
-// exact norm and of the fp64 one.  Otherwise (about one key in 200) the thread redoes
-// the sum in fp64 in index order and rounds that.
+// is accumulated in index order.  The fast path sums the exact fp32 squares (fp16
+// squares fit in fp32) in a fixed tree (at most 11 roundings on any term's path, so
+// relative error <= gamma_11 ~ 11 u, u = 2^-24), takes the IEEE root (root of the sum's
+// error 5.5 u, plus u for the root's rounding) and checks that n (1 - 2^-21) and
+// n (1 + 2^-21) round to the same fp16 value (8 u covers those 6.5 u, the u of the
+// product's rounding and the fp64 reference's 2^-46); then that value is the rounding
+// of the fp64 norm.  Otherwise (about one key in 600 of LogNormal keys) the key is
+// queued in shared memory and, once the CTA's tiles are done, the epilogue threads
+// redo those sums in fp64 in index order, one key per thread, reading the keys from
+// global memory: a dependent chain of 128 fp64 operations costs about a microsecond,
+// and run inline it would hold its whole warp (and through it the accumulator and the
+// stage) while 31 lanes idle.  A key that finds the queue full takes the same sum
+// inline from the tile in shared memory.
 // Sign bits: bit = 1 iff the fp32 accumulator's sign bit is clear.  An exactly zero
 // projection of a nonzero key lies inside the tolerance band whatever its sign; a zero
 // key (sum of squares 0) gets all bits set, since every projection is exactly 0.
@@ -60,6 +67,7 @@ constexpr int kTileBytes = 2 * kHalfBytes;
 constexpr int kThreads = 320;             // producer, MMA, 2 x 4 epilogue warps
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccStride = 256;     // TMEM columns between the two accumulators
+constexpr int kSlowCap = 256;            // keys whose norm is deferred to the slow path, per CTA
 
 enum : unsigned int {
     kErrProducer = 0x101,
@@ -209,19 +217,25 @@ __device__ __forceinline__ float row_sum_squares(const uint8_t* st, int row) {
     return s[0];
 }
 
-// fp16 bits of the norm: the fp32 fast path when both ends of n (1 -+ 2^-19) round to
-// the same fp16 value, else the defining sequence (fp64 sum in index order, IEEE root,
-// one rounding to fp16).
-__device__ __forceinline__ uint16_t norm_f16_bits(const uint8_t* st, int row, float ss) {
+// The fp32 fast path: true, with the fp16 bits of the norm, when both ends of
+// n (1 -+ 2^-21) round to the same fp16 value.
+__device__ __forceinline__ bool norm_f16_fast(float ss, uint16_t& bits) {
     const float n = __fsqrt_rn(ss);
-    const __half lo = __float2half_rn(__fmul_rn(n, 1.0f - 1.9073486328125e-06f));
-    const __half hi = __float2half_rn(__fmul_rn(n, 1.0f + 1.9073486328125e-06f));
-    if (__half_as_ushort(lo) == __half_as_ushort(hi)) return __half_as_ushort(lo);
+    const __half lo = __float2half_rn(__fmul_rn(n, 1.0f - 0x1p-21f));
+    const __half hi = __float2half_rn(__fmul_rn(n, 1.0f + 0x1p-21f));
+    bits = __half_as_ushort(lo);
+    return __half_as_ushort(lo) == __half_as_ushort(hi);
+}
+
+// The defining sequence: fp64 sum of the squares in index order, IEEE root, one
+// rounding to fp16.  chunk(c) gives the c-th 8 components (16 bytes) of the key.
+template <class Chunk>
+__device__ __forceinline__ uint16_t norm_f16_index_order(Chunk chunk) {
     double s64 = 0.0;
 #pragma unroll 1
     for (int c = 0; c < 16; ++c) {
-        const uint4 v = tile_chunk(st, row, c);
-        const __half* h = reinterpret_cast<const __half*>(&v);
+        const uint4 x = chunk(c);
+        const __half* h = reinterpret_cast<const __half*>(&x);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const double d = (double)__half2float(h[i]);
@@ -240,12 +254,14 @@ struct Smem {
 template <bool kSketchOut>
 __global__ void __launch_bounds__(kThreads, 1)
 qjl_mma_kernel(const __grid_constant__ CUtensorMap tmap_rows,
-               const __grid_constant__ CUtensorMap tmap_s, int64_t n_rows, int m,
-               uint32_t* __restrict__ words, uint16_t* __restrict__ norms,
-               float* __restrict__ sketch_out) {
+               const __grid_constant__ CUtensorMap tmap_s, const uint16_t* __restrict__ rows,
+               int64_t n_rows, int m, uint32_t* __restrict__ words,
+               uint16_t* __restrict__ norms, float* __restrict__ sketch_out) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag_storage;
+    __shared__ int slow_count;
+    __shared__ uint32_t slow_keys[kSlowCap];
     volatile int* abort_flag = &abort_flag_storage;
 
     const uint32_t raw = smem_u32(smem_raw);
@@ -268,6 +284,7 @@ qjl_mma_kernel(const __grid_constant__ CUtensorMap tmap_rows,
 
     if (threadIdx.x == 0) {
         abort_flag_storage = 0;
+        slow_count = 0;
         for (int s = 0; s < kStages; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 4);
@@ -360,6 +377,7 @@ qjl_mma_kernel(const __grid_constant__ CUtensorMap tmap_rows,
             const int64_t key = tile * kBM + row;
             float ss = 0.0f;
             uint16_t nbits = 0;
+            bool deferred = false;
             if constexpr (!kSketchOut) {
                 // The norm needs only the landed tile: compute it while the MMA runs.
                 const uint32_t ph = (uint32_t)(it / kStages) & 1u;
@@ -367,7 +385,15 @@ qjl_mma_kernel(const __grid_constant__ CUtensorMap tmap_rows,
                 if (!__all_sync(0xffffffffu, okf)) break;
                 const uint8_t* st = base_ptr + (stage_base - base) + (size_t)stage * kTileBytes;
                 ss = row_sum_squares(st, row);
-                nbits = norm_f16_bits(st, row, ss);
+                if (!norm_f16_fast(ss, nbits) && key < n_rows) {
+                    const int slot = key <= 0xFFFFFFFFll ? atomicAdd(&slow_count, 1) : kSlowCap;
+                    if (slot < kSlowCap) {
+                        slow_keys[slot] = (uint32_t)key;
+                        deferred = true;
+                    } else {
+                        nbits = norm_f16_index_order([&](int c) { return tile_chunk(st, row, c); });
+                    }
+                }
             }
             const bool ok = mbar_wait(tfull_bar(acc), aph, abort_flag, kErrEpilogue);
             if (!__all_sync(0xffffffffu, ok)) break;  // warp-uniform: tcgen05.ld is .aligned
@@ -409,7 +435,7 @@ qjl_mma_kernel(const __grid_constant__ CUtensorMap tmap_rows,
                         for (int c = 0; c < 8; ++c)
                             if (c < nw) dst[c] = wbits[c];
                     }
-                    norms[key] = nbits;
+                    if (!deferred) norms[key] = nbits;
                 }
             } else {
                 float* dst = sketch_out + key * m;
@@ -432,6 +458,19 @@ qjl_mma_kernel(const __grid_constant__ CUtensorMap tmap_rows,
                     mbar_arrive(tempty_bar(acc));
                     mbar_arrive(empty_bar(stage));
                 }
+            }
+        }
+        if constexpr (!kSketchOut) {
+            // The deferred norms, one key per epilogue thread, from global memory (rows
+            // are 256 bytes, so 16-byte aligned).  The barrier over the 256 epilogue
+            // threads makes every queued key visible; every epilogue warp reaches it,
+            // also after leaving its loop early.
+            asm volatile("bar.sync 1, 256;" ::: "memory");
+            const int cnt = min(slow_count, kSlowCap);
+            for (int i = (int)threadIdx.x - 64; i < cnt; i += 256) {
+                const uint32_t key = slow_keys[i];
+                const uint4* src = reinterpret_cast<const uint4*>(rows + (size_t)key * kDim);
+                norms[key] = norm_f16_index_order([&](int c) { return __ldg(src + c); });
             }
         }
     }
@@ -497,8 +536,8 @@ cudaError_t launch_mma(const uint16_t* rows, int64_t n_rows, const uint16_t* S, 
     const int64_t n_tiles = (n_rows + kBM - 1) / kBM;
     const int64_t sms = device_sm_count();
     const int grid = (int)(n_tiles < sms ? n_tiles : sms);
-    qjl_mma_kernel<kSketchOut><<<grid, kThreads, smem, st>>>(map_rows, map_s, n_rows, m, words,
-                                                             norms, sketch);
+    qjl_mma_kernel<kSketchOut><<<grid, kThreads, smem, st>>>(map_rows, map_s, rows, n_rows, m,
+                                                             words, norms, sketch);
     return cudaGetLastError();
 }
 

@@ -249,6 +249,33 @@ def test_qjl_parallel_key_and_scaling():
     assert np.all(wz == 0xFFFFFFFF) and float(nz[0]) == 0.0
 
 
+
+def tie_keys():
+    """Keys whose exact norm is an fp16 rounding midpoint (ulp 2 at 2048, 2^-7 at 8)."""
+    rows = np.zeros((6, 128), np.float16)
+    rows[0, :3] = [2048, 64, 1]                 # 2048^2 + 64^2 + 1 = 2049^2: tie -> even 2048
+    rows[1, :4] = [2048, 110, 14, 1]            # = 2051^2: tie between 2050 and 2052 -> 2052
+    rows[2, :3] = [8, 0.25, 2.0 ** -8]          # = 8.00390625^2: tie -> 8
+    rows[3] = rows[2]
+    rows[3, 3:10] = 2.0 ** -24                  # seven 2^-48 squares after 64: each below
+    #                                             half an ulp of the partial sum, dropped
+    rows[4, 100:103] = [8, 0.25, 2.0 ** -8]
+    rows[4, 0:7] = 2.0 ** -24                   # the same squares first: 7 * 2^-48 is exact,
+    #                                             then 64 + 7 * 2^-48 rounds to 64 + 2^-45
+    rows[5] = rows[2]
+    rows[5, 3] = 2.0 ** -12                     # a 2^-24 square is kept: above the midpoint
+    return rows
+
+
+def test_qjl_norm_fp64_index_order_and_ties():
+    """The stored norm is the fp16 rounding (nearest, ties to even) of the root of the
+    fp64 sum of squares taken in index order: exact midpoints pin the tie rule; the same
+    multiset of squares in two orders pins the order (the exact norm would round up in
+    both); a kept small square pins that the sum is not a coarser one."""
+    S = inputs.sketch_matrix(32, 128)
+    _, norms = oracle.qjl_encode(tie_keys(), S)
+    assert [float(x) for x in norms] == [2048.0, 2052.0, 8.0, 8.0, 8.0078125, 8.0078125]
+
 # ----------------------------------------------------------------------------------
 # Decode step: softmax invariants, special cases, fp64 brute force with the page's GQA
 # broadcast (unsqueeze(2).expand(...).reshape(...))

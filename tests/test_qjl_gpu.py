@@ -56,6 +56,64 @@ def test_encode_special_keys(kvq):
     assert np.array_equal(w[1], w[2])
 
 
+def _near_midpoint_pairs(scale, count, rng, within):
+    """fp16 pairs (a, b) whose fp64 norm lies within `within` (relative) of a midpoint
+    between two fp16 values."""
+    out = []
+    while len(out) < count:
+        a = rng.uniform(0.5, 1.0, 4096).astype(np.float16) * np.float16(scale)
+        b = rng.uniform(0.5, 1.0, 4096).astype(np.float16) * np.float16(scale)
+        n = np.hypot(a.astype(np.float64), b.astype(np.float64))
+        lo = n.astype(np.float16).astype(np.float64)
+        nxt = np.nextafter(n.astype(np.float16), np.float16(np.inf)).astype(np.float64)
+        prv = np.nextafter(n.astype(np.float16), np.float16(-np.inf)).astype(np.float64)
+        mid = np.where(n >= lo, (lo + nxt) / 2, (lo + prv) / 2)
+        hit = np.abs(n / mid - 1) < within
+        out += list(zip(a[hit], b[hit]))
+    return out[:count]
+
+
+def test_encode_norm_slow_paths(kvq):
+    """Norms near fp16 rounding midpoints, bit-exact against the oracle: two large
+    components within 2^-20 of a midpoint (either side of the fp32 fast path's 2^-21
+    margin); the same at 2^-19 with subnormal components added, whose squares span more
+    than 53 bits; exact midpoints (the tie rule); and exact midpoints with small squares
+    that the index-order fp64 sum drops or keeps depending on their position, scaled by
+    powers of two."""
+    from tests.test_oracle_pins import tie_keys
+    rng = np.random.default_rng(77)
+    keys = np.zeros((256, 128), np.float16)
+    for i, (a, b) in enumerate(_near_midpoint_pairs(1.0, 128, rng, 2.0 ** -20)):
+        keys[i, 3], keys[i, 90] = a, b
+    for i, (a, b) in enumerate(_near_midpoint_pairs(256.0, 128, rng, 2.0 ** -19)):
+        keys[128 + i, 0], keys[128 + i, 127] = a, b
+        keys[128 + i, 1:120:7] = np.float16(2.0 ** -24) * (1 + i % 5)
+    ties = tie_keys()
+    scaled = [ties[:2] * np.float16(2.0 ** k) for k in range(-8, 5)]
+    scaled += [ties[2:] * np.float16(2.0 ** k) for k in range(0, 8)]
+    keys = np.concatenate([keys] + scaled)
+    S = inputs.sketch_matrix(256, 128)
+    _encode_and_compare(kvq, keys, S)
+
+
+def test_encode_norm_slow_queue_overflow(kvq):
+    """Every key takes the slow norm and each CTA gets three tiles (384 such keys, more
+    than its 256-entry queue): queued keys and the overflow computed inline, all
+    bit-exact against the oracle."""
+    from tests.test_oracle_pins import tie_keys
+    rng = np.random.default_rng(78)
+    base = np.zeros((96, 128), np.float16)
+    for i, (a, b) in enumerate(_near_midpoint_pairs(4.0, 96, rng, 2.0 ** -22)):
+        base[i, i % 128], base[i, (i * 37 + 5) % 128] = a, b   # distinct: 36 i != -5 mod 128
+    ties = tie_keys()
+    base = np.concatenate([base] + [ties * np.float16(2.0 ** k) for k in range(0, 5)])
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    n = sms * 128 * 3
+    keys = np.ascontiguousarray(np.resize(base, (n, 128)))
+    S = inputs.sketch_matrix(256, 128)
+    _encode_and_compare(kvq, keys, S)
+
+
 def test_encode_full_size_sampled(kvq):
     """The key-sketch workload: keys [1, 32, 32768, 128] (1,048,576 keys, per-channel
     LogNormal std), S [256, 128] from seed 7; 2048 sampled keys checked against the oracle."""
