@@ -322,6 +322,77 @@ __device__ __forceinline__ void nibbles8(uint32_t w, uint64_t* c) {
                     pack2(-kRoundMagic, -kRoundMagic));
 }
 
+// A lane's view of the byte tables when it scores its own token: the 32 entries of a
+// token are read at positions rotated by x = lane & 7 (both the 16-byte entry within
+// an 8-entry group and the byte order within a word pair), so that the eight lanes of a
+// shared-memory phase hit distinct banks.
+struct LutLane {
+    uint32_t off16[8];
+    uint32_t sel[4];
+    bool swap_words;
+    __device__ explicit LutLane(int lane) {
+        const int x = lane & 7;
+        swap_words = (x & 4) != 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) off16[e] = (uint32_t)((e ^ x) * 16);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sel[e] = 0x6504u | ((uint32_t)((e ^ x) & 3) << 4);
+    }
+};
+
+// The estimator's table sum for one token: sc[g] = sum over the 32 byte positions of
+// the token's sign words w[0..7] of entry (pos, byte) for head g (tables at shared
+// address lut_s, the layout of build_sign_tables).
+template <int G>
+__device__ __forceinline__ void lut_token_sums(const uint32_t* w, uint32_t lut_s, const LutLane& L, float* sc) {
+    constexpr int HALF_FLOATS = 256 * 16 * 4;
+#pragma unroll
+    for (int g = 0; g < G; ++g) sc[g] = 0.0f;
+    uint64_t s01 = 0ull, s23 = 0ull, t01 = 0ull, t23 = 0ull;
+#pragma unroll
+    for (int pr = 0; pr < 4; ++pr) {
+        const uint32_t wa = L.swap_words ? w[2 * pr + 1] : w[2 * pr];
+        const uint32_t wb = L.swap_words ? w[2 * pr] : w[2 * pr + 1];
+        const uint32_t half_off = (uint32_t)((pr >> 1) * HALF_FLOATS * 4 + (pr & 1) * 128);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const uint32_t o = __byte_perm(e < 4 ? wa : wb, L.off16[e], L.sel[e & 3]);
+            const uint32_t addr = lut_s + half_off + o;
+            if constexpr (G == 4) {
+                float4 f;
+                asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                             : "=f"(f.x), "=f"(f.y), "=f"(f.z), "=f"(f.w) : "r"(addr));
+                if (e & 1) {
+                    t01 = add2(t01, pack2(f.x, f.y));
+                    t23 = add2(t23, pack2(f.z, f.w));
+                } else {
+                    s01 = add2(s01, pack2(f.x, f.y));
+                    s23 = add2(s23, pack2(f.z, f.w));
+                }
+            } else if constexpr (G == 2) {
+                float2 f;
+                asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(f.x), "=f"(f.y) : "r"(addr));
+                if (e & 1) t01 = add2(t01, pack2(f.x, f.y));
+                else s01 = add2(s01, pack2(f.x, f.y));
+            } else {
+                float f;
+                asm volatile("ld.shared.f32 %0, [%1];" : "=f"(f) : "r"(addr));
+                sc[0] += f;
+            }
+        }
+    }
+    if constexpr (G >= 2) {
+        const float2 a = unpack2(add2(s01, t01));
+        sc[0] = a.x;
+        sc[1] = a.y;
+    }
+    if constexpr (G == 4) {
+        const float2 a = unpack2(add2(s23, t23));
+        sc[2] = a.x;
+        sc[3] = a.y;
+    }
+}
+
 template <int G, bool V4>
 __global__ void __launch_bounds__(kI8Threads, int8_ctas_per_sm(G))
 decode_int8_kernel(const DecodeParams p) {
@@ -1050,14 +1121,7 @@ decode_qjl_pf_kernel(const DecodeParams p) {
     float* qgs = qs + G * kD;
     const uint32_t bar = dev::smem_u32(bars) + 8u * warp;
 
-    const int x = lane & 7;
-    const bool swap_words = (x & 4) != 0;
-    uint32_t off16[8];
-    uint32_t sel[4];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) off16[e] = (uint32_t)((e ^ x) * 16);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) sel[e] = 0x6504u | ((uint32_t)((e ^ x) & 3) << 4);
+    const LutLane lut_lane(lane);
     const uint32_t lut_s = (uint32_t)__cvta_generic_to_shared(lut);
 
     if (threadIdx.x == 0) {
@@ -1151,51 +1215,7 @@ decode_qjl_pf_kernel(const DecodeParams p) {
             if (!aborted) {
                 // ---- estimator: 32 byte-table lookups ----
                 float sc[G];
-#pragma unroll
-                for (int g = 0; g < G; ++g) sc[g] = 0.0f;
-                uint64_t s01 = 0ull, s23 = 0ull, t01 = 0ull, t23 = 0ull;
-#pragma unroll
-                for (int pr = 0; pr < 4; ++pr) {
-                    const uint32_t wa = swap_words ? w[2 * pr + 1] : w[2 * pr];
-                    const uint32_t wb = swap_words ? w[2 * pr] : w[2 * pr + 1];
-                    const uint32_t half_off = (uint32_t)((pr >> 1) * HALF_FLOATS * 4 + (pr & 1) * 128);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const uint32_t o = __byte_perm(e < 4 ? wa : wb, off16[e], sel[e & 3]);
-                        const uint32_t addr = lut_s + half_off + o;
-                        if constexpr (G == 4) {
-                            float4 f;
-                            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                                         : "=f"(f.x), "=f"(f.y), "=f"(f.z), "=f"(f.w) : "r"(addr));
-                            if (e & 1) {
-                                t01 = add2(t01, pack2(f.x, f.y));
-                                t23 = add2(t23, pack2(f.z, f.w));
-                            } else {
-                                s01 = add2(s01, pack2(f.x, f.y));
-                                s23 = add2(s23, pack2(f.z, f.w));
-                            }
-                        } else if constexpr (G == 2) {
-                            float2 f;
-                            asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(f.x), "=f"(f.y) : "r"(addr));
-                            if (e & 1) t01 = add2(t01, pack2(f.x, f.y));
-                            else s01 = add2(s01, pack2(f.x, f.y));
-                        } else {
-                            float f;
-                            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(f) : "r"(addr));
-                            sc[0] += f;
-                        }
-                    }
-                }
-                if constexpr (G >= 2) {
-                    const float2 a = unpack2(add2(s01, t01));
-                    sc[0] = a.x;
-                    sc[1] = a.y;
-                }
-                if constexpr (G == 4) {
-                    const float2 a = unpack2(add2(s23, t23));
-                    sc[2] = a.x;
-                    sc[3] = a.y;
-                }
+                lut_token_sums<G>(w, lut_s, lut_lane, sc);
                 float score[G];
 #pragma unroll
                 for (int g = 0; g < G; ++g) score[g] = p.qjl_c * nrm * sc[g];
@@ -1359,6 +1379,367 @@ decode_qjl_pf_kernel(const DecodeParams p) {
     __syncwarp();
 }
 
+// -----------------------------------------------------------------------------------
+// QJL keys, value pass on the tensor cores.  The range streams in chunks of 128 tokens
+// of one unit through a 4-stage ring: the value rows by a TMA tile with the 128-byte
+// swizzle (token rows of 128 INT8 codes, which the tensor core reads as the MN-major
+// operand A = V^T [128 dims x 128 tokens]), the sign words, norms and value scales by
+// bulk copies.  Warp roles (448 threads, one CTA per SM):
+//   warp 0       producer;
+//   warp 1       TMEM and the MMA thread: per chunk four tcgen05.mma kind::i8, slice k
+//                (tokens 32 k .. 32 k + 31) into its own 16-column int32 accumulator;
+//   warps 2..9   scorers in two groups of four that take alternate chunks, one token per
+//                thread: the estimator from the byte tables; per warp (32 tokens, one
+//                MMA slice) the max M of the log2-domain logits of each head and the max
+//                value scale smax; the weight w = 2^(s - M) * vscale as a 24-bit
+//                fixed-point integer W = round(w (2^24 - 1) / smax), split into three
+//                unsigned bytes that form rows 3 g + k of the operand B [16 x 128
+//                tokens] (K-major); the warp's sum of 2^(s - M) in fixed point by one
+//                integer warp reduction;
+//   warps 10..13 accumulators, one value dimension per thread: per slice, sum_t W_t c_t
+//                = D2 2^16 + D1 2^8 + D0 (exact in int32: |c| <= 127, bytes <= 255, 32
+//                tokens), rescaled by smax / (2^24 - 1), merged over the slices by their
+//                maxima and into the running online-softmax state of each head.
+// The INT8 codes enter the product unconverted and every product and sum is exact; the
+// approximations are the weights' 24-bit fixed point (absolute error at most 2^-25 smax
+// per token), the sums' 2^-24 fixed point, and the fp32 merges.
+constexpr int kTcTok = 128;                 // tokens per chunk
+constexpr int kTcStages = 4;
+constexpr int kTcScorerWarps = 8;
+constexpr int kTcThreads = 32 * (2 + kTcScorerWarps + 4);
+constexpr int kTcVBytes = kTcTok * kD;      // value tile: 16 KB
+constexpr int kTcStageBytes = 21 * 1024;    // tile | words (<= 4 KB) | norms | scales
+constexpr int kTcWordsOff = kTcVBytes;
+constexpr int kTcNormsOff = kTcWordsOff + kTcTok * 32;
+constexpr int kTcScalesOff = kTcNormsOff + kTcTok * 2;
+static_assert(kTcScalesOff + kTcTok * 4 <= kTcStageBytes, "stage layout");
+constexpr int kTcBBytes = 2048;             // operand B: 16 rows x 128 bytes
+constexpr int kTcAcc = 4;                   // chunks in flight between scorers and accumulators
+constexpr uint32_t kTcTmemCols = kTcAcc * 4 * 16;
+constexpr float kTcWmax = 16777215.0f;      // 2^24 - 1
+// instruction descriptor: int32 accumulator, A signed 8-bit MN-major, B unsigned 8-bit
+// K-major, N = 16, M = 128
+constexpr uint32_t kTcIdesc = (2u << 4) | (1u << 7) | (0u << 10) | (1u << 15) | (0u << 16) |
+                              ((16u >> 3) << 17) | ((128u >> 4) << 24);
+
+enum : unsigned int { kErrTcProducer = 0x211, kErrTcMma = 0x212, kErrTcScore = 0x213, kErrTcAcc = 0x214 };
+
+struct TcSlice {              // per chunk and MMA slice, from a scorer warp to the accumulators
+    float M[4];               // max of the slice's log2-domain logits, per head
+    float L[4];               // sum of 2^(s - M), per head
+    float inv_scale;          // smax / (2^24 - 1)
+    float pad[3];
+};
+
+__host__ __device__ constexpr size_t tc_smem_bytes() {
+    return 1024 /* alignment */ + 2 * 65536 /* tables */ + (size_t)kTcStages * kTcStageBytes +
+           kTcAcc * kTcBBytes + kTcAcc * 4 * sizeof(TcSlice) + (2 * kTcStages + 3 * kTcAcc + 1) * 8;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kTcThreads, 1)
+decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap vmap) {
+    extern __shared__ uint8_t tc_raw[];
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_storage;
+    volatile int* abort_flag = &abort_storage;
+    const uint32_t raw = dev::smem_u32(tc_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* bp = tc_raw + (base - raw);
+    float* lut = reinterpret_cast<float*>(bp);                         // 128 KB
+    const uint32_t lut_s = base;
+    const uint32_t stage_s = base + 2 * 65536;
+    uint8_t* stage_p = bp + 2 * 65536;
+    const uint32_t b_s = stage_s + kTcStages * kTcStageBytes;          // 1024-aligned
+    uint8_t* b_p = stage_p + kTcStages * kTcStageBytes;
+    TcSlice* slices = reinterpret_cast<TcSlice*>(b_p + kTcAcc * kTcBBytes);   // [kTcAcc][4]
+    const uint32_t bars = dev::smem_u32(slices + kTcAcc * 4);
+    auto full_bar = [&](int s) { return bars + 8u * s; };
+    auto empty_bar = [&](int s) { return bars + 8u * (kTcStages + s); };
+    auto bready_bar = [&](int a) { return bars + 8u * (2 * kTcStages + a); };
+    auto tfull_bar = [&](int a) { return bars + 8u * (2 * kTcStages + kTcAcc + a); };
+    auto tempty_bar = [&](int a) { return bars + 8u * (2 * kTcStages + 2 * kTcAcc + a); };
+    const uint32_t done_bar = bars + 8u * (2 * kTcStages + 3 * kTcAcc);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int cta = blockIdx.x;
+    const RangeWalk walk(p, cta);
+    const int nseg = walk.count();
+    const int nw = p.m / 32;
+
+    if (threadIdx.x == 0) {
+        abort_storage = 0;
+        for (int s = 0; s < kTcStages; ++s) {
+            dev::mbar_init(full_bar(s), 1);
+            dev::mbar_init(empty_bar(s), 1);
+        }
+        for (int a = 0; a < kTcAcc; ++a) {
+            dev::mbar_init(bready_bar(a), 4);
+            dev::mbar_init(tfull_bar(a), 1);
+            dev::mbar_init(tempty_bar(a), 4);
+        }
+        dev::mbar_init(done_bar, 1);
+        dev::mbar_init_fence();
+    }
+    // operand B: rows 3 G .. 15 stay zero
+    for (int i = threadIdx.x; i < kTcAcc * kTcBBytes / 16; i += kTcThreads)
+        reinterpret_cast<uint4*>(b_p)[i] = make_uint4(0u, 0u, 0u, 0u);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (warp == 1) dev::tmem_alloc(dev::smem_u32(&tmem_slot), kTcTmemCols);
+    dev::tc_fence_before();
+    __syncthreads();
+    dev::tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    dev::griddep_launch_dependents();  // the combine kernel may be scheduled (it waits)
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
+            int c = 0;
+            bool ok = true;
+            for (int jj = 0; ok && jj < nseg; ++jj) {
+                const Segment sg = walk.seg(jj);
+                const int64_t row0 = sg.u * p.cap;
+                for (int64_t t = sg.t0; t < sg.t1; t += kTcTok, ++c) {
+                    const int s = c % kTcStages;
+                    const uint32_t ph = (uint32_t)(c / kTcStages) & 1u;
+                    if (!dev::mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, &g_decode_error, kErrTcProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t n = (uint32_t)min((int64_t)kTcTok, sg.t1 - t);
+                    const int64_t r = row0 + t;
+                    const uint32_t dst = stage_s + (uint32_t)s * kTcStageBytes;
+                    dev::mbar_arrive_expect_tx(full_bar(s), (uint32_t)kTcVBytes + n * (uint32_t)nw * 4u + n * 2u + n * 4u);
+                    dev::tma_load_2d(dst, &vmap, full_bar(s), 0, (int)r);
+                    dev::bulk_g2s(dst + kTcWordsOff, p.kw + r * nw, n * (uint32_t)nw * 4u, full_bar(s));
+                    dev::bulk_g2s(dst + kTcNormsOff, p.kn + r, n * 2u, full_bar(s));
+                    dev::bulk_g2s(dst + kTcScalesOff, p.vs + r, n * 4u, full_bar(s));
+                }
+            }
+            // never leave the CTA with a copy in flight: wait for the last fill of each stage
+            for (int k = max(0, c - kTcStages); k < c; ++k)
+                dev::mbar_drain(full_bar(k % kTcStages), (uint32_t)(k / kTcStages) & 1u);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            int c = 0;
+            bool ok = true;
+            for (int jj = 0; ok && jj < nseg; ++jj) {
+                const Segment sg = walk.seg(jj);
+                for (int64_t t = sg.t0; t < sg.t1; t += kTcTok, ++c) {
+                    const int s = c % kTcStages;
+                    const uint32_t ph = (uint32_t)(c / kTcStages) & 1u;
+                    const int a = c % kTcAcc;
+                    const uint32_t aph = (uint32_t)(c / kTcAcc) & 1u;
+                    if (!dev::mbar_wait(full_bar(s), ph, abort_flag, &g_decode_error, kErrTcMma) ||
+                        !dev::mbar_wait(bready_bar(a), aph, abort_flag, &g_decode_error, kErrTcMma)) {
+                        ok = false;
+                        break;
+                    }
+                    dev::tc_fence_after();
+                    const uint32_t va = stage_s + (uint32_t)s * kTcStageBytes;
+                    const uint32_t bb = b_s + (uint32_t)a * kTcBBytes;
+                    const int nk = (int)((min((int64_t)kTcTok, sg.t1 - t) + 31) / 32);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if (k < nk)
+                            dev::tc_mma_i8(tmem + (uint32_t)(a * 4 + k) * 16u,
+                                           dev::smem_desc_sw128(va + (uint32_t)k * 4096u),
+                                           dev::smem_desc_sw128(bb + (uint32_t)k * 32u), kTcIdesc, 0u);
+                    dev::tc_commit(tfull_bar(a));
+                    dev::tc_commit(empty_bar(s));
+                }
+            }
+            dev::tc_commit(done_bar);
+            dev::mbar_drain(done_bar, 0);
+        }
+    } else if (warp < 2 + kTcScorerWarps) {
+        // ---------------- scorers: group gi takes the chunks c with c % 2 == gi ----------------
+        const int gi = (warp - 2) >> 2;
+        const int sw = (warp - 2) & 3;                  // MMA slice: tokens 32 sw .. 32 sw + 31
+        const int st = sw * 32 + lane;                  // this thread's token of the chunk
+        const LutLane lut_lane(lane);
+        const int kb = st >> 4, kx = st & 15;          // its byte in a row of B
+        int c = 0;
+        bool ok = true;
+        for (int jj = 0; jj < nseg; ++jj) {
+            const Segment sg = walk.seg(jj);
+            const int64_t b = sg.u / p.Hkv;
+            const int kvh = (int)(sg.u % p.Hkv);
+            // the tables are rebuilt per unit by all scorers; every scorer reaches both
+            // barriers, also after an abort (they then skip the work in between)
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcScorerWarps) : "memory");
+            if (ok)
+                build_sign_tables<G>(lut, p.sketch_v + (b * p.Hq + (int64_t)kvh * G) * p.m, p.m, p.m,
+                                     threadIdx.x - 64, 32 * kTcScorerWarps);
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcScorerWarps) : "memory");
+            for (int64_t t = sg.t0; t < sg.t1; t += kTcTok, ++c) {
+                if (!ok || (c & 1) != gi) continue;
+                const int s = c % kTcStages;
+                const uint32_t ph = (uint32_t)(c / kTcStages) & 1u;
+                const int a = c % kTcAcc;
+                const uint32_t aph = (uint32_t)(c / kTcAcc) & 1u;
+                const int n = (int)min((int64_t)kTcTok, sg.t1 - t);
+                ok = __all_sync(0xffffffffu, dev::mbar_wait(full_bar(s), ph, abort_flag, &g_decode_error, kErrTcScore));
+                if (!ok) continue;
+                const bool valid = st < n;
+                const uint8_t* sp = stage_p + (size_t)s * kTcStageBytes;
+                uint32_t w[8];
+                if (nw == 8) {
+                    const uint4 x0 = reinterpret_cast<const uint4*>(sp + kTcWordsOff)[2 * st];
+                    const uint4 x1 = reinterpret_cast<const uint4*>(sp + kTcWordsOff)[2 * st + 1];
+                    w[0] = x0.x; w[1] = x0.y; w[2] = x0.z; w[3] = x0.w;
+                    w[4] = x1.x; w[5] = x1.y; w[6] = x1.z; w[7] = x1.w;
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        w[k] = k < nw ? reinterpret_cast<const uint32_t*>(sp + kTcWordsOff)[st * nw + k] : 0u;
+                }
+                const float nrm = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(sp + kTcNormsOff)[st]));
+                const float vsc = valid ? reinterpret_cast<const float*>(sp + kTcScalesOff)[st] : 0.0f;
+                float sc[G];
+                lut_token_sums<G>(w, lut_s, lut_lane, sc);
+                float lg[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float score = p.qjl_c * nrm * sc[g];
+                    lg[g] = valid ? score * p.scale_log2 : -INFINITY;
+                    if (p.scores_out != nullptr && valid)
+                        p.scores_out[(b * p.Hq + (int64_t)kvh * G + g) * p.T + t + st] = score;
+                }
+                const float smax = warp_max(vsc);
+                const float rscale = smax > 0.0f ? kTcWmax / smax : 0.0f;
+                float M[G];
+                uint32_t W[G], Lq[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    M[g] = warp_max(lg[g]);      // -inf for a slice without valid tokens
+                    const float pe = valid ? fast_exp2(lg[g] - M[g]) : 0.0f;
+                    W[g] = min(__float2uint_rn(pe * vsc * rscale), 0xFFFFFFu);
+                    Lq[g] = __reduce_add_sync(0xffffffffu, __float2uint_rn(pe * 16777216.0f));
+                }
+                // operand B and the slice stats of buffer a are free once chunk c - kTcAcc is merged
+                ok = __all_sync(0xffffffffu, dev::mbar_wait(tempty_bar(a), aph ^ 1u, abort_flag, &g_decode_error,
+                                                            kErrTcScore));
+                if (!ok) continue;
+                uint8_t* bq = b_p + a * kTcBBytes;
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int k = 0; k < 3; ++k) {
+                        const int row = 3 * g + k;
+                        bq[(row >> 3) * 1024 + (row & 7) * 128 + ((kb ^ (row & 7)) << 4) + kx] =
+                            (uint8_t)(W[g] >> (8 * k));
+                    }
+                if (lane == 0) {
+                    TcSlice& S = slices[a * 4 + sw];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        S.M[g] = M[g];
+                        S.L[g] = (float)Lq[g] * 5.9604644775390625e-8f;   // 2^-24
+                    }
+                    S.inv_scale = smax / kTcWmax;
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) dev::mbar_arrive(bready_bar(a));
+            }
+        }
+    } else {
+        // ---------------- accumulators: value dimension d ----------------
+        const int quarter = warp & 3;
+        const int d = quarter * 32 + lane;
+        int c = 0;
+        bool ok = true;
+        for (int jj = 0; ok && jj < nseg; ++jj) {
+            const Segment sg = walk.seg(jj);
+            float mrun[G], lrun[G], o[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) mrun[g] = -INFINITY, lrun[g] = 0.0f, o[g] = 0.0f;
+            for (int64_t t = sg.t0; t < sg.t1; t += kTcTok, ++c) {
+                const int a = c % kTcAcc;
+                const uint32_t aph = (uint32_t)(c / kTcAcc) & 1u;
+                const int nk = (int)((min((int64_t)kTcTok, sg.t1 - t) + 31) / 32);
+                // the scorers' arrival on bready publishes the slice stats; the MMA's
+                // completion, the accumulators
+                ok = __all_sync(0xffffffffu,
+                                dev::mbar_wait(bready_bar(a), aph, abort_flag, &g_decode_error, kErrTcAcc) &&
+                                    dev::mbar_wait(tfull_bar(a), aph, abort_flag, &g_decode_error, kErrTcAcc));
+                if (!ok) break;  // warp-uniform: tcgen05.ld is .aligned
+                dev::tc_fence_after();
+                // the chunk's four slices (64 contiguous columns) in one load, the slice
+                // stats into registers, then the buffer goes back to the scorers
+                uint32_t r[64];
+                dev::tmem_ld_32x32b_x64(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 4) * 16u, r);
+                float sM[4][G], sL[4][G], sinv[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const TcSlice& S = slices[a * 4 + k];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {   // slices past the chunk's tokens: never written
+                        sM[k][g] = k < nk ? S.M[g] : -INFINITY;
+                        sL[k][g] = k < nk ? S.L[g] : 0.0f;
+                    }
+                    sinv[k] = k < nk ? S.inv_scale : 0.0f;
+                }
+                dev::tmem_ld_wait();
+                dev::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) dev::mbar_arrive(tempty_bar(a));
+                float Mc[G], num[G], L[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    Mc[g] = fmaxf(fmaxf(sM[0][g], sM[1][g]), fmaxf(sM[2][g], sM[3][g]));
+                    num[g] = 0.0f;
+                    L[g] = 0.0f;
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        // a slice past the chunk's tokens, or without valid ones, has M = -inf
+                        const float f = sM[k][g] == -INFINITY ? 0.0f : fast_exp2(sM[k][g] - Mc[g]);
+                        const float x = __fmaf_rn((float)(int)r[16 * k + 3 * g + 2], 65536.0f,
+                                                  __fmaf_rn((float)(int)r[16 * k + 3 * g + 1], 256.0f,
+                                                            (float)(int)r[16 * k + 3 * g]));
+                        num[g] = __fmaf_rn(x * sinv[k], f, num[g]);
+                        L[g] = __fmaf_rn(sL[k][g], f, L[g]);
+                    }
+                }
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float mn = fmaxf(mrun[g], Mc[g]);
+                    const float al = fast_exp2(mrun[g] - mn);
+                    const float be = fast_exp2(Mc[g] - mn);
+                    o[g] = __fmaf_rn(o[g], al, num[g] * be);
+                    lrun[g] = __fmaf_rn(lrun[g], al, L[g] * be);
+                    mrun[g] = mn;
+                }
+            }
+            if (!ok) break;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float* slot = p.ws + (((int64_t)cta * p.maxj + jj) * G + g) * (2 + kD);
+                slot[2 + d] = o[g];
+                if (d == 0) {
+                    slot[0] = mrun[g];
+                    slot[1] = lrun[g];
+                }
+            }
+        }
+    }
+
+    __syncwarp();  // reconverge warps 0 and 1, whose lane 0 ran the role loop alone
+    dev::tc_fence_before();
+    __syncthreads();
+    dev::tc_fence_after();
+    if (warp == 1) dev::tmem_dealloc(tmem, kTcTmemCols);
+}
+
 // out[b][h][d]: merge, over the CTAs whose ranges covered unit u = b * Hkv + h / G,
 // acc_s[d] 2^(m_s - M) / sum_s l_s 2^(m_s - M).
 __global__ void __launch_bounds__(kD)
@@ -1442,8 +1823,30 @@ cudaError_t run_qjl_pf(const DecodeParams& p, int ctas, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// The tensor-core QJL decode applies when every chunk's copies are 16-byte aligned:
+// chunk starts and lengths are multiples of 8 tokens (T and the unit capacity are), the
+// arrays are 16-byte aligned, and the value rows fit a TMA row coordinate.
+bool qjl_tc_applies(const DecodeParams& p) {
+    const auto al16 = [](const void* x) { return reinterpret_cast<uintptr_t>(x) % 16 == 0; };
+    const int64_t units = p.T > 0 ? p.total / p.T : 0;
+    return p.knew == nullptr && p.want_out && p.k4p == nullptr && p.m <= 256 && p.m % 32 == 0 &&
+           p.T % 8 == 0 && p.cap % 8 == 0 && al16(p.kw) && al16(p.kn) && al16(p.vs) && al16(p.vc) &&
+           units * p.cap <= (int64_t)INT32_MAX;
+}
+
 template <int G>
 cudaError_t run_qjl(const DecodeParams& p, int ctas, cudaStream_t st) {
+    if (qjl_tc_applies(p)) {
+        CUtensorMap vmap;
+        if (make_u8_rows_map(&vmap, p.vc, (p.total / p.T) * p.cap, kTcTok)) {
+            auto kern = decode_qjl_tc_kernel<G>;
+            const size_t smem = tc_smem_bytes();
+            const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            kern<<<ctas, kTcThreads, smem, st>>>(p, vmap);
+            return cudaGetLastError();
+        }
+    }
     if (p.knew == nullptr && p.m <= 256) {
         auto kern = decode_qjl_pf_kernel<G>;
         const size_t smem = qjl_pf_smem<G>();

@@ -1,6 +1,7 @@
 // Internal declarations shared by the library's translation units (host side).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -38,6 +39,9 @@ cudaError_t launch_dequantize_int8_channelwise(const int8_t* codes, const float*
 // Returns cudaErrorNotSupported when the driver's tensor-map encoder is unavailable.
 cudaError_t launch_qjl_encode(const uint16_t* keys, int64_t n_keys, const uint16_t* S, int m,
                               uint32_t* words, uint16_t* norms, cudaStream_t st);
+// TMA descriptor of a byte tensor [rows][128] (box 128 bytes x box_rows, 128-byte
+// swizzle); false if the driver's encoder is unavailable or rejects the arguments.
+bool make_u8_rows_map(CUtensorMap* map, const void* ptr, int64_t rows, int box_rows);
 cudaError_t launch_qjl_query_sketch(const uint16_t* q, int64_t n_q, const uint16_t* S, int m,
                                     float* v, cudaStream_t st);
 cudaError_t read_and_clear_device_error(uint32_t* code);

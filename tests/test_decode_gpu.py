@@ -100,6 +100,34 @@ def test_decode_qjl_parity(kvq, B, Hq, Hkv, T, m):
     assert np.all(err <= tol), float((err / tol).max())
 
 
+# Shapes whose token count and capacity are multiples of 8 take the tensor-core value
+# pass (chunks of 128 tokens): one partial chunk, several chunks with a partial tail,
+# CTA ranges that span many short units (several segments and table builds per CTA),
+# one, two and four query heads per KV head, m = 32, 128 and 256.
+@pytest.mark.parametrize("B,Hq,Hkv,T,m", [(1, 4, 1, 8, 256), (2, 8, 2, 1504, 256), (1, 32, 8, 2048, 256),
+                                          (1, 4, 4, 704, 128), (1, 2, 1, 336, 32), (16, 32, 8, 8, 256),
+                                          (4, 8, 4, 96, 256), (3, 12, 3, 5000, 256)])
+def test_decode_qjl_tc_parity(kvq, B, Hq, Hkv, T, m):
+    test_decode_qjl_parity(kvq, B, Hq, Hkv, T, m)
+
+
+def test_decode_qjl_tc_zero_value_chunk(kvq):
+    """Value rows that are all zero (scale 0) over whole 128-token chunks and over a
+    partial one: those chunks add nothing to the weighted sum but still to the softmax
+    sum.  Against the oracle on the same codes and scales."""
+    B, Hq, Hkv, T, m = 1, 8, 2, 1000, 256
+    q, S, w, n, vc, vs = _qjl_cache(900, B, Hkv, T, Hq, m)
+    vc[0, 0, 128:384] = 0
+    vs[0, 0, 128:384] = 0.0
+    vc[0, 1, 900:] = 0
+    vs[0, 1, 900:] = 0.0
+    ref = oracle.decode_attention(q, k_words=w, k_norms=n, S=S, v_codes=vc, v_scales=vs)
+    qg, Sg, wg, ng, vcg, vsg = _cuda(q, S, w.view(np.int32), n, vc, vs)
+    out, _ = kvq.kvq_decode_attention(qg, k_words=wg, k_norms=ng, sketch=Sg, v_codes=vcg, v_scales=vsg)
+    assert np.abs(to_np(out) - ref["out"]).max() <= OUT_TOL
+    assert kvq.kvq_device_error() == 0
+
+
 def test_decode_int8_llama7b_layer_sampled(kvq):
     """One layer of the 7B-shaped cache (batch 8, 32 heads, 4096 tokens): GPU quantize
     then GPU decode; 6 sampled (batch, head) units re-done by the oracle from the fp16
