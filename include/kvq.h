@@ -147,6 +147,13 @@ kvq_status kvq_qjl_query_sketch(const uint16_t* q_f16, int64_t n_q, int32_t d,
  * otherwise); QJL needs m a multiple of 32 in [32, 256]; Hq % Hkv == 0; T >= 1
  * (a softmax over no tokens is undefined: KVQ_ERR_INVALID_ARG).  sm_scale == 0 selects
  * 1/sqrt(head_dim).
+ * Precision: scores and the softmax in fp32 (exponentials by the hardware 2^x); out
+ * within 2e-3 absolute of the fp64 value of the formula above.  With QJL keys, when T
+ * is a multiple of 8 and k_words, k_norms, v_codes and v_scales are 16-byte aligned,
+ * the weighted sum runs on the tensor cores: per block of 32 tokens and head, the
+ * weights p_t * sv_t relative to the block's largest p and sv become 24-bit fixed-point
+ * integers that multiply the INT8 codes exactly in int32 (error at most 2^-25 of the
+ * block's largest sv per token); otherwise in fp32 on the CUDA cores.
  * workspace: caller-owned device memory of at least kvq_decode_workspace_bytes(a)
  * bytes, 256-byte aligned (KVQ_ERR_WORKSPACE otherwise).  It holds per-split partial
  * softmax states and the query sketches; its contents on entry do not matter.
