@@ -333,8 +333,9 @@ size_t kvq_decode_int4v_workspace_bytes(const kvq_decode_int4v_args* a);
  *              results yields M and L).  base.scores_out may be NULL: the scores then
  *              go to the workspace.
  *   attn_mass: [batch][seq_len] fp32, 4-byte aligned, read and written (start it at 0).
- * Workspace from kvq_decode_mass_workspace_bytes.  Three launches; errors as
- * kvq_decode_attention, KVQ_ERR_INVALID_ARG for a missing base.out or attn_mass.
+ * Workspace from kvq_decode_mass_workspace_bytes.  Three launches (four with QJL keys:
+ * the query sketch); errors as kvq_decode_attention, KVQ_ERR_INVALID_ARG for a missing
+ * base.out or attn_mass.
  */
 typedef struct kvq_decode_mass_args {
     kvq_decode_args base;

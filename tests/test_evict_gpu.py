@@ -71,7 +71,8 @@ def _mass_tol(ref, Hq):
 @pytest.mark.parametrize("fmt,B,Hq,Hkv,T", [("int8", 1, 1, 1, 1), ("int8", 2, 8, 2, 33),
                                             ("int8", 1, 8, 1, 1000), ("int8", 2, 16, 4, 4097),
                                             ("int8", 3, 24, 3, 70), ("qjl", 1, 4, 1, 7),
-                                            ("qjl", 2, 8, 2, 1500), ("qjl", 1, 32, 8, 2049)])
+                                            ("qjl", 2, 8, 2, 1500), ("qjl", 1, 32, 8, 2049),
+                                            ("qjl", 1, 4, 1, 8), ("qjl", 2, 8, 2, 1504)])
 @pytest.mark.parametrize("want_scores", [False, True])
 def test_mass_decode_parity(kvq, fmt, B, Hq, Hkv, T, want_scores):
     make = _int8_cache if fmt == "int8" else _qjl_cache
