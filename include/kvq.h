@@ -149,8 +149,8 @@ kvq_status kvq_qjl_query_sketch(const uint16_t* q_f16, int64_t n_q, int32_t d,
  * 1/sqrt(head_dim).
  * Precision: scores and the softmax in fp32 (exponentials by the hardware 2^x); out
  * within 2e-3 absolute of the fp64 value of the formula above.  With QJL keys, when T
- * is a multiple of 8 and k_words, k_norms, v_codes and v_scales are 16-byte aligned,
- * the weighted sum runs on the tensor cores: per block of 32 tokens and head, the
+ * is a multiple of 8, k_words, k_norms, v_codes and v_scales are 16-byte aligned and
+ * the cache has fewer than 2^31 token rows, the weighted sum runs on the tensor cores: per block of 32 tokens and head, the
  * weights p_t * sv_t relative to the block's largest p and sv become 24-bit fixed-point
  * integers that multiply the INT8 codes exactly in int32 (error at most 2^-25 of the
  * block's largest sv per token); otherwise in fp32 on the CUDA cores.
