@@ -144,9 +144,13 @@ kvq_status kvq_qjl_query_sketch(const uint16_t* q_f16, int64_t n_q, int32_t d,
  *   out        [B][Hq][D] fp32 or NULL
  *   scores_out [B][Hq][T] fp32 raw scores (before sm_scale) or NULL
  * out and scores_out may not both be NULL.  head_dim must be 128 (KVQ_ERR_UNSUPPORTED
- * otherwise); QJL needs m a multiple of 32 in [32, 256]; Hq % Hkv == 0; T >= 1
- * (a softmax over no tokens is undefined: KVQ_ERR_INVALID_ARG).  sm_scale == 0 selects
- * 1/sqrt(head_dim).
+ * otherwise); QJL needs m a multiple of 32 in [32, 256]; Hq % Hkv == 0, any group size
+ * G = Hq / Hkv (MHA G = 1, GQA, MQA Hkv = 1); T >= 1 (a softmax over no tokens is
+ * undefined: KVQ_ERR_INVALID_ARG).  sm_scale == 0 selects 1/sqrt(head_dim).
+ * Group sizes: one CTA serves up to 8 query heads of a KV head with INT8 keys and up
+ * to 4 with QJL keys (the largest power of two dividing G); a larger G is served by
+ * G / that CTAs per token range, which stream the same cache bytes side by side (the
+ * second read mostly from L2).
  * Precision: scores and the softmax in fp32 (exponentials by the hardware 2^x); out
  * within 2e-3 absolute of the fp64 value of the formula above.  With QJL keys, when T
  * is a multiple of 8, k_words, k_norms, v_codes and v_scales are 16-byte aligned and
@@ -158,6 +162,9 @@ kvq_status kvq_qjl_query_sketch(const uint16_t* q_f16, int64_t n_q, int32_t d,
  * bytes, 256-byte aligned (KVQ_ERR_WORKSPACE otherwise).  It holds per-split partial
  * softmax states and the query sketches; its contents on entry do not matter.
  * Launches 2 kernels (INT8 keys) or 3 (QJL keys) on `stream`; no host synchronisation.
+ * If a decode kernel records a device-side error (see kvq_device_error), the outputs of
+ * this and of every later decode call are NaN until kvq_device_error() reads and clears
+ * the error: out is valid only while kvq_device_error() reports 0.
  */
 typedef struct kvq_decode_args {
     int64_t batch;
@@ -407,7 +414,7 @@ kvq_status kvq_gather_rows_multi(const kvq_gather_array* arrays, int32_t n_array
  *   base:      key_format = KVQ_KEYS_QJL with k_words / k_norms_f16 = the residual's
  *              sign words and fp16 norms, sketch_f16 / sketch_dim = S and m (128 or
  *              256, else KVQ_ERR_UNSUPPORTED); everything else as kvq_decode_attention
- *              (G = Hq / Hkv in {1, 2, 4}).
+ *              (any group size G = Hq / Hkv).
  *   k_packed4: [B][Hkv][T][D/2] INT4 codes (16-byte aligned); k_scales4, k_zeros4:
  *              [B][Hkv][T][D/k_group] fp32 (4-byte aligned); k_group 32, 64 or 128.
  * Workspace from kvq_decode_qjlres_workspace_bytes.  Errors as kvq_decode_attention.

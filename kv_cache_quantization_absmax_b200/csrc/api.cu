@@ -55,13 +55,6 @@ kvq_status check_decode(const kvq_decode_args* a) {
     if (a->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
     if (!a->out && !a->scores_out) return KVQ_ERR_INVALID_ARG;
     if (!(a->sm_scale == a->sm_scale) || a->sm_scale < 0.0f) return KVQ_ERR_INVALID_ARG;
-    {
-        // Query heads per KV head served by one CTA: INT8 keys up to 8, QJL keys up to 4
-        // (four 32 KB byte tables fill the shared memory a CTA may use).
-        const int64_t G = a->n_q_heads / a->n_kv_heads;
-        const bool pow2 = G == 1 || G == 2 || G == 4 || G == 8;
-        if (!pow2 || (a->key_format == KVQ_KEYS_QJL && G > 4)) return KVQ_ERR_UNSUPPORTED;
-    }
     if (a->batch == 0) return KVQ_OK;
     if (!a->q_f16 || !aligned(a->q_f16, 16)) return KVQ_ERR_INVALID_ARG;
     if (a->key_format == KVQ_KEYS_INT8) {

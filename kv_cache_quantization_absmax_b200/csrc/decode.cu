@@ -68,6 +68,9 @@ struct DecodeParams {
     int64_t total;          // units * T
     int Hq;
     int Hkv;
+    int Gt;                 // query heads per KV head (Hq / Hkv)
+    int nsub;               // head subgroups per KV head: the kernel's G heads each; CTA c
+                            // covers token range c / nsub for heads of subgroup c % nsub
     int maxj;               // unit segments a range can touch
     int m;
     float scale_log2;       // sm_scale * log2(e)
@@ -415,7 +418,7 @@ decode_int8_kernel(const DecodeParams p) {
     const int cta = blockIdx.x;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const RangeWalk walk(p, cta);
+    const RangeWalk walk(p, cta / p.nsub);
     const int nseg = walk.count();
     const uint32_t ring = dev::smem_u32(smem_raw);
     float* red = reinterpret_cast<float*>(smem_raw + kI8Stages * kI8StageBytes);  // [warps][G][2+D]
@@ -541,11 +544,11 @@ decode_int8_kernel(const DecodeParams p) {
         const int64_t row0 = sg.u * p.cap;
         const int64_t b = sg.u / p.Hkv;
         const int kvh = (int)(sg.u % p.Hkv);
+        const int64_t hb = b * p.Hq + (int64_t)kvh * p.Gt + (int64_t)(cta % p.nsub) * G;
         uint64_t qp[G][NP];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const int64_t h = (int64_t)kvh * G + g;
-            const uint4* src = reinterpret_cast<const uint4*>(p.q + (b * p.Hq + h) * kD + sub * DPL);
+            const uint4* src = reinterpret_cast<const uint4*>(p.q + (hb + g) * kD + sub * DPL);
 #pragma unroll
             for (int v = 0; v < DPL / 8; ++v) {
                 const uint4 a = __ldg(src + v);
@@ -675,7 +678,7 @@ decode_int8_kernel(const DecodeParams p) {
                     if (valid[u]) {
 #pragma unroll
                         for (int g = 0; g < G; ++g)
-                            p.scores_out[(b * p.Hq + (int64_t)kvh * G + g) * p.T + tstage + tok0 + u] =
+                            p.scores_out[(hb + g) * p.T + tstage + tok0 + u] =
                                 score[u][g];
                     }
             }
@@ -814,7 +817,7 @@ decode_qjl_kernel(const DecodeParams p) {
     const int cta = blockIdx.x;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const RangeWalk walk(p, cta);
+    const RangeWalk walk(p, cta / p.nsub);
     const int nseg = walk.count();
     const int nw = p.m / 32;
     const int npos = p.m / 8;
@@ -866,6 +869,7 @@ decode_qjl_kernel(const DecodeParams p) {
         const int64_t row0 = sg.u * p.cap;
         const int64_t b = sg.u / p.Hkv;
         const int kvh = (int)(sg.u % p.Hkv);
+        const int64_t hb = b * p.Hq + (int64_t)kvh * p.Gt + (int64_t)(cta % p.nsub) * G;
         __syncthreads();  // the previous segment's merge no longer reads red[]
         // ---- byte tables ----
         if (threadIdx.x < 512) {
@@ -874,7 +878,7 @@ decode_qjl_kernel(const DecodeParams p) {
             float v[G][8];
     #pragma unroll
             for (int g = 0; g < G; ++g) {
-                const float* src = p.sketch_v + (b * p.Hq + (int64_t)kvh * G + g) * p.m + pos * 8;
+                const float* src = p.sketch_v + (hb + g) * p.m + pos * 8;
     #pragma unroll
                 for (int k = 0; k < 8; ++k) v[g][k] = pos < npos ? __ldg(src + k) : 0.0f;
             }
@@ -994,7 +998,7 @@ decode_qjl_kernel(const DecodeParams p) {
             if (p.scores_out != nullptr && valid) {
 #pragma unroll
                 for (int g = 0; g < G; ++g)
-                    p.scores_out[(b * p.Hq + (int64_t)kvh * G + g) * p.T + t0 + lane] = score[g];
+                    p.scores_out[(hb + g) * p.T + t0 + lane] = score[g];
             }
             if (!p.want_out) continue;
             // ---- online softmax at warp granularity ----
@@ -1108,7 +1112,7 @@ decode_qjl_pf_kernel(const DecodeParams p) {
     const int cta = blockIdx.x;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const RangeWalk walk(p, cta);
+    const RangeWalk walk(p, cta / p.nsub);
     const int nseg = walk.count();
     const int nw = p.m / 32;
     float* lut = dsmem;                              // 2 halves x [256][16] x 4 floats
@@ -1142,12 +1146,13 @@ decode_qjl_pf_kernel(const DecodeParams p) {
         const int64_t row0 = sg.u * p.cap;
         const int64_t b = sg.u / p.Hkv;
         const int kvh = (int)(sg.u % p.Hkv);
+        const int64_t hb = b * p.Hq + (int64_t)kvh * p.Gt + (int64_t)(cta % p.nsub) * G;
         __syncthreads();  // the previous segment's merge no longer reads red[]
-        build_sign_tables<G>(lut, p.sketch_v + (b * p.Hq + (int64_t)kvh * G) * p.m, p.m, p.m, threadIdx.x,
+        build_sign_tables<G>(lut, p.sketch_v + hb * p.m, p.m, p.m, threadIdx.x,
                              kQpfThreads);
         if constexpr (RES) {
             for (int i = threadIdx.x; i < G * kD; i += kQpfThreads)
-                qs[i] = __half2float(__ushort_as_half(p.q[(b * p.Hq + (int64_t)kvh * G) * kD + i]));
+                qs[i] = __half2float(__ushort_as_half(p.q[hb * kD + i]));
         }
         __syncthreads();
         if constexpr (RES) {
@@ -1276,7 +1281,7 @@ decode_qjl_pf_kernel(const DecodeParams p) {
                 if (p.scores_out != nullptr && valid) {
 #pragma unroll
                     for (int g = 0; g < G; ++g)
-                        p.scores_out[(b * p.Hq + (int64_t)kvh * G + g) * p.T + t0 + lane] = score[g];
+                        p.scores_out[(hb + g) * p.T + t0 + lane] = score[g];
                 }
                 if (p.want_out) {
                     // ---- online softmax at warp granularity ----
@@ -1464,7 +1469,7 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int cta = blockIdx.x;
-    const RangeWalk walk(p, cta);
+    const RangeWalk walk(p, cta / p.nsub);
     const int nseg = walk.count();
     const int nw = p.m / 32;
 
@@ -1570,11 +1575,12 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
             const Segment sg = walk.seg(jj);
             const int64_t b = sg.u / p.Hkv;
             const int kvh = (int)(sg.u % p.Hkv);
+            const int64_t hb = b * p.Hq + (int64_t)kvh * p.Gt + (int64_t)(cta % p.nsub) * G;
             // the tables are rebuilt per unit by all scorers; every scorer reaches both
             // barriers, also after an abort (they then skip the work in between)
             asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcScorerWarps) : "memory");
             if (ok)
-                build_sign_tables<G>(lut, p.sketch_v + (b * p.Hq + (int64_t)kvh * G) * p.m, p.m, p.m,
+                build_sign_tables<G>(lut, p.sketch_v + hb * p.m, p.m, p.m,
                                      threadIdx.x - 64, 32 * kTcScorerWarps);
             asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcScorerWarps) : "memory");
             for (int64_t t = sg.t0; t < sg.t1; t += kTcTok, ++c) {
@@ -1609,7 +1615,7 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
                     const float score = p.qjl_c * nrm * sc[g];
                     lg[g] = valid ? score * p.scale_log2 : -INFINITY;
                     if (p.scores_out != nullptr && valid)
-                        p.scores_out[(b * p.Hq + (int64_t)kvh * G + g) * p.T + t + st] = score;
+                        p.scores_out[(hb + g) * p.T + t + st] = score;
                 }
                 const float smax = warp_max(vsc);
                 const float rscale = smax > 0.0f ? kTcWmax / smax : 0.0f;
@@ -1740,26 +1746,35 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
     if (warp == 1) dev::tmem_dealloc(tmem, kTcTmemCols);
 }
 
-// out[b][h][d]: merge, over the CTAs whose ranges covered unit u = b * Hkv + h / G,
-// acc_s[d] 2^(m_s - M) / sum_s l_s 2^(m_s - M).
+// out[b][h][d]: merge, over the token ranges that covered KV unit u = b * Hkv + h / Gt,
+// acc_s[d] 2^(m_s - M) / sum_s l_s 2^(m_s - M).  The states of query head h were written by
+// the CTAs of its head subgroup (h % Gt) / G, one per range.  If a decode kernel recorded
+// an error (a bounded wait gave up and the CTA skipped its work), the states are not
+// complete and the head's output is NaN.
 __global__ void __launch_bounds__(kD)
-decode_combine_kernel(const float* __restrict__ ws, int64_t T, int64_t W, int maxj, int Hq, int Hkv,
-                      float* __restrict__ out, float* __restrict__ fin_ml) {
+decode_combine_kernel(const float* __restrict__ ws, int64_t T, int64_t W, int maxj, int Hq, int Hkv, int G,
+                      int nsub, float* __restrict__ out, float* __restrict__ fin_ml) {
     // Launched as a programmatic dependent of the decode kernel: nothing is read before
     // that kernel has completed and its partial states are visible.
     dev::griddep_wait();
     const int64_t bh = blockIdx.x;
     const int64_t b = bh / Hq;
     const int h = (int)(bh % Hq);
-    const int G = Hq / Hkv;
-    const int64_t u = b * Hkv + h / G;
+    const int Gt = Hq / Hkv;
+    const int64_t u = b * Hkv + h / Gt;
+    const int sub = (h % Gt) / G;
     const int gh = h % G;
     const int64_t c0 = (u * T) / W;
     const int64_t c1 = ((u + 1) * T - 1) / W;
     const int d = threadIdx.x;
+    if (*reinterpret_cast<volatile unsigned int*>(&g_decode_error) != 0u) {
+        out[bh * kD + d] = __int_as_float(0x7fc00000);
+        if (fin_ml != nullptr && d == 0) fin_ml[2 * bh] = fin_ml[2 * bh + 1] = __int_as_float(0x7fc00000);
+        return;
+    }
     auto slot = [&](int64_t c) {
         const int64_t j = u - (c * W) / T;
-        return ws + ((c * maxj + j) * G + gh) * (2 + kD);
+        return ws + (((c * nsub + sub) * maxj + j) * G + gh) * (2 + kD);
     };
     float mx = -INFINITY;
     for (int64_t c = c0; c <= c1; ++c) mx = fmaxf(mx, slot(c)[0]);
@@ -1909,21 +1924,38 @@ cudaError_t read_and_clear_decode_error(uint32_t* code) {
     return e;
 }
 
+// Query heads one CTA serves per KV head: up to 8 with INT8 keys, up to 4 with QJL keys
+// (four 32 KB byte tables fill the shared memory a CTA may use); the largest such
+// power of two that divides Hq / Hkv.
+int decode_group_size(const kvq_decode_args* a) {
+    const int64_t Gt = a->n_q_heads / a->n_kv_heads;
+    const int cap = a->key_format == KVQ_KEYS_QJL ? 4 : 8;
+    int g = cap;
+    while (g > 1 && Gt % g != 0) g >>= 1;
+    return g;
+}
+
 DecodePlan plan_decode(const kvq_decode_args* a, int sm_count) {
     DecodePlan pl{};
-    const int64_t G = a->n_q_heads / a->n_kv_heads;
+    const int64_t Gt = a->n_q_heads / a->n_kv_heads;
+    const int G = decode_group_size(a);
     const bool qjl = a->key_format == KVQ_KEYS_QJL;
+    pl.G = G;
+    pl.nsub = (int)(Gt / G);
     pl.units = a->batch * a->n_kv_heads;
     const int64_t T = a->seq_len;
     const int64_t total = pl.units * T;
     // As many CTAs as can be resident at once: up to three 68 KB-ring INT8 CTAs per SM,
-    // or one 512-thread QJL CTA per SM (its byte tables fill shared memory).
+    // or one 512-thread QJL CTA per SM (its byte tables fill shared memory); the token
+    // space is cut into one range per nsub of them (the CTAs of a range stream the same
+    // bytes side by side, each for its own head subgroup).
     // (residual keys run the QJL decode kernel: their key_format is QJL too)
-    const int64_t resident = (int64_t)sm_count * (qjl ? 1 : int8_ctas_per_sm((int)G));
-    int64_t W = total > 0 ? (total + resident - 1) / resident : kRange;
+    const int64_t resident = (int64_t)sm_count * (qjl ? 1 : int8_ctas_per_sm(G));
+    const int64_t ranges = resident / pl.nsub > 0 ? resident / pl.nsub : 1;
+    int64_t W = total > 0 ? (total + ranges - 1) / ranges : kRange;
     W = (W + kRange - 1) / kRange * kRange;
     pl.W = W;
-    pl.ctas = total > 0 ? (int)((total + W - 1) / W) : 0;
+    pl.ctas = total > 0 ? (int)((total + W - 1) / W) * pl.nsub : 0;
     pl.maxj = (int)((W + T - 1) / T + 1);
     pl.partial_bytes = align256((size_t)pl.ctas * pl.maxj * G * (2 + kD) * sizeof(float));
     pl.sketch_bytes = qjl ? align256((size_t)a->batch * a->n_q_heads * a->sketch_dim * sizeof(float)) : 0;
@@ -1938,7 +1970,7 @@ float decode_scale_log2(const kvq_decode_args* a) {
 
 cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaStream_t st,
                           const AppendSpec* app, const Int4Values* v4, float* fin_ml, const Int4Keys* k4) {
-    const int G = (int)(a->n_q_heads / a->n_kv_heads);
+    const int G = pl.G;
     const bool qjl = a->key_format == KVQ_KEYS_QJL;
     char* ws = static_cast<char*>(a->workspace);
     DecodeParams p{};
@@ -1969,6 +2001,8 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
     p.total = pl.units * a->seq_len;
     p.Hq = (int)a->n_q_heads;
     p.Hkv = (int)a->n_kv_heads;
+    p.Gt = (int)(a->n_q_heads / a->n_kv_heads);
+    p.nsub = pl.nsub;
     p.maxj = pl.maxj;
     p.m = qjl ? a->sketch_dim : 0;
     p.scale_log2 = decode_scale_log2(a);
@@ -2009,7 +2043,8 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const float* ws_c = p.ws;
-    return cudaLaunchKernelEx(&cfg, decode_combine_kernel, ws_c, p.T, p.W, p.maxj, p.Hq, p.Hkv, a->out, fin_ml);
+    return cudaLaunchKernelEx(&cfg, decode_combine_kernel, ws_c, p.T, p.W, p.maxj, p.Hq, p.Hkv, G, p.nsub,
+                              a->out, fin_ml);
 }
 
 }  // namespace kvq

@@ -48,9 +48,11 @@ cudaError_t read_and_clear_device_error(uint32_t* code);
 
 // decode.cu
 struct DecodePlan {
+    int G;                // query heads per CTA (a power of two dividing Hq / Hkv)
+    int nsub;             // head subgroups per KV head: (Hq / Hkv) / G
     int64_t units;        // B * Hkv
-    int ctas;             // CTAs of the partial kernel (one contiguous token range each)
-    int64_t W;            // tokens per CTA range
+    int ctas;             // CTAs of the partial kernel: nsub per contiguous token range
+    int64_t W;            // tokens per range
     int maxj;             // unit segments one range can touch
     size_t partial_bytes; // per-segment softmax states
     size_t sketch_bytes;  // query sketches (QJL)

@@ -289,7 +289,7 @@ def kvq_decode_attention(q, *, k_codes=None, k_scales=None, k_words=None, k_norm
     need = kvq_decode_workspace_bytes(a)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
-    a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     _check("kvq_decode_attention", lib.kvq_decode_attention(ctypes.byref(a), _stream(stream)))
     return (out if want_out else None), (scores_out if want_scores else None)
 
@@ -361,7 +361,7 @@ def kvq_decode_append(q, k_new, v_new, *, T, k_codes=None, k_scales=None, k_word
     need = int(lib.kvq_decode_append_workspace_bytes(ctypes.byref(a)))
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
-    a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     _check("kvq_decode_append", lib.kvq_decode_append(ctypes.byref(a), _stream(stream)))
     return (out if want_out else None), (scores_out if want_scores else None)
 
@@ -454,7 +454,7 @@ def kvq_decode_attention_int4v(q, *, k_codes, k_scales, v_packed, v_scales4, v_z
     need = int(lib.kvq_decode_int4v_workspace_bytes(ctypes.byref(a)))
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
-    a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     _check("kvq_decode_attention_int4v", lib.kvq_decode_attention_int4v(ctypes.byref(a), _stream(stream)))
     return out, (scores_out if want_scores else None)
 
@@ -492,7 +492,7 @@ def kvq_decode_attention_mass(q, attn_mass, *, k_codes=None, k_scales=None, k_wo
     need = int(lib.kvq_decode_mass_workspace_bytes(ctypes.byref(a)))
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
-    a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     _check("kvq_decode_attention_mass", lib.kvq_decode_attention_mass(ctypes.byref(a), _stream(stream)))
     return out, (scores_out if want_scores else None)
 
@@ -587,7 +587,7 @@ def kvq_decode_attention_qjlres(q, *, k_packed4, k_scales4, k_zeros4, k_group, k
     need = int(lib.kvq_decode_qjlres_workspace_bytes(ctypes.byref(a)))
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
-    a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    a.base.workspace, a.base.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     _check("kvq_decode_attention_qjlres", lib.kvq_decode_attention_qjlres(ctypes.byref(a), _stream(stream)))
     return (out if want_out else None), (scores_out if want_scores else None)
 

@@ -250,6 +250,33 @@ def decode_attention(q_f16, *, k_codes=None, k_scales=None, k_words=None, k_norm
     return {"out": out, "scores": scores, "probs": probs}
 
 
+def decode_from_scores(scores, values, sm_scale=0.0):
+    """The decode step after its scores, in fp64 ("QJL" abstract and "GPU-Accelerated INT8
+    Quantization ..." abstract: attention over the compressed cache; "Q-TensorFormer" model
+    card, section 4: query head h reads KV head h // G).  For each (b, h):
+        p_t = exp(sigma s_t - max_t sigma s_t) / sum_t exp(...),   out = sum_t p_t v_t,
+    sigma = sm_scale, or the fp32 value of 1/sqrt(D) when 0 (as decode_attention).
+    scores [B, Hq, T] (any float dtype, used in fp64); values [B, Hkv, T, D] (the
+    dequantized value rows, used in fp64).  Returns (out fp64 [B, Hq, D], p fp64
+    [B, Hq, T])."""
+    s = np.asarray(scores, np.float64)
+    v = np.asarray(values, np.float64)
+    B, Hq, T = s.shape
+    Hkv, D = v.shape[1], v.shape[3]
+    assert v.shape == (B, Hkv, T, D) and Hq % Hkv == 0
+    G = Hq // Hkv
+    # the fp32 value of 1/sqrt(D) that decode_attention uses
+    sigma = float(sm_scale) if sm_scale != 0.0 else float(np.float32(1.0) / np.sqrt(np.float32(D)))
+    lg = sigma * s
+    e = np.exp(lg - lg.max(axis=-1, keepdims=True))
+    p = e / e.sum(axis=-1, keepdims=True)
+    out = np.empty((B, Hq, D), np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            out[b, h] = p[b, h] @ v[b, h // G]
+    return out, p
+
+
 def decode_append(q_f16, k_new_f16, v_new_f16, *, T, k_codes=None, k_scales=None, k_words=None,
                   k_norms=None, S=None, v_codes=None, v_scales=None, sm_scale=0.0,
                   want_out=True, want_scores=False):

@@ -89,14 +89,18 @@ def test_decode_rejects_bad_arguments(kvq):
     assert call(_args(kvq, head_dim=100)) == E
     assert call(_args(kvq, out=None)) == E                     # nothing requested
     assert call(_args(kvq, key_format=5)) == E
-    assert call(_args(kvq, n_q_heads=6, n_kv_heads=2)) == U    # G = 3
+    # any group size is served (here valid arguments without a workspace)
+    for hq, hkv in ((6, 2), (16, 1), (32, 1), (24, 2)):
+        assert call(_args(kvq, n_q_heads=hq, n_kv_heads=hkv)) == kvq.KVQ_ERR_WORKSPACE
+        assert L.kvq_decode_workspace_bytes(ctypes.byref(_args(kvq, n_q_heads=hq, n_kv_heads=hkv))) > 0
     assert call(_args(kvq, k_codes=A16 + 1)) == E
     assert call(_args(kvq, q_f16=None)) == E
     assert call(_args(kvq, sm_scale=-1.0)) == E
     qjl = dict(key_format=kvq.KVQ_KEYS_QJL, k_words=A16, k_norms_f16=A16, sketch_f16=A16)
     assert call(_args(kvq, sketch_dim=100, **qjl)) == E
     assert call(_args(kvq, sketch_dim=512, **qjl)) == U
-    assert call(_args(kvq, sketch_dim=256, n_q_heads=16, **qjl)) == U   # QJL with G = 8
+    for hq in (16, 32, 6):                                              # QJL with G = 8, 16, 3
+        assert call(_args(kvq, sketch_dim=256, n_q_heads=hq, **qjl)) == kvq.KVQ_ERR_WORKSPACE
     assert call(_args(kvq, sketch_dim=256, sketch_f16=A16 + 2,
                       **{k: v for k, v in qjl.items() if k != "sketch_f16"})) == E
     # valid arguments but no workspace

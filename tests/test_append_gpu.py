@@ -4,7 +4,8 @@ The new token's key / value rows are encoded inside the decode kernel and stored
 token T of caches with a per-head capacity above T + 1.  Checked: the appended INT8
 codes and scales and the QJL norms bit-exact; QJL sign bits exact outside the band
 |(S k)_i| < 1e-4 ||k||; every other cache row untouched; decode outputs within 2e-3
-max-abs of the oracle; raw scores within the fp32 summation bound (INT8 keys) or the
+max-abs of the oracle and within the arithmetic bound (tests/_helpers.py,
+check_decode_bound); raw scores within the fp32 summation bound (INT8 keys) or the
 estimator bound on the same stored bits (QJL keys).
 """
 import numpy as np
@@ -13,7 +14,7 @@ import torch
 
 import oracle
 from kv_cache_quantization_absmax_b200 import inputs
-from tests._helpers import bit_mismatch_outside_band, score_tolerance, to_np, words_u32
+from tests._helpers import bit_mismatch_outside_band, check_decode_bound, score_tolerance, to_np, words_u32
 
 pytestmark = pytest.mark.gpu
 
@@ -44,6 +45,12 @@ def _case(seed, B, Hq, Hkv, T, cap):
     return q, k[:, :, T].copy(), v[:, :, T].copy(), k[:, :, :T], kc, ks, vc, vs
 
 
+def _vals(vc, vs):
+    """Dequantized value rows [B, Hkv, T, D]."""
+    vc, vs = np.ascontiguousarray(vc), np.ascontiguousarray(vs)
+    return oracle.dequantize_int8(vc.reshape(-1, 128), vs.reshape(-1)).reshape(vc.shape)
+
+
 def _cuda(*arrs):
     return [torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in arrs]
 
@@ -68,6 +75,8 @@ def test_append_int8(kvq, B, Hq, Hkv, T, cap):
     terms = np.abs(np.repeat(kfull, G, axis=1) * q.astype(np.float64)[:, :, None, :]).sum(-1)
     err = np.abs(to_np(scores).astype(np.float64) - ref["scores"])
     assert np.all(err <= 2 * 128 * 2.0 ** -24 * terms + 1e-30)
+    vals = _vals(ref["v_codes"][:, :, :T + 1], ref["v_scales"][:, :, :T + 1])
+    check_decode_bound(to_np(out), to_np(scores), ref["scores"], vals, qjl=False)
     assert kvq.kvq_device_error() == 0
 
 
@@ -130,6 +139,9 @@ def test_append_qjl(kvq, B, Hq, Hkv, T, cap, m):
                           v64, m)
     err = np.abs(to_np(scores).astype(np.float64) - ref2["scores"]).reshape(B * Hq, T + 1)
     assert np.all(err <= tol)
+    vs1 = ref["v_scales"][:, :, :T + 1]
+    check_decode_bound(to_np(out), to_np(scores), ref2["scores"], _vals(ref["v_codes"][:, :, :T + 1], vs1),
+                       qjl=True, v_scales=vs1)
     assert kvq.kvq_device_error() == 0
 
 

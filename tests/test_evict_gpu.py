@@ -1,7 +1,8 @@
 """GPU parity of attention-sink eviction ("Q-TensorFormer" model card, section 6,
 Attention-Sink Dynamic Eviction) against the CPU oracle.
 
-- Mass decode: the decode output as the plain decode step (max-abs 2e-3); the added
+- Mass decode: the decode output as the plain decode step (max-abs 2e-3 and the
+  arithmetic bound of tests/_helpers.py, check_decode_bound); the added
   attention mass within 2e-5 relative + 1e-7 per head of the oracle's (fp32 scores
   and exp2 on the GPU against the oracle's exactly summed scores).
 - Selection: bit-exact (same int32 indices) against the oracle run on the same fp32
@@ -14,7 +15,7 @@ import torch
 
 import oracle
 from kv_cache_quantization_absmax_b200 import inputs
-from tests._helpers import to_np
+from tests._helpers import check_decode_bound, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -64,6 +65,12 @@ def _gpu_kwargs(c):
     return g
 
 
+def _vals(c):
+    """The cache's dequantized value rows [B, Hkv, T, D]."""
+    vc, vs = c["v_codes"], c["v_scales"]
+    return oracle.dequantize_int8(vc.reshape(-1, 128), vs.reshape(-1)).reshape(vc.shape)
+
+
 def _mass_tol(ref, Hq):
     return 2e-5 * np.abs(ref) + 1e-7 * Hq
 
@@ -77,13 +84,20 @@ def _mass_tol(ref, Hq):
 def test_mass_decode_parity(kvq, fmt, B, Hq, Hkv, T, want_scores):
     make = _int8_cache if fmt == "int8" else _qjl_cache
     q, c = make(500 + T, B, Hkv, T, Hq)
-    ref_out = oracle.decode_attention(q, **c)["out"]
+    ref = oracle.decode_attention(q, want_scores=True, **c)
+    ref_out = ref["out"]
     ref_mass = oracle.attention_mass(q, **c)
     init = np.random.default_rng(T).random((B, T), dtype=np.float32)
     mass = _cuda(init)[0]
     g = _gpu_kwargs(c)
     out, scores = kvq.kvq_decode_attention_mass(_cuda(q)[0], mass, want_scores=want_scores, **g)
     assert np.abs(to_np(out) - ref_out).max() <= OUT_TOL
+    if scores is None:   # the same kernel's scores, from the plain decode step
+        _, scores = kvq.kvq_decode_attention(_cuda(q)[0], want_scores=True, **g)
+    check_decode_bound(to_np(out), to_np(scores), ref["scores"], _vals(c), qjl=fmt == "qjl",
+                       v_scales=c["v_scales"] if fmt == "qjl" else None)
+    if not want_scores:
+        scores = None
     err = np.abs(to_np(mass).astype(np.float64) - (init.astype(np.float64) + ref_mass))
     assert np.all(err <= _mass_tol(ref_mass, Hq) + 2.0 ** -23 * (init + ref_mass)), float(err.max())
     assert (scores is not None) == want_scores
@@ -237,9 +251,11 @@ def test_evict_pipeline_end_to_end(kvq, fmt):
             want = cc["k_words"].view(np.int32) if k == "k_words" else cc[k]
             assert np.array_equal(to_np(gc[k]), want), k
     q = inputs.gaussian_queries(720, B, Hq)
-    out, _ = kvq.kvq_decode_attention(_cuda(q)[0], **gc)
-    ref = oracle.decode_attention(q, **cc)["out"]
-    assert np.abs(to_np(out) - ref).max() <= OUT_TOL
+    out, scores = kvq.kvq_decode_attention(_cuda(q)[0], want_scores=True, **gc)
+    ref = oracle.decode_attention(q, want_scores=True, **cc)
+    assert np.abs(to_np(out) - ref["out"]).max() <= OUT_TOL
+    check_decode_bound(to_np(out), to_np(scores), ref["scores"], _vals(cc), qjl=fmt == "qjl",
+                       v_scales=cc["v_scales"] if fmt == "qjl" else None)
     assert kvq.kvq_device_error() == 0
 
 

@@ -3,7 +3,8 @@ outputs are sampled and re-done one by one by the oracle (from the same fp16/fp3
 inputs, copied back to the host).
 
   * throughput sweep: 1e9 elements at D = 128, 1024, 8192, fp32 and fp16;
-  * the 7B-shaped cache: all 32 layers x {K, V} quantized in one launch, decode sampled;
+  * the 7B-shaped cache: all 32 layers x {K, V} quantized in one launch, decode sampled
+    (outputs within 2e-3 and within the arithmetic bound of tests/_helpers.py);
   * the key-sketch workload: estimator scores of one query per head over 32768 keys.
 """
 import numpy as np
@@ -12,7 +13,7 @@ import torch
 
 import oracle
 from kv_cache_quantization_absmax_b200 import inputs
-from tests._helpers import score_tolerance, to_np
+from tests._helpers import check_decode_unit, decode_chain, score_tolerance, sm_count, softmax_scale, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -51,11 +52,12 @@ def test_llama7b_cache_full_sampled(kvq):
     cache = inputs.lognormal_cache_device(3, (L, 2, B, H, T, 128), n_sigma_dims=(0, 1, 3, 5), device="cuda")
     q = inputs.gaussian_queries_device(30, (L, B, H, 128), "cuda")
     codes, scales = kvq.kvq_quantize_int8(cache)          # one launch over 134M rows
-    outs = []
+    outs, scs = [], []
     for l in (0, 17, 31):
-        out, _ = kvq.kvq_decode_attention(q[l], k_codes=codes[l, 0], k_scales=scales[l, 0],
-                                          v_codes=codes[l, 1], v_scales=scales[l, 1])
+        out, sc = kvq.kvq_decode_attention(q[l], k_codes=codes[l, 0], k_scales=scales[l, 0],
+                                           v_codes=codes[l, 1], v_scales=scales[l, 1], want_scores=True)
         outs.append(to_np(out))
+        scs.append(to_np(sc))
     torch.cuda.synchronize()
     rng = np.random.default_rng(7)
     flat = cache.view(-1, 128)
@@ -70,8 +72,11 @@ def test_llama7b_cache_full_sampled(kvq):
         vc, vs = oracle.quantize_int8(to_np(cache[l, 1, b, h]))
         ref = oracle.decode_attention(to_np(q[l, b, h])[None, None], k_codes=kc[None, None],
                                       k_scales=ks[None, None], v_codes=vc[None, None],
-                                      v_scales=vs[None, None])
+                                      v_scales=vs[None, None], want_scores=True)
         assert np.abs(outs[i][b, h] - ref["out"][0, 0]).max() <= 2e-3
+        n_chain, n_rescale = decode_chain(B, H, T, H, sm_count(), qjl=False)
+        check_decode_unit(outs[i][b, h][None], scs[i][b, h][None], ref["scores"][0],
+                          oracle.dequantize_int8(vc, vs), softmax_scale(), n_chain, n_rescale)
 
 
 def test_key_sketch_scores_full_size(kvq):

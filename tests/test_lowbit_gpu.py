@@ -1,12 +1,15 @@
 """GPU parity of channel-wise INT8 and group-wise INT4 quantize / dequantize against the
-CPU oracle: codes, packed nibbles, scales, zero points and dequantized values bit-exact."""
+CPU oracle: codes, packed nibbles, scales, zero points and dequantized values bit-exact.
+Decode over INT4 values: outputs within 2e-3 max-abs of the oracle and within the
+arithmetic bound (tests/_helpers.py, check_decode_bound), on the INT4 reconstructions."""
 import numpy as np
 import pytest
 import torch
 
 import oracle
 from kv_cache_quantization_absmax_b200 import inputs
-from tests._helpers import to_np
+from tests._helpers import (check_decode_bound, check_decode_unit, decode_chain, sm_count, softmax_scale,
+                            to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -81,6 +84,25 @@ def test_channelwise_int8_bit_exact(kvq, dtype, nb, rows, d):
 OUT_TOL = 2e-3
 
 
+def _vals4(vp, vs4, vz4, g):
+    """The INT4 reconstructions [..., T, D] of packed values [..., T, D/2]."""
+    lead = vp.shape[:-1]
+    return oracle.dequantize_int4_group(vp.reshape(-1, 64), vs4.reshape(-1, 128 // g),
+                                        vz4.reshape(-1, 128 // g), g).reshape(lead + (128,))
+
+
+def _abs4(vp, vs4, vz4, g):
+    """|c s| + |z| per element [..., T, D]: the two parts the kernel sums separately."""
+    lead = vp.shape[:-1]
+    p = vp.reshape(-1, 64)
+    c = np.empty((p.shape[0], 128), np.float64)
+    c[:, 0::2] = p & 15
+    c[:, 1::2] = p >> 4
+    s = np.repeat(vs4.reshape(-1, 128 // g).astype(np.float64), g, axis=1)
+    z = np.repeat(vz4.reshape(-1, 128 // g).astype(np.float64), g, axis=1)
+    return (np.abs(c * s) + np.abs(z)).reshape(lead + (128,))
+
+
 @pytest.mark.parametrize("B,Hq,Hkv,T,g", [(1, 4, 4, 5, 32), (2, 8, 2, 33, 64), (1, 8, 1, 1000, 128),
                                           (2, 16, 4, 4097, 32), (16, 16, 8, 3, 32), (1, 8, 8, 1501, 32),
                                           (4, 8, 8, 100, 64)])
@@ -101,6 +123,8 @@ def test_decode_int4_values(kvq, B, Hq, Hkv, T, g):
     xh = kc.astype(np.float64) * ks.astype(np.float64)[..., None]
     terms = np.abs(np.repeat(xh, Hq // Hkv, axis=1) * q.astype(np.float64)[:, :, None, :]).sum(-1)
     assert np.all(np.abs(to_np(scores).astype(np.float64) - ref["scores"]) <= 2 * 128 * 2.0 ** -24 * terms + 1e-30)
+    check_decode_bound(to_np(out), to_np(scores), ref["scores"], _vals4(vp, vs4, vz4, g), qjl=False,
+                       vabs=_abs4(vp, vs4, vz4, g))
     assert kvq.kvq_device_error() == 0
 
 
@@ -112,17 +136,21 @@ def test_decode_int4_values_7b_layer_sampled(kvq):
     q = inputs.gaussian_queries_device(31, (B, H, 128), "cuda")
     kc, ks = kvq.kvq_quantize_int8(kv[0])
     vp, vs4, vz4 = kvq.kvq_quantize_int4(kv[1], 32)
-    out, _ = kvq.kvq_decode_attention_int4v(q, k_codes=kc, k_scales=ks, v_packed=vp, v_scales4=vs4,
-                                            v_zeros4=vz4, v_group=32)
-    out = to_np(out)
+    out, scores = kvq.kvq_decode_attention_int4v(q, k_codes=kc, k_scales=ks, v_packed=vp, v_scales4=vs4,
+                                                 v_zeros4=vz4, v_group=32, want_scores=True)
+    out, scores = to_np(out), to_np(scores)
+    n_chain, n_rescale = decode_chain(B, H, T, H, sm_count(), qjl=False)
     rng = np.random.default_rng(8)
     for b, h in zip(rng.integers(0, B, 6), rng.integers(0, H, 6)):
         kc_r, ks_r = oracle.quantize_int8(to_np(kv[0, b, h]))
         vp_r, vs_r, vz_r = oracle.quantize_int4_group(to_np(kv[1, b, h]), 32)
         ref = oracle.decode_attention(to_np(q[b, h])[None, None], k_codes=kc_r[None, None],
                                       k_scales=ks_r[None, None],
-                                      v4=(vp_r[None, None], vs_r[None, None], vz_r[None, None], 32))
+                                      v4=(vp_r[None, None], vs_r[None, None], vz_r[None, None], 32),
+                                      want_scores=True)
         assert np.abs(out[b, h] - ref["out"][0, 0]).max() <= OUT_TOL
+        check_decode_unit(out[b, h][None], scores[b, h][None], ref["scores"][0], _vals4(vp_r, vs_r, vz_r, 32),
+                          softmax_scale(), n_chain, n_rescale, vabs=_abs4(vp_r, vs_r, vz_r, 32))
 
 
 def test_decode_int4_values_unaligned_group_params(kvq):
@@ -134,7 +162,8 @@ def test_decode_int4_values_unaligned_group_params(kvq):
     vp, vs4, vz4 = oracle.quantize_int4_group(v.reshape(-1, 128), g)
     shp = (B, Hkv, T)
     ref = oracle.decode_attention(q, k_codes=kc.reshape(shp + (128,)), k_scales=ks.reshape(shp),
-                                  v4=(vp.reshape(shp + (64,)), vs4.reshape(shp + (4,)), vz4.reshape(shp + (4,)), g))
+                                  v4=(vp.reshape(shp + (64,)), vs4.reshape(shp + (4,)), vz4.reshape(shp + (4,)), g),
+                                  want_scores=True)
     # copy the parameters into buffers offset by one float
     sbuf = torch.zeros(vs4.size + 1, dtype=torch.float32, device="cuda")
     zbuf = torch.zeros(vz4.size + 1, dtype=torch.float32, device="cuda")
@@ -142,6 +171,9 @@ def test_decode_int4_values_unaligned_group_params(kvq):
     zbuf[1:] = torch.from_numpy(vz4.reshape(-1)).cuda()
     qg, kcg, ksg, vpg = [torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in
                          (q, kc.reshape(shp + (128,)), ks.reshape(shp), vp.reshape(shp + (64,)))]
-    out, _ = kvq.kvq_decode_attention_int4v(qg, k_codes=kcg, k_scales=ksg, v_packed=vpg,
-                                            v_scales4=sbuf[1:], v_zeros4=zbuf[1:], v_group=g)
+    out, scores = kvq.kvq_decode_attention_int4v(qg, k_codes=kcg, k_scales=ksg, v_packed=vpg,
+                                                 v_scales4=sbuf[1:], v_zeros4=zbuf[1:], v_group=g, want_scores=True)
     assert np.abs(to_np(out) - ref["out"]).max() <= OUT_TOL
+    check_decode_bound(to_np(out), to_np(scores), ref["scores"],
+                       _vals4(vp.reshape(shp + (64,)), vs4, vz4, g), qjl=False,
+                       vabs=_abs4(vp.reshape(shp + (64,)), vs4, vz4, g))

@@ -362,6 +362,33 @@ def test_decode_qjl_brute_force(T):
     assert np.allclose(r["out"], out, rtol=0, atol=1e-5)
 
 
+@pytest.mark.parametrize("T,Hq,Hkv", [(1, 4, 2), (5, 4, 2), (33, 4, 1), (40, 6, 3)])
+def test_decode_from_scores_pins(T, Hq, Hkv):
+    """The fp64 definition after the scores (used as the reference of the arithmetic
+    bound): equals the page's GQA broadcast in fp64 brute force; T = 1 gives the value
+    row; equal scores give the mean of the values; it agrees with decode_attention's fp32
+    output on the same scores within the fp32 summation error."""
+    rng = np.random.default_rng(T + Hq)
+    D = 8
+    sc = rng.standard_normal((1, Hq, T)) * 30
+    vdeq = rng.standard_normal((1, Hkv, T, D))
+    sigma = float(np.float32(1.0) / np.sqrt(np.float32(D)))
+    out, p = oracle.decode_from_scores(sc, vdeq)
+    ref, _, pr = _brute_force(np.zeros((1, Hq, D)), sc, vdeq, Hq, sigma, scores_given=True)
+    assert np.allclose(out, ref, rtol=0, atol=1e-13) and np.allclose(p, pr, rtol=0, atol=1e-15)
+    if T == 1:
+        assert np.array_equal(out[0], np.repeat(vdeq[0, :, 0], Hq // Hkv, axis=0))
+    flat, _ = oracle.decode_from_scores(np.full((1, Hq, T), 2.5), vdeq)
+    assert np.allclose(flat[0], np.repeat(vdeq[0].mean(axis=1), Hq // Hkv, axis=0), rtol=0, atol=1e-14)
+    # against the C oracle's fp32 decode of an INT8 cache, on the C oracle's own scores
+    k, q, kc, ks, vc, vs = _tiny_cache(T, D=D, Hq=Hq, Hkv=Hkv, seed=T)
+    r = oracle.decode_attention(q, k_codes=kc, k_scales=ks, v_codes=vc, v_scales=vs, want_scores=True)
+    o64, p64 = oracle.decode_from_scores(r["scores"], _fl32_product(vc, vs))
+    vabs = np.repeat(np.abs(_fl32_product(vc, vs)), Hq // Hkv, axis=1)
+    tol = (T + 4) * 2.0 ** -23 * np.einsum("bht,bhtd->bhd", p64, vabs) + 1e-30
+    assert np.all(np.abs(r["out"] - o64) <= tol)
+
+
 def test_decode_equal_logits_give_mean_of_values():
     T = 40
     _, q, kc, ks, vc, vs = _tiny_cache(T)

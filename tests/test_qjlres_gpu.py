@@ -4,7 +4,8 @@ residual's sign sketch; the "TurboQuant" news page's two stages) against the CPU
 - Encode: INT4 codes, scales, zero points, the fp16 residual and its fp16 norm
   bit-exact; sign bits exact except where the oracle's |(S r)_i| < 1e-4 ||r|| (the GPU
   projects in fp32 on the tensor cores).
-- Decode (same encoded cache on both sides): outputs max-abs <= 2e-3; scores within
+- Decode (same encoded cache on both sides): outputs max-abs <= 2e-3 and within the
+  arithmetic bound (tests/_helpers.py, check_decode_bound); scores within
   32 * 2^-24 * sum_j |q_j| (|c_j s_g| + |z_g|) (fp32 factored INT4 dot against the
   oracle's fp64 sum of rounded reconstructions) + 1e-4 * c ||r|| ||S q||_2 (the
   residual estimator's natural scale, as for QJL keys).
@@ -17,7 +18,9 @@ import torch
 
 import oracle
 from kv_cache_quantization_absmax_b200 import inputs
-from tests._helpers import to_np, words_u32
+from tests import _oracle_pool
+from tests._helpers import (check_decode_bound, check_decode_unit, decode_chain, sm_count, softmax_scale, to_np,
+                            words_u32)
 
 pytestmark = pytest.mark.gpu
 
@@ -108,6 +111,9 @@ def test_decode_qjlres_parity(kvq, B, Hq, Hkv, T, g, m):
     err = np.abs(to_np(scores).astype(np.float64) - ref["scores"])
     tol = _score_tol(q, c, Hq)
     assert np.all(err <= tol), float((err / tol).max())
+    vc, vs = c["v_codes"], c["v_scales"]
+    vals = oracle.dequantize_int8(vc.reshape(-1, 128), vs.reshape(-1)).reshape(vc.shape)
+    check_decode_bound(to_np(out), to_np(scores), ref["scores"], vals, qjl=True)
     assert kvq.kvq_device_error() == 0
 
 
@@ -147,29 +153,58 @@ def test_decode_qjlres_beats_plain_qjl_on_scores(kvq):
     assert e_res < 0.5 * e_qjl, (e_res, e_qjl)
 
 
-def test_qjlres_gqa_long_context_sampled(kvq):
+def test_qjlres_gqa_long_context_all_units(kvq):
     """Long-context GQA cache (batch 4, 32 query / 8 KV heads, 131072 tokens): keys
     encoded as INT4 + residual sketch and values INT8-quantized on the GPU, one decode
-    step; one sampled KV unit (4 query heads) re-done by the oracle from the GPU's own
-    encoding (the encode is checked separately)."""
+    step.  Every one of the 32 KV units is re-done end to end by the oracle from the fp16
+    cache (in spawned worker processes): the INT4 stage and residual norms bit-exact, sign
+    bits exact outside the band, scores within their tolerance wherever both sides hold
+    the same bits, outputs within 2e-3 and within the arithmetic bound."""
     B, Hq, Hkv, T = 4, 32, 8, 131072
+    G = Hq // Hkv
     kv = inputs.lognormal_cache_device(5, (2, B, Hkv, T, 128), n_sigma_dims=(0, 2, 4), device="cuda")
     q = inputs.gaussian_queries_device(50, (B, Hq, 128), "cuda")
     S_np = inputs.sketch_matrix(256, 128)
     S = torch.from_numpy(S_np).cuda()
     e = kvq.kvq_qjl_residual_encode(kv[0], 32, S)
     vc, vs = kvq.kvq_quantize_int8(kv[1])
-    del kv
-    out, _ = kvq.kvq_decode_attention_qjlres(q, k_packed4=e["packed"], k_scales4=e["scales"], k_zeros4=e["zeros"],
-                                             k_group=32, k_words=e["words"], k_norms=e["rnorms"], sketch=S,
-                                             v_codes=vc, v_scales=vs)
-    out = to_np(out)
+    out, scores = kvq.kvq_decode_attention_qjlres(q, k_packed4=e["packed"], k_scales4=e["scales"],
+                                                  k_zeros4=e["zeros"], k_group=32, k_words=e["words"],
+                                                  k_norms=e["rnorms"], sketch=S, v_codes=vc, v_scales=vs,
+                                                  want_scores=True)
+    out, scores = to_np(out), to_np(scores)
     assert kvq.kvq_device_error() == 0
-    b, u = 1, 6
-    c = dict(k4=(to_np(e["packed"][b:b + 1, u:u + 1]), to_np(e["scales"][b:b + 1, u:u + 1]),
-                 to_np(e["zeros"][b:b + 1, u:u + 1]), 32),
-             k_words=words_u32(e["words"][b:b + 1, u:u + 1]), k_norms=to_np(e["rnorms"][b:b + 1, u:u + 1]), S=S_np,
-             v_codes=to_np(vc[b:b + 1, u:u + 1]), v_scales=to_np(vs[b:b + 1, u:u + 1]))
-    qs = to_np(q[b:b + 1, u * 4:(u + 1) * 4])
-    ref = oracle.decode_attention(qs, **c)
-    assert np.abs(out[b, u * 4:(u + 1) * 4] - ref["out"][0]).max() <= OUT_TOL
+    q_np = to_np(q)
+    units = [(b, g) for b in range(B) for g in range(Hkv)]
+    jobs = [(to_np(kv[0, b, g]), to_np(kv[1, b, g]), q_np[b, g * G:(g + 1) * G], S_np, 32) for b, g in units]
+    del kv
+    refs = _oracle_pool.run_units(_oracle_pool.qjlres_unit, jobs)
+    n_chain, n_rescale = decode_chain(B, Hkv, T, Hq, sm_count(), qjl=True)
+    for (b, g), job, r in zip(units, jobs, refs):
+        assert np.array_equal(to_np(e["packed"][b, g]), r["packed"])
+        assert np.array_equal(to_np(e["scales"][b, g]).view(np.uint32), r["scales"].view(np.uint32))
+        assert np.array_equal(to_np(e["zeros"][b, g]).view(np.uint32), r["zeros"].view(np.uint32))
+        assert np.array_equal(to_np(e["rnorms"][b, g]).view(np.uint16), r["rnorms"].view(np.uint16))
+        assert np.array_equal(to_np(e["residual"][b, g]).view(np.uint16), r["r"].view(np.uint16))
+        assert np.array_equal(to_np(vc[b, g]), r["v_codes"])
+        assert np.array_equal(to_np(vs[b, g]).view(np.uint32), r["v_scales"].view(np.uint32))
+        gw = words_u32(e["words"][b, g])
+        same = np.all(gw == r["words"], axis=1)
+        if not np.all(same):
+            t_diff = np.flatnonzero(~same)
+            resid = r["r"][t_diff]
+            u = resid.astype(np.float64) @ S_np.astype(np.float64).T
+            n64 = np.linalg.norm(resid.astype(np.float64), axis=1)
+            band = np.abs(u) < 1e-4 * n64[:, None]
+            diff = gw[t_diff] ^ r["words"][t_diff]
+            bits = ((diff[:, :, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(len(t_diff), 256).astype(bool)
+            assert not np.any(bits & ~band)
+        hs = slice(g * G, (g + 1) * G)
+        c = dict(k4=(r["packed"][None, None], r["scales"].reshape(1, 1, T, 4), r["zeros"].reshape(1, 1, T, 4), 32),
+                 k_words=r["words"][None, None], k_norms=r["rnorms"][None, None], S=S_np)
+        tol = _score_tol(job[2][None], c, G)[0]
+        err = np.abs(scores[b, hs].astype(np.float64) - r["scores"])
+        assert np.all(err[:, same] <= tol[:, same])
+        assert np.abs(out[b, hs] - r["out"]).max() <= OUT_TOL
+        check_decode_unit(out[b, hs], scores[b, hs], r["scores"], oracle.dequantize_int8(r["v_codes"], r["v_scales"]),
+                          softmax_scale(), n_chain, n_rescale)

@@ -4,10 +4,11 @@ It serves callers that can neither allocate device memory nor lend a workspace (
 engine that has reserved all device memory through its own allocator, or a path where
 an allocation is not allowed).  The test calls it through the C ABI twice in a row --
 an INT8 GQA step, then a QJL GQA step, both sharing the one scratch array -- and
-checks each result against kvq_decode_attention with a caller-owned workspace, within
-the decode tolerance the other tests use (2e-3 max-abs).  It also checks that a request
-larger than the scratch is refused before anything is launched.  This file is collected
-last so that a failure here cannot hide the other tests.
+checks each result against kvq_decode_attention with a caller-owned workspace and
+against the oracle, within the decode tolerance the other tests use (2e-3 max-abs), and
+against the oracle within the arithmetic bound of tests/_helpers.py.  It also checks
+that a request larger than the scratch is refused before anything is launched.  This
+file is collected last so that a failure here cannot hide the other tests.
 """
 import ctypes
 
@@ -17,6 +18,7 @@ import torch
 
 import oracle
 from kv_cache_quantization_absmax_b200 import inputs
+from tests._helpers import check_decode_bound, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -36,8 +38,11 @@ def _int8_case(B=2, Hq=16, Hkv=4, T=3001):
     vc, vs = oracle.quantize_int8(v.reshape(-1, 128))
     shp = (B, Hkv, T)
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
-    return dict(q=t(q), k_codes=t(kc.reshape(shp + (128,))), k_scales=t(ks.reshape(shp)),
-                v_codes=t(vc.reshape(shp + (128,))), v_scales=t(vs.reshape(shp)))
+    ref = oracle.decode_attention(q, k_codes=kc.reshape(shp + (128,)), k_scales=ks.reshape(shp),
+                                  v_codes=vc.reshape(shp + (128,)), v_scales=vs.reshape(shp), want_scores=True)
+    ref.update(vals=oracle.dequantize_int8(vc, vs).reshape(shp + (128,)), qjl=False, vs=None)
+    return ref, dict(q=t(q), k_codes=t(kc.reshape(shp + (128,))), k_scales=t(ks.reshape(shp)),
+                     v_codes=t(vc.reshape(shp + (128,))), v_scales=t(vs.reshape(shp)))
 
 
 def _qjl_case(B=1, Hq=32, Hkv=8, T=5000):
@@ -48,18 +53,29 @@ def _qjl_case(B=1, Hq=32, Hkv=8, T=5000):
     vc, vs = oracle.quantize_int8(v.reshape(-1, 128))
     shp = (B, Hkv, T)
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
-    return dict(q=t(q), k_words=t(w.view(np.int32).reshape(shp + (8,))), k_norms=t(n.reshape(shp)),
-                sketch=t(S), v_codes=t(vc.reshape(shp + (128,))), v_scales=t(vs.reshape(shp)))
+    ref = oracle.decode_attention(q, k_words=w.reshape(shp + (8,)), k_norms=n.reshape(shp), S=S,
+                                  v_codes=vc.reshape(shp + (128,)), v_scales=vs.reshape(shp), want_scores=True)
+    ref.update(vals=oracle.dequantize_int8(vc, vs).reshape(shp + (128,)), qjl=True, vs=vs.reshape(shp))
+    return ref, dict(q=t(q), k_words=t(w.view(np.int32).reshape(shp + (8,))), k_norms=t(n.reshape(shp)),
+                     sketch=t(S), v_codes=t(vc.reshape(shp + (128,))), v_scales=t(vs.reshape(shp)))
 
 
 def _noalloc(kvq, case):
     q = case["q"]
     out = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
     rest = {k: v for k, v in case.items() if k != "q"}
-    a = kvq.make_decode_args(q, out=out, **rest)
+    T = rest["v_codes"].shape[2]
+    scores = torch.full((q.shape[0], q.shape[1], T), float("nan"), dtype=torch.float32, device="cuda")
+    a = kvq.make_decode_args(q, out=out, scores_out=scores, **rest)
     st = kvq.lib.kvq_decode_attention_noalloc(ctypes.byref(a), None)
     assert st == kvq.KVQ_OK, kvq.lib.kvq_status_string(st)
-    return out
+    return out, scores
+
+
+def _check_oracle(got, ref):
+    out, scores = to_np(got[0]), to_np(got[1])
+    assert np.abs(out - ref["out"]).max() <= TOL
+    check_decode_bound(out, scores, ref["scores"], ref["vals"], qjl=ref["qjl"], v_scales=ref["vs"])
 
 
 def _with_workspace(kvq, case):
@@ -69,18 +85,21 @@ def _with_workspace(kvq, case):
 
 
 def test_noalloc_matches_workspace_entry_point_two_calls(kvq):
-    c1, c2 = _int8_case(), _qjl_case()
+    (o1, c1), (o2, c2) = _int8_case(), _qjl_case()
     ref1, ref2 = _with_workspace(kvq, c1), _with_workspace(kvq, c2)
     got1 = _noalloc(kvq, c1)            # first call on this device sets the scratch up
     got2 = _noalloc(kvq, c2)            # second call reuses the same scratch
     torch.cuda.synchronize()
     assert kvq.kvq_device_error() == 0
-    assert torch.isfinite(got1).all() and torch.isfinite(got2).all()
-    assert (got1 - ref1).abs().max().item() <= TOL
-    assert (got2 - ref2).abs().max().item() <= TOL
+    assert torch.isfinite(got1[0]).all() and torch.isfinite(got2[0]).all()
+    assert (got1[0] - ref1).abs().max().item() <= TOL
+    assert (got2[0] - ref2).abs().max().item() <= TOL
+    _check_oracle(got1, o1)
+    _check_oracle(got2, o2)
     got1b = _noalloc(kvq, c1)           # and once more, after the other case used it
     torch.cuda.synchronize()
-    assert (got1b - ref1).abs().max().item() <= TOL
+    assert (got1b[0] - ref1).abs().max().item() <= TOL
+    _check_oracle(got1b, o1)
 
 
 def test_noalloc_refuses_requests_larger_than_its_scratch(kvq):
