@@ -55,7 +55,7 @@ typedef enum { KVQ_F32 = 0, KVQ_F16 = 1 } kvq_dtype;
 
 typedef enum { KVQ_KEYS_INT8 = 0, KVQ_KEYS_QJL = 1 } kvq_key_format;
 
-#define KVQ_ABI_VERSION 1
+#define KVQ_ABI_VERSION 2
 
 int kvq_abi_version(void);
 const char* kvq_status_string(kvq_status s);
@@ -158,6 +158,9 @@ kvq_status kvq_qjl_query_sketch(const uint16_t* q_f16, int64_t n_q, int32_t d,
  * weights p_t * sv_t relative to the block's largest p and sv become 24-bit fixed-point
  * integers that multiply the INT8 codes exactly in int32 (error at most 2^-25 of the
  * block's largest sv per token); otherwise in fp32 on the CUDA cores.
+ * flags (KVQ_DECODE_*): KVQ_DECODE_CUDA_CORES keeps the whole step on the CUDA cores
+ * (QJL keys: the weighted sum in fp32 FMAs even where the tensor-core value pass
+ * applies); 0 lets the library choose; other bits: KVQ_ERR_INVALID_ARG.
  * workspace: caller-owned device memory of at least kvq_decode_workspace_bytes(a)
  * bytes, 256-byte aligned (KVQ_ERR_WORKSPACE otherwise).  It holds per-split partial
  * softmax states and the query sketches; its contents on entry do not matter.
@@ -187,7 +190,10 @@ typedef struct kvq_decode_args {
     float* scores_out;
     void* workspace;
     size_t workspace_bytes;
+    uint32_t flags;                /* KVQ_DECODE_* */
 } kvq_decode_args;
+
+#define KVQ_DECODE_CUDA_CORES 1u   /* no tensor-core value pass */
 
 kvq_status kvq_decode_attention(const kvq_decode_args* a, kvq_stream_t stream);
 

@@ -79,6 +79,7 @@ struct DecodeParams {
     int scales_bulk;        // INT8: scales 16-byte aligned per stage -> bulk-copied too
     int qjl_bulk;           // QJL: value rows 16-byte aligned -> each warp's next 32 value
                             // rows come by one bulk copy
+    int cuda_cores;         // the caller asked for no tensor-core value pass
 };
 
 // The unit segments of CTA `cta`'s range: unit u, tokens [t0, t1) of that unit, slot j.
@@ -1844,7 +1845,7 @@ cudaError_t run_qjl_pf(const DecodeParams& p, int ctas, cudaStream_t st) {
 bool qjl_tc_applies(const DecodeParams& p) {
     const auto al16 = [](const void* x) { return reinterpret_cast<uintptr_t>(x) % 16 == 0; };
     const int64_t units = p.T > 0 ? p.total / p.T : 0;
-    return p.knew == nullptr && p.want_out && p.k4p == nullptr && p.m <= 256 && p.m % 32 == 0 &&
+    return !p.cuda_cores && p.knew == nullptr && p.want_out && p.k4p == nullptr && p.m <= 256 && p.m % 32 == 0 &&
            p.T % 8 == 0 && p.cap % 8 == 0 && al16(p.kw) && al16(p.kn) && al16(p.vs) && al16(p.vc) &&
            units * p.cap <= (int64_t)INT32_MAX;
 }
@@ -2008,6 +2009,7 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
     p.scale_log2 = decode_scale_log2(a);
     p.qjl_c = qjl ? (float)(1.2533141373155002512 / (double)a->sketch_dim) : 0.0f;  // sqrt(pi/2)/m
     p.want_out = a->out != nullptr;
+    p.cuda_cores = (a->flags & KVQ_DECODE_CUDA_CORES) != 0u;
     if (k4 != nullptr) {
         p.k4p = k4->packed;
         p.k4s = k4->scales;

@@ -18,6 +18,8 @@ from . import build as _build
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CUDA, KVQ_ERR_WORKSPACE, KVQ_ERR_DEVICE = range(6)
 KVQ_F32, KVQ_F16 = 0, 1
 KVQ_KEYS_INT8, KVQ_KEYS_QJL = 0, 1
+KVQ_DECODE_CUDA_CORES = 1
+ABI_VERSION = 2
 
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -32,7 +34,7 @@ class DecodeArgs(ctypes.Structure):
         ("q_f16", _P), ("k_codes", _P), ("k_scales", _P), ("k_words", _P), ("k_norms_f16", _P),
         ("sketch_f16", _P), ("sketch_dim", _I32), ("sm_scale", ctypes.c_float),
         ("v_codes", _P), ("v_scales", _P), ("out", _P), ("scores_out", _P),
-        ("workspace", _P), ("workspace_bytes", ctypes.c_size_t),
+        ("workspace", _P), ("workspace_bytes", ctypes.c_size_t), ("flags", ctypes.c_uint32),
     ]
 
 
@@ -122,8 +124,8 @@ def _load():
     for f in ("kvq_quantize_int8", "kvq_dequantize_int8", "kvq_int8_scores", "kvq_qjl_encode",
               "kvq_qjl_query_sketch", "kvq_decode_attention", "kvq_device_error"):
         getattr(so, f).restype = ctypes.c_int
-    if so.kvq_abi_version() != 1:
-        raise RuntimeError(f"libkvq ABI version {so.kvq_abi_version()} != 1")
+    if so.kvq_abi_version() != ABI_VERSION:
+        raise RuntimeError(f"libkvq ABI version {so.kvq_abi_version()} != {ABI_VERSION}")
     return so
 
 
@@ -241,7 +243,7 @@ def kvq_qjl_query_sketch(q, sketch, out=None, stream=None):
 
 def make_decode_args(q, *, k_codes=None, k_scales=None, k_words=None, k_norms=None, sketch=None,
                      v_codes=None, v_scales=None, out=None, scores_out=None, sm_scale=0.0,
-                     workspace=None):
+                     workspace=None, flags=0):
     """Fill a ``kvq_decode_args`` from tensors (q [B, Hq, D] fp16; cache [B, Hkv, T, ...])."""
     B, Hq, D = q.shape
     a = DecodeArgs()
@@ -261,6 +263,7 @@ def make_decode_args(q, *, k_codes=None, k_scales=None, k_words=None, k_norms=No
     a.out = out.data_ptr() if out is not None else None
     a.scores_out = scores_out.data_ptr() if scores_out is not None else None
     a.sm_scale = float(sm_scale)
+    a.flags = int(flags)
     if workspace is not None:
         a.workspace, a.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     return a
@@ -272,8 +275,9 @@ def kvq_decode_workspace_bytes(args: DecodeArgs) -> int:
 
 def kvq_decode_attention(q, *, k_codes=None, k_scales=None, k_words=None, k_norms=None, sketch=None,
                          v_codes=None, v_scales=None, want_out=True, want_scores=False,
-                         sm_scale=0.0, workspace=None, out=None, scores_out=None, stream=None):
-    """One decode step; returns (out [B, Hq, D] fp32 or None, scores [B, Hq, T] or None)."""
+                         sm_scale=0.0, workspace=None, out=None, scores_out=None, stream=None, flags=0):
+    """One decode step; returns (out [B, Hq, D] fp32 or None, scores [B, Hq, T] or None).
+    flags: KVQ_DECODE_CUDA_CORES keeps the weighted value sum on the CUDA cores."""
     _need_cuda(q, k_codes, k_scales, k_words, k_norms, sketch, v_codes, v_scales)
     B, Hq, D = q.shape
     ref = k_words if k_words is not None else k_codes
@@ -285,7 +289,7 @@ def kvq_decode_attention(q, *, k_codes=None, k_scales=None, k_words=None, k_norm
     a = make_decode_args(q, k_codes=k_codes, k_scales=k_scales, k_words=k_words, k_norms=k_norms,
                          sketch=sketch, v_codes=v_codes if want_out else None,
                          v_scales=v_scales if want_out else None, out=out if want_out else None,
-                         scores_out=scores_out if want_scores else None, sm_scale=sm_scale)
+                         scores_out=scores_out if want_scores else None, sm_scale=sm_scale, flags=flags)
     need = kvq_decode_workspace_bytes(a)
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)

@@ -18,14 +18,29 @@ from . import build as _build
 F32, F16 = 0, 1
 KEYS_INT8, KEYS_QJL, KEYS_QJLRES = 0, 1, 2
 
-_lib = None
+_libs = {}
+_all_cores = False
+
+
+def use_all_cores(on: bool = True) -> None:
+    """Run the calls that follow on the all-cores build of the same C source (OpenMP over
+    rows, keys or (batch, head) units; every result identical), or, with on=False, on the
+    single-threaded build (the default)."""
+    global _all_cores
+    _all_cores = bool(on)
+
+
+def threads() -> int:
+    """Threads the current build runs its outer loops on (1 for the single-threaded one)."""
+    return int(_load().ora_max_threads())
 
 
 def _load():
-    global _lib
-    if _lib is None:
-        path = _build.build()
+    key = _all_cores
+    if key not in _libs:
+        path = _build.build(all_cores=key)
         lib = ctypes.CDLL(path)
+        lib.ora_max_threads.restype = ctypes.c_int
         P = ctypes.c_void_p
         I64 = ctypes.c_int64
         I32 = ctypes.c_int
@@ -57,8 +72,8 @@ def _load():
                   "ora_qjl_encode", "ora_qjl_query_sketch", "ora_qjl_scores",
                   "ora_decode_attention"):
             getattr(lib, f).restype = ctypes.c_int
-        _lib = lib
-    return _lib
+        _libs[key] = lib
+    return _libs[key]
 
 
 def _ptr(a):

@@ -52,6 +52,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORA_F32 0
 #define ORA_F16 1
@@ -63,6 +66,18 @@
  * IEEE-754 binary16 <-> binary64, written from the format's definition
  * (1 sign bit, 5 exponent bits with bias 15, 10 fraction bits).
  * ------------------------------------------------------------------------------- */
+/* The all-cores build (-fopenmp) runs the outer loops over rows, keys or (batch, head)
+ * units in parallel; every row, key or unit is computed by one thread exactly as in the
+ * plain build, so the results are identical.  Threads the all-cores build uses (1 in
+ * the plain build). */
+int ora_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
 double ora_half_to_double(uint16_t h) {
     int sign = (h >> 15) & 1;
     int e = (h >> 10) & 0x1f;
@@ -110,6 +125,7 @@ static float load_elem(const void* x, int dtype, int64_t i) {
 int ora_quantize_int8(const void* x, int dtype, int64_t n_rows, int64_t d,
                       int8_t* codes, float* scales) {
     if (n_rows < 0 || d <= 0) return 1;
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < n_rows; ++r) {
         float a = 0.0f;
         for (int64_t j = 0; j < d; ++j) {
@@ -138,6 +154,7 @@ int ora_quantize_int8(const void* x, int dtype, int64_t n_rows, int64_t d,
 int ora_dequantize_int8(const int8_t* codes, const float* scales, int64_t n_rows,
                         int64_t d, void* out, int out_dtype) {
     if (n_rows < 0 || d <= 0) return 1;
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < n_rows; ++r) {
         for (int64_t j = 0; j < d; ++j) {
             float v = (float)codes[r * d + j] * scales[r];
@@ -160,6 +177,7 @@ int ora_dequantize_int8(const int8_t* codes, const float* scales, int64_t n_rows
 int ora_quantize_int8_channelwise(const void* x, int dtype, int64_t n_blocks, int64_t rows,
                                   int64_t d, int8_t* codes, float* scales) {
     if (n_blocks < 0 || rows <= 0 || d <= 0) return 1;
+#pragma omp parallel for collapse(2) schedule(static)
     for (int64_t b = 0; b < n_blocks; ++b) {
         for (int64_t j = 0; j < d; ++j) {
             float a = 0.0f;
@@ -189,6 +207,7 @@ int ora_quantize_int8_channelwise(const void* x, int dtype, int64_t n_blocks, in
 int ora_dequantize_int8_channelwise(const int8_t* codes, const float* scales, int64_t n_blocks,
                                     int64_t rows, int64_t d, void* out, int out_dtype) {
     if (n_blocks < 0 || rows <= 0 || d <= 0) return 1;
+#pragma omp parallel for collapse(2) schedule(static)
     for (int64_t b = 0; b < n_blocks; ++b)
         for (int64_t r = 0; r < rows; ++r)
             for (int64_t j = 0; j < d; ++j) {
@@ -211,6 +230,7 @@ int ora_quantize_int4_group(const void* x, int dtype, int64_t n_rows, int64_t d,
                             uint8_t* packed, float* scales, float* zeros) {
     if (n_rows < 0 || d <= 0 || g <= 0 || (d % g) != 0 || (g % 2) != 0) return 1;
     int64_t ng = d / g;
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < n_rows; ++r) {
         for (int64_t k = 0; k < ng; ++k) {
             int64_t o = r * d + k * g;
@@ -255,6 +275,7 @@ static float int4_value(const uint8_t* packed, const float* scales, const float*
 int ora_dequantize_int4_group(const uint8_t* packed, const float* scales, const float* zeros,
                               int64_t n_rows, int64_t d, int g, void* out, int out_dtype) {
     if (n_rows < 0 || d <= 0 || g <= 0 || (d % g) != 0 || (g % 2) != 0) return 1;
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < n_rows; ++r)
         for (int64_t j = 0; j < d; ++j) {
             float v = int4_value(packed, scales, zeros, r, d, g, j);
@@ -283,6 +304,7 @@ int ora_int8_scores(const void* q, int q_dtype, const int8_t* codes, const float
     float* qf = (float*)malloc(sizeof(float) * (size_t)d);
     if (!qf) return 2;
     for (int64_t j = 0; j < d; ++j) qf[j] = load_elem(q, q_dtype, j);
+#pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < n_rows; ++r)
         scores[r] = int8_row_score(qf, codes + r * d, scales[r], d);
     free(qf);
@@ -300,25 +322,34 @@ int ora_qjl_encode(const uint16_t* keys_f16, int64_t n_keys, int d, const double
                    int m, uint32_t* words, uint16_t* norms_f16, double* u_out) {
     if (n_keys < 0 || d <= 0 || m <= 0 || (m % 32) != 0) return 1;
     int nw = m / 32;
-    double* k = (double*)malloc(sizeof(double) * (size_t)d);
-    if (!k) return 2;
-    for (int64_t n = 0; n < n_keys; ++n) {
-        double ss = 0.0;
-        for (int j = 0; j < d; ++j) {
-            k[j] = ora_half_to_double(keys_f16[n * d + j]);
-            ss += k[j] * k[j];
+    int fail = 0;
+#pragma omp parallel
+    {
+        double* k = (double*)malloc(sizeof(double) * (size_t)d);   /* one per thread */
+        if (!k) {
+#pragma omp atomic write
+            fail = 1;
         }
-        for (int w = 0; w < nw; ++w) words[n * nw + w] = 0u;
-        for (int i = 0; i < m; ++i) {
-            double u = 0.0;
-            for (int j = 0; j < d; ++j) u += S[(int64_t)i * d + j] * k[j];
-            if (u_out) u_out[n * m + i] = u;
-            if (u >= 0.0) words[n * nw + i / 32] |= (1u << (i % 32));
+#pragma omp for schedule(static)
+        for (int64_t n = 0; n < n_keys; ++n) {
+            if (!k) continue;
+            double ss = 0.0;
+            for (int j = 0; j < d; ++j) {
+                k[j] = ora_half_to_double(keys_f16[n * d + j]);
+                ss += k[j] * k[j];
+            }
+            for (int w = 0; w < nw; ++w) words[n * nw + w] = 0u;
+            for (int i = 0; i < m; ++i) {
+                double u = 0.0;
+                for (int j = 0; j < d; ++j) u += S[(int64_t)i * d + j] * k[j];
+                if (u_out) u_out[n * m + i] = u;
+                if (u >= 0.0) words[n * nw + i / 32] |= (1u << (i % 32));
+            }
+            norms_f16[n] = ora_double_to_half(sqrt(ss));
         }
-        norms_f16[n] = ora_double_to_half(sqrt(ss));
+        free(k);
     }
-    free(k);
-    return 0;
+    return fail ? 2 : 0;
 }
 
 /* [QJL] the query side: the plain (unquantized) JL transform v = S q, fp64, returned in
@@ -454,17 +485,26 @@ int ora_decode_attention(int64_t B, int64_t Hq, int64_t Hkv, int64_t T, int D,
     int64_t G = Hq / Hkv;
     int nw = m / 32;
     float sigma = sm_scale != 0.0f ? sm_scale : 1.0f / sqrtf((float)D);
+    int fail = 0;
+#pragma omp parallel
+    {
+    /* scratch, one set per thread */
     float* qf = (float*)malloc(sizeof(float) * (size_t)D);
     float* score = (float*)malloc(sizeof(float) * (size_t)T);
     float* e = (float*)malloc(sizeof(float) * (size_t)T);
     double* v64 = (double*)malloc(sizeof(double) * (size_t)(m > 0 ? m : 1));
     double* vst = (double*)malloc(sizeof(double) * (size_t)(m > 0 ? m : 1));
-    if (!qf || !score || !e || !v64 || !vst) {
-        free(qf); free(score); free(e); free(v64); free(vst);
-        return 2;
+    int ok = qf && score && e && v64 && vst;
+    if (!ok) {
+#pragma omp atomic write
+        fail = 2;
     }
-    for (int64_t b = 0; b < B; ++b) {
-        for (int64_t h = 0; h < Hq; ++h) {
+    /* one (batch, query head) pair per iteration */
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < B * Hq; ++bh) {
+        if (!ok) continue;
+        {
+            int64_t b = bh / Hq, h = bh % Hq;
             int64_t kvh = h / G;
             int64_t qo = (b * Hq + h) * D;
             int64_t base = (b * Hkv + kvh) * T;   /* first token row of this KV head */
@@ -519,5 +559,6 @@ int ora_decode_attention(int64_t B, int64_t Hq, int64_t Hkv, int64_t T, int D,
         }
     }
     free(qf); free(score); free(e); free(v64); free(vst);
-    return 0;
+    }
+    return fail;
 }

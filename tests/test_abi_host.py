@@ -28,7 +28,7 @@ def test_exports_every_declared_symbol(kvq):
             "kvq_decode_attention"} <= set(names)
     for n in names:
         assert hasattr(kvq.lib, n), n
-    assert kvq.lib.kvq_abi_version() == 1
+    assert kvq.lib.kvq_abi_version() == kvq.ABI_VERSION == 2
 
 
 def test_status_strings(kvq):
@@ -96,6 +96,8 @@ def test_decode_rejects_bad_arguments(kvq):
     assert call(_args(kvq, k_codes=A16 + 1)) == E
     assert call(_args(kvq, q_f16=None)) == E
     assert call(_args(kvq, sm_scale=-1.0)) == E
+    assert call(_args(kvq, flags=2)) == E                      # unknown flag bit
+    assert call(_args(kvq, flags=kvq.KVQ_DECODE_CUDA_CORES)) == kvq.KVQ_ERR_WORKSPACE
     qjl = dict(key_format=kvq.KVQ_KEYS_QJL, k_words=A16, k_norms_f16=A16, sketch_f16=A16)
     assert call(_args(kvq, sketch_dim=100, **qjl)) == E
     assert call(_args(kvq, sketch_dim=512, **qjl)) == U

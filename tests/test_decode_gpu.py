@@ -103,13 +103,13 @@ def _qjl_cache(seed, B, Hkv, T, Hq, m=256):
                                           (1, 32, 8, 2049, 256), (1, 4, 4, 700, 128), (1, 2, 1, 333, 32),
                                           (16, 32, 8, 3, 256), (4, 8, 4, 100, 256),
                                           (2, 16, 1, 1000, 256), (1, 12, 2, 801, 256), (1, 3, 1, 257, 64)])
-def test_decode_qjl_parity(kvq, B, Hq, Hkv, T, m):
+def test_decode_qjl_parity(kvq, B, Hq, Hkv, T, m, flags=0):
     q, S, w, n, vc, vs = _qjl_cache(100 + T, B, Hkv, T, Hq, m)
     ref = oracle.decode_attention(q, k_words=w, k_norms=n, S=S, v_codes=vc, v_scales=vs,
                                   want_scores=True)
     qg, Sg, wg, ng, vcg, vsg = _cuda(q, S, w.view(np.int32), n, vc, vs)
     out, scores = kvq.kvq_decode_attention(qg, k_words=wg, k_norms=ng, sketch=Sg, v_codes=vcg,
-                                           v_scales=vsg, want_scores=True)
+                                           v_scales=vsg, want_scores=True, flags=flags)
     out, scores = to_np(out), to_np(scores)
     assert np.abs(out - ref["out"]).max() <= OUT_TOL
     v64, _ = oracle.qjl_query_sketch(q.reshape(-1, 128), S)
@@ -132,6 +132,14 @@ def test_decode_qjl_parity(kvq, B, Hq, Hkv, T, m):
                                           (1, 8, 1, 1504, 256), (1, 16, 2, 2048, 256), (1, 32, 1, 4096, 256)])
 def test_decode_qjl_tc_parity(kvq, B, Hq, Hkv, T, m):
     test_decode_qjl_parity(kvq, B, Hq, Hkv, T, m)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T,m", [(2, 8, 2, 1504, 256), (1, 32, 8, 2048, 256), (16, 32, 8, 8, 256),
+                                          (1, 16, 2, 2048, 256), (1, 4, 4, 704, 128)])
+def test_decode_qjl_cuda_cores_flag_parity(kvq, B, Hq, Hkv, T, m):
+    """KVQ_DECODE_CUDA_CORES on shapes that would take the tensor-core value pass: the
+    weighted sum runs in fp32 on the CUDA cores, against the same oracle and bounds."""
+    test_decode_qjl_parity(kvq, B, Hq, Hkv, T, m, flags=kvq.KVQ_DECODE_CUDA_CORES)
 
 
 @pytest.mark.parametrize("key_format,T", [("int8", 4096), ("qjl", 4096), ("qjl", 1000)])
