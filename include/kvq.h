@@ -154,10 +154,11 @@ kvq_status kvq_qjl_query_sketch(const uint16_t* q_f16, int64_t n_q, int32_t d,
  * Precision: scores and the softmax in fp32 (exponentials by the hardware 2^x); out
  * within 2e-3 absolute of the fp64 value of the formula above.  With QJL keys, when T
  * is a multiple of 8, k_words, k_norms, v_codes and v_scales are 16-byte aligned and
- * the cache has fewer than 2^31 token rows, the weighted sum runs on the tensor cores: per block of 32 tokens and head, the
- * weights p_t * sv_t relative to the block's largest p and sv become 24-bit fixed-point
- * integers that multiply the INT8 codes exactly in int32 (error at most 2^-25 of the
- * block's largest sv per token); otherwise in fp32 on the CUDA cores.
+ * the cache has fewer than 2^31 token rows, the weighted sum runs on the tensor cores:
+ * per block of 32 tokens and head, the weights p_t * sv_t relative to the block's
+ * largest p become integers in units of 2^-E, smax 2^E in [2^23, 2^24) for the block's
+ * largest value scale smax, that multiply the INT8 codes exactly in int32 (error at most
+ * 2^-24 smax per token); otherwise in fp32 on the CUDA cores.
  * flags (KVQ_DECODE_*): KVQ_DECODE_CUDA_CORES keeps the whole step on the CUDA cores
  * (QJL keys: the weighted sum in fp32 FMAs even where the tensor-core value pass
  * applies); 0 lets the library choose; other bits: KVQ_ERR_INVALID_ARG.

@@ -1387,41 +1387,48 @@ decode_qjl_pf_kernel(const DecodeParams p) {
 
 // -----------------------------------------------------------------------------------
 // QJL keys, value pass on the tensor cores.  The range streams in chunks of 128 tokens
-// of one unit through a 4-stage ring: the value rows by a TMA tile with the 128-byte
-// swizzle (token rows of 128 INT8 codes, which the tensor core reads as the MN-major
-// operand A = V^T [128 dims x 128 tokens]), the sign words, norms and value scales by
-// bulk copies.  Warp roles (448 threads, one CTA per SM):
+// of one unit through two rings: a key ring (the chunk's sign words, fp16 norms and
+// value scales, by bulk copies) that the producer fills kTcLookahead chunks ahead of a
+// value ring (the chunk's 128 value rows by a TMA tile with the 128-byte swizzle, which
+// the tensor core reads as the MN-major operand A = V^T [128 dims x 128 tokens]).  The
+// scorers take each chunk's keys as soon as they land and release the key stage once
+// they hold its data in registers, so a chunk's weights are usually ready before its
+// value tile lands, and a value stage is held only for its load and its MMA.
+// Warp roles (one CTA per SM):
 //   warp 0       producer;
 //   warp 1       TMEM and the MMA thread: per chunk four tcgen05.mma kind::i8, slice k
 //                (tokens 32 k .. 32 k + 31) into its own 16-column int32 accumulator;
-//   warps 2..9   scorers in two groups of four that take alternate chunks, one token per
+//   warps 2..    scorers in groups of four that take chunks in turn, one token per
 //                thread: the estimator from the byte tables; per warp (32 tokens, one
 //                MMA slice) the max M of the log2-domain logits of each head and the max
 //                value scale smax; the weight w = 2^(s - M) * vscale as a 24-bit
-//                fixed-point integer W = round(w (2^24 - 1) / smax), split into three
-//                unsigned bytes that form rows 3 g + k of the operand B [16 x 128
-//                tokens] (K-major); the warp's sum of 2^(s - M) in fixed point by one
-//                integer warp reduction;
-//   warps 10..13 accumulators, one value dimension per thread: per slice, sum_t W_t c_t
+//                fixed-point integer W = round(w 2^E) with 2^E the power of two that puts
+//                smax 2^E in [2^23, 2^24), split into three unsigned bytes that form rows
+//                3 g + k of the operand B [16 x 128 tokens] (K-major); the warp's sum of
+//                2^(s - Mc) in fixed point by one integer warp reduction;
+//   last 4 warps accumulators, one value dimension per thread: per slice, sum_t W_t c_t
 //                = D2 2^16 + D1 2^8 + D0 (exact in int32: |c| <= 127, bytes <= 255, 32
-//                tokens), rescaled by smax / (2^24 - 1), merged over the slices by their
-//                maxima and into the running online-softmax state of each head.
+//                tokens), times the slice's factor, summed over the slices and merged into
+//                the running online-softmax state of each head.
 // The INT8 codes enter the product unconverted and every product and sum is exact; the
-// approximations are the weights' 24-bit fixed point (absolute error at most 2^-25 smax
-// per token), the sums' 2^-24 fixed point, and the fp32 merges.
+// approximations are the weights' fixed point (absolute error at most 2^-24 smax per
+// token), the sums' 2^-24 fixed point, and the fp32 merges.
 constexpr int kTcTok = 128;                 // tokens per chunk
-constexpr int kTcStages = 4;
-constexpr int kTcScorerWarps = 8;
+constexpr int kTcValueStages = 3;           // value ring: 16 KB tiles
+constexpr int kTcKeyStages = 5;             // key ring: words, norms and scales of a chunk
+constexpr int kTcLookahead = 3;             // key loads run this many chunks ahead of value loads
+static_assert(kTcLookahead + 2 <= kTcKeyStages, "the key ring holds the look-ahead and two chunks in scoring");
+constexpr int kTcScorerGroups = 3;          // groups of four scorer warps, chunk c to group c % 3
+constexpr int kTcScorerWarps = 4 * kTcScorerGroups;
 constexpr int kTcThreads = 32 * (2 + kTcScorerWarps + 4);
 constexpr int kTcVBytes = kTcTok * kD;      // value tile: 16 KB
-constexpr int kTcStageBytes = 21 * 1024;    // tile | words (<= 4 KB) | norms | scales
-constexpr int kTcWordsOff = kTcVBytes;
+constexpr int kTcWordsOff = 0;              // key stage: words (<= 4 KB) | norms | scales
 constexpr int kTcNormsOff = kTcWordsOff + kTcTok * 32;
 constexpr int kTcScalesOff = kTcNormsOff + kTcTok * 2;
-static_assert(kTcScalesOff + kTcTok * 4 <= kTcStageBytes, "stage layout");
+constexpr int kTcKeyBytes = kTcScalesOff + kTcTok * 4;
 constexpr int kTcBBytes = 2048;             // operand B: 16 rows x 128 bytes
-constexpr int kTcAcc = 4;                   // chunks in flight between scorers and accumulators
-constexpr uint32_t kTcTmemCols = kTcAcc * 4 * 16;
+constexpr int kTcAcc = 2 * kTcScorerGroups;  // chunks in flight between scorers and accumulators
+constexpr uint32_t kTcTmemCols = kTcAcc * 16 <= 32 ? 32 : (kTcAcc * 16 <= 64 ? 64 : (kTcAcc * 16 <= 128 ? 128 : 256));
 constexpr float kTcWmax = 16777215.0f;      // 2^24 - 1
 // instruction descriptor: int32 accumulator, A signed 8-bit MN-major, B unsigned 8-bit
 // K-major, N = 16, M = 128
@@ -1430,17 +1437,31 @@ constexpr uint32_t kTcIdesc = (2u << 4) | (1u << 7) | (0u << 10) | (1u << 15) | 
 
 enum : unsigned int { kErrTcProducer = 0x211, kErrTcMma = 0x212, kErrTcScore = 0x213, kErrTcAcc = 0x214 };
 
-struct TcSlice {              // per chunk and MMA slice, from a scorer warp to the accumulators
-    float M[4];               // max of the slice's log2-domain logits, per head
-    float L[4];               // sum of 2^(s - M), per head
-    float inv_scale;          // smax / (2^24 - 1)
+struct TcChunk {              // per chunk in flight, from the scorer group to the accumulators
+    float Mk[4][4];           // [slice][head] max of the slice's log2-domain logits (group scratch)
+    float Sk[4];              // [slice] max value scale of the slice (group scratch)
+    float Mc[4];              // [head] the chunk's max logit
+    float inv;                // 2^-E: the value of one unit of the weights' fixed point
     float pad[3];
+    float Lf[4][4];           // [slice][head] sum over the slice of 2^(s - Mc)
 };
 
+// Shared memory, from a 1024-byte aligned base: byte tables | value ring | operand B
+// buffers | key ring | per-chunk statistics | mbarriers.
+constexpr size_t kTcLutOff = 0;
+constexpr size_t kTcValueOff = kTcLutOff + 2 * 65536;
+constexpr size_t kTcBOff = kTcValueOff + (size_t)kTcValueStages * kTcVBytes;
+constexpr size_t kTcKeyOff = kTcBOff + (size_t)kTcAcc * kTcBBytes;
+constexpr size_t kTcSliceOff = kTcKeyOff + (size_t)kTcKeyStages * kTcKeyBytes;
+constexpr size_t kTcBarOff = kTcSliceOff + (size_t)kTcAcc * sizeof(TcChunk);
+constexpr int kTcBars = 2 * kTcKeyStages + 2 * kTcValueStages + 3 * kTcAcc + 1;
+static_assert(kTcValueOff % 1024 == 0 && kTcBOff % 1024 == 0, "swizzled operands need 1024-byte alignment");
+static_assert(kTcKeyBytes % 16 == 0 && kTcSliceOff % 16 == 0, "bulk copy destinations are 16-byte aligned");
+
 __host__ __device__ constexpr size_t tc_smem_bytes() {
-    return 1024 /* alignment */ + 2 * 65536 /* tables */ + (size_t)kTcStages * kTcStageBytes +
-           kTcAcc * kTcBBytes + kTcAcc * 4 * sizeof(TcSlice) + (2 * kTcStages + 3 * kTcAcc + 1) * 8;
+    return 1024 /* alignment */ + kTcBarOff + (size_t)kTcBars * 8;
 }
+static_assert(tc_smem_bytes() + 64 <= 232448, "shared memory of one CTA");
 
 template <int G>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -1452,20 +1473,24 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
     const uint32_t raw = dev::smem_u32(tc_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* bp = tc_raw + (base - raw);
-    float* lut = reinterpret_cast<float*>(bp);                         // 128 KB
-    const uint32_t lut_s = base;
-    const uint32_t stage_s = base + 2 * 65536;
-    uint8_t* stage_p = bp + 2 * 65536;
-    const uint32_t b_s = stage_s + kTcStages * kTcStageBytes;          // 1024-aligned
-    uint8_t* b_p = stage_p + kTcStages * kTcStageBytes;
-    TcSlice* slices = reinterpret_cast<TcSlice*>(b_p + kTcAcc * kTcBBytes);   // [kTcAcc][4]
-    const uint32_t bars = dev::smem_u32(slices + kTcAcc * 4);
-    auto full_bar = [&](int s) { return bars + 8u * s; };
-    auto empty_bar = [&](int s) { return bars + 8u * (kTcStages + s); };
-    auto bready_bar = [&](int a) { return bars + 8u * (2 * kTcStages + a); };
-    auto tfull_bar = [&](int a) { return bars + 8u * (2 * kTcStages + kTcAcc + a); };
-    auto tempty_bar = [&](int a) { return bars + 8u * (2 * kTcStages + 2 * kTcAcc + a); };
-    const uint32_t done_bar = bars + 8u * (2 * kTcStages + 3 * kTcAcc);
+    float* lut = reinterpret_cast<float*>(bp + kTcLutOff);               // 128 KB
+    const uint32_t lut_s = base + (uint32_t)kTcLutOff;
+    const uint32_t val_s = base + (uint32_t)kTcValueOff;
+    const uint32_t b_s = base + (uint32_t)kTcBOff;
+    uint8_t* b_p = bp + kTcBOff;
+    const uint32_t key_s = base + (uint32_t)kTcKeyOff;
+    const uint8_t* key_p = bp + kTcKeyOff;
+    TcChunk* chunks = reinterpret_cast<TcChunk*>(bp + kTcSliceOff);   // [kTcAcc]
+    const uint32_t bars = base + (uint32_t)kTcBarOff;
+    auto kfull_bar = [&](int s) { return bars + 8u * s; };
+    auto kempty_bar = [&](int s) { return bars + 8u * (kTcKeyStages + s); };
+    auto vfull_bar = [&](int s) { return bars + 8u * (2 * kTcKeyStages + s); };
+    auto vempty_bar = [&](int s) { return bars + 8u * (2 * kTcKeyStages + kTcValueStages + s); };
+    constexpr int kAccBar0 = 2 * kTcKeyStages + 2 * kTcValueStages;
+    auto bready_bar = [&](int a) { return bars + 8u * (kAccBar0 + a); };
+    auto tfull_bar = [&](int a) { return bars + 8u * (kAccBar0 + kTcAcc + a); };
+    auto tempty_bar = [&](int a) { return bars + 8u * (kAccBar0 + 2 * kTcAcc + a); };
+    const uint32_t done_bar = bars + 8u * (kAccBar0 + 3 * kTcAcc);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -1476,9 +1501,13 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
 
     if (threadIdx.x == 0) {
         abort_storage = 0;
-        for (int s = 0; s < kTcStages; ++s) {
-            dev::mbar_init(full_bar(s), 1);
-            dev::mbar_init(empty_bar(s), 1);
+        for (int s = 0; s < kTcKeyStages; ++s) {
+            dev::mbar_init(kfull_bar(s), 1);
+            dev::mbar_init(kempty_bar(s), 4);     // the four warps of the scorer group
+        }
+        for (int s = 0; s < kTcValueStages; ++s) {
+            dev::mbar_init(vfull_bar(s), 1);
+            dev::mbar_init(vempty_bar(s), 1);     // the MMA's commit
         }
         for (int a = 0; a < kTcAcc; ++a) {
             dev::mbar_init(bready_bar(a), 4);
@@ -1503,31 +1532,56 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
         // ---------------- producer ----------------
         if (lane == 0) {
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
-            int c = 0;
+            // chunk i's keys are issued at step i, its value tile at step i + kTcLookahead
+            int nk = 0, nv = 0;            // key / value loads issued
             bool ok = true;
-            for (int jj = 0; ok && jj < nseg; ++jj) {
-                const Segment sg = walk.seg(jj);
-                const int64_t row0 = sg.u * p.cap;
-                for (int64_t t = sg.t0; t < sg.t1; t += kTcTok, ++c) {
-                    const int s = c % kTcStages;
-                    const uint32_t ph = (uint32_t)(c / kTcStages) & 1u;
-                    if (!dev::mbar_wait(empty_bar(s), ph ^ 1u, abort_flag, &g_decode_error, kErrTcProducer)) {
+            int js = 0;                    // segment and token of the next key load
+            int64_t ts = nseg > 0 ? walk.seg(0).t0 : 0;
+            int jv = 0;                    // segment and token of the next value load
+            int64_t tv = ts;
+            auto next = [&](int& j, int64_t& t) {
+                t += kTcTok;
+                if (t >= walk.seg(j).t1 && ++j < nseg) t = walk.seg(j).t0;
+            };
+            while (ok && jv < nseg) {
+                if (js < nseg) {
+                    const Segment sg = walk.seg(js);
+                    const int s = nk % kTcKeyStages;
+                    const uint32_t ph = (uint32_t)(nk / kTcKeyStages) & 1u;
+                    if (!dev::mbar_wait(kempty_bar(s), ph ^ 1u, abort_flag, &g_decode_error, kErrTcProducer)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t n = (uint32_t)min((int64_t)kTcTok, sg.t1 - t);
-                    const int64_t r = row0 + t;
-                    const uint32_t dst = stage_s + (uint32_t)s * kTcStageBytes;
-                    dev::mbar_arrive_expect_tx(full_bar(s), (uint32_t)kTcVBytes + n * (uint32_t)nw * 4u + n * 2u + n * 4u);
-                    dev::tma_load_2d(dst, &vmap, full_bar(s), 0, (int)r);
-                    dev::bulk_g2s(dst + kTcWordsOff, p.kw + r * nw, n * (uint32_t)nw * 4u, full_bar(s));
-                    dev::bulk_g2s(dst + kTcNormsOff, p.kn + r, n * 2u, full_bar(s));
-                    dev::bulk_g2s(dst + kTcScalesOff, p.vs + r, n * 4u, full_bar(s));
+                    const uint32_t n = (uint32_t)min((int64_t)kTcTok, sg.t1 - ts);
+                    const int64_t r = sg.u * p.cap + ts;
+                    const uint32_t dst = key_s + (uint32_t)s * kTcKeyBytes;
+                    dev::mbar_arrive_expect_tx(kfull_bar(s), n * (uint32_t)nw * 4u + n * 2u + n * 4u);
+                    dev::bulk_g2s(dst + kTcWordsOff, p.kw + r * nw, n * (uint32_t)nw * 4u, kfull_bar(s));
+                    dev::bulk_g2s(dst + kTcNormsOff, p.kn + r, n * 2u, kfull_bar(s));
+                    dev::bulk_g2s(dst + kTcScalesOff, p.vs + r, n * 4u, kfull_bar(s));
+                    ++nk;
+                    next(js, ts);
+                }
+                if (nk > nv + kTcLookahead || js >= nseg) {
+                    const Segment sg = walk.seg(jv);
+                    const int s = nv % kTcValueStages;
+                    const uint32_t ph = (uint32_t)(nv / kTcValueStages) & 1u;
+                    if (!dev::mbar_wait(vempty_bar(s), ph ^ 1u, abort_flag, &g_decode_error, kErrTcProducer)) {
+                        ok = false;
+                        break;
+                    }
+                    dev::mbar_arrive_expect_tx(vfull_bar(s), (uint32_t)kTcVBytes);
+                    dev::tma_load_2d(val_s + (uint32_t)s * kTcVBytes, &vmap, vfull_bar(s), 0,
+                                     (int)(sg.u * p.cap + tv));
+                    ++nv;
+                    next(jv, tv);
                 }
             }
             // never leave the CTA with a copy in flight: wait for the last fill of each stage
-            for (int k = max(0, c - kTcStages); k < c; ++k)
-                dev::mbar_drain(full_bar(k % kTcStages), (uint32_t)(k / kTcStages) & 1u);
+            for (int k = max(0, nk - kTcKeyStages); k < nk; ++k)
+                dev::mbar_drain(kfull_bar(k % kTcKeyStages), (uint32_t)(k / kTcKeyStages) & 1u);
+            for (int k = max(0, nv - kTcValueStages); k < nv; ++k)
+                dev::mbar_drain(vfull_bar(k % kTcValueStages), (uint32_t)(k / kTcValueStages) & 1u);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -1537,39 +1591,41 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
             for (int jj = 0; ok && jj < nseg; ++jj) {
                 const Segment sg = walk.seg(jj);
                 for (int64_t t = sg.t0; t < sg.t1; t += kTcTok, ++c) {
-                    const int s = c % kTcStages;
-                    const uint32_t ph = (uint32_t)(c / kTcStages) & 1u;
+                    const int s = c % kTcValueStages;
+                    const uint32_t ph = (uint32_t)(c / kTcValueStages) & 1u;
                     const int a = c % kTcAcc;
                     const uint32_t aph = (uint32_t)(c / kTcAcc) & 1u;
-                    if (!dev::mbar_wait(full_bar(s), ph, abort_flag, &g_decode_error, kErrTcMma) ||
-                        !dev::mbar_wait(bready_bar(a), aph, abort_flag, &g_decode_error, kErrTcMma)) {
+                    if (!dev::mbar_wait(bready_bar(a), aph, abort_flag, &g_decode_error, kErrTcMma) ||
+                        !dev::mbar_wait(vfull_bar(s), ph, abort_flag, &g_decode_error, kErrTcMma)) {
                         ok = false;
                         break;
                     }
                     dev::tc_fence_after();
-                    const uint32_t va = stage_s + (uint32_t)s * kTcStageBytes;
+                    const uint32_t va = val_s + (uint32_t)s * kTcVBytes;
                     const uint32_t bb = b_s + (uint32_t)a * kTcBBytes;
                     const int nk = (int)((min((int64_t)kTcTok, sg.t1 - t) + 31) / 32);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
                         if (k < nk)
-                            dev::tc_mma_i8(tmem + (uint32_t)(a * 4 + k) * 16u,
-                                           dev::smem_desc_sw128(va + (uint32_t)k * 4096u),
-                                           dev::smem_desc_sw128(bb + (uint32_t)k * 32u), kTcIdesc, 0u);
+                            dev::tc_mma_i8(tmem + (uint32_t)a * 16u, dev::smem_desc_sw128(va + (uint32_t)k * 4096u),
+                                           dev::smem_desc_sw128(bb + (uint32_t)k * 32u), kTcIdesc, k > 0 ? 1u : 0u);
                     dev::tc_commit(tfull_bar(a));
-                    dev::tc_commit(empty_bar(s));
+                    dev::tc_commit(vempty_bar(s));
                 }
             }
             dev::tc_commit(done_bar);
             dev::mbar_drain(done_bar, 0);
         }
     } else if (warp < 2 + kTcScorerWarps) {
-        // ---------------- scorers: group gi takes the chunks c with c % 2 == gi ----------------
+        // ---------------- scorers: group gi takes the chunks c with c % kTcScorerGroups == gi ----------------
         const int gi = (warp - 2) >> 2;
         const int sw = (warp - 2) & 3;                  // MMA slice: tokens 32 sw .. 32 sw + 31
         const int st = sw * 32 + lane;                  // this thread's token of the chunk
         const LutLane lut_lane(lane);
         const int kb = st >> 4, kx = st & 15;          // its byte in a row of B
+        int boff[8];                                    // ... under the 128-byte swizzle of row r
+#pragma unroll
+        for (int r7 = 0; r7 < 8; ++r7) boff[r7] = ((kb ^ r7) << 4) + kx;
         int c = 0;
         bool ok = true;
         for (int jj = 0; jj < nseg; ++jj) {
@@ -1581,79 +1637,112 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
             // barriers, also after an abort (they then skip the work in between)
             asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcScorerWarps) : "memory");
             if (ok)
-                build_sign_tables<G>(lut, p.sketch_v + hb * p.m, p.m, p.m,
-                                     threadIdx.x - 64, 32 * kTcScorerWarps);
+                build_sign_tables<G>(lut, p.sketch_v + hb * p.m, p.m, p.m, threadIdx.x - 64, 32 * kTcScorerWarps);
             asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcScorerWarps) : "memory");
             for (int64_t t = sg.t0; t < sg.t1; t += kTcTok, ++c) {
-                if (!ok || (c & 1) != gi) continue;
-                const int s = c % kTcStages;
-                const uint32_t ph = (uint32_t)(c / kTcStages) & 1u;
+                if (c % kTcScorerGroups != gi) continue;
+                // every warp of the group passes the group barrier below on every chunk of
+                // the group, also after an abort (it then skips the work around it)
+                const int s = c % kTcKeyStages;
+                const uint32_t ph = (uint32_t)(c / kTcKeyStages) & 1u;
                 const int a = c % kTcAcc;
                 const uint32_t aph = (uint32_t)(c / kTcAcc) & 1u;
                 const int n = (int)min((int64_t)kTcTok, sg.t1 - t);
-                ok = __all_sync(0xffffffffu, dev::mbar_wait(full_bar(s), ph, abort_flag, &g_decode_error, kErrTcScore));
-                if (!ok) continue;
-                const bool valid = st < n;
-                const uint8_t* sp = stage_p + (size_t)s * kTcStageBytes;
-                uint32_t w[8];
-                if (nw == 8) {
-                    const uint4 x0 = reinterpret_cast<const uint4*>(sp + kTcWordsOff)[2 * st];
-                    const uint4 x1 = reinterpret_cast<const uint4*>(sp + kTcWordsOff)[2 * st + 1];
-                    w[0] = x0.x; w[1] = x0.y; w[2] = x0.z; w[3] = x0.w;
-                    w[4] = x1.x; w[5] = x1.y; w[6] = x1.z; w[7] = x1.w;
-                } else {
+                float M[G], lgk[G], smax = 0.0f, vsck = 0.0f;
+                bool validk = false;
+                if (ok)
+                    ok = __all_sync(0xffffffffu,
+                                    dev::mbar_wait(kfull_bar(s), ph, abort_flag, &g_decode_error, kErrTcScore));
+                if (ok) {
+                    const bool valid = st < n;
+                    const uint8_t* kp = key_p + (size_t)s * kTcKeyBytes;
+                    uint32_t w[8];
+                    if (nw == 8) {
+                        const uint4 x0 = reinterpret_cast<const uint4*>(kp + kTcWordsOff)[2 * st];
+                        const uint4 x1 = reinterpret_cast<const uint4*>(kp + kTcWordsOff)[2 * st + 1];
+                        w[0] = x0.x; w[1] = x0.y; w[2] = x0.z; w[3] = x0.w;
+                        w[4] = x1.x; w[5] = x1.y; w[6] = x1.z; w[7] = x1.w;
+                    } else {
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        w[k] = k < nw ? reinterpret_cast<const uint32_t*>(sp + kTcWordsOff)[st * nw + k] : 0u;
-                }
-                const float nrm = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(sp + kTcNormsOff)[st]));
-                const float vsc = valid ? reinterpret_cast<const float*>(sp + kTcScalesOff)[st] : 0.0f;
-                float sc[G];
-                lut_token_sums<G>(w, lut_s, lut_lane, sc);
-                float lg[G];
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float score = p.qjl_c * nrm * sc[g];
-                    lg[g] = valid ? score * p.scale_log2 : -INFINITY;
-                    if (p.scores_out != nullptr && valid)
-                        p.scores_out[(hb + g) * p.T + t + st] = score;
-                }
-                const float smax = warp_max(vsc);
-                const float rscale = smax > 0.0f ? kTcWmax / smax : 0.0f;
-                float M[G];
-                uint32_t W[G], Lq[G];
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    M[g] = warp_max(lg[g]);      // -inf for a slice without valid tokens
-                    const float pe = valid ? fast_exp2(lg[g] - M[g]) : 0.0f;
-                    W[g] = min(__float2uint_rn(pe * vsc * rscale), 0xFFFFFFu);
-                    Lq[g] = __reduce_add_sync(0xffffffffu, __float2uint_rn(pe * 16777216.0f));
-                }
-                // operand B and the slice stats of buffer a are free once chunk c - kTcAcc is merged
-                ok = __all_sync(0xffffffffu, dev::mbar_wait(tempty_bar(a), aph ^ 1u, abort_flag, &g_decode_error,
-                                                            kErrTcScore));
-                if (!ok) continue;
-                uint8_t* bq = b_p + a * kTcBBytes;
-#pragma unroll
-                for (int g = 0; g < G; ++g)
-#pragma unroll
-                    for (int k = 0; k < 3; ++k) {
-                        const int row = 3 * g + k;
-                        bq[(row >> 3) * 1024 + (row & 7) * 128 + ((kb ^ (row & 7)) << 4) + kx] =
-                            (uint8_t)(W[g] >> (8 * k));
+                        for (int k = 0; k < 8; ++k)
+                            w[k] = k < nw ? reinterpret_cast<const uint32_t*>(kp + kTcWordsOff)[st * nw + k] : 0u;
                     }
-                if (lane == 0) {
-                    TcSlice& S = slices[a * 4 + sw];
+                    const float nrm = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(kp + kTcNormsOff)[st]));
+                    const float vsc = valid ? reinterpret_cast<const float*>(kp + kTcScalesOff)[st] : 0.0f;
+                    // the key stage is read: the producer may refill it
+                    __syncwarp();
+                    if (lane == 0) dev::mbar_arrive(kempty_bar(s));
+                    float sc[G];
+                    lut_token_sums<G>(w, lut_s, lut_lane, sc);
+                    float lg[G];
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
-                        S.M[g] = M[g];
-                        S.L[g] = (float)Lq[g] * 5.9604644775390625e-8f;   // 2^-24
+                        const float score = p.qjl_c * nrm * sc[g];
+                        lg[g] = valid ? score * p.scale_log2 : -INFINITY;
+                        if (p.scores_out != nullptr && valid)
+                            p.scores_out[(hb + g) * p.T + t + st] = score;
                     }
-                    S.inv_scale = smax / kTcWmax;
+                    // the slice's maxima; the group agrees on the chunk's before quantizing
+                    smax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(vsc)));   // vsc >= 0
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        M[g] = warp_max(lg[g]);      // -inf for a slice without valid tokens
+                        lgk[g] = lg[g];
+                    }
+                    vsck = vsc;
+                    validk = valid;
+                    // operand B and the statistics of buffer a are free once chunk c - kTcAcc is merged
+                    ok = __all_sync(0xffffffffu, dev::mbar_wait(tempty_bar(a), aph ^ 1u, abort_flag,
+                                                                &g_decode_error, kErrTcScore));
+                    if (ok && lane == 0) {
+#pragma unroll
+                        for (int g = 0; g < G; ++g) chunks[a].Mk[sw][g] = M[g];
+                        chunks[a].Sk[sw] = smax;
+                    }
                 }
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) dev::mbar_arrive(bready_bar(a));
+                asm volatile("bar.sync %0, 128;" ::"r"(2 + gi) : "memory");   // the group's slice maxima
+                if (ok) {
+                    TcChunk& X = chunks[a];
+                    // the chunk's max logit per head and max value scale; weights 2^(s - Mc) v
+                    // in fixed point against an exact power of two 2^E with smax 2^E in
+                    // [2^23, 2^24) (from smax's exponent; chunks whose values are all below
+                    // 2^-100 count as zero), so the scale itself is not rounded
+                    float Mc[G];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) Mc[g] = fmaxf(fmaxf(X.Mk[0][g], X.Mk[1][g]), fmaxf(X.Mk[2][g], X.Mk[3][g]));
+                    const float sc_max = fmaxf(fmaxf(X.Sk[0], X.Sk[1]), fmaxf(X.Sk[2], X.Sk[3]));
+                    const uint32_t sexp = __float_as_uint(sc_max) >> 23;
+                    const float rscale = sexp >= 28u ? __uint_as_float((277u - sexp) << 23) : 0.0f;
+                    uint32_t W[G];
+                    float Lsl[G];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const float pe = validk ? fast_exp2(lgk[g] - Mc[g]) : 0.0f;
+                        W[g] = min(__float2uint_rn(pe * vsck * rscale), 0xFFFFFFu);
+                        Lsl[g] = (float)__reduce_add_sync(0xffffffffu, __float2uint_rn(pe * 16777216.0f)) *
+                                 5.9604644775390625e-8f;   // 2^-24
+                    }
+                    uint8_t* bq = b_p + a * kTcBBytes;
+#pragma unroll
+                    for (int g = 0; g < G; ++g)
+#pragma unroll
+                        for (int k = 0; k < 3; ++k) {
+                            const int row = 3 * g + k;
+                            bq[(row >> 3) * 1024 + (row & 7) * 128 + boff[row & 7]] = (uint8_t)(W[g] >> (8 * k));
+                        }
+                    if (lane == 0) {
+#pragma unroll
+                        for (int g = 0; g < G; ++g) X.Lf[sw][g] = Lsl[g];
+                        if (sw == 0) {
+#pragma unroll
+                            for (int g = 0; g < G; ++g) X.Mc[g] = Mc[g];
+                            X.inv = sexp >= 28u ? __uint_as_float((sexp - 23u) << 23) : 0.0f;
+                        }
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) dev::mbar_arrive(bready_bar(a));
+                }
             }
         }
     } else {
@@ -1670,51 +1759,38 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
             for (int64_t t = sg.t0; t < sg.t1; t += kTcTok, ++c) {
                 const int a = c % kTcAcc;
                 const uint32_t aph = (uint32_t)(c / kTcAcc) & 1u;
-                const int nk = (int)((min((int64_t)kTcTok, sg.t1 - t) + 31) / 32);
-                // the scorers' arrival on bready publishes the slice stats; the MMA's
+                // the scorers' arrival on bready publishes the chunk's statistics; the MMA's
                 // completion, the accumulators
                 ok = __all_sync(0xffffffffu,
                                 dev::mbar_wait(bready_bar(a), aph, abort_flag, &g_decode_error, kErrTcAcc) &&
                                     dev::mbar_wait(tfull_bar(a), aph, abort_flag, &g_decode_error, kErrTcAcc));
                 if (!ok) break;  // warp-uniform: tcgen05.ld is .aligned
                 dev::tc_fence_after();
-                // the chunk's four slices (64 contiguous columns) in one load, the slice
-                // stats into registers, then the buffer goes back to the scorers
-                uint32_t r[64];
-                dev::tmem_ld_32x32b_x64(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 4) * 16u, r);
-                float sM[4][G], sL[4][G], sinv[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const TcSlice& S = slices[a * 4 + k];
-#pragma unroll
-                    for (int g = 0; g < G; ++g) {   // slices past the chunk's tokens: never written
-                        sM[k][g] = k < nk ? S.M[g] : -INFINITY;
-                        sL[k][g] = k < nk ? S.L[g] : 0.0f;
-                    }
-                    sinv[k] = k < nk ? S.inv_scale : 0.0f;
-                }
-                dev::tmem_ld_wait();
-                dev::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) dev::mbar_arrive(tempty_bar(a));
+                // the chunk's statistics and its 16-column accumulator (the four slices summed
+                // by the tensor core), then the buffer goes back to the scorers
+                const TcChunk& X = chunks[a];
+                const float inv = X.inv;
                 float Mc[G], num[G], L[G];
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    Mc[g] = fmaxf(fmaxf(sM[0][g], sM[1][g]), fmaxf(sM[2][g], sM[3][g]));
-                    num[g] = 0.0f;
-                    L[g] = 0.0f;
+                    Mc[g] = X.Mc[g];
+                    L[g] = (X.Lf[0][g] + X.Lf[1][g]) + (X.Lf[2][g] + X.Lf[3][g]);
                 }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
+                {
+                    uint32_t r[16];
+                    dev::tmem_ld_32x32b_x16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)a * 16u, r);
+                    dev::tmem_ld_wait();
+                    dev::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) dev::mbar_arrive(tempty_bar(a));
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
-                        // a slice past the chunk's tokens, or without valid ones, has M = -inf
-                        const float f = sM[k][g] == -INFINITY ? 0.0f : fast_exp2(sM[k][g] - Mc[g]);
-                        const float x = __fmaf_rn((float)(int)r[16 * k + 3 * g + 2], 65536.0f,
-                                                  __fmaf_rn((float)(int)r[16 * k + 3 * g + 1], 256.0f,
-                                                            (float)(int)r[16 * k + 3 * g]));
-                        num[g] = __fmaf_rn(x * sinv[k], f, num[g]);
-                        L[g] = __fmaf_rn(sL[k][g], f, L[g]);
+                        // sum_t W c = D2 2^16 + (D1 2^8 + D0): the low part exact in int32
+                        // (|.| < 2^31), D2 (|D2| < 2^22) converted exactly through the
+                        // 1.5 * 2^23 bias
+                        const int lo = (int)r[3 * g + 1] * 256 + (int)r[3 * g];
+                        const float d2 = __int_as_float((int)r[3 * g + 2] + 0x4B400000) - kRoundMagic;
+                        num[g] = __fmaf_rn(d2, 65536.0f, (float)lo) * inv;
                     }
                 }
 #pragma unroll

@@ -43,7 +43,7 @@ def score_tolerance(ref, norms, v, m, rel=1e-4):
 #
 #   |out_gpu - out_ref| <= e^(2 Dm) [ sum_t P_t (rho_t + expm1(delta_t)) |v_t - out_ref| ]
 #                          + (n_chain + 66) 2^-24 (sum_t P_t |v_t| + |out_ref|)
-#                          + [tensor-core value pass] 2^-25 * 32 * 127 * smax + 2^-20 |out_ref|
+#                          + [tensor-core value pass] 2^-24 * 128 * 127 * smax + 2^-20 |out_ref|
 #
 #  * P_t, out_ref: fp64 softmax and weighted sum of the oracle's scores;
 #  * delta_t = sigma |s_gpu,t - s_ref,t|: the GPU's own score deviation (itself held to the
@@ -56,10 +56,10 @@ def score_tolerance(ref, norms, v, m, rel=1e-4):
 #  * n_chain: the longest sequential fp32 accumulation in any kernel: a CTA range of W
 #    tokens is split over at least 16 lane groups / warps / chunks, then the lane, warp and
 #    range merges (W <= ceil(B Hkv T nsub / SMs), rounded up to 64);
-#  * the tensor-core value pass rounds each weight to 24-bit fixed point relative to its
-#    32-token slice (2^-25 smax |c| per token, |c| <= 127) and the softmax sum to 2^-24
-#    per token; both are relative to a slice maximum of weight 1, so their share of the
-#    output is at most the largest slice's.
+#  * the tensor-core value pass rounds each weight of a 128-token chunk to an integer
+#    multiple of 2^-E with smax 2^E in [2^23, 2^24) (at most 2^-24 smax |c| per token,
+#    |c| <= 127) and the softmax sum to 2^-24 per token; both are relative to the chunk's
+#    maximum weight 1, so their share of the output is at most the largest chunk's.
 # Dm = max_t (delta_t + rho_t).  Every term is a worst case, not an estimate.
 
 EX2_REL = 2.0 ** -21
@@ -116,7 +116,7 @@ def decode_out_bound(out_ref, p, vals, s_gpu, s_ref, sigma, n_chain, n_rescale, 
     acc = (n_chain + 66) * 2.0 ** -24 * (p @ (np.abs(vals) if vabs is None else vabs) + np.abs(out_ref))
     b = Ew + acc + 1e-30
     if tc_smax is not None:
-        b += 2.0 ** -25 * 32 * 127 * float(tc_smax) + 2.0 ** -20 * np.abs(out_ref)
+        b += 2.0 ** -24 * 128 * 127 * float(tc_smax) + 2.0 ** -20 * np.abs(out_ref)
     return b
 
 
