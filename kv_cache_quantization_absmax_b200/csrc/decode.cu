@@ -1387,47 +1387,46 @@ decode_qjl_pf_kernel(const DecodeParams p) {
 
 // -----------------------------------------------------------------------------------
 // QJL keys, value pass on the tensor cores.  The range streams in chunks of 128 tokens
-// of one unit through two rings: a key ring (the chunk's sign words, fp16 norms and
-// value scales, by bulk copies) that the producer fills kTcLookahead chunks ahead of a
-// value ring (the chunk's 128 value rows by a TMA tile with the 128-byte swizzle, which
-// the tensor core reads as the MN-major operand A = V^T [128 dims x 128 tokens]).  The
-// scorers take each chunk's keys as soon as they land and release the key stage once
-// they hold its data in registers, so a chunk's weights are usually ready before its
-// value tile lands, and a value stage is held only for its load and its MMA.
-// Warp roles (one CTA per SM):
-//   warp 0       producer;
+// of one unit through two rings, each filled by its own producer thread: a key ring (the
+// chunk's sign words, by bulk copies) and a value ring (the
+// chunk's 128 value rows by a TMA tile with the 128-byte swizzle, which the tensor core
+// reads as the MN-major operand A = V^T [128 dims x 128 tokens]).  A scorer takes a
+// chunk's sign words as soon as they land and releases the key stage once it holds them
+// in registers (the norms and value scales it loads itself), so a chunk's weights are
+// usually ready before its value tile lands, and a value stage is held only for its load
+// and its MMA.
+// Warp roles (480 threads, one CTA per SM):
+//   warp 0       key producer; warp 14 value producer;
 //   warp 1       TMEM and the MMA thread: per chunk four tcgen05.mma kind::i8, slice k
-//                (tokens 32 k .. 32 k + 31) into its own 16-column int32 accumulator;
-//   warps 2..    scorers in groups of four that take chunks in turn, one token per
-//                thread: the estimator from the byte tables; per warp (32 tokens, one
-//                MMA slice) the max M of the log2-domain logits of each head and the max
-//                value scale smax; the weight w = 2^(s - M) * vscale as a 24-bit
-//                fixed-point integer W = round(w 2^E) with 2^E the power of two that puts
+//                (tokens 32 k .. 32 k + 31), all into the chunk's 16-column int32
+//                accumulator;
+//   warps 2..9   scorers, one warp per chunk (chunk c to warp c % 8), four tokens per
+//                thread (tokens 32 i + lane, i = 0 .. 3, i.e. slice i): the estimator from
+//                the byte tables; the chunk's max logit Mc of each head and max value scale
+//                smax by warp reductions; the weight w = 2^(s - Mc) * vscale as a 24-bit
+//                fixed-point integer W = round(w 2^E), 2^E the power of two that puts
 //                smax 2^E in [2^23, 2^24), split into three unsigned bytes that form rows
-//                3 g + k of the operand B [16 x 128 tokens] (K-major); the warp's sum of
-//                2^(s - Mc) in fixed point by one integer warp reduction;
-//   last 4 warps accumulators, one value dimension per thread: per slice, sum_t W_t c_t
-//                = D2 2^16 + D1 2^8 + D0 (exact in int32: |c| <= 127, bytes <= 255, 32
-//                tokens), times the slice's factor, summed over the slices and merged into
-//                the running online-softmax state of each head.
+//                3 g + k of the operand B [16 x 128 tokens] (K-major); the chunk's sum of
+//                2^(s - Mc) in fixed point by one integer warp reduction per head;
+//   warps 10..13 accumulators, one value dimension per thread: sum_t W_t c_t = D2 2^16 +
+//                D1 2^8 + D0 (exact in int32: |c| <= 127, bytes <= 255, 128 tokens), times
+//                2^-E, merged into the running online-softmax state of each head.
 // The INT8 codes enter the product unconverted and every product and sum is exact; the
 // approximations are the weights' fixed point (absolute error at most 2^-24 smax per
 // token), the sums' 2^-24 fixed point, and the fp32 merges.
 constexpr int kTcTok = 128;                 // tokens per chunk
 constexpr int kTcValueStages = 3;           // value ring: 16 KB tiles
-constexpr int kTcKeyStages = 5;             // key ring: words, norms and scales of a chunk
-constexpr int kTcLookahead = 3;             // key loads run this many chunks ahead of value loads
-static_assert(kTcLookahead + 2 <= kTcKeyStages, "the key ring holds the look-ahead and two chunks in scoring");
-constexpr int kTcScorerGroups = 3;          // groups of four scorer warps, chunk c to group c % 3
-constexpr int kTcScorerWarps = 4 * kTcScorerGroups;
-constexpr int kTcThreads = 32 * (2 + kTcScorerWarps + 4);
+constexpr int kTcScorerWarps = 8;           // one scorer warp per chunk, chunk c to warp c % 8
+// Key stages: the sign words of a chunk, one stage per scorer warp (chunk c in stage c % 8),
+// so that each stage has one consumer that takes its fills in order (mbarrier phases are
+// told apart by parity only: a consumer must never be more than one fill ahead).
+constexpr int kTcKeyStages = kTcScorerWarps;
+constexpr int kTcValueWarp = 2 + kTcScorerWarps + 4;   // the value producer, after the accumulators
+constexpr int kTcThreads = 32 * (kTcValueWarp + 1);
 constexpr int kTcVBytes = kTcTok * kD;      // value tile: 16 KB
-constexpr int kTcWordsOff = 0;              // key stage: words (<= 4 KB) | norms | scales
-constexpr int kTcNormsOff = kTcWordsOff + kTcTok * 32;
-constexpr int kTcScalesOff = kTcNormsOff + kTcTok * 2;
-constexpr int kTcKeyBytes = kTcScalesOff + kTcTok * 4;
+constexpr int kTcKeyBytes = kTcTok * 32;    // key stage: the chunk's sign words (<= 4 KB)
 constexpr int kTcBBytes = 2048;             // operand B: 16 rows x 128 bytes
-constexpr int kTcAcc = 2 * kTcScorerGroups;  // chunks in flight between scorers and accumulators
+constexpr int kTcAcc = kTcScorerWarps;       // chunks in flight between scorers and accumulators
 constexpr uint32_t kTcTmemCols = kTcAcc * 16 <= 32 ? 32 : (kTcAcc * 16 <= 64 ? 64 : (kTcAcc * 16 <= 128 ? 128 : 256));
 constexpr float kTcWmax = 16777215.0f;      // 2^24 - 1
 // instruction descriptor: int32 accumulator, A signed 8-bit MN-major, B unsigned 8-bit
@@ -1437,13 +1436,11 @@ constexpr uint32_t kTcIdesc = (2u << 4) | (1u << 7) | (0u << 10) | (1u << 15) | 
 
 enum : unsigned int { kErrTcProducer = 0x211, kErrTcMma = 0x212, kErrTcScore = 0x213, kErrTcAcc = 0x214 };
 
-struct TcChunk {              // per chunk in flight, from the scorer group to the accumulators
-    float Mk[4][4];           // [slice][head] max of the slice's log2-domain logits (group scratch)
-    float Sk[4];              // [slice] max value scale of the slice (group scratch)
+struct TcChunk {              // per chunk in flight, from its scorer warp to the accumulators
     float Mc[4];              // [head] the chunk's max logit
+    float L[4];               // [head] sum over the chunk of 2^(s - Mc)
     float inv;                // 2^-E: the value of one unit of the weights' fixed point
     float pad[3];
-    float Lf[4][4];           // [slice][head] sum over the slice of 2^(s - Mc)
 };
 
 // Shared memory, from a 1024-byte aligned base: byte tables | value ring | operand B
@@ -1503,14 +1500,14 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
         abort_storage = 0;
         for (int s = 0; s < kTcKeyStages; ++s) {
             dev::mbar_init(kfull_bar(s), 1);
-            dev::mbar_init(kempty_bar(s), 4);     // the four warps of the scorer group
+            dev::mbar_init(kempty_bar(s), 1);     // the chunk's scorer warp
         }
         for (int s = 0; s < kTcValueStages; ++s) {
             dev::mbar_init(vfull_bar(s), 1);
             dev::mbar_init(vempty_bar(s), 1);     // the MMA's commit
         }
         for (int a = 0; a < kTcAcc; ++a) {
-            dev::mbar_init(bready_bar(a), 4);
+            dev::mbar_init(bready_bar(a), 1);
             dev::mbar_init(tfull_bar(a), 1);
             dev::mbar_init(tempty_bar(a), 4);
         }
@@ -1528,60 +1525,48 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
     const uint32_t tmem = tmem_slot;
     dev::griddep_launch_dependents();  // the combine kernel may be scheduled (it waits)
 
-    if (warp == 0) {
-        // ---------------- producer ----------------
+    if (warp == 0 || warp == kTcValueWarp) {
+        // ---------------- producers: warp 0 the key ring, warp kTcValueWarp the value ring ----------------
+        // Two threads, so that a value tile is never held back behind a key load: at the
+        // start of a new unit the scorers that have finished the old one wait for the
+        // others at the table rebuild, and those may need the old unit's last value tiles.
         if (lane == 0) {
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
-            // chunk i's keys are issued at step i, its value tile at step i + kTcLookahead
-            int nk = 0, nv = 0;            // key / value loads issued
+            const bool keys = warp == 0;
+            if (!keys)
+                asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
+            int i = 0;
             bool ok = true;
-            int js = 0;                    // segment and token of the next key load
-            int64_t ts = nseg > 0 ? walk.seg(0).t0 : 0;
-            int jv = 0;                    // segment and token of the next value load
-            int64_t tv = ts;
-            auto next = [&](int& j, int64_t& t) {
-                t += kTcTok;
-                if (t >= walk.seg(j).t1 && ++j < nseg) t = walk.seg(j).t0;
-            };
-            while (ok && jv < nseg) {
-                if (js < nseg) {
-                    const Segment sg = walk.seg(js);
-                    const int s = nk % kTcKeyStages;
-                    const uint32_t ph = (uint32_t)(nk / kTcKeyStages) & 1u;
-                    if (!dev::mbar_wait(kempty_bar(s), ph ^ 1u, abort_flag, &g_decode_error, kErrTcProducer)) {
-                        ok = false;
-                        break;
+            for (int jj = 0; ok && jj < nseg; ++jj) {
+                const Segment sg = walk.seg(jj);
+                for (int64_t t = sg.t0; t < sg.t1; t += kTcTok, ++i) {
+                    const int64_t r = sg.u * p.cap + t;
+                    if (keys) {
+                        const int s = i % kTcKeyStages;
+                        const uint32_t ph = (uint32_t)(i / kTcKeyStages) & 1u;
+                        if (!dev::mbar_wait(kempty_bar(s), ph ^ 1u, abort_flag, &g_decode_error, kErrTcProducer)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint32_t n = (uint32_t)min((int64_t)kTcTok, sg.t1 - t);
+                        dev::mbar_arrive_expect_tx(kfull_bar(s), n * (uint32_t)nw * 4u);
+                        dev::bulk_g2s(key_s + (uint32_t)s * kTcKeyBytes, p.kw + r * nw, n * (uint32_t)nw * 4u,
+                                      kfull_bar(s));
+                    } else {
+                        const int s = i % kTcValueStages;
+                        const uint32_t ph = (uint32_t)(i / kTcValueStages) & 1u;
+                        if (!dev::mbar_wait(vempty_bar(s), ph ^ 1u, abort_flag, &g_decode_error, kErrTcProducer)) {
+                            ok = false;
+                            break;
+                        }
+                        dev::mbar_arrive_expect_tx(vfull_bar(s), (uint32_t)kTcVBytes);
+                        dev::tma_load_2d(val_s + (uint32_t)s * kTcVBytes, &vmap, vfull_bar(s), 0, (int)r);
                     }
-                    const uint32_t n = (uint32_t)min((int64_t)kTcTok, sg.t1 - ts);
-                    const int64_t r = sg.u * p.cap + ts;
-                    const uint32_t dst = key_s + (uint32_t)s * kTcKeyBytes;
-                    dev::mbar_arrive_expect_tx(kfull_bar(s), n * (uint32_t)nw * 4u + n * 2u + n * 4u);
-                    dev::bulk_g2s(dst + kTcWordsOff, p.kw + r * nw, n * (uint32_t)nw * 4u, kfull_bar(s));
-                    dev::bulk_g2s(dst + kTcNormsOff, p.kn + r, n * 2u, kfull_bar(s));
-                    dev::bulk_g2s(dst + kTcScalesOff, p.vs + r, n * 4u, kfull_bar(s));
-                    ++nk;
-                    next(js, ts);
-                }
-                if (nk > nv + kTcLookahead || js >= nseg) {
-                    const Segment sg = walk.seg(jv);
-                    const int s = nv % kTcValueStages;
-                    const uint32_t ph = (uint32_t)(nv / kTcValueStages) & 1u;
-                    if (!dev::mbar_wait(vempty_bar(s), ph ^ 1u, abort_flag, &g_decode_error, kErrTcProducer)) {
-                        ok = false;
-                        break;
-                    }
-                    dev::mbar_arrive_expect_tx(vfull_bar(s), (uint32_t)kTcVBytes);
-                    dev::tma_load_2d(val_s + (uint32_t)s * kTcVBytes, &vmap, vfull_bar(s), 0,
-                                     (int)(sg.u * p.cap + tv));
-                    ++nv;
-                    next(jv, tv);
                 }
             }
             // never leave the CTA with a copy in flight: wait for the last fill of each stage
-            for (int k = max(0, nk - kTcKeyStages); k < nk; ++k)
-                dev::mbar_drain(kfull_bar(k % kTcKeyStages), (uint32_t)(k / kTcKeyStages) & 1u);
-            for (int k = max(0, nv - kTcValueStages); k < nv; ++k)
-                dev::mbar_drain(vfull_bar(k % kTcValueStages), (uint32_t)(k / kTcValueStages) & 1u);
+            const int stages = keys ? kTcKeyStages : kTcValueStages;
+            for (int k = max(0, i - stages); k < i; ++k)
+                dev::mbar_drain(keys ? kfull_bar(k % stages) : vfull_bar(k % stages), (uint32_t)(k / stages) & 1u);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -1617,15 +1602,15 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
             dev::mbar_drain(done_bar, 0);
         }
     } else if (warp < 2 + kTcScorerWarps) {
-        // ---------------- scorers: group gi takes the chunks c with c % kTcScorerGroups == gi ----------------
-        const int gi = (warp - 2) >> 2;
-        const int sw = (warp - 2) & 3;                  // MMA slice: tokens 32 sw .. 32 sw + 31
-        const int st = sw * 32 + lane;                  // this thread's token of the chunk
+        // ---------------- scorers: warp sw takes the chunks c with c % kTcScorerWarps == sw ----------------
+        // lane l scores tokens 32 i + l of the chunk, i = 0 .. 3 (MMA slice i), in two pairs
+        const int sw = warp - 2;
         const LutLane lut_lane(lane);
-        const int kb = st >> 4, kx = st & 15;          // its byte in a row of B
-        int boff[8];                                    // ... under the 128-byte swizzle of row r
-#pragma unroll
-        for (int r7 = 0; r7 < 8; ++r7) boff[r7] = ((kb ^ r7) << 4) + kx;
+        // the byte of token 32 i + lane in row r of B under the 128-byte swizzle:
+        // ((2 i + lane / 16) ^ (r % 8)) * 16 + lane % 16, split into a compile-time part
+        // and one of two per-lane offsets
+        const int bo_even = ((lane >> 4) << 4) + (lane & 15);
+        const int bo_odd = (((lane >> 4) ^ 1) << 4) + (lane & 15);
         int c = 0;
         bool ok = true;
         for (int jj = 0; jj < nseg; ++jj) {
@@ -1640,112 +1625,123 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
                 build_sign_tables<G>(lut, p.sketch_v + hb * p.m, p.m, p.m, threadIdx.x - 64, 32 * kTcScorerWarps);
             asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcScorerWarps) : "memory");
             for (int64_t t = sg.t0; t < sg.t1; t += kTcTok, ++c) {
-                if (c % kTcScorerGroups != gi) continue;
-                // every warp of the group passes the group barrier below on every chunk of
-                // the group, also after an abort (it then skips the work around it)
+                if (!ok || c % kTcScorerWarps != sw) continue;
                 const int s = c % kTcKeyStages;
                 const uint32_t ph = (uint32_t)(c / kTcKeyStages) & 1u;
                 const int a = c % kTcAcc;
                 const uint32_t aph = (uint32_t)(c / kTcAcc) & 1u;
                 const int n = (int)min((int64_t)kTcTok, sg.t1 - t);
-                float M[G], lgk[G], smax = 0.0f, vsck = 0.0f;
-                bool validk = false;
-                if (ok)
-                    ok = __all_sync(0xffffffffu,
-                                    dev::mbar_wait(kfull_bar(s), ph, abort_flag, &g_decode_error, kErrTcScore));
-                if (ok) {
-                    const bool valid = st < n;
-                    const uint8_t* kp = key_p + (size_t)s * kTcKeyBytes;
-                    uint32_t w[8];
+                // the four tokens' norms and value scales straight from global memory
+                // (coalesced across the warp; in flight during the table lookups)
+                const int64_t r0 = sg.u * p.cap + t;
+                uint16_t nrm_b[4];
+                float vsc[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const bool v = 32 * i + lane < n;
+                    nrm_b[i] = v ? __ldcs(p.kn + r0 + 32 * i + lane) : (uint16_t)0;
+                    vsc[i] = v ? __ldcs(p.vs + r0 + 32 * i + lane) : 0.0f;
+                }
+                ok = __all_sync(0xffffffffu, dev::mbar_wait(kfull_bar(s), ph, abort_flag, &g_decode_error, kErrTcScore));
+                if (!ok) continue;
+                const uint8_t* kp = key_p + (size_t)s * kTcKeyBytes;
+                float lg[4][G];
+#pragma unroll
+                for (int pr = 0; pr < 2; ++pr) {
+                    uint32_t wA[8], wB[8];
+                    const int tA = 64 * pr + lane, tB = tA + 32;
                     if (nw == 8) {
-                        const uint4 x0 = reinterpret_cast<const uint4*>(kp + kTcWordsOff)[2 * st];
-                        const uint4 x1 = reinterpret_cast<const uint4*>(kp + kTcWordsOff)[2 * st + 1];
-                        w[0] = x0.x; w[1] = x0.y; w[2] = x0.z; w[3] = x0.w;
-                        w[4] = x1.x; w[5] = x1.y; w[6] = x1.z; w[7] = x1.w;
+                        const uint4* wp = reinterpret_cast<const uint4*>(kp);
+                        const uint4 a0 = wp[2 * tA], a1 = wp[2 * tA + 1], b0 = wp[2 * tB], b1 = wp[2 * tB + 1];
+                        wA[0] = a0.x; wA[1] = a0.y; wA[2] = a0.z; wA[3] = a0.w;
+                        wA[4] = a1.x; wA[5] = a1.y; wA[6] = a1.z; wA[7] = a1.w;
+                        wB[0] = b0.x; wB[1] = b0.y; wB[2] = b0.z; wB[3] = b0.w;
+                        wB[4] = b1.x; wB[5] = b1.y; wB[6] = b1.z; wB[7] = b1.w;
                     } else {
+                        const uint32_t* wp = reinterpret_cast<const uint32_t*>(kp);
 #pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            w[k] = k < nw ? reinterpret_cast<const uint32_t*>(kp + kTcWordsOff)[st * nw + k] : 0u;
+                        for (int k = 0; k < 8; ++k) {
+                            wA[k] = k < nw ? wp[tA * nw + k] : 0u;
+                            wB[k] = k < nw ? wp[tB * nw + k] : 0u;
+                        }
                     }
-                    const float nrm = __half2float(__ushort_as_half(reinterpret_cast<const uint16_t*>(kp + kTcNormsOff)[st]));
-                    const float vsc = valid ? reinterpret_cast<const float*>(kp + kTcScalesOff)[st] : 0.0f;
-                    // the key stage is read: the producer may refill it
-                    __syncwarp();
-                    if (lane == 0) dev::mbar_arrive(kempty_bar(s));
-                    float sc[G];
-                    lut_token_sums<G>(w, lut_s, lut_lane, sc);
-                    float lg[G];
+                    const bool vA = tA < n, vB = tB < n;
+                    if (pr == 1) {
+                        // the key stage is read: the producer may refill it
+                        __syncwarp();
+                        if (lane == 0) dev::mbar_arrive(kempty_bar(s));
+                    }
+                    float scA[G], scB[G];
+                    lut_token_sums<G>(wA, lut_s, lut_lane, scA);
+                    lut_token_sums<G>(wB, lut_s, lut_lane, scB);
+                    const float nA = __half2float(__ushort_as_half(nrm_b[2 * pr]));
+                    const float nB = __half2float(__ushort_as_half(nrm_b[2 * pr + 1]));
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
-                        const float score = p.qjl_c * nrm * sc[g];
-                        lg[g] = valid ? score * p.scale_log2 : -INFINITY;
-                        if (p.scores_out != nullptr && valid)
-                            p.scores_out[(hb + g) * p.T + t + st] = score;
-                    }
-                    // the slice's maxima; the group agrees on the chunk's before quantizing
-                    smax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(vsc)));   // vsc >= 0
-#pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        M[g] = warp_max(lg[g]);      // -inf for a slice without valid tokens
-                        lgk[g] = lg[g];
-                    }
-                    vsck = vsc;
-                    validk = valid;
-                    // operand B and the statistics of buffer a are free once chunk c - kTcAcc is merged
-                    ok = __all_sync(0xffffffffu, dev::mbar_wait(tempty_bar(a), aph ^ 1u, abort_flag,
-                                                                &g_decode_error, kErrTcScore));
-                    if (ok && lane == 0) {
-#pragma unroll
-                        for (int g = 0; g < G; ++g) chunks[a].Mk[sw][g] = M[g];
-                        chunks[a].Sk[sw] = smax;
+                        const float sa = p.qjl_c * nA * scA[g], sb = p.qjl_c * nB * scB[g];
+                        lg[2 * pr][g] = vA ? sa * p.scale_log2 : -INFINITY;
+                        lg[2 * pr + 1][g] = vB ? sb * p.scale_log2 : -INFINITY;
+                        if (p.scores_out != nullptr) {
+                            if (vA) p.scores_out[(hb + g) * p.T + t + tA] = sa;
+                            if (vB) p.scores_out[(hb + g) * p.T + t + tB] = sb;
+                        }
                     }
                 }
-                asm volatile("bar.sync %0, 128;" ::"r"(2 + gi) : "memory");   // the group's slice maxima
-                if (ok) {
+                // the chunk's max logit per head and max value scale (value scales are >= 0:
+                // their bit patterns order like the values); weights 2^(s - Mc) v in fixed
+                // point against an exact power of two 2^E with smax 2^E in [2^23, 2^24)
+                // (from smax's exponent; chunks whose values are all below 2^-100 count as
+                // zero), so the scale itself is not rounded
+                float Mc[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+                    Mc[g] = warp_max(fmaxf(fmaxf(lg[0][g], lg[1][g]), fmaxf(lg[2][g], lg[3][g])));
+                const uint32_t sexp =
+                    __reduce_max_sync(0xffffffffu, __float_as_uint(fmaxf(fmaxf(vsc[0], vsc[1]), fmaxf(vsc[2], vsc[3])))) >> 23;
+                const float rscale = sexp >= 28u ? __uint_as_float((277u - sexp) << 23) : 0.0f;
+                uint32_t W[4][G];
+                float L[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    uint32_t lq = 0u;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float pe = fast_exp2(lg[i][g] - Mc[g]);   // 0 for an invalid token
+                        W[i][g] = min(__float2uint_rn(pe * vsc[i] * rscale), 0xFFFFFFu);
+                        lq += __float2uint_rn(pe * 16777216.0f);
+                    }
+                    L[g] = (float)__reduce_add_sync(0xffffffffu, lq) * 5.9604644775390625e-8f;   // 2^-24
+                }
+                // operand B and the statistics of buffer a are free once chunk c - kTcAcc is merged
+                ok = __all_sync(0xffffffffu, dev::mbar_wait(tempty_bar(a), aph ^ 1u, abort_flag,
+                                                            &g_decode_error, kErrTcScore));
+                if (!ok) continue;
+                uint8_t* bq = b_p + a * kTcBBytes;
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int k = 0; k < 3; ++k) {
+                        const int row = 3 * g + k, r7 = row & 7;
+                        uint8_t* rp = bq + (row >> 3) * 1024 + r7 * 128 + ((r7 & 1) ? bo_odd : bo_even);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            rp[(((2 * i) ^ r7) & 6) << 4] = (uint8_t)(W[i][g] >> (8 * k));
+                    }
+                if (lane == 0) {
                     TcChunk& X = chunks[a];
-                    // the chunk's max logit per head and max value scale; weights 2^(s - Mc) v
-                    // in fixed point against an exact power of two 2^E with smax 2^E in
-                    // [2^23, 2^24) (from smax's exponent; chunks whose values are all below
-                    // 2^-100 count as zero), so the scale itself is not rounded
-                    float Mc[G];
-#pragma unroll
-                    for (int g = 0; g < G; ++g) Mc[g] = fmaxf(fmaxf(X.Mk[0][g], X.Mk[1][g]), fmaxf(X.Mk[2][g], X.Mk[3][g]));
-                    const float sc_max = fmaxf(fmaxf(X.Sk[0], X.Sk[1]), fmaxf(X.Sk[2], X.Sk[3]));
-                    const uint32_t sexp = __float_as_uint(sc_max) >> 23;
-                    const float rscale = sexp >= 28u ? __uint_as_float((277u - sexp) << 23) : 0.0f;
-                    uint32_t W[G];
-                    float Lsl[G];
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
-                        const float pe = validk ? fast_exp2(lgk[g] - Mc[g]) : 0.0f;
-                        W[g] = min(__float2uint_rn(pe * vsck * rscale), 0xFFFFFFu);
-                        Lsl[g] = (float)__reduce_add_sync(0xffffffffu, __float2uint_rn(pe * 16777216.0f)) *
-                                 5.9604644775390625e-8f;   // 2^-24
+                        X.Mc[g] = Mc[g];
+                        X.L[g] = L[g];
                     }
-                    uint8_t* bq = b_p + a * kTcBBytes;
-#pragma unroll
-                    for (int g = 0; g < G; ++g)
-#pragma unroll
-                        for (int k = 0; k < 3; ++k) {
-                            const int row = 3 * g + k;
-                            bq[(row >> 3) * 1024 + (row & 7) * 128 + boff[row & 7]] = (uint8_t)(W[g] >> (8 * k));
-                        }
-                    if (lane == 0) {
-#pragma unroll
-                        for (int g = 0; g < G; ++g) X.Lf[sw][g] = Lsl[g];
-                        if (sw == 0) {
-#pragma unroll
-                            for (int g = 0; g < G; ++g) X.Mc[g] = Mc[g];
-                            X.inv = sexp >= 28u ? __uint_as_float((sexp - 23u) << 23) : 0.0f;
-                        }
-                    }
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    __syncwarp();
-                    if (lane == 0) dev::mbar_arrive(bready_bar(a));
+                    X.inv = sexp >= 28u ? __uint_as_float((sexp - 23u) << 23) : 0.0f;
                 }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) dev::mbar_arrive(bready_bar(a));
             }
         }
-    } else {
+    } else if (warp < kTcValueWarp) {
         // ---------------- accumulators: value dimension d ----------------
         const int quarter = warp & 3;
         const int d = quarter * 32 + lane;
@@ -1774,7 +1770,7 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
                     Mc[g] = X.Mc[g];
-                    L[g] = (X.Lf[0][g] + X.Lf[1][g]) + (X.Lf[2][g] + X.Lf[3][g]);
+                    L[g] = X.L[g];
                 }
                 {
                     uint32_t r[16];
