@@ -45,7 +45,8 @@ struct DecodeParams {
     const uint16_t* kn;
     const int8_t* vc;
     const float* vs;
-    const float* sketch_v;  // [B * Hq][m] fp32 (QJL)
+    float* sketch_v;        // QJL: the query projections [B * Hq][m] fp32 that a separate kernel
+                            // writes; the tensor-core kernel's own slots [ctas][maxj - 1][G][256]
     float* scores_out;
     float* ws;              // partial states [ctas][maxj][G][2 + D]
     int64_t T;              // tokens attended per unit
@@ -260,11 +261,43 @@ __host__ __device__ constexpr int int8_ctas_per_sm(int G) { return G == 1 ? 3 : 
 // The byte tables of the sign-sketch estimator (the layout of the QJL decode kernel's
 // tables, described there): entry (pos, b) holds, for each of the G
 // heads, sum_{k<8} v[8 pos + k] * (bit k of b ? +1 : -1), at byte offset
-// (pos / 16) * 64 KB + b * 256 + (pos % 16) * 16.  Built by `nthr` threads.
+// (pos / 16) * 64 KB + b * 256 + (pos % 16) * 16.
+//
+// The 16 entries (pos, b) with high nibble c of b, from the eight projections vv[g][k] =
+// v[8 pos + k] of each head: the low nibble walks a Gray code, one sign flip per entry.
+template <int G>
+__device__ __forceinline__ void write_sign_entries(float* lut, int pos, int c, const float (&vv)[G][8]) {
+    constexpr int HALF_FLOATS = 256 * 16 * 4;
+    float val[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        float sacc = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sacc -= vv[g][k];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) sacc += ((c >> k) & 1) ? vv[g][4 + k] : -vv[g][4 + k];
+        val[g] = sacc;
+    }
+    float* base = lut + (pos >> 4) * HALF_FLOATS + (c * 16 * 16 + (pos & 15)) * 4;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int gray = i ^ (i >> 1);
+        if (i > 0) {
+            const int k = (i & 1) ? 0 : ((i & 2) ? 1 : ((i & 4) ? 2 : 3));   // the bit that flips at step i
+            const bool on = (gray >> k) & 1;
+#pragma unroll
+            for (int g = 0; g < G; ++g) val[g] += on ? 2.0f * vv[g][k] : -2.0f * vv[g][k];
+        }
+        *reinterpret_cast<float4*>(base + gray * 16 * 4) =
+            make_float4(val[0], G > 1 ? val[G > 1 ? 1 : 0] : 0.0f, G > 2 ? val[G > 2 ? 2 : 0] : 0.0f,
+                        G > 3 ? val[G > 3 ? 3 : 0] : 0.0f);
+    }
+}
+
+// All the tables, from the projections v (fp32, head g at v + g * vstride), by `nthr` threads.
 template <int G>
 __device__ __forceinline__ void build_sign_tables(float* lut, const float* v, int m, int64_t vstride, int tid,
                                                   int nthr) {
-    constexpr int HALF_FLOATS = 256 * 16 * 4;
     const int npos = m / 8;
     for (int item = tid; item < 512; item += nthr) {
         const int pos = item & 31;
@@ -274,31 +307,24 @@ __device__ __forceinline__ void build_sign_tables(float* lut, const float* v, in
         for (int g = 0; g < G; ++g)
 #pragma unroll
             for (int k = 0; k < 8; ++k) vv[g][k] = pos < npos ? __ldg(v + g * vstride + pos * 8 + k) : 0.0f;
-        float val[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            float sacc = 0.0f;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) sacc -= vv[g][k];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) sacc += ((c >> k) & 1) ? vv[g][4 + k] : -vv[g][4 + k];
-            val[g] = sacc;
-        }
-        float* base = lut + (pos >> 4) * HALF_FLOATS + (c * 16 * 16 + (pos & 15)) * 4;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int gray = i ^ (i >> 1);
-            if (i > 0) {
-                const int k = __ffs(i) - 1;           // the bit that flips at step i
-                const bool on = (gray >> k) & 1;
-#pragma unroll
-                for (int g = 0; g < G; ++g) val[g] += on ? 2.0f * vv[g][k] : -2.0f * vv[g][k];
-            }
-            *reinterpret_cast<float4*>(base + gray * 16 * 4) =
-                make_float4(val[0], G > 1 ? val[G > 1 ? 1 : 0] : 0.0f, G > 2 ? val[G > 2 ? 2 : 0] : 0.0f,
-                            G > 3 ? val[G > 3 ? 3 : 0] : 0.0f);
-        }
+        write_sign_entries<G>(lut, pos, c, vv);
     }
+}
+
+// All the tables, by eight warps, from projections held one sketch row per thread: lane
+// `lane` of warp w holds v[g][32 w + lane] in sv[g] and the warp writes the entries of
+// positions 4 w .. 4 w + 3, whose eight rows each it holds, exchanged by shuffles (lane:
+// position 4 w + lane / 8, high nibbles lane % 8 and lane % 8 + 8).
+template <int G>
+__device__ __forceinline__ void build_sign_tables_from_rows(float* lut, const float (&sv)[G], int w, int lane) {
+    float vv[G][8];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) vv[g][k] = __shfl_sync(0xffffffffu, sv[g], (lane & ~7) + k);
+    const int pos = 4 * w + (lane >> 3);
+    write_sign_entries<G>(lut, pos, lane & 7, vv);
+    write_sign_entries<G>(lut, pos, (lane & 7) + 8, vv);
 }
 
 // A lane's BYTES consecutive bytes of a shared-memory row (16, 8 or 4) as 32-bit words.
@@ -1421,6 +1447,10 @@ constexpr int kTcScorerWarps = 8;           // one scorer warp per chunk, chunk 
 // so that each stage has one consumer that takes its fills in order (mbarrier phases are
 // told apart by parity only: a consumer must never be more than one fill ahead).
 constexpr int kTcKeyStages = kTcScorerWarps;
+static_assert(kTcScorerWarps == 8, "the scorers build the tables as eight warps of four positions");
+// Units a CTA range may touch (the projections of all but the first wait in the workspace;
+// shorter units go to the CUDA-core kernel)
+constexpr int kTcMaxUnits = 9;
 constexpr int kTcValueWarp = 2 + kTcScorerWarps + 4;   // the value producer, after the accumulators
 constexpr int kTcThreads = 32 * (kTcValueWarp + 1);
 constexpr int kTcVBytes = kTcTok * kD;      // value tile: 16 KB
@@ -1428,7 +1458,6 @@ constexpr int kTcKeyBytes = kTcTok * 32;    // key stage: the chunk's sign words
 constexpr int kTcBBytes = 2048;             // operand B: 16 rows x 128 bytes
 constexpr int kTcAcc = kTcScorerWarps;       // chunks in flight between scorers and accumulators
 constexpr uint32_t kTcTmemCols = kTcAcc * 16 <= 32 ? 32 : (kTcAcc * 16 <= 64 ? 64 : (kTcAcc * 16 <= 128 ? 128 : 256));
-constexpr float kTcWmax = 16777215.0f;      // 2^24 - 1
 // instruction descriptor: int32 accumulator, A signed 8-bit MN-major, B unsigned 8-bit
 // K-major, N = 16, M = 128
 constexpr uint32_t kTcIdesc = (2u << 4) | (1u << 7) | (0u << 10) | (1u << 15) | (0u << 16) |
@@ -1451,7 +1480,7 @@ constexpr size_t kTcBOff = kTcValueOff + (size_t)kTcValueStages * kTcVBytes;
 constexpr size_t kTcKeyOff = kTcBOff + (size_t)kTcAcc * kTcBBytes;
 constexpr size_t kTcSliceOff = kTcKeyOff + (size_t)kTcKeyStages * kTcKeyBytes;
 constexpr size_t kTcBarOff = kTcSliceOff + (size_t)kTcAcc * sizeof(TcChunk);
-constexpr int kTcBars = 2 * kTcKeyStages + 2 * kTcValueStages + 3 * kTcAcc + 1;
+constexpr int kTcBars = 2 * kTcKeyStages + 2 * kTcValueStages + 3 * kTcAcc + 2;
 static_assert(kTcValueOff % 1024 == 0 && kTcBOff % 1024 == 0, "swizzled operands need 1024-byte alignment");
 static_assert(kTcKeyBytes % 16 == 0 && kTcSliceOff % 16 == 0, "bulk copy destinations are 16-byte aligned");
 
@@ -1488,6 +1517,7 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
     auto tfull_bar = [&](int a) { return bars + 8u * (kAccBar0 + kTcAcc + a); };
     auto tempty_bar = [&](int a) { return bars + 8u * (kAccBar0 + 2 * kTcAcc + a); };
     const uint32_t done_bar = bars + 8u * (kAccBar0 + 3 * kTcAcc);
+    const uint32_t pro_bar = bars + 8u * (kAccBar0 + 3 * kTcAcc + 1);   // the projection inputs
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -1495,6 +1525,10 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
     const RangeWalk walk(p, cta / p.nsub);
     const int nseg = walk.count();
     const int nw = p.m / 32;
+    // the first of the G query heads this CTA serves for unit u
+    const auto tc_head0 = [&](int64_t u) {
+        return (u / p.Hkv) * p.Hq + (u % p.Hkv) * p.Gt + (int64_t)(cta % p.nsub) * G;
+    };
 
     if (threadIdx.x == 0) {
         abort_storage = 0;
@@ -1512,6 +1546,7 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
             dev::mbar_init(tempty_bar(a), 4);
         }
         dev::mbar_init(done_bar, 1);
+        dev::mbar_init(pro_bar, 1);
         dev::mbar_init_fence();
     }
     // operand B: rows 3 G .. 15 stay zero
@@ -1534,6 +1569,16 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
             const bool keys = warp == 0;
             if (!keys)
                 asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
+            if (keys) {
+                // the projection inputs, into the table space the scorers fill only after
+                // they have used them: S (m rows of kD fp16) at 0 and the G query rows
+                // of each unit this CTA visits after 64 KB
+                dev::mbar_arrive_expect_tx(pro_bar, (uint32_t)(p.m * kD * 2 + nseg * G * kD * 2));
+                dev::bulk_g2s(lut_s, p.S, (uint32_t)(p.m * kD * 2), pro_bar);
+                for (int jj = 0; jj < nseg; ++jj)
+                    dev::bulk_g2s(lut_s + 65536u + (uint32_t)(jj * G * kD * 2), p.q + tc_head0(walk.seg(jj).u) * kD,
+                                  (uint32_t)(G * kD * 2), pro_bar);
+            }
             int i = 0;
             bool ok = true;
             for (int jj = 0; ok && jj < nseg; ++jj) {
@@ -1567,6 +1612,7 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
             const int stages = keys ? kTcKeyStages : kTcValueStages;
             for (int k = max(0, i - stages); k < i; ++k)
                 dev::mbar_drain(keys ? kfull_bar(k % stages) : vfull_bar(k % stages), (uint32_t)(k / stages) & 1u);
+            if (keys) dev::mbar_drain(pro_bar, 0);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -1611,18 +1657,65 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
         // and one of two per-lane offsets
         const int bo_even = ((lane >> 4) << 4) + (lane & 15);
         const int bo_odd = (((lane >> 4) ^ 1) << 4) + (lane & 15);
+        // The query projections v[g][i] = sum_d S[i][d] q[g][d] (fp32) of every unit this
+        // CTA visits, formed once, from S and the queries staged in the table space: thread
+        // i (sketch row 32 sw + lane; zero for i >= m) sums its row over the 16-byte column
+        // blocks in the rotated order b = (k + lane) % 16, k = 0 .. 15, so that a warp's
+        // reads of 32 rows fall in distinct banks.  The first unit's projections build its
+        // tables at once; the others wait in this CTA's slots of the workspace (written and
+        // read back by the same thread).
+        const int row = 32 * sw + lane;
+        float* proj = p.sketch_v + (size_t)cta * (size_t)(p.maxj - 1) * G * 256;
+        float sv0[G];
+        bool ok = __all_sync(0xffffffffu, dev::mbar_wait(pro_bar, 0, abort_flag, &g_decode_error, kErrTcScore));
+        if (ok) {
+            const uint4* srow = reinterpret_cast<const uint4*>(lut) + row * (kD / 8);
+            const uint4* qrows = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(lut) + 65536);
+            for (int jj = 0; jj < nseg; ++jj) {
+                float sv[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) sv[g] = 0.0f;
+                if (row < p.m) {
+#pragma unroll 4
+                    for (int k = 0; k < kD / 8; ++k) {
+                        const int blk = (k + lane) & (kD / 8 - 1);
+                        const uint4 s8 = srow[blk];
+                        const __half2* sh = reinterpret_cast<const __half2*>(&s8);
+#pragma unroll
+                        for (int g = 0; g < G; ++g) {
+                            const uint4 q8 = qrows[(jj * G + g) * (kD / 8) + blk];
+                            const __half2* qh = reinterpret_cast<const __half2*>(&q8);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 a = __half22float2(sh[e]), b = __half22float2(qh[e]);
+                                sv[g] = fmaf(a.x, b.x, sv[g]);
+                                sv[g] = fmaf(a.y, b.y, sv[g]);
+                            }
+                        }
+                    }
+                }
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    if (jj == 0) sv0[g] = sv[g];
+                    else proj[((size_t)(jj - 1) * G + g) * 256 + row] = sv[g];
+                }
+            }
+        }
+        // every scorer is done with the staged inputs before the first tables overwrite them
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcScorerWarps) : "memory");
         int c = 0;
-        bool ok = true;
         for (int jj = 0; jj < nseg; ++jj) {
             const Segment sg = walk.seg(jj);
-            const int64_t b = sg.u / p.Hkv;
-            const int kvh = (int)(sg.u % p.Hkv);
-            const int64_t hb = b * p.Hq + (int64_t)kvh * p.Gt + (int64_t)(cta % p.nsub) * G;
+            const int64_t hb = tc_head0(sg.u);
             // the tables are rebuilt per unit by all scorers; every scorer reaches both
             // barriers, also after an abort (they then skip the work in between)
-            asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcScorerWarps) : "memory");
-            if (ok)
-                build_sign_tables<G>(lut, p.sketch_v + hb * p.m, p.m, p.m, threadIdx.x - 64, 32 * kTcScorerWarps);
+            if (jj > 0) asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcScorerWarps) : "memory");
+            if (ok) {
+                float sv[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) sv[g] = jj == 0 ? sv0[g] : proj[((size_t)(jj - 1) * G + g) * 256 + row];
+                build_sign_tables_from_rows<G>(lut, sv, sw, lane);
+            }
             asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcScorerWarps) : "memory");
             for (int64_t t = sg.t0; t < sg.t1; t += kTcTok, ++c) {
                 if (!ok || c % kTcScorerWarps != sw) continue;
@@ -1918,22 +2011,27 @@ bool qjl_tc_applies(const DecodeParams& p) {
     const auto al16 = [](const void* x) { return reinterpret_cast<uintptr_t>(x) % 16 == 0; };
     const int64_t units = p.T > 0 ? p.total / p.T : 0;
     return !p.cuda_cores && p.knew == nullptr && p.want_out && p.k4p == nullptr && p.m <= 256 && p.m % 32 == 0 &&
-           p.T % 8 == 0 && p.cap % 8 == 0 && al16(p.kw) && al16(p.kn) && al16(p.vs) && al16(p.vc) &&
+           p.maxj <= kTcMaxUnits &&
+           p.T % 8 == 0 && p.cap % 8 == 0 && al16(p.kw) && al16(p.vc) && al16(p.q) && al16(p.S) &&
            units * p.cap <= (int64_t)INT32_MAX;
 }
 
+// The tensor-core kernel applies and its value map could be made.  That kernel projects
+// the queries on the sketch itself; the other QJL kernels read the projections that a
+// separate kernel writes to the workspace first.
+bool qjl_tc_map(const DecodeParams& p, CUtensorMap* vmap) {
+    return qjl_tc_applies(p) && make_u8_rows_map(vmap, p.vc, (p.total / p.T) * p.cap, kTcTok);
+}
+
 template <int G>
-cudaError_t run_qjl(const DecodeParams& p, int ctas, cudaStream_t st) {
-    if (qjl_tc_applies(p)) {
-        CUtensorMap vmap;
-        if (make_u8_rows_map(&vmap, p.vc, (p.total / p.T) * p.cap, kTcTok)) {
-            auto kern = decode_qjl_tc_kernel<G>;
-            const size_t smem = tc_smem_bytes();
-            const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            if (e != cudaSuccess) return e;
-            kern<<<ctas, kTcThreads, smem, st>>>(p, vmap);
-            return cudaGetLastError();
-        }
+cudaError_t run_qjl(const DecodeParams& p, int ctas, cudaStream_t st, const CUtensorMap* vmap) {
+    if (vmap != nullptr) {
+        auto kern = decode_qjl_tc_kernel<G>;
+        const size_t smem = tc_smem_bytes();
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        kern<<<ctas, kTcThreads, smem, st>>>(p, *vmap);
+        return cudaGetLastError();
     }
     if (p.knew == nullptr && p.m <= 256) {
         auto kern = decode_qjl_pf_kernel<G>;
@@ -1951,7 +2049,10 @@ cudaError_t run_qjl(const DecodeParams& p, int ctas, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-cudaError_t run_partial(bool qjl, int G, const DecodeParams& p, int ctas, cudaStream_t st) {
+// The partial-state kernel for the format and group size; vmap (QJL keys only) selects
+// the tensor-core QJL kernel.
+cudaError_t run_partial(bool qjl, int G, const DecodeParams& p, int ctas, cudaStream_t st,
+                        const CUtensorMap* vmap) {
     if (p.k4p != nullptr) {
         switch (G) {
             case 1: return run_qjl_pf<1, true>(p, ctas, st);
@@ -1962,9 +2063,9 @@ cudaError_t run_partial(bool qjl, int G, const DecodeParams& p, int ctas, cudaSt
     }
     if (qjl) {
         switch (G) {
-            case 1: return run_qjl<1>(p, ctas, st);
-            case 2: return run_qjl<2>(p, ctas, st);
-            case 4: return run_qjl<4>(p, ctas, st);
+            case 1: return run_qjl<1>(p, ctas, st, vmap);
+            case 2: return run_qjl<2>(p, ctas, st, vmap);
+            case 4: return run_qjl<4>(p, ctas, st, vmap);
             default: return cudaErrorNotSupported;
         }
     }
@@ -2031,7 +2132,12 @@ DecodePlan plan_decode(const kvq_decode_args* a, int sm_count) {
     pl.ctas = total > 0 ? (int)((total + W - 1) / W) * pl.nsub : 0;
     pl.maxj = (int)((W + T - 1) / T + 1);
     pl.partial_bytes = align256((size_t)pl.ctas * pl.maxj * G * (2 + kD) * sizeof(float));
-    pl.sketch_bytes = qjl ? align256((size_t)a->batch * a->n_q_heads * a->sketch_dim * sizeof(float)) : 0;
+    // QJL: the query projections, or (tensor-core kernel) the slots of the units after a
+    // CTA's first
+    const size_t proj_pre = (size_t)a->batch * a->n_q_heads * a->sketch_dim;
+    const size_t proj_tc = pl.maxj <= kTcMaxUnits ? (size_t)pl.ctas * (size_t)(pl.maxj - 1) * G * 256 : 0;
+    const size_t proj = proj_pre > proj_tc ? proj_pre : proj_tc;
+    pl.sketch_bytes = qjl ? align256(proj * sizeof(float)) : 0;
     pl.total_bytes = pl.partial_bytes + pl.sketch_bytes;
     return pl;
 }
@@ -2096,12 +2202,14 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
                     reinterpret_cast<uintptr_t>(a->k_scales) % 16 == 0 &&
                     (a->out == nullptr || reinterpret_cast<uintptr_t>(a->v_scales) % 16 == 0);
     cudaError_t e;
-    if (qjl) {
+    CUtensorMap vmap;
+    const bool tc = qjl && qjl_tc_map(p, &vmap);
+    if (qjl && !tc) {
         e = launch_qjl_query_sketch(a->q_f16, a->batch * a->n_q_heads, a->sketch_f16, a->sketch_dim,
                                     const_cast<float*>(p.sketch_v), st);
         if (e != cudaSuccess) return e;
     }
-    e = run_partial(qjl, G, p, pl.ctas, st);
+    e = run_partial(qjl, G, p, pl.ctas, st, tc ? &vmap : nullptr);
     if (e != cudaSuccess || !a->out) return e;
     // The combine kernel is scheduled as the decode kernel's CTAs retire (programmatic
     // dependent launch) instead of after it has fully drained, hiding its launch latency;
