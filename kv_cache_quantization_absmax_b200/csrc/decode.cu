@@ -1912,11 +1912,19 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
     if (warp == 1) dev::tmem_dealloc(tmem, kTcTmemCols);
 }
 
+// a / b for non-negative 64-bit a, b > 0, through the 32-bit divide when both fit.
+__device__ __forceinline__ int64_t div_nonneg(int64_t a, int64_t b) {
+    if (((uint64_t)a | (uint64_t)b) >> 32 == 0) return (int64_t)((uint32_t)a / (uint32_t)b);
+    return a / b;
+}
+
 // out[b][h][d]: merge, over the token ranges that covered KV unit u = b * Hkv + h / Gt,
 // acc_s[d] 2^(m_s - M) / sum_s l_s 2^(m_s - M).  The states of query head h were written by
 // the CTAs of its head subgroup (h % Gt) / G, one per range.  If a decode kernel recorded
 // an error (a bounded wait gave up and the CTA skipped its work), the states are not
-// complete and the head's output is NaN.
+// complete and the head's output is NaN.  Up to eight ranges (the usual case) are read in
+// one batch of independent loads, issued together with the error flag's, so the merge
+// costs one trip to L2 after the decode kernel drains.
 __global__ void __launch_bounds__(kD)
 decode_combine_kernel(const float* __restrict__ ws, int64_t T, int64_t W, int maxj, int Hq, int Hkv, int G,
                       int nsub, float* __restrict__ out, float* __restrict__ fin_ml) {
@@ -1930,27 +1938,47 @@ decode_combine_kernel(const float* __restrict__ ws, int64_t T, int64_t W, int ma
     const int64_t u = b * Hkv + h / Gt;
     const int sub = (h % Gt) / G;
     const int gh = h % G;
-    const int64_t c0 = (u * T) / W;
-    const int64_t c1 = ((u + 1) * T - 1) / W;
+    const int64_t c0 = div_nonneg(u * T, W);
+    const int64_t c1 = div_nonneg((u + 1) * T - 1, W);
     const int d = threadIdx.x;
-    if (*reinterpret_cast<volatile unsigned int*>(&g_decode_error) != 0u) {
-        out[bh * kD + d] = __int_as_float(0x7fc00000);
-        if (fin_ml != nullptr && d == 0) fin_ml[2 * bh] = fin_ml[2 * bh + 1] = __int_as_float(0x7fc00000);
-        return;
-    }
     auto slot = [&](int64_t c) {
-        const int64_t j = u - (c * W) / T;
+        const int64_t j = u - div_nonneg(c * W, T);
         return ws + (((c * nsub + sub) * maxj + j) * G + gh) * (2 + kD);
     };
-    float mx = -INFINITY;
-    for (int64_t c = c0; c <= c1; ++c) mx = fmaxf(mx, slot(c)[0]);
-    float l = 0.0f, a = 0.0f;
-    for (int64_t c = c0; c <= c1; ++c) {
-        const float* sl = slot(c);
-        const float f = exp2f(sl[0] - mx);
-        l += sl[1] * f;
-        a += sl[2 + d] * f;
+    const bool failed = *reinterpret_cast<volatile unsigned int*>(&g_decode_error) != 0u;
+    float mx = -INFINITY, l = 0.0f, a = 0.0f;
+    if (c1 - c0 < 8) {
+        float m8[8], l8[8], a8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if (k <= c1 - c0) {
+                const float* sl = slot(c0 + k);
+                m8[k] = sl[0];
+                l8[k] = sl[1];
+                a8[k] = sl[2 + d];
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (k <= c1 - c0) mx = fmaxf(mx, m8[k]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if (k <= c1 - c0) {
+                const float f = exp2f(m8[k] - mx);
+                l += l8[k] * f;
+                a += a8[k] * f;
+            }
+        }
+    } else {
+        for (int64_t c = c0; c <= c1; ++c) mx = fmaxf(mx, slot(c)[0]);
+        for (int64_t c = c0; c <= c1; ++c) {
+            const float* sl = slot(c);
+            const float f = exp2f(sl[0] - mx);
+            l += sl[1] * f;
+            a += sl[2 + d] * f;
+        }
     }
+    if (failed) mx = l = a = __int_as_float(0x7fc00000);
     out[bh * kD + d] = a / l;
     if (fin_ml != nullptr && d == 0) {  // the head's final softmax max (log2 domain) and sum
         fin_ml[2 * bh] = mx;
