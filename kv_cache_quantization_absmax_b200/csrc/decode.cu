@@ -1912,6 +1912,461 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
     if (warp == 1) dev::tmem_dealloc(tmem, kTcTmemCols);
 }
 
+// -----------------------------------------------------------------------------------
+// INT8 keys and values, both contractions on the tensor cores.  The range streams in
+// chunks of 128 tokens of one unit through a key ring and a value ring, each filled by
+// TMA tiles (128 rows of 128 bytes, 128-byte swizzle) that its own producer thread issues.
+// Per chunk:
+//   scores: one tcgen05.mma kind::i8 per 32 dims, D1 [128 tokens x N] = K [128 x 128]
+//           (K-major) x Qb^T, where Qb [N x 128 dims] holds, in rows 3 g + k, the base-256
+//           digits k (each in -128 .. 127) of the query of head g as a fixed-point integer
+//           q_fix = round(q 2^E) with max |q| 2^E in [2^21, 2^22): sum_d c_d q_fix,d =
+//           D1[3g] + 2^8 D1[3g+1] + 2^16 D1[3g+2] exactly (|D1| < 2^21 in int32);
+//   softmax: four warps, one per 32-token slice (the TMEM lane quarter of its tokens),
+//           one token per thread: the logit k_scale 2^-E sum_d c_d q_fix,d * sigma log2 e,
+//           the slice's max logit Mc per head, and the weight 2^(s - Mc) v_scale as a
+//           24-bit fixed-point integer W against the power of two 2^E' that puts the
+//           slice's max value scale into [2^23, 2^24), whose three bytes are rows
+//           3 g + k of the value operand B [N x 128 tokens] (K-major); the slice's sum of
+//           2^(s - Mc) in 2^-24 fixed point by one integer warp reduction;
+//   values: one MMA per slice, D2_i [128 dims x N] = V_i^T [128 x 32 tokens] (MN-major) x
+//           W_i^T, each slice into its own accumulator;
+//   merge:  four warps, one value dimension per thread: sum_t W_t c_t of each slice (exact
+//           in int32), times 2^-E', merged slice by slice into the running online-softmax
+//           state of each head.
+// Warp roles (one CTA per SM): warp 0 key producer; warp 1 TMEM and the score MMAs; warp
+// 2 value producer; warp 3 the value MMAs (each issued as soon as its chunk's weights and
+// value tile are in, so that a value stage is held no longer than that); then
+// `groups` softmax groups of four warps (group i takes the chunks c with c % groups == i,
+// each in its own TMEM and operand buffer i, so that several chunks are scored at once);
+// then four merge warps.  The query digits of every unit the CTA visits are formed once,
+// at the start, by softmax group 0.
+// The products and the per-slice sums are exact; the approximations are the query's
+// fixed point (at most 2^-23 max |q| per element), the weights' fixed point (at most
+// 2^-24 of the slice's max value scale per token), the sums' 2^-24 fixed point, and the
+// fp32 rounding of the score and of the merges.
+// -----------------------------------------------------------------------------------
+constexpr int kI8TcTok = 128;
+constexpr int kI8TcKStages = 6;
+constexpr int kI8TcVStages = 6;
+constexpr int kI8TcMaxUnits = 4;       // units a CTA range may touch (query digits held)
+constexpr int kI8TcSoft0 = 4;          // first softmax warp
+constexpr int kI8TcTile = kI8TcTok * kD;   // 16 KB
+
+enum : unsigned int { kErrI8TcProducer = 0x221, kErrI8TcMma = 0x222, kErrI8TcSoft = 0x223, kErrI8TcAcc = 0x224 };
+
+template <int G>
+struct I8Tc {
+    static constexpr int N = G == 8 ? 32 : 16;                // MMA N: rows 3 g + k
+    static constexpr int acc = G == 8 ? 2 : 4;                // chunks in flight after their scores
+    static constexpr int groups = acc;                        // softmax groups: group i owns buffer i
+    static constexpr int acc0 = kI8TcSoft0 + 4 * groups;      // first merge warp
+    static constexpr int threads = 32 * (acc0 + 4);
+    static constexpr int ob = N * 128;                        // an operand of N rows of 128 bytes
+    static constexpr uint32_t cols = 5 * N * acc <= 256 ? 256u : 512u;
+    struct Slice {                                            // per chunk and slice
+        float Mc[G];                                          // max logit per head (-inf: empty)
+        float L[G];                                           // sum of 2^(s - Mc) per head
+        float inv;                                            // 2^-E' of the weights
+    };
+    // shared memory from a 1024-byte aligned base
+    static constexpr size_t k_off = 0;
+    static constexpr size_t v_off = k_off + (size_t)kI8TcKStages * kI8TcTile;
+    static constexpr size_t w_off = v_off + (size_t)kI8TcVStages * kI8TcTile;
+    static constexpr size_t q_off = w_off + (size_t)acc * ob;
+    static constexpr size_t st_off = q_off + (size_t)kI8TcMaxUnits * ob;
+    static constexpr size_t qi_off = st_off + (size_t)acc * 4 * sizeof(Slice);
+    static constexpr size_t red_off = qi_off + (size_t)kI8TcMaxUnits * G * sizeof(float);
+    static constexpr size_t bar_off = (red_off + 4 * G * sizeof(float) + 7) & ~(size_t)7;
+    static constexpr int nbars = 2 * kI8TcKStages + 2 * kI8TcVStages + 5 * acc + 3;
+    static constexpr size_t smem = 1024 + bar_off + (size_t)nbars * 8;
+    static_assert(smem + 64 <= 232448, "shared memory of one CTA");
+    static_assert(w_off % 1024 == 0 && q_off % 1024 == 0 && ob % 1024 == 0, "swizzled operands");
+    // instruction descriptors (int32 accumulator, M = 128): scores: A signed K-major,
+    // B signed K-major; values: A signed MN-major, B unsigned K-major
+    static constexpr uint32_t idesc_qk = (2u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (0u << 16) |
+                                         ((uint32_t)(N >> 3) << 17) | ((128u >> 4) << 24);
+    static constexpr uint32_t idesc_pv = (2u << 4) | (1u << 7) | (0u << 10) | (1u << 15) | (0u << 16) |
+                                         ((uint32_t)(N >> 3) << 17) | ((128u >> 4) << 24);
+};
+
+// Byte (row r, column k) of a K-major operand of rows of 128 bytes, 128-byte swizzle.
+__device__ __forceinline__ int sw128_byte(int r, int k) {
+    const int r7 = r & 7;
+    return (r >> 3) * 1024 + r7 * 128 + ((((k >> 4) ^ r7) & 7) << 4) + (k & 15);
+}
+
+template <int G>
+__global__ void __launch_bounds__(I8Tc<G>::threads, 1)
+decode_int8_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap kmap,
+                      const __grid_constant__ CUtensorMap vmap) {
+    using C = I8Tc<G>;
+    using Slice = typename C::Slice;
+    constexpr int N = C::N;
+    constexpr int ACC = C::acc;
+    extern __shared__ uint8_t i8tc_raw[];
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_storage;
+    volatile int* abort_flag = &abort_storage;
+    const uint32_t raw = dev::smem_u32(i8tc_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* bp = i8tc_raw + (base - raw);
+    const uint32_t k_s = base + (uint32_t)C::k_off;
+    const uint32_t v_s = base + (uint32_t)C::v_off;
+    const uint32_t w_s = base + (uint32_t)C::w_off;
+    uint8_t* w_p = bp + C::w_off;
+    const uint32_t q_s = base + (uint32_t)C::q_off;
+    uint8_t* q_p = bp + C::q_off;
+    Slice* slices = reinterpret_cast<Slice*>(bp + C::st_off);       // [ACC][4]
+    float* qinv = reinterpret_cast<float*>(bp + C::qi_off);         // [units][G] 2^-E
+    float* qred = reinterpret_cast<float*>(bp + C::red_off);        // [4][G]
+    const uint32_t bars = base + (uint32_t)C::bar_off;
+    auto kfull_bar = [&](int s) { return bars + 8u * s; };
+    auto kempty_bar = [&](int s) { return bars + 8u * (kI8TcKStages + s); };
+    auto vfull_bar = [&](int s) { return bars + 8u * (2 * kI8TcKStages + s); };
+    auto vempty_bar = [&](int s) { return bars + 8u * (2 * kI8TcKStages + kI8TcVStages + s); };
+    constexpr int kA0 = 2 * kI8TcKStages + 2 * kI8TcVStages;
+    auto sfull_bar = [&](int a) { return bars + 8u * (kA0 + a); };             // scores in TMEM
+    auto sempty_bar = [&](int a) { return bars + 8u * (kA0 + ACC + a); };      // scores read
+    auto bready_bar = [&](int a) { return bars + 8u * (kA0 + 2 * ACC + a); };  // weights written
+    auto tfull_bar = [&](int a) { return bars + 8u * (kA0 + 3 * ACC + a); };   // value sums in TMEM
+    auto tempty_bar = [&](int a) { return bars + 8u * (kA0 + 4 * ACC + a); };  // value sums read
+    const uint32_t qready_bar = bars + 8u * (kA0 + 5 * ACC);
+    const uint32_t done_bar = bars + 8u * (kA0 + 5 * ACC + 1);      // the score MMAs, at the end
+    const uint32_t vdone_bar = bars + 8u * (kA0 + 5 * ACC + 2);     // the value MMAs, at the end
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int cta = blockIdx.x;
+    const RangeWalk walk(p, cta / p.nsub);
+    const int nseg = walk.count();
+    const auto head0 = [&](int64_t u) {
+        return (u / p.Hkv) * p.Hq + (u % p.Hkv) * p.Gt + (int64_t)(cta % p.nsub) * G;
+    };
+
+    if (threadIdx.x == 0) {
+        abort_storage = 0;
+        for (int s = 0; s < kI8TcKStages; ++s) {
+            dev::mbar_init(kfull_bar(s), 1);
+            dev::mbar_init(kempty_bar(s), 1);     // the score MMAs' commit
+        }
+        for (int s = 0; s < kI8TcVStages; ++s) {
+            dev::mbar_init(vfull_bar(s), 1);
+            dev::mbar_init(vempty_bar(s), 1);     // the value MMAs' commit
+        }
+        for (int a = 0; a < ACC; ++a) {
+            dev::mbar_init(sfull_bar(a), 1);
+            dev::mbar_init(sempty_bar(a), 4);     // the softmax warps
+            dev::mbar_init(bready_bar(a), 4);
+            dev::mbar_init(tfull_bar(a), 1);
+            dev::mbar_init(tempty_bar(a), 4);     // the merge warps
+        }
+        dev::mbar_init(qready_bar, 1);
+        dev::mbar_init(done_bar, 1);
+        dev::mbar_init(vdone_bar, 1);
+        dev::mbar_init_fence();
+    }
+    // the operands B (weights and query digits): rows 3 G .. N - 1 stay zero
+    for (int i = threadIdx.x; i < (ACC + kI8TcMaxUnits) * C::ob / 16; i += C::threads)
+        reinterpret_cast<uint4*>(w_p)[i] = make_uint4(0u, 0u, 0u, 0u);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (warp == 1) dev::tmem_alloc(dev::smem_u32(&tmem_slot), C::cols);
+    dev::tc_fence_before();
+    __syncthreads();
+    dev::tc_fence_after();
+    const uint32_t tmem = tmem_slot;
+    const uint32_t tmem_s = tmem;                          // [ACC][N] scores
+    const uint32_t tmem_o = tmem + (uint32_t)(ACC * N);    // [ACC][4][N] value sums
+    dev::griddep_launch_dependents();  // the combine kernel may be scheduled (it waits)
+
+    if (warp == 0 || warp == 2) {
+        // ---------------- producers: warp 0 the key ring, warp 2 the value ring ----------------
+        if (lane == 0) {
+            const bool keys = warp == 0;
+            const CUtensorMap* map = keys ? &kmap : &vmap;
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+            const int stages = keys ? kI8TcKStages : kI8TcVStages;
+            const uint32_t ring = keys ? k_s : v_s;
+            const int err = kErrI8TcProducer;
+            int i = 0;
+            bool ok = true;
+            for (int jj = 0; ok && jj < nseg; ++jj) {
+                const Segment sg = walk.seg(jj);
+                for (int64_t t = sg.t0; t < sg.t1; t += kI8TcTok, ++i) {
+                    const int s = i % stages;
+                    const uint32_t ph = (uint32_t)(i / stages) & 1u;
+                    const uint32_t full = keys ? kfull_bar(s) : vfull_bar(s);
+                    const uint32_t empty = keys ? kempty_bar(s) : vempty_bar(s);
+                    if (!dev::mbar_wait(empty, ph ^ 1u, abort_flag, &g_decode_error, err)) {
+                        ok = false;
+                        break;
+                    }
+                    dev::mbar_arrive_expect_tx(full, (uint32_t)kI8TcTile);
+                    dev::tma_load_2d(ring + (uint32_t)s * kI8TcTile, map, full, 0, (int)(sg.u * p.cap + t));
+                }
+            }
+            // never leave the CTA with a copy in flight: wait for the last fill of each stage
+            for (int k = max(0, i - stages); k < i; ++k)
+                dev::mbar_drain(keys ? kfull_bar(k % stages) : vfull_bar(k % stages), (uint32_t)(k / stages) & 1u);
+        }
+    } else if (warp == 1) {
+        // ---------------- the score MMAs ----------------
+        if (lane == 0) {
+            bool ok = dev::mbar_wait(qready_bar, 0u, abort_flag, &g_decode_error, kErrI8TcMma);
+            int c = 0;
+            for (int jj = 0; ok && jj < nseg; ++jj) {
+                const Segment sg = walk.seg(jj);
+                for (int64_t t = sg.t0; ok && t < sg.t1; t += kI8TcTok, ++c) {
+                    const int a = c % ACC;
+                    const int s = c % kI8TcKStages;
+                    if (!dev::mbar_wait(sempty_bar(a), ((uint32_t)(c / ACC) & 1u) ^ 1u, abort_flag, &g_decode_error,
+                                        kErrI8TcMma) ||
+                        !dev::mbar_wait(kfull_bar(s), (uint32_t)(c / kI8TcKStages) & 1u, abort_flag, &g_decode_error,
+                                        kErrI8TcMma)) {
+                        ok = false;
+                        break;
+                    }
+                    dev::tc_fence_after();
+                    const uint32_t ka = k_s + (uint32_t)s * kI8TcTile;
+                    const uint32_t qb = q_s + (uint32_t)jj * C::ob;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        dev::tc_mma_i8(tmem_s + (uint32_t)(a * N), dev::smem_desc_sw128(ka + (uint32_t)k * 32u),
+                                       dev::smem_desc_sw128(qb + (uint32_t)k * 32u), C::idesc_qk, k > 0 ? 1u : 0u);
+                    dev::tc_commit(sfull_bar(a));
+                    dev::tc_commit(kempty_bar(s));
+                }
+            }
+            dev::tc_commit(done_bar);
+            dev::mbar_drain(done_bar, 0);
+        }
+    } else if (warp == 3) {
+        // ---------------- the value MMAs: a chunk's as soon as its weights and values are in ----------------
+        if (lane == 0) {
+            int j = 0;
+            bool ok = true;
+            for (int jj = 0; ok && jj < nseg; ++jj) {
+                const Segment sg = walk.seg(jj);
+                for (int64_t t = sg.t0; ok && t < sg.t1; t += kI8TcTok, ++j) {
+                    const int a = j % ACC;
+                    const int s = j % kI8TcVStages;
+                    if (!dev::mbar_wait(bready_bar(a), (uint32_t)(j / ACC) & 1u, abort_flag, &g_decode_error,
+                                        kErrI8TcMma) ||
+                        !dev::mbar_wait(vfull_bar(s), (uint32_t)(j / kI8TcVStages) & 1u, abort_flag, &g_decode_error,
+                                        kErrI8TcMma)) {
+                        ok = false;
+                        break;
+                    }
+                    dev::tc_fence_after();
+                    const uint32_t va = v_s + (uint32_t)s * kI8TcTile;
+                    const uint32_t wb = w_s + (uint32_t)a * C::ob;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dev::tc_mma_i8(tmem_o + (uint32_t)((a * 4 + i) * N),
+                                       dev::smem_desc_sw128(va + (uint32_t)i * 4096u),
+                                       dev::smem_desc_sw128(wb + (uint32_t)i * 32u), C::idesc_pv, 0u);
+                    dev::tc_commit(tfull_bar(a));
+                    dev::tc_commit(vempty_bar(s));
+                }
+            }
+            dev::tc_commit(vdone_bar);
+            dev::mbar_drain(vdone_bar, 0);
+        }
+    } else if (warp < C::acc0) {
+        // ---------------- softmax: group grp takes the chunks c with c % groups == grp (its
+        // buffer); warp quarter q of the group, token 32 q + lane of the chunk ----------------
+        const int q = warp & 3;
+        const int grp = (warp - kI8TcSoft0) >> 2;
+        const int tid = threadIdx.x - 32 * kI8TcSoft0;     // group 0: 0 .. 127, a query dimension
+        // The query digits of every unit, formed once by group 0: thread tid takes dimension
+        // tid of the G heads; the max |q| of each head over the 128 dimensions by warp
+        // reductions and a pass through shared memory.
+        for (int jj = 0; grp == 0 && jj < nseg; ++jj) {
+            const int64_t hb = head0(walk.seg(jj).u);
+            float qv[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                qv[g] = __half2float(__ushort_as_half(p.q[(hb + g) * kD + tid]));
+                const unsigned int m = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(qv[g])));
+                if (lane == 0) qred[(warp - kI8TcSoft0) * G + g] = __uint_as_float(m);
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float amax = fmaxf(fmaxf(qred[g], qred[G + g]), fmaxf(qred[2 * G + g], qred[3 * G + g]));
+                // 2^E with amax 2^E in [2^21, 2^22) (fp16 queries: 6 <= E <= 45); all
+                // digits zero for a zero query
+                const int e = (int)(__float_as_uint(amax) >> 23) - 127;
+                const int E = amax > 0.0f ? 21 - e : 0;
+                const int qf = __float2int_rn(qv[g] * __uint_as_float((uint32_t)(127 + E) << 23));
+                const int d0 = ((qf + 128) & 255) - 128;
+                const int r1 = (qf - d0) >> 8;
+                const int d1 = ((r1 + 128) & 255) - 128;
+                const int d2 = (r1 - d1) >> 8;
+                uint8_t* qb = q_p + jj * C::ob;
+                qb[sw128_byte(3 * g, tid)] = (uint8_t)d0;
+                qb[sw128_byte(3 * g + 1, tid)] = (uint8_t)d1;
+                qb[sw128_byte(3 * g + 2, tid)] = (uint8_t)d2;
+                if (tid == 0) qinv[jj * G + g] = __uint_as_float((uint32_t)(127 - E) << 23);
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+        }
+        if (grp == 0) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (tid == 0) dev::mbar_arrive(qready_bar);
+        }
+        // the query scales 2^-E of every unit are in shared memory once the digits are
+        bool ok = __all_sync(0xffffffffu, dev::mbar_wait(qready_bar, 0u, abort_flag, &g_decode_error, kErrI8TcSoft));
+
+        const int tl = 32 * q + lane;
+        int c = 0;
+        for (int jj = 0; jj < nseg; ++jj) {
+            const Segment sg = walk.seg(jj);
+            const int64_t hb = head0(sg.u);
+            float qsc[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) qsc[g] = qinv[jj * G + g];
+            for (int64_t t = sg.t0; ok && t < sg.t1; t += kI8TcTok, ++c) {
+                if (c % C::groups != grp) continue;
+                const int a = c % ACC;
+                const uint32_t aph = (uint32_t)(c / ACC) & 1u;
+                const bool valid = t + tl < sg.t1;
+                const int64_t r = sg.u * p.cap + t + tl;
+                const float ksc = valid ? __ldcs(p.ks + r) : 0.0f;
+                const float vsc = valid ? __ldcs(p.vs + r) : 0.0f;
+                ok = __all_sync(0xffffffffu, dev::mbar_wait(sfull_bar(a), aph, abort_flag, &g_decode_error, kErrI8TcSoft));
+                if (!ok) break;
+                dev::tc_fence_after();
+                uint32_t d[N];
+                if constexpr (N == 16) dev::tmem_ld_32x32b_x16(tmem_s + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * N), d);
+                else dev::tmem_ld_32x32b_x32(tmem_s + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * N), d);
+                dev::tmem_ld_wait();
+                dev::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) dev::mbar_arrive(sempty_bar(a));
+                float lg[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const int lo = (int)d[3 * g + 1] * 256 + (int)d[3 * g];
+                    const float dot = __fmaf_rn((float)(int)d[3 * g + 2], 65536.0f, (float)lo);
+                    const float s = dot * (ksc * qsc[g]);
+                    lg[g] = valid ? s * p.scale_log2 : -INFINITY;
+                    if (p.scores_out != nullptr && valid) p.scores_out[(hb + g) * p.T + t + tl] = s;
+                }
+                // the slice's max logit per head and max value scale (value scales are
+                // >= 0: their bit patterns order like the values); weights in fixed point
+                // against 2^E' (from smax's exponent; slices whose values are all below
+                // 2^-100 count as zero)
+                float Mc[G], L[G];
+                uint32_t W[G];
+                const uint32_t sexp = __reduce_max_sync(0xffffffffu, __float_as_uint(vsc)) >> 23;
+                const float rscale = sexp >= 28u ? __uint_as_float((277u - sexp) << 23) : 0.0f;
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    Mc[g] = warp_max(lg[g]);
+                    const float pe = valid ? fast_exp2(lg[g] - Mc[g]) : 0.0f;
+                    W[g] = min(__float2uint_rn(pe * vsc * rscale), 0xFFFFFFu);
+                    L[g] = (float)__reduce_add_sync(0xffffffffu, __float2uint_rn(pe * 16777216.0f)) *
+                           5.9604644775390625e-8f;   // 2^-24
+                }
+                // the weights' buffer and the statistics of buffer a are free once chunk
+                // c - ACC is merged
+                ok = __all_sync(0xffffffffu,
+                                dev::mbar_wait(tempty_bar(a), aph ^ 1u, abort_flag, &g_decode_error, kErrI8TcSoft));
+                if (!ok) break;
+                uint8_t* wq = w_p + a * C::ob;
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int k = 0; k < 3; ++k) wq[sw128_byte(3 * g + k, tl)] = (uint8_t)(W[g] >> (8 * k));
+                if (lane == 0) {
+                    Slice& X = slices[a * 4 + q];
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        X.Mc[g] = Mc[g];
+                        X.L[g] = L[g];
+                    }
+                    X.inv = sexp >= 28u ? __uint_as_float((sexp - 23u) << 23) : 0.0f;
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) dev::mbar_arrive(bready_bar(a));
+            }
+        }
+    } else {
+        // ---------------- merge: value dimension d ----------------
+        const int quarter = warp & 3;
+        const int d = quarter * 32 + lane;
+        int c = 0;
+        bool ok = true;
+        for (int jj = 0; jj < nseg; ++jj) {
+            const Segment sg = walk.seg(jj);
+            float mrun[G], lrun[G], o[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) mrun[g] = -INFINITY, lrun[g] = 0.0f, o[g] = 0.0f;
+            for (int64_t t = sg.t0; ok && t < sg.t1; t += kI8TcTok, ++c) {
+                const int a = c % ACC;
+                const uint32_t aph = (uint32_t)(c / ACC) & 1u;
+                // the softmax warps' arrivals on bready publish the statistics; the MMA's
+                // completion, the sums
+                ok = __all_sync(0xffffffffu,
+                                dev::mbar_wait(bready_bar(a), aph, abort_flag, &g_decode_error, kErrI8TcAcc) &&
+                                    dev::mbar_wait(tfull_bar(a), aph, abort_flag, &g_decode_error, kErrI8TcAcc));
+                if (!ok) break;  // warp-uniform: tcgen05.ld is .aligned
+                dev::tc_fence_after();
+                const uint32_t ta = tmem_o + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(a * 4 * N);
+                // the four slices' sums, two slices per load
+                uint32_t rr[2 * N];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    if ((i & 1) == 0) {
+                        if constexpr (N == 16) dev::tmem_ld_32x32b_x32(ta + (uint32_t)(i * N), rr);
+                        else dev::tmem_ld_32x32b_x64(ta + (uint32_t)(i * N), rr);
+                        dev::tmem_ld_wait();
+                    }
+                    const uint32_t* r = rr + (i & 1) * N;
+                    const Slice& X = slices[a * 4 + i];
+                    if (X.Mc[0] == -INFINITY) continue;   // a slice without tokens
+                    const float inv = X.inv;
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const int lo = (int)r[3 * g + 1] * 256 + (int)r[3 * g];
+                        const float num = __fmaf_rn((float)(int)r[3 * g + 2], 65536.0f, (float)lo) * inv;
+                        const float mc = X.Mc[g];
+                        const float mn = fmaxf(mrun[g], mc);
+                        const float al = fast_exp2(mrun[g] - mn);
+                        const float be = fast_exp2(mc - mn);
+                        o[g] = __fmaf_rn(o[g], al, num * be);
+                        lrun[g] = __fmaf_rn(lrun[g], al, X.L[g] * be);
+                        mrun[g] = mn;
+                    }
+                }
+                // the sums and the statistics are read: buffer a goes back to the softmax warps
+                dev::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) dev::mbar_arrive(tempty_bar(a));
+            }
+            if (!ok) break;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float* slot = p.ws + (((int64_t)cta * p.maxj + jj) * G + g) * (2 + kD);
+                slot[2 + d] = o[g];
+                if (d == 0) {
+                    slot[0] = mrun[g];
+                    slot[1] = lrun[g];
+                }
+            }
+        }
+    }
+
+    __syncwarp();  // reconverge warps 0..3, whose lane 0 ran the role loop alone
+    dev::tc_fence_before();
+    __syncthreads();
+    dev::tc_fence_after();
+    if (warp == 1) dev::tmem_dealloc(tmem, C::cols);
+}
+
 // a / b for non-negative 64-bit a, b > 0, through the 32-bit divide when both fit.
 __device__ __forceinline__ int64_t div_nonneg(int64_t a, int64_t b) {
     if (((uint64_t)a | (uint64_t)b) >> 32 == 0) return (int64_t)((uint32_t)a / (uint32_t)b);
@@ -2077,6 +2532,29 @@ cudaError_t run_qjl(const DecodeParams& p, int ctas, cudaStream_t st, const CUte
     return cudaGetLastError();
 }
 
+template <int G>
+cudaError_t run_int8_tc_g(const DecodeParams& p, int ctas, cudaStream_t st, const CUtensorMap& kmap,
+                          const CUtensorMap& vmap) {
+    auto kern = decode_int8_tc_kernel<G>;
+    const size_t smem = I8Tc<G>::smem;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    kern<<<ctas, I8Tc<G>::threads, smem, st>>>(p, kmap, vmap);
+    return cudaGetLastError();
+}
+
+// The tensor-core INT8 kernel for the group size.
+cudaError_t run_int8_tc(int G, const DecodeParams& p, int ctas, cudaStream_t st, const CUtensorMap& kmap,
+                        const CUtensorMap& vmap) {
+    switch (G) {
+        case 1: return run_int8_tc_g<1>(p, ctas, st, kmap, vmap);
+        case 2: return run_int8_tc_g<2>(p, ctas, st, kmap, vmap);
+        case 4: return run_int8_tc_g<4>(p, ctas, st, kmap, vmap);
+        case 8: return run_int8_tc_g<8>(p, ctas, st, kmap, vmap);
+        default: return cudaErrorNotSupported;
+    }
+}
+
 // The partial-state kernel for the format and group size; vmap (QJL keys only) selects
 // the tensor-core QJL kernel.
 cudaError_t run_partial(bool qjl, int G, const DecodeParams& p, int ctas, cudaStream_t st,
@@ -2137,7 +2615,18 @@ int decode_group_size(const kvq_decode_args* a) {
     return g;
 }
 
-DecodePlan plan_decode(const kvq_decode_args* a, int sm_count) {
+// The tensor-core INT8 kernel may run this decode: an output, no request for the CUDA
+// cores, contexts of at least four chunks, and 16-byte aligned code arrays whose rows a
+// TMA coordinate reaches.  (Whether its ranges touch few enough units is checked on the
+// plan.)
+bool int8_tc_eligible(const kvq_decode_args* a) {
+    return a->key_format == KVQ_KEYS_INT8 && a->out != nullptr && (a->flags & KVQ_DECODE_CUDA_CORES) == 0u &&
+           a->seq_len >= 4 * kI8TcTok && reinterpret_cast<uintptr_t>(a->k_codes) % 16 == 0 &&
+           reinterpret_cast<uintptr_t>(a->v_codes) % 16 == 0 &&
+           a->batch * a->n_kv_heads * a->seq_len <= (int64_t)INT32_MAX;
+}
+
+DecodePlan plan_decode(const kvq_decode_args* a, int sm_count, bool tc_capable) {
     DecodePlan pl{};
     const int64_t Gt = a->n_q_heads / a->n_kv_heads;
     const int G = decode_group_size(a);
@@ -2147,18 +2636,26 @@ DecodePlan plan_decode(const kvq_decode_args* a, int sm_count) {
     pl.units = a->batch * a->n_kv_heads;
     const int64_t T = a->seq_len;
     const int64_t total = pl.units * T;
-    // As many CTAs as can be resident at once: up to three 68 KB-ring INT8 CTAs per SM,
-    // or one 512-thread QJL CTA per SM (its byte tables fill shared memory); the token
-    // space is cut into one range per nsub of them (the CTAs of a range stream the same
-    // bytes side by side, each for its own head subgroup).
+    // The token space is cut into one range per nsub resident CTAs (the CTAs of a range
+    // stream the same bytes side by side, each for its own head subgroup).
+    const auto cut = [&](int64_t resident) {
+        const int64_t ranges = resident / pl.nsub > 0 ? resident / pl.nsub : 1;
+        int64_t W = total > 0 ? (total + ranges - 1) / ranges : kRange;
+        W = (W + kRange - 1) / kRange * kRange;
+        pl.W = W;
+        pl.ctas = total > 0 ? (int)((total + W - 1) / W) * pl.nsub : 0;
+        pl.maxj = (int)((W + T - 1) / T + 1);
+    };
+    // As many CTAs as can be resident at once: one tensor-core INT8 CTA per SM (when its
+    // ranges touch few enough units), else up to three 68 KB-ring INT8 CTAs per SM, or one
+    // QJL CTA per SM (its byte tables fill shared memory).
     // (residual keys run the QJL decode kernel: their key_format is QJL too)
-    const int64_t resident = (int64_t)sm_count * (qjl ? 1 : int8_ctas_per_sm(G));
-    const int64_t ranges = resident / pl.nsub > 0 ? resident / pl.nsub : 1;
-    int64_t W = total > 0 ? (total + ranges - 1) / ranges : kRange;
-    W = (W + kRange - 1) / kRange * kRange;
-    pl.W = W;
-    pl.ctas = total > 0 ? (int)((total + W - 1) / W) * pl.nsub : 0;
-    pl.maxj = (int)((W + T - 1) / T + 1);
+    pl.int8_tc = false;
+    if (tc_capable && int8_tc_eligible(a)) {
+        cut(sm_count);
+        pl.int8_tc = pl.maxj <= kI8TcMaxUnits;
+    }
+    if (!pl.int8_tc) cut((int64_t)sm_count * (qjl ? 1 : int8_ctas_per_sm(G)));
     pl.partial_bytes = align256((size_t)pl.ctas * pl.maxj * G * (2 + kD) * sizeof(float));
     // QJL: the query projections, or (tensor-core kernel) the slots of the units after a
     // CTA's first
@@ -2237,7 +2734,16 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
                                     const_cast<float*>(p.sketch_v), st);
         if (e != cudaSuccess) return e;
     }
-    e = run_partial(qjl, G, p, pl.ctas, st, tc ? &vmap : nullptr);
+    bool done = false;
+    if (pl.int8_tc && p.v4p == nullptr && p.knew == nullptr) {
+        CUtensorMap kmap, vmap8;
+        const int64_t rows = pl.units * p.cap;
+        if (make_u8_rows_map(&kmap, p.kc, rows, kI8TcTok) && make_u8_rows_map(&vmap8, p.vc, rows, kI8TcTok)) {
+            e = run_int8_tc(G, p, pl.ctas, st, kmap, vmap8);
+            done = true;
+        }
+    }
+    if (!done) e = run_partial(qjl, G, p, pl.ctas, st, tc ? &vmap : nullptr);
     if (e != cudaSuccess || !a->out) return e;
     // The combine kernel is scheduled as the decode kernel's CTAs retire (programmatic
     // dependent launch) instead of after it has fully drained, hiding its launch latency;

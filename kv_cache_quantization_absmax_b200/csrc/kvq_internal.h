@@ -54,11 +54,14 @@ struct DecodePlan {
     int ctas;             // CTAs of the partial kernel: nsub per contiguous token range
     int64_t W;            // tokens per range
     int maxj;             // unit segments one range can touch
+    bool int8_tc;         // INT8 keys: the tensor-core kernel, one CTA per SM
     size_t partial_bytes; // per-segment softmax states
     size_t sketch_bytes;  // query sketches (QJL)
     size_t total_bytes;
 };
-DecodePlan plan_decode(const kvq_decode_args* a, int sm_count);
+// tc_capable: the call may run the tensor-core INT8 kernel (plain decodes with INT8
+// values; not the append or INT4-value entry points)
+DecodePlan plan_decode(const kvq_decode_args* a, int sm_count, bool tc_capable = true);
 cudaError_t read_and_clear_decode_error(uint32_t* code);
 // Append-on-decode: the new token (row T - 1 of every unit, a->seq_len = T) is encoded
 // by the decode kernel itself; the cache arrays have `capacity` rows per unit.

@@ -277,7 +277,8 @@ def kvq_decode_attention(q, *, k_codes=None, k_scales=None, k_words=None, k_norm
                          v_codes=None, v_scales=None, want_out=True, want_scores=False,
                          sm_scale=0.0, workspace=None, out=None, scores_out=None, stream=None, flags=0):
     """One decode step; returns (out [B, Hq, D] fp32 or None, scores [B, Hq, T] or None).
-    flags: KVQ_DECODE_CUDA_CORES keeps the weighted value sum on the CUDA cores."""
+    flags: KVQ_DECODE_CUDA_CORES keeps the scores and the weighted value sum on the CUDA
+    cores (no tensor-core kernel)."""
     _need_cuda(q, k_codes, k_scales, k_words, k_norms, sketch, v_codes, v_scales)
     B, Hq, D = q.shape
     ref = k_words if k_words is not None else k_codes

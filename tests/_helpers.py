@@ -69,9 +69,11 @@ def decode_chain(batch, n_kv_heads, seq_len, n_q_heads, n_sm, qjl=False):
     """(n_chain, n_rescale) for the bound above.  A CTA range holds at most
     W = ceil(units * T * nsub / SMs) tokens (rounded up to 64), nsub = head subgroups per
     KV head (G / 8 for INT8 keys, G / 4 for QJL keys, at least 1).  Within a range:
-      INT8 keys: 32 lane groups (16 from four heads per CTA up) each sum their own tokens;
-                 a group rescales at most once per pipeline stage (128 tokens for one head
-                 per CTA, else 64);
+      INT8 keys: on the CUDA cores 32 lane groups (16 from four heads per CTA up) each
+                 sum their own tokens and rescale at most once per pipeline stage (64 or 128
+                 tokens); on the tensor cores one running state per range takes one exact
+                 32-token slice sum at a time (one rescale per slice); the bound takes the
+                 larger of the two;
       QJL keys:  32 (warp, token parity) chains on the CUDA cores, or one running state per
                  128-token chunk on the tensor cores; at most one rescale per 128 tokens."""
     G = n_q_heads // n_kv_heads
@@ -86,7 +88,7 @@ def decode_chain(batch, n_kv_heads, seq_len, n_q_heads, n_sm, qjl=False):
     if qjl:
         groups, stage = 32, 128
     else:
-        groups, stage = (32 if g <= 2 else 16), (128 if g == 1 else 64)
+        groups, stage = 16, 32
     n_chain = W // groups + 64 + (-(-seq_len // W)) + 2
     n_rescale = W // stage + 8
     return n_chain, n_rescale
@@ -150,8 +152,10 @@ def softmax_scale(sm_scale=0.0, head_dim=128):
 def check_decode_bound(out_gpu, s_gpu, s_ref, vals, *, qjl, v_scales=None, sm_scale=0.0, n_sm=None, vabs=None):
     """check_decode_unit for every (batch, KV head) of a decode step: out_gpu [B, Hq, D],
     s_gpu / s_ref [B, Hq, T] raw scores, vals [B, Hkv, T, D] dequantized values (fp32 or
-    fp64); v_scales [B, Hkv, T] when the tensor-core value pass may run (QJL keys); vabs
-    [B, Hkv, T, D] as for decode_out_bound.  Returns the largest err / bound."""
+    fp64); v_scales [B, Hkv, T] when the tensor-core value pass may run (QJL keys; for
+    INT8 values without it, the unit's largest value scale is max |vals| / 127, which the
+    largest code of absmax rows makes exact); vabs [B, Hkv, T, D] as for decode_out_bound
+    (INT4 values, which never take the tensor-core pass).  Returns the largest err / bound."""
     out_gpu, s_gpu, s_ref = (np.asarray(a) for a in (out_gpu, s_gpu, s_ref))
     B, Hq, T = s_ref.shape
     Hkv = vals.shape[1]
@@ -162,7 +166,12 @@ def check_decode_bound(out_gpu, s_gpu, s_ref, vals, *, qjl, v_scales=None, sm_sc
     for b in range(B):
         for g in range(Hkv):
             hs = slice(g * G, (g + 1) * G)
-            smax = float(np.asarray(v_scales)[b, g].max()) if v_scales is not None else None
+            if v_scales is not None:
+                smax = float(np.asarray(v_scales)[b, g].max())
+            elif not qjl and vabs is None:
+                smax = float(np.abs(np.asarray(vals[b, g])).max()) / 127.0
+            else:
+                smax = None
             worst = max(worst, check_decode_unit(out_gpu[b, hs], s_gpu[b, hs], s_ref[b, hs],
                                                  np.asarray(vals[b, g], np.float64), sigma, n_chain,
                                                  n_rescale, smax, None if vabs is None else vabs[b, g]))

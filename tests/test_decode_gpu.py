@@ -55,24 +55,35 @@ def _int8_score_bound(q, kc, ks, G):
 
 
 # MHA, GQA (G = 2, 4, 8, and G = 3, 6 that are not powers of two), MQA (Hkv = 1, G up to
-# 32: query heads split over several CTAs per token range)
+# 32: query heads split over several CTAs per token range).  Contexts of 512 tokens and
+# more take the tensor-core kernel (128-token chunks, partial chunks at range and unit
+# edges, ranges over up to four units): G = 1 .. 8 and MQA among them.
 @pytest.mark.parametrize("B,Hq,Hkv,T", [(1, 1, 1, 1), (1, 4, 4, 5), (2, 8, 2, 33), (1, 8, 1, 1000),
                                         (2, 16, 4, 4097), (1, 8, 8, 300), (1, 16, 2, 2500),
                                         (16, 16, 8, 3), (4, 8, 8, 100), (3, 24, 3, 70),
                                         (1, 16, 1, 1000), (2, 32, 1, 700), (1, 32, 2, 3000),
-                                        (1, 12, 2, 500), (2, 6, 2, 301)])
-def test_decode_int8_parity(kvq, B, Hq, Hkv, T):
+                                        (1, 12, 2, 500), (2, 6, 2, 301), (2, 4, 4, 1030),
+                                        (1, 2, 1, 777), (3, 6, 3, 2000), (8, 8, 8, 600)])
+def test_decode_int8_parity(kvq, B, Hq, Hkv, T, flags=0):
     q, kc, ks, vc, vs = _int8_cache(10 + T, B, Hkv, T, Hq)
     ref = oracle.decode_attention(q, k_codes=kc, k_scales=ks, v_codes=vc, v_scales=vs,
                                   want_scores=True)
     qg, kcg, ksg, vcg, vsg = _cuda(q, kc, ks, vc, vs)
     out, scores = kvq.kvq_decode_attention(qg, k_codes=kcg, k_scales=ksg, v_codes=vcg,
-                                           v_scales=vsg, want_scores=True)
+                                           v_scales=vsg, want_scores=True, flags=flags)
     out, scores = to_np(out), to_np(scores)
     assert np.abs(out - ref["out"]).max() <= OUT_TOL
-    # raw scores: fp32 summation bound on the same codes
+    # raw scores: fp32 summation bound on the same codes (the tensor-core kernel's exact
+    # fixed-point sums, from a query rounded by at most 2^-22 max |q|, stay well inside it)
     assert np.all(np.abs(scores.astype(np.float64) - ref["scores"]) <= _int8_score_bound(q, kc, ks, Hq // Hkv))
     check_decode_bound(out, scores, ref["scores"], _vals(vc, vs), qjl=False)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T", [(2, 16, 4, 4097), (1, 16, 1, 1000), (2, 4, 4, 1030)])
+def test_decode_int8_cuda_cores_flag_parity(kvq, B, Hq, Hkv, T):
+    """KVQ_DECODE_CUDA_CORES on shapes that would take the tensor-core kernel: scores and
+    weighted sum in fp32 on the CUDA cores, against the same oracle and bounds."""
+    test_decode_int8_parity(kvq, B, Hq, Hkv, T, flags=kvq.KVQ_DECODE_CUDA_CORES)
 
 
 def test_decode_scores_only_outlier_layer(kvq):
@@ -203,7 +214,7 @@ def test_decode_int8_llama7b_layer_sampled(kvq):
         # the unit's bound, with the chain lengths of the whole layer's launch
         n_chain, n_rescale = decode_chain(B, H, T, H, sm_count(), qjl=False)
         check_decode_unit(out[b, h][None], scores[b, h][None], ref["scores"][0], _vals(vc_r, vs_r),
-                          softmax_scale(), n_chain, n_rescale)
+                          softmax_scale(), n_chain, n_rescale, tc_smax=float(vs_r.max()))
 
 
 def test_decode_qjl_gqa_long_context_all_units(kvq):

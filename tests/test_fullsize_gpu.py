@@ -76,7 +76,8 @@ def test_llama7b_cache_full_sampled(kvq):
         assert np.abs(outs[i][b, h] - ref["out"][0, 0]).max() <= 2e-3
         n_chain, n_rescale = decode_chain(B, H, T, H, sm_count(), qjl=False)
         check_decode_unit(outs[i][b, h][None], scs[i][b, h][None], ref["scores"][0],
-                          oracle.dequantize_int8(vc, vs), softmax_scale(), n_chain, n_rescale)
+                          oracle.dequantize_int8(vc, vs), softmax_scale(), n_chain, n_rescale,
+                          tc_smax=float(vs.max()))
 
 
 def test_key_sketch_scores_full_size(kvq):
