@@ -76,7 +76,9 @@ def decode_keys(llama=LLAMA, gqa=GQA):
             + gqa["batch"] * gqa["kv_heads"] * gqa["seq"])
 
 
-LAUNCHES_PER_STEP = 1 + LLAMA["layers"] * 2 + 1 + 1 + 1 + 3
+# quantize; per layer the INT8 decode and its combine; dequantize; QJL encode; value
+# quantize; the tensor-core QJL decode (which projects the queries itself) and its combine
+LAUNCHES_PER_STEP = 1 + LLAMA["layers"] * 2 + 1 + 1 + 1 + 2
 
 
 def max_over_ranks(value: float, group=None) -> float:
@@ -481,9 +483,12 @@ def measure_next_rows(wl, stream, reps=3):
     ag = kvq.make_decode_append_args(wl.qg, gnew[0], gnew[1], T=gt - 1, k_words=wl.words,
                                      k_norms=wl.norms, sketch=wl.S, v_codes=wl.vcodes,
                                      v_scales=wl.vscales, out=wl.outg, workspace=wl.wsg)
+    # the append entry point keeps the CUDA-core kernels (more CTAs per SM than the
+    # tensor-core decode): its workspace is sized on its own, once
+    need = max(lib.kvq_decode_append_workspace_bytes(ctypes.byref(a)) for a in a7 + [ag])
+    wsa = torch.empty(int(need), dtype=torch.uint8, device=wl.cache.device)
     for a in a7 + [ag]:
-        if lib.kvq_decode_append_workspace_bytes(ctypes.byref(a)) > a.base.workspace_bytes:
-            raise RuntimeError("append workspace larger than the decode workspace")
+        a.base.workspace, a.base.workspace_bytes = wsa.data_ptr(), int(need)
 
     def run(args_list):
         for a in args_list:
@@ -556,13 +561,35 @@ def measure_next_rows(wl, stream, reps=3):
     ms = timed(dec_cc)
     row("decode_qjl_cuda_cores", ms, row_bytes()["decode_qjl"],
         "GQA [4, 32q/8kv, 131072]: the decode_qjl row of the step with KVQ_DECODE_CUDA_CORES")
+    # ---- the 7B-shaped INT8 decode with scores and value sum on the CUDA cores ----
+    a7cc = [kvq.make_decode_args(wl.q7[l], k_codes=wl.codes[l, 0], k_scales=wl.scales[l, 0],
+                                 v_codes=wl.codes[l, 1], v_scales=wl.scales[l, 1], out=wl.out7[l],
+                                 flags=kvq.KVQ_DECODE_CUDA_CORES) for l in range(L)]
+    wscc = torch.empty(int(lib.kvq_decode_workspace_bytes(ctypes.byref(a7cc[0]))), dtype=torch.uint8,
+                       device=wl.cache.device)
+    for a in a7cc:
+        a.workspace, a.workspace_bytes = wscc.data_ptr(), wscc.numel()
+
+    def dec8_cc():
+        for a in a7cc:
+            st = lib.kvq_decode_attention(ctypes.byref(a), s)
+            if st != kvq.KVQ_OK:
+                raise kvq.KvqError("kvq_decode_attention", st)
+    ms = timed(dec8_cc) / L
+    row("decode_int8_cuda_cores", ms, row_bytes()["decode_int8"] / L,
+        "7B-shaped layer [8, 32, 4096, 128]: the decode_int8 row of the step with KVQ_DECODE_CUDA_CORES, per layer")
+    del wscc
     ms = timed(lambda: kvq.kvq_quantize_int4(wl.cache, g, v4p, v4s, v4z, stream=stream))
     row("int4_quantize", ms, elems * (2 + 0.5) + elems // g * 8, cache_desc + ", groups of 32")
     ms = timed(lambda: kvq.kvq_dequantize_int4(v4p, v4s, v4z, g, out=wl.deq, stream=stream))
     row("int4_dequantize", ms, elems * (0.5 + 2) + elems // g * 8, cache_desc + " -> fp16")
     a4 = [kvq.make_decode_int4v_args(wl.q7[l], k_codes=wl.codes[l, 0], k_scales=wl.scales[l, 0],
                                      v_packed=v4p[l, 1], v_scales4=v4s[l, 1], v_zeros4=v4z[l, 1],
-                                     v_group=g, out=wl.out7[l], workspace=wl.ws7) for l in range(L)]
+                                     v_group=g, out=wl.out7[l]) for l in range(L)]
+    ws4 = torch.empty(int(lib.kvq_decode_int4v_workspace_bytes(ctypes.byref(a4[0]))), dtype=torch.uint8,
+                      device=wl.cache.device)
+    for a in a4:
+        a.base.workspace, a.base.workspace_bytes = ws4.data_ptr(), ws4.numel()
 
     def dec4():
         for a in a4:
@@ -1066,8 +1093,8 @@ def run_profile_case(case: str, reps: int = 3, layers: int = 1):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(0)
     B, H, T, D = LLAMA["batch"], LLAMA["heads"], LLAMA["seq"], LLAMA["dim"]
-    if case in ("quantize", "dequantize", "decode_int8"):
-        shape = (2 * (layers if case != "decode_int8" else 1), B, H, T, D)
+    if case in ("quantize", "dequantize", "decode_int8", "decode_int8_cuda_cores"):
+        shape = (2 * (layers if not case.startswith("decode_int8") else 1), B, H, T, D)
         kv = inputs.lognormal_cache_device(3, shape, n_sigma_dims=(0, 2, 4), device=dev)
         codes, scales = kvq.kvq_quantize_int8(kv)
         out = torch.empty_like(kv)
@@ -1079,7 +1106,8 @@ def run_profile_case(case: str, reps: int = 3, layers: int = 1):
                 kvq.kvq_dequantize_int8(codes, scales, out=out)
             else:
                 kvq.kvq_decode_attention(q, k_codes=codes[0], k_scales=scales[0], v_codes=codes[1],
-                                         v_scales=scales[1])
+                                         v_scales=scales[1],
+                                         flags=kvq.KVQ_DECODE_CUDA_CORES if case.endswith("cores") else 0)
     elif case in ("qjl_encode", "decode_qjl"):
         gb, gq, gk, gt, m = (GQA[k] for k in ("batch", "q_heads", "kv_heads", "seq", "m"))
         if case == "qjl_encode":
@@ -1171,7 +1199,7 @@ def main(argv=None):
     p.add_argument("--no-sweep", action="store_true", help="skip the quantize/dequantize throughput sweep")
     p.add_argument("--profile-case", default=None,
                    help="run one small single-kernel case (quantize, dequantize, decode_int8, "
-                        "qjl_encode, decode_qjl, int4_quantize, int4_dequantize, cw_quantize, "
+                        "decode_int8_cuda_cores, qjl_encode, decode_qjl, int4_quantize, int4_dequantize, cw_quantize, "
                         "cw_dequantize, decode_int4v, decode_mass, evict_select, evict_compact, qjlres_encode, "
                         "decode_qjlres) for an ncu "
                         "capture, then exit")

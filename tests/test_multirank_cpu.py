@@ -69,7 +69,9 @@ def test_row_bytes_match_the_workload():
     assert b["dequantize_cache"] == rows * (128 + 4 + 2 * 128)
     keys = 4 * 8 * 131072
     assert b["decode_qjl"] == keys * (32 + 2 + 128 + 4) + 256 * 128 * 2 + 4 * 32 * 128 * 6
-    assert bench.LAUNCHES_PER_STEP == 71
+    # quantize, 32 x (INT8 decode + combine), dequantize, QJL encode, value quantize,
+    # tensor-core QJL decode + combine
+    assert bench.LAUNCHES_PER_STEP == 1 + 32 * 2 + 3 + 2
 
 
 def test_reference_arm_other_ranks_exit_without_work():
