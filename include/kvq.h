@@ -152,20 +152,29 @@ kvq_status kvq_qjl_query_sketch(const uint16_t* q_f16, int64_t n_q, int32_t d,
  * G / that CTAs per token range, which stream the same cache bytes side by side (the
  * second read mostly from L2).
  * Precision: scores and the softmax in fp32 (exponentials by the hardware 2^x); out
- * within 2e-3 absolute of the fp64 value of the formula above.  With QJL keys, when T
- * is a multiple of 8, k_words, k_norms, v_codes and v_scales are 16-byte aligned and
- * the cache has fewer than 2^31 token rows, the weighted sum runs on the tensor cores:
- * per block of 32 tokens and head, the weights p_t * sv_t relative to the block's
- * largest p become integers in units of 2^-E, smax 2^E in [2^23, 2^24) for the block's
- * largest value scale smax, that multiply the INT8 codes exactly in int32 (error at most
- * 2^-24 smax per token); otherwise in fp32 on the CUDA cores.
+ * within 2e-3 absolute of the fp64 value of the formula above.  Unless
+ * KVQ_DECODE_CUDA_CORES is set, the contractions run on the tensor cores where they
+ * apply, as exact integer products:
+ *   QJL keys (T a multiple of 8, k_words and v_codes 16-byte aligned, at most 9 units
+ *   per CTA range, fewer than 2^31 token rows): the weighted sum, per chunk of 128 tokens
+ *   and head, with the weights p_t * sv_t relative to the chunk's largest p as integers
+ *   in units of 2^-E, smax 2^E in [2^23, 2^24) for the chunk's largest value scale smax,
+ *   multiplying the INT8 codes exactly in int32 (error at most 2^-24 smax per token);
+ *   INT8 keys (T >= 512, k_codes and v_codes 16-byte aligned, at most 4 units per CTA
+ *   range, fewer than 2^31 token rows): the scores, as exact int32 sums of the key codes
+ *   times the query written as the fixed-point integer round(q 2^E), max|q| 2^E in
+ *   [2^21, 2^22) (error at most 2^-23 max|q| per query entry), rounded once to fp32 and
+ *   multiplied by s_t; and the weighted sum as for QJL keys, per block of 32 tokens.
+ * Everything else runs in fp32 on the CUDA cores.
  * flags (KVQ_DECODE_*): KVQ_DECODE_CUDA_CORES keeps the whole step on the CUDA cores
- * (QJL keys: the weighted sum in fp32 FMAs even where the tensor-core value pass
- * applies); 0 lets the library choose; other bits: KVQ_ERR_INVALID_ARG.
+ * (fp32 scores and weighted sum even where the tensor-core kernels apply); 0 lets the
+ * library choose; other bits: KVQ_ERR_INVALID_ARG.
  * workspace: caller-owned device memory of at least kvq_decode_workspace_bytes(a)
  * bytes, 256-byte aligned (KVQ_ERR_WORKSPACE otherwise).  It holds per-split partial
- * softmax states and the query sketches; its contents on entry do not matter.
- * Launches 2 kernels (INT8 keys) or 3 (QJL keys) on `stream`; no host synchronisation.
+ * softmax states and, for QJL keys, the query projections; its contents on entry do not
+ * matter.
+ * Launches 2 kernels (the decode and the merge of its partial states), 3 with QJL keys
+ * on the CUDA cores (the query projections first), on `stream`; no host synchronisation.
  * If a decode kernel records a device-side error (see kvq_device_error), the outputs of
  * this and of every later decode call are NaN until kvq_device_error() reads and clears
  * the error: out is valid only while kvq_device_error() reports 0.
@@ -194,7 +203,7 @@ typedef struct kvq_decode_args {
     uint32_t flags;                /* KVQ_DECODE_* */
 } kvq_decode_args;
 
-#define KVQ_DECODE_CUDA_CORES 1u   /* no tensor-core value pass */
+#define KVQ_DECODE_CUDA_CORES 1u   /* no tensor-core contraction */
 
 kvq_status kvq_decode_attention(const kvq_decode_args* a, kvq_stream_t stream);
 
