@@ -300,9 +300,11 @@ kvq_status kvq_qjl_residual_encode(const uint16_t* keys_f16, int64_t n_keys, int
  *              0 .. T are neither read nor written.
  *   k_new_f16, v_new_f16: [B][Hkv][D] fp16, 16-byte aligned; v_new_f16 may be NULL
  *              when base.out is NULL (the value rows are then not appended).
- * The appended rows are written by the decode kernel itself, which uses them in the
- * same launch.  Workspace as kvq_decode_attention, sized by
- * kvq_decode_append_workspace_bytes.  Errors as kvq_decode_attention.
+ * The appended rows are written before the attention reads them: by a small kernel
+ * ahead of the decode where a tensor-core decode kernel runs (see kvq_decode_attention),
+ * else by the CUDA-core decode kernel itself in the same launch.  Workspace as
+ * kvq_decode_attention, sized by kvq_decode_append_workspace_bytes.  Errors as
+ * kvq_decode_attention.
  */
 typedef struct kvq_decode_append_args {
     kvq_decode_args base;

@@ -268,7 +268,7 @@ kvq_status check_append(const kvq_decode_append_args* a, kvq_decode_args* view) 
 KVQ_API size_t kvq_decode_append_workspace_bytes(const kvq_decode_append_args* a) {
     kvq_decode_args view;
     if (check_append(a, &view) != KVQ_OK) return 0;
-    return kvq::plan_decode(&view, kvq::device_sm_count(), false).total_bytes;
+    return kvq::plan_decode(&view, kvq::device_sm_count()).total_bytes;
 }
 
 KVQ_API kvq_status kvq_decode_append(const kvq_decode_append_args* a, kvq_stream_t stream) {
@@ -276,7 +276,7 @@ KVQ_API kvq_status kvq_decode_append(const kvq_decode_append_args* a, kvq_stream
     const kvq_status st = check_append(a, &view);
     if (st != KVQ_OK) return st;
     if (view.batch == 0) return KVQ_OK;
-    const kvq::DecodePlan plan = kvq::plan_decode(&view, kvq::device_sm_count(), false);
+    const kvq::DecodePlan plan = kvq::plan_decode(&view, kvq::device_sm_count());
     if (!view.workspace || !aligned(view.workspace, 256) || view.workspace_bytes < plan.total_bytes)
         return KVQ_ERR_WORKSPACE;
     const kvq::AppendSpec app{a->capacity, a->k_new_f16, a->v_new_f16};

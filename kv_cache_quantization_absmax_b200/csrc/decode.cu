@@ -191,6 +191,31 @@ __device__ __forceinline__ uint16_t append_norm_bits(const uint16_t* k) {
     return __half_as_ushort(__double2half(__dsqrt_rn(s64)));
 }
 
+// The append of every unit's new token as a kernel of its own, for decodes that then run
+// a tensor-core kernel (which does not encode it): one CTA per unit stores row T - 1.
+// INT8 keys: warp 0 the key row, warp 1 the value row.  QJL keys: warps 0 .. m/32 - 1 one
+// sign word each, warp m/32 the norm, warp m/32 + 1 the value row.  The rows are the same
+// bits as the encode kernels' (and as the decode kernels' own append prologues).
+__global__ void __launch_bounds__(32 * 10)
+append_encode_kernel(const DecodeParams p, int qjl) {
+    const int64_t u = blockIdx.x;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t row = u * p.cap + p.T - 1;
+    const uint16_t* kn = p.knew + u * kD;
+    const int nw = qjl ? p.m / 32 : 1;
+    if (qjl && warp < nw) {
+        const uint32_t word = append_sign_word(p.S, kn, warp, lane);
+        if (lane == 0) const_cast<uint32_t*>(p.kw)[row * nw + warp] = word;
+    } else if (qjl && warp == nw) {
+        if (lane == 0) const_cast<uint16_t*>(p.kn)[row] = append_norm_bits(kn);
+    } else if (!qjl && warp == 0) {
+        append_int8_row(kn, const_cast<int8_t*>(p.kc) + row * kD, const_cast<float*>(p.ks) + row, lane);
+    } else if (warp == nw + (qjl ? 1 : 0) && p.vnew != nullptr) {
+        append_int8_row(p.vnew + u * kD, const_cast<int8_t*>(p.vc) + row * kD, const_cast<float*>(p.vs) + row, lane);
+    }
+}
+
 // Merge of per-warp softmax states (m, l, acc[D]) through shared memory into the
 // segment's partial slot.  red: [WARPS][G][2 + kD] floats, already written.
 template <int G, int WARPS>
@@ -2727,6 +2752,20 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
                     reinterpret_cast<uintptr_t>(a->k_scales) % 16 == 0 &&
                     (a->out == nullptr || reinterpret_cast<uintptr_t>(a->v_scales) % 16 == 0);
     cudaError_t e;
+    if (p.knew != nullptr) {
+        // append: where a tensor-core kernel runs the decode, the new token is encoded by
+        // a kernel of its own first (the CUDA-core kernels encode it themselves)
+        DecodeParams na = p;
+        na.knew = nullptr;
+        na.vnew = nullptr;
+        if (qjl ? qjl_tc_applies(na) : (pl.int8_tc && p.v4p == nullptr)) {
+            append_encode_kernel<<<(unsigned)pl.units, qjl ? 32 * (p.m / 32 + 2) : 64, 0, st>>>(p, qjl ? 1 : 0);
+            e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+            p.knew = nullptr;
+            p.vnew = nullptr;
+        }
+    }
     CUtensorMap vmap;
     const bool tc = qjl && qjl_tc_map(p, &vmap);
     if (qjl && !tc) {

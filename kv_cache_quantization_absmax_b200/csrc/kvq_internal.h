@@ -59,8 +59,8 @@ struct DecodePlan {
     size_t sketch_bytes;  // query sketches (QJL)
     size_t total_bytes;
 };
-// tc_capable: the call may run the tensor-core INT8 kernel (plain decodes with INT8
-// values; not the append or INT4-value entry points)
+// tc_capable: the call may run the tensor-core INT8 kernel (decodes and appends with INT8
+// values; not the INT4-value entry point)
 DecodePlan plan_decode(const kvq_decode_args* a, int sm_count, bool tc_capable = true);
 cudaError_t read_and_clear_decode_error(uint32_t* code);
 // Append-on-decode: the new token (row T - 1 of every unit, a->seq_len = T) is encoded

@@ -55,6 +55,8 @@ def _cuda(*arrs):
     return [torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in arrs]
 
 
+# T + 1 >= 512 takes the tensor-core decode, with the append encoded by a kernel of its
+# own first; the shorter contexts encode inside the CUDA-core kernel.
 @pytest.mark.parametrize("B,Hq,Hkv,T,cap", [(1, 4, 4, 0, 8), (2, 8, 2, 33, 40), (1, 8, 1, 999, 1000),
                                             (2, 16, 4, 4095, 4096), (16, 16, 8, 2, 3),
                                             (3, 24, 3, 70, 77), (1, 8, 8, 1500, 1501)])
@@ -97,9 +99,13 @@ def test_append_int8_scores_only(kvq):
     assert np.all(np.abs(to_np(scores).astype(np.float64) - ref["scores"]) <= 2 * 128 * 2.0 ** -24 * terms)
 
 
+# T + 1 and the capacity multiples of 8 take the tensor-core decode, with the append
+# encoded by a kernel of its own first: (1, 32, 8, 2047, 2048), (2, 16, 2, 1535, 1536),
+# (1, 8, 4, 4095, 4104, m = 128); the others encode inside the CUDA-core kernel.
 @pytest.mark.parametrize("B,Hq,Hkv,T,cap,m", [(1, 4, 1, 0, 4, 256), (2, 8, 2, 100, 128, 256),
                                               (1, 32, 8, 2047, 2048, 256), (1, 4, 4, 333, 400, 128),
-                                              (4, 8, 4, 5000, 5001, 64)])
+                                              (4, 8, 4, 5000, 5001, 64), (2, 16, 2, 1535, 1536, 256),
+                                              (1, 8, 4, 4095, 4104, 128)])
 def test_append_qjl(kvq, B, Hq, Hkv, T, cap, m):
     q, kn, vn, kprev, _, _, vc, vs = _case(90 + T, B, Hq, Hkv, T, cap)
     S = inputs.sketch_matrix(m, 128)
