@@ -168,7 +168,8 @@ kvq_status kvq_qjl_query_sketch(const uint16_t* q_f16, int64_t n_q, int32_t d,
  * Everything else runs in fp32 on the CUDA cores.
  * flags (KVQ_DECODE_*): KVQ_DECODE_CUDA_CORES keeps the whole step on the CUDA cores
  * (fp32 scores and weighted sum even where the tensor-core kernels apply); 0 lets the
- * library choose; other bits: KVQ_ERR_INVALID_ARG.
+ * library choose; KVQ_DECODE_TEST_EXPIRE is for testing the failure path (below the
+ * struct); other bits: KVQ_ERR_INVALID_ARG.
  * workspace: caller-owned device memory of at least kvq_decode_workspace_bytes(a)
  * bytes, 256-byte aligned (KVQ_ERR_WORKSPACE otherwise).  It holds per-split partial
  * softmax states and, for QJL keys, the query projections; its contents on entry do not
@@ -204,6 +205,12 @@ typedef struct kvq_decode_args {
 } kvq_decode_args;
 
 #define KVQ_DECODE_CUDA_CORES 1u   /* no tensor-core contraction */
+/* For testing the failure path only: the tensor-core decode kernels issue none of their
+ * key loads, so the bounded waits of the roles that consume them expire (after about 2 s
+ * each): the call completes, kvq_device_error() then reports the kernel's code, and the
+ * outputs are NaN.  No fault and no hang: every wait is bounded.  The CUDA-core kernels
+ * ignore it. */
+#define KVQ_DECODE_TEST_EXPIRE 2u
 
 kvq_status kvq_decode_attention(const kvq_decode_args* a, kvq_stream_t stream);
 

@@ -55,7 +55,7 @@ kvq_status check_decode(const kvq_decode_args* a) {
     if (a->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
     if (!a->out && !a->scores_out) return KVQ_ERR_INVALID_ARG;
     if (!(a->sm_scale == a->sm_scale) || a->sm_scale < 0.0f) return KVQ_ERR_INVALID_ARG;
-    if ((a->flags & ~KVQ_DECODE_CUDA_CORES) != 0u) return KVQ_ERR_INVALID_ARG;
+    if ((a->flags & ~(KVQ_DECODE_CUDA_CORES | KVQ_DECODE_TEST_EXPIRE)) != 0u) return KVQ_ERR_INVALID_ARG;
     if (a->batch == 0) return KVQ_OK;
     if (!a->q_f16 || !aligned(a->q_f16, 16)) return KVQ_ERR_INVALID_ARG;
     if (a->key_format == KVQ_KEYS_INT8) {

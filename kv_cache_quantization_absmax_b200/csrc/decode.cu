@@ -81,6 +81,7 @@ struct DecodeParams {
     int qjl_bulk;           // QJL: value rows 16-byte aligned -> each warp's next 32 value
                             // rows come by one bulk copy
     int cuda_cores;         // the caller asked for no tensor-core value pass
+    int test_expire;        // testing the failure path: the tensor-core kernels issue no key loads
 };
 
 // The unit segments of CTA `cta`'s range: unit u, tokens [t0, t1) of that unit, slot j.
@@ -1590,7 +1591,8 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
         // Two threads, so that a value tile is never held back behind a key load: at the
         // start of a new unit the scorers that have finished the old one wait for the
         // others at the table rebuild, and those may need the old unit's last value tiles.
-        if (lane == 0) {
+        // (KVQ_DECODE_TEST_EXPIRE: the key producer issues nothing, its consumers' waits expire)
+        if (lane == 0 && !(warp == 0 && p.test_expire)) {
             const bool keys = warp == 0;
             if (!keys)
                 asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&vmap)) : "memory");
@@ -2106,7 +2108,8 @@ decode_int8_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap 
 
     if (warp == 0 || warp == 2) {
         // ---------------- producers: warp 0 the key ring, warp 2 the value ring ----------------
-        if (lane == 0) {
+        // (KVQ_DECODE_TEST_EXPIRE: the key producer issues nothing, its consumers' waits expire)
+        if (lane == 0 && !(warp == 0 && p.test_expire)) {
             const bool keys = warp == 0;
             const CUtensorMap* map = keys ? &kmap : &vmap;
             asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -2738,6 +2741,7 @@ cudaError_t launch_decode(const kvq_decode_args* a, const DecodePlan& pl, cudaSt
     p.qjl_c = qjl ? (float)(1.2533141373155002512 / (double)a->sketch_dim) : 0.0f;  // sqrt(pi/2)/m
     p.want_out = a->out != nullptr;
     p.cuda_cores = (a->flags & KVQ_DECODE_CUDA_CORES) != 0u;
+    p.test_expire = (a->flags & KVQ_DECODE_TEST_EXPIRE) != 0u;
     if (k4 != nullptr) {
         p.k4p = k4->packed;
         p.k4s = k4->scales;

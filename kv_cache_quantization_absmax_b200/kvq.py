@@ -19,6 +19,7 @@ KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CUDA, KVQ_ERR_WORKSPAC
 KVQ_F32, KVQ_F16 = 0, 1
 KVQ_KEYS_INT8, KVQ_KEYS_QJL = 0, 1
 KVQ_DECODE_CUDA_CORES = 1
+KVQ_DECODE_TEST_EXPIRE = 2
 ABI_VERSION = 2
 
 _P = ctypes.c_void_p

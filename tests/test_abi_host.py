@@ -96,8 +96,9 @@ def test_decode_rejects_bad_arguments(kvq):
     assert call(_args(kvq, k_codes=A16 + 1)) == E
     assert call(_args(kvq, q_f16=None)) == E
     assert call(_args(kvq, sm_scale=-1.0)) == E
-    assert call(_args(kvq, flags=2)) == E                      # unknown flag bit
+    assert call(_args(kvq, flags=4)) == E                      # unknown flag bit
     assert call(_args(kvq, flags=kvq.KVQ_DECODE_CUDA_CORES)) == kvq.KVQ_ERR_WORKSPACE
+    assert call(_args(kvq, flags=kvq.KVQ_DECODE_TEST_EXPIRE)) == kvq.KVQ_ERR_WORKSPACE
     qjl = dict(key_format=kvq.KVQ_KEYS_QJL, k_words=A16, k_norms_f16=A16, sketch_f16=A16)
     assert call(_args(kvq, sketch_dim=100, **qjl)) == E
     assert call(_args(kvq, sketch_dim=512, **qjl)) == U
