@@ -1974,8 +1974,8 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
 // fp32 rounding of the score and of the merges.
 // -----------------------------------------------------------------------------------
 constexpr int kI8TcTok = 128;
-constexpr int kI8TcKStages = 6;
-constexpr int kI8TcVStages = 6;
+constexpr int kI8TcKStages = 4;
+constexpr int kI8TcVStages = 8;
 constexpr int kI8TcMaxUnits = 4;       // units a CTA range may touch (query digits held)
 constexpr int kI8TcSoft0 = 4;          // first softmax warp
 constexpr int kI8TcTile = kI8TcTok * kD;   // 16 KB
