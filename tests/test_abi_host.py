@@ -220,3 +220,20 @@ def test_gather_multi_rejects_bad_arguments(kvq):
     assert L.kvq_gather_rows_multi(arr, 2, 2, 4, _p(A16 + 2), 10, None) == E    # kept alignment
     assert L.kvq_gather_rows_multi(arr, 0, 2, 4, None, 10, None) == kvq.KVQ_OK
     assert L.kvq_gather_rows_multi(arr, 2, 2, 4, None, 0, None) == kvq.KVQ_OK
+
+
+def test_decode_plan_takes_the_tensor_core_int8_kernel_from_512_tokens(kvq):
+    """The INT8 decode's plan (host side, no GPU: the library then assumes 148 SMs): from
+    512 tokens, with 16-byte aligned code arrays and an output, it runs the tensor-core
+    kernel, one CTA per SM, so its partial states take less workspace than the CUDA-core
+    plan's three CTAs per SM that KVQ_DECODE_CUDA_CORES selects; below 512 tokens, or
+    without an output, both plans are the CUDA-core one."""
+    ws = lambda **kw: kvq.lib.kvq_decode_workspace_bytes(ctypes.byref(_args(kvq, **kw)))
+    cc = kvq.KVQ_DECODE_CUDA_CORES
+    llama = dict(batch=8, n_q_heads=32, n_kv_heads=32, seq_len=4096)      # one 7B-shaped layer
+    assert 0 < ws(**llama) < ws(flags=cc, **llama)
+    assert ws(**llama) == ws(flags=kvq.KVQ_DECODE_TEST_EXPIRE, **llama)
+    short = dict(batch=8, n_q_heads=32, n_kv_heads=32, seq_len=511)
+    assert ws(**short) == ws(flags=cc, **short) > 0
+    # scores only (no output): the CUDA-core kernel
+    assert ws(out=None, scores_out=A16, **llama) == ws(out=None, scores_out=A16, flags=cc, **llama)
