@@ -159,11 +159,12 @@ kvq_status kvq_qjl_query_sketch(const uint16_t* q_f16, int64_t n_q, int32_t d,
  *   per CTA range, fewer than 2^31 token rows): the weighted sum, per chunk of 128 tokens
  *   and head, with the weights p_t * sv_t relative to the chunk's largest p as integers
  *   in units of 2^-E, smax 2^E in [2^23, 2^24) for the chunk's largest value scale smax,
- *   multiplying the INT8 codes exactly in int32 (error at most 2^-24 smax per token);
+ *   multiplying the INT8 codes exactly in int32 (error below 2^-23 smax per token: the
+ *   product p_t * sv_t is rounded to fp32 before its rounding to the fixed point);
  *   INT8 keys (T >= 512, k_codes and v_codes 16-byte aligned, at most 4 units per CTA
  *   range, fewer than 2^31 token rows): the scores, as exact int32 sums of the key codes
  *   times the query written as the fixed-point integer round(q 2^E), max|q| 2^E in
- *   [2^21, 2^22) (error at most 2^-23 max|q| per query entry), rounded once to fp32 and
+ *   [2^21, 2^22) (error at most 2^-22 max|q| per query entry), rounded once to fp32 and
  *   multiplied by s_t; and the weighted sum as for QJL keys, per block of 32 tokens.
  * Everything else runs in fp32 on the CUDA cores.
  * flags (KVQ_DECODE_*): KVQ_DECODE_CUDA_CORES keeps the whole step on the CUDA cores

@@ -1464,8 +1464,9 @@ decode_qjl_pf_kernel(const DecodeParams p) {
 //                D1 2^8 + D0 (exact in int32: |c| <= 127, bytes <= 255, 128 tokens), times
 //                2^-E, merged into the running online-softmax state of each head.
 // The INT8 codes enter the product unconverted and every product and sum is exact; the
-// approximations are the weights' fixed point (absolute error at most 2^-24 smax per
-// token), the sums' 2^-24 fixed point, and the fp32 merges.
+// approximations are the weights' fixed point (absolute error below 2^-23 smax per
+// token: the product is rounded to fp32 before its rounding to the fixed point), the
+// sums' 2^-24 fixed point (at most 2^-25 per token), and the fp32 merges.
 constexpr int kTcTok = 128;                 // tokens per chunk
 constexpr int kTcValueStages = 3;           // value ring: 16 KB tiles
 constexpr int kTcScorerWarps = 8;           // one scorer warp per chunk, chunk c to warp c % 8
@@ -1969,8 +1970,8 @@ decode_qjl_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap v
 // then four merge warps.  The query digits of every unit the CTA visits are formed once,
 // at the start, by softmax group 0.
 // The products and the per-slice sums are exact; the approximations are the query's
-// fixed point (at most 2^-23 max |q| per element), the weights' fixed point (at most
-// 2^-24 of the slice's max value scale per token), the sums' 2^-24 fixed point, and the
+// fixed point (at most 2^-22 max |q| per element), the weights' fixed point (below
+// 2^-23 of the slice's max value scale per token), the sums' 2^-24 fixed point, and the
 // fp32 rounding of the score and of the merges.
 // -----------------------------------------------------------------------------------
 constexpr int kI8TcTok = 128;

@@ -56,10 +56,13 @@ def score_tolerance(ref, norms, v, m, rel=1e-4):
 #  * n_chain: the longest sequential fp32 accumulation in any kernel: a CTA range of W
 #    tokens is split over at least 16 lane groups / warps / chunks, then the lane, warp and
 #    range merges (W <= ceil(B Hkv T nsub / SMs), rounded up to 64);
-#  * the tensor-core value pass rounds each weight of a 128-token chunk to an integer
-#    multiple of 2^-E with smax 2^E in [2^23, 2^24) (at most 2^-24 smax |c| per token,
-#    |c| <= 127) and the softmax sum to 2^-24 per token; both are relative to the chunk's
-#    maximum weight 1, so their share of the output is at most the largest chunk's.
+#  * the tensor-core value pass rounds each weight of a 128-token chunk (or 32-token
+#    slice) to an integer multiple of 2^-E with smax 2^E in [2^23, 2^24), after rounding
+#    the product p * s to fp32 (below 2^-23 smax |c| per token, |c| <= 127), and each
+#    token's share of the softmax sum to 2^-24 (at most 2^-25 per token, 2^-18 relative
+#    for a chunk, whose sum is at least 1); both are relative to the chunk's maximum
+#    weight 1, so their share of the output is at most the largest chunk's
+#    (tests/test_fixedpoint_cpu.py checks these roundings).
 # Dm = max_t (delta_t + rho_t).  Every term is a worst case, not an estimate.
 
 EX2_REL = 2.0 ** -21
@@ -118,7 +121,7 @@ def decode_out_bound(out_ref, p, vals, s_gpu, s_ref, sigma, n_chain, n_rescale, 
     acc = (n_chain + 66) * 2.0 ** -24 * (p @ (np.abs(vals) if vabs is None else vabs) + np.abs(out_ref))
     b = Ew + acc + 1e-30
     if tc_smax is not None:
-        b += 2.0 ** -24 * 128 * 127 * float(tc_smax) + 2.0 ** -20 * np.abs(out_ref)
+        b += 2.0 ** -23 * 128 * 127 * float(tc_smax) + 2.0 ** -18 * np.abs(out_ref)
     return b
 
 
