@@ -43,7 +43,7 @@ def score_tolerance(ref, norms, v, m, rel=1e-4):
 #
 #   |out_gpu - out_ref| <= e^(2 Dm) [ sum_t P_t (rho_t + expm1(delta_t)) |v_t - out_ref| ]
 #                          + (n_chain + 66) 2^-24 (sum_t P_t |v_t| + |out_ref|)
-#                          + [tensor-core value pass] 2^-24 * 128 * 127 * smax + 2^-20 |out_ref|
+#                          + [tensor-core value pass] 2^-23 * 128 * 127 * smax + 2^-18 |out_ref|
 #
 #  * P_t, out_ref: fp64 softmax and weighted sum of the oracle's scores;
 #  * delta_t = sigma |s_gpu,t - s_ref,t|: the GPU's own score deviation (itself held to the
